@@ -1,0 +1,16 @@
+"""CPU oracle for the STQ1_0 matmul -- test infrastructure, never part of the product path.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+and reference legs may import this package.
+"""
+
+from .stq1 import *  # noqa: F401,F403
+from .stq1 import (  # noqa: F401
+    BLOCK_BYTES, BLOCK_WEIGHTS, GROUP, GROUPS_PER_BLOCK, FLAG_WEIGHT_UP,
+    OracleValueError, codebook, pattern_of_code, code_of, code_parts,
+    fp16_bits, fp16_value, bf16_bits_rne, bf16_to_f64,
+    pack_blocks, unpack_blocks, packed_size,
+    encode_plain, encode_sherry, wls_scale, zero_lane_choice, weighted_error,
+    decode, dequant_bf16, gemv, gemv_abs, tolerance, route_pairs, moe_gateup,
+    half_from_struct,
+)

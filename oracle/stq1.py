@@ -1,0 +1,443 @@
+"""CPU oracle for the STQ1_0 quantized matmul -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this module.  The
+library under ``sub_bit_sparse_b200/`` never imports it and has no CPU
+fallback.
+
+Plain, slow and obviously correct: NumPy, fp64 wherever a real number is
+involved, no blocking or fusion beyond what the definitions say.  It shares no
+code with the CUDA path.
+
+Sources (page title, then the section):
+
+* [LEM] lemmy.durstig.online post 66506 (Tencent Hunyuan quantization
+  breakdown): "Four weights, five bits"; "Scale and zero position are fit
+  together"; "Runtime".
+* [AGI] "Tencent compresses 770B Hunyuan Hy4 Preview into 214 GiB at ~2.38
+  bits per weight": "Four weights, five bits"; "Fitting and runtime".
+* [TRA] "Tencent's 200GB Hy4-preview: a 7x compression claim that needs a
+  second look": "MIX-STQ1_0: where the bits go".
+* [ALS] "AngelSlim Shrinks Tencent's 1.5TB Hy4-Preview to 214 GiB at 6x
+  Compression": "How STQ1_0 works" and the bullet list at the top.
+
+What the pages fix: every group of four weights takes values in {-d, 0, +d}
+with exactly one zero lane; 4 zero positions x 8 sign patterns = 32 patterns
+in 5 bits [LEM "Four weights, five bits"]; the 5 bits are a 4-bit code plus a
+1-bit table-select into a 32-entry codebook, and one fp16 scale is shared by
+256 weights, 42 bytes per block, 1.3125 bits per weight [ALS "How STQ1_0
+works"].  The original encoder scales by amax [ALS bullets]; the improved one
+alternates a weighted-least-squares fit of d with an importance-weighted
+choice of the zero lane, three rounds [LEM "Scale and zero position are fit
+together"].
+
+What the pages leave open, and the reading taken here (each is listed in the
+design notes):
+
+1. Block layout (little-endian, 42 bytes, no padding): bytes 0-1 the fp16
+   scale d; bytes 2-33 ``qs[32]``, the 4-bit code of group g is
+   ``(qs[g >> 1] >> 4 * (g & 1)) & 0xF``; bytes 34-41 ``qh[8]``, the select
+   bit of group g is ``(qh[g >> 3] >> (g & 7)) & 1``.  Group g covers the
+   columns 256 b + 4 g + l, l = 0..3.  Blocks are stored row-major: block
+   (j, b) starts at byte (j * K / 256 + b) * 42.
+2. Codebook: with n the 4-bit code and t the select bit, the zero lane is
+   z = n >> 2; the other lanes in ascending order a < b < c carry +1, then
+   -1 if bit 1 of n is set (else +1), then -1 if bit 0 of n is set (else
+   +1); table t = 1 is the negation of table t = 0.
+3. Plain encoder (E0): d = amax of the block, rounded to fp16; in each
+   group the lane of smallest |w| is zeroed (ties: lowest lane) and the
+   others take the sign of w (-0.0 counts as +).
+4. Sherry encoder (E1): start from E0's zero lanes; each round fits d by
+   weighted least squares over the non-zero lanes, then re-picks every
+   group's zero lane as the one whose zeroing adds the least weighted error
+   h_l * d * (2|w_l| - d) (ties: lowest lane); after the last round d is
+   refit for the final zero lanes and rounded to fp16.  All in fp64,
+   sums in ascending column order, the unrounded d between rounds.  If the
+   importance of a whole block is zero the block uses h = 1; if a fit's
+   denominator is zero that fit uses h = 1.
+5. fp64 -> fp16 rounding is direct round-to-nearest-even, saturating at
+   65504 instead of overflowing to infinity.
+6. Matmul: y[t, j] = sum_k W^[j, k] x[t, k] with W^ = pattern * fp32(d).
+   MoE gate/up: y[t, s, :] = W^_{ids[t, s]} x_t, unweighted unless flag bit 0
+   asks to scale the up half (rows N/2..N-1) by the routing weight.
+"""
+
+from __future__ import annotations
+
+import struct
+from typing import Iterable
+
+import numpy as np
+
+BLOCK_WEIGHTS = 256
+GROUP = 4
+GROUPS_PER_BLOCK = BLOCK_WEIGHTS // GROUP   # 64
+BLOCK_BYTES = 42
+OFF_D = 0
+OFF_QS = 2
+OFF_QH = 34
+FP16_MAX = 65504.0
+
+FLAG_WEIGHT_UP = 1
+
+
+class OracleValueError(ValueError):
+    """Non-finite weights, negative importance, or a shape the format cannot hold."""
+
+
+# ---------------------------------------------------------------------------
+# Codebook  [LEM "Four weights, five bits"], [ALS "How STQ1_0 works"]
+# ---------------------------------------------------------------------------
+
+
+def code_parts(code: int):
+    """5-bit code -> (t, n, z, beta, gamma)."""
+    t = (code >> 4) & 1
+    n = code & 0xF
+    return t, n, n >> 2, (n >> 1) & 1, n & 1
+
+
+def pattern_of_code(code: int) -> list[int]:
+    """The 4-lane pattern in {-1, 0, +1} that code ``code`` (0..31) stands for."""
+    t, _, z, beta, gamma = code_parts(code)
+    a, b, c = [lane for lane in range(GROUP) if lane != z]
+    p = [0, 0, 0, 0]
+    p[a] = 1
+    p[b] = -1 if beta else 1
+    p[c] = -1 if gamma else 1
+    if t:
+        p = [-v for v in p]
+    return p
+
+
+def codebook() -> np.ndarray:
+    """All 32 patterns, int8 [32, 4], row = code."""
+    return np.array([pattern_of_code(c) for c in range(32)], dtype=np.int8)
+
+
+def code_of(z: int, negative: Iterable[bool]) -> int:
+    """Encoder side: zero lane z and the sign of each lane (True = negative) -> code.
+
+    t is the sign of the first non-zero lane; bits 1 and 0 of n say whether
+    the second and third non-zero lanes differ in sign from the first.
+    """
+    neg = list(negative)
+    a, b, c = [lane for lane in range(GROUP) if lane != z]
+    t = 1 if neg[a] else 0
+    bit1 = 1 if neg[b] != neg[a] else 0
+    bit0 = 1 if neg[c] != neg[a] else 0
+    return (t << 4) | (z << 2) | (bit1 << 1) | bit0
+
+
+def _code_table() -> np.ndarray:
+    """[4 zero lanes, 16 sign masks] -> code; sign mask bit l = lane l negative."""
+    tab = np.zeros((GROUP, 16), dtype=np.uint8)
+    for z in range(GROUP):
+        for m in range(16):
+            tab[z, m] = code_of(z, [(m >> lane) & 1 == 1 for lane in range(GROUP)])
+    return tab
+
+
+_CODE_TABLE = _code_table()
+_CODEBOOK_F64 = codebook().astype(np.float64)
+
+
+def codes_from_choice(zero_lane: np.ndarray, w_groups: np.ndarray) -> np.ndarray:
+    """Vectorised ``code_of``: zero_lane [..., 64] int, w_groups [..., 64, 4] fp -> codes uint8."""
+    neg = (w_groups < 0).astype(np.int64)   # -0.0 < 0 is False: counts as +
+    mask = neg[..., 0] | (neg[..., 1] << 1) | (neg[..., 2] << 2) | (neg[..., 3] << 3)
+    return _CODE_TABLE[zero_lane, mask]
+
+
+# ---------------------------------------------------------------------------
+# fp16 / bf16 rounding
+# ---------------------------------------------------------------------------
+
+
+def fp16_bits(x) -> np.ndarray:
+    """fp64 -> fp16 bits, round to nearest even, saturating at +/-65504.
+
+    NumPy's float64 -> float16 cast rounds once, directly from double.  NaN or
+    infinite inputs raise ``OracleValueError``.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if not np.all(np.isfinite(x)):
+        raise OracleValueError("non-finite value cannot be stored as an STQ1_0 scale")
+    with np.errstate(over="ignore"):
+        h = x.astype(np.float16)
+    h = np.where(np.isinf(h), np.copysign(np.float16(FP16_MAX), x), h).astype(np.float16)
+    return h.view(np.uint16)
+
+
+def fp16_value(bits) -> np.ndarray:
+    """fp16 bits -> fp64 (exact)."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def bf16_bits_rne(x32: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bits, round to nearest even (finite inputs)."""
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + (((u >> 16) & 1) + 0x7FFF)) >> 16).astype(np.uint16)
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    """bf16 bits -> fp64 (exact)."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Block packing (layout reading 1)
+# ---------------------------------------------------------------------------
+
+
+def pack_blocks(d_bits: np.ndarray, codes: np.ndarray) -> np.ndarray:
+    """d_bits uint16 [B], codes uint8 [B, 64] -> bytes uint8 [B * 42]."""
+    d_bits = np.asarray(d_bits, dtype=np.uint16).reshape(-1)
+    codes = np.asarray(codes, dtype=np.uint8).reshape(-1, GROUPS_PER_BLOCK)
+    nb = d_bits.shape[0]
+    out = np.zeros((nb, BLOCK_BYTES), dtype=np.uint8)
+    out[:, OFF_D] = d_bits & 0xFF
+    out[:, OFF_D + 1] = d_bits >> 8
+    n = codes & 0xF
+    t = (codes >> 4) & 1
+    for g in range(GROUPS_PER_BLOCK):
+        out[:, OFF_QS + (g >> 1)] |= (n[:, g] << (4 * (g & 1))).astype(np.uint8)
+        out[:, OFF_QH + (g >> 3)] |= (t[:, g] << (g & 7)).astype(np.uint8)
+    return out.reshape(-1)
+
+
+def unpack_blocks(packed: np.ndarray):
+    """bytes uint8 [B * 42] -> (d_bits uint16 [B], codes uint8 [B, 64])."""
+    blk = np.asarray(packed, dtype=np.uint8).reshape(-1, BLOCK_BYTES)
+    d_bits = blk[:, OFF_D].astype(np.uint16) | (blk[:, OFF_D + 1].astype(np.uint16) << 8)
+    codes = np.zeros((blk.shape[0], GROUPS_PER_BLOCK), dtype=np.uint8)
+    for g in range(GROUPS_PER_BLOCK):
+        n = (blk[:, OFF_QS + (g >> 1)] >> (4 * (g & 1))) & 0xF
+        t = (blk[:, OFF_QH + (g >> 3)] >> (g & 7)) & 1
+        codes[:, g] = n | (t << 4)
+    return d_bits, codes
+
+
+def packed_size(n: int, k: int) -> int:
+    """Bytes of an [n, k] STQ1_0 matrix."""
+    return n * (k // BLOCK_WEIGHTS) * BLOCK_BYTES
+
+
+def _as_blocks(w: np.ndarray) -> np.ndarray:
+    """[N, K] -> [N * K / 256, 64, 4] in block storage order (row-major blocks)."""
+    n, k = w.shape
+    if k % BLOCK_WEIGHTS:
+        raise OracleValueError("K must be a multiple of 256")
+    return w.reshape(n * (k // BLOCK_WEIGHTS), GROUPS_PER_BLOCK, GROUP)
+
+
+# ---------------------------------------------------------------------------
+# E0: the plain amax encoder  [ALS bullets], [AGI "Fitting and runtime"]
+# ---------------------------------------------------------------------------
+
+
+def encode_plain(w: np.ndarray) -> np.ndarray:
+    """Amax-scaled ternary encoding with the smallest-magnitude lane zeroed."""
+    w = np.asarray(w, dtype=np.float32)
+    if not np.all(np.isfinite(w)):
+        raise OracleValueError("non-finite weight")
+    blocks = _as_blocks(w)
+    aw = np.abs(blocks)
+    amax = aw.reshape(blocks.shape[0], -1).max(axis=1).astype(np.float64)
+    d_bits = fp16_bits(amax)
+    z = np.argmin(aw, axis=2)              # first minimum: lowest lane on ties
+    codes = codes_from_choice(z, blocks)
+    return pack_blocks(d_bits, codes)
+
+
+# ---------------------------------------------------------------------------
+# E1: the Sherry encoder  [LEM "Scale and zero position are fit together"]
+# ---------------------------------------------------------------------------
+
+
+def _nonzero_mask(z: np.ndarray) -> np.ndarray:
+    """zero lanes [B, 64] -> bool [B, 256], True on the lanes that stay non-zero."""
+    lanes = np.arange(GROUP)[None, None, :]
+    return (lanes != z[:, :, None]).reshape(z.shape[0], BLOCK_WEIGHTS)
+
+
+def wls_scale(aw: np.ndarray, h: np.ndarray, z: np.ndarray) -> np.ndarray:
+    """Weighted least-squares scale for fixed zero lanes.
+
+    With s_k = sign(w_k) on the non-zero lanes, the minimiser of
+    sum_k h_k (w_k - d s_k)^2 is d = sum h_k |w_k| / sum h_k over those lanes.
+    Sums run over k in ascending order (sequential fp64).  A zero denominator
+    falls back to h = 1 for that fit.  aw, h: fp64 [B, 256]; z: [B, 64].
+    """
+    nz = _nonzero_mask(z)
+    num = np.zeros(aw.shape[0])
+    den = np.zeros(aw.shape[0])
+    num1 = np.zeros(aw.shape[0])
+    for k in range(BLOCK_WEIGHTS):
+        m = nz[:, k]
+        num = num + np.where(m, h[:, k] * aw[:, k], 0.0)
+        den = den + np.where(m, h[:, k], 0.0)
+        num1 = num1 + np.where(m, aw[:, k], 0.0)
+    zero_den = den == 0.0
+    count = float(BLOCK_WEIGHTS - GROUPS_PER_BLOCK)
+    safe_den = np.where(zero_den, 1.0, den)
+    return np.where(zero_den, num1 / count, num / safe_den)
+
+
+def zero_lane_choice(aw: np.ndarray, h: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """Per group, the lane whose zeroing adds the least weighted error.
+
+    Zeroing lane l instead of giving it sign(w_l) * d raises h_l * w_l^2 -
+    h_l * (|w_l| - d)^2 = h_l * d * (2|w_l| - d); evaluated as
+    (h_l * d) * (2 |w_l| - d).  Ties go to the lowest lane.
+    """
+    B = aw.shape[0]
+    a4 = aw.reshape(B, GROUPS_PER_BLOCK, GROUP)
+    h4 = h.reshape(B, GROUPS_PER_BLOCK, GROUP)
+    dd = d[:, None, None]
+    delta = (h4 * dd) * (2.0 * a4 - dd)
+    return np.argmin(delta, axis=2)
+
+
+def weighted_error(w_blocks: np.ndarray, h: np.ndarray, d: np.ndarray, z: np.ndarray) -> np.ndarray:
+    """sum_k h_k (w_k - d s_k)^2 per block for zero lanes z and s_k = sign(w_k) (fp64)."""
+    aw = np.abs(w_blocks.reshape(w_blocks.shape[0], -1).astype(np.float64))
+    nz = _nonzero_mask(z)
+    r = np.where(nz, aw - d[:, None], aw)
+    return np.sum(h * r * r, axis=1)
+
+
+def encode_sherry(w: np.ndarray, h: np.ndarray | None = None, rounds: int = 3, trace: bool = False):
+    """Alternating WLS scale / importance-weighted zero placement, ``rounds`` rounds.
+
+    ``h`` is the per-column importance (diagonal imatrix), shared by all rows;
+    ``None`` means h = 1.  With ``trace=True`` also returns the per-round
+    scales and zero lanes (for the brute-force checks).
+    """
+    w = np.asarray(w, dtype=np.float32)
+    if not np.all(np.isfinite(w)):
+        raise OracleValueError("non-finite weight")
+    n, k = w.shape
+    blocks = _as_blocks(w)
+    B = blocks.shape[0]
+    if h is None:
+        hcol = np.ones(k)
+    else:
+        hcol = np.asarray(h, dtype=np.float32).astype(np.float64)
+        if hcol.shape != (k,) or not np.all(np.isfinite(hcol)) or np.any(hcol < 0):
+            raise OracleValueError("importance must be finite, >= 0, one value per column")
+    hb = np.broadcast_to(hcol.reshape(1, k), (n, k)).reshape(B, BLOCK_WEIGHTS).copy()
+    all_zero = ~np.any(hb != 0.0, axis=1)
+    hb[all_zero] = 1.0
+    aw = np.abs(blocks.reshape(B, BLOCK_WEIGHTS).astype(np.float64))
+
+    z = np.argmin(np.abs(blocks), axis=2)     # round 0: E0's zero lanes
+    hist = [(None, z.copy())]
+    for _ in range(rounds):
+        d = wls_scale(aw, hb, z)
+        z = zero_lane_choice(aw, hb, d)
+        hist.append((d.copy(), z.copy()))
+    d_final = wls_scale(aw, hb, z)
+    packed = pack_blocks(fp16_bits(d_final), codes_from_choice(z, blocks))
+    if trace:
+        return packed, {"rounds": hist, "d_final": d_final, "h_blocks": hb}
+    return packed
+
+
+# ---------------------------------------------------------------------------
+# Decoder and dequantization
+# ---------------------------------------------------------------------------
+
+
+def decode(packed: np.ndarray, n: int, k: int) -> np.ndarray:
+    """STQ1_0 bytes -> W^ fp64 [n, k], W^ = pattern * fp32(d) (exact)."""
+    if k % BLOCK_WEIGHTS:
+        raise OracleValueError("K must be a multiple of 256")
+    d_bits, codes = unpack_blocks(packed)
+    if d_bits.shape[0] != n * (k // BLOCK_WEIGHTS):
+        raise OracleValueError("packed size does not match the shape")
+    d = fp16_value(d_bits)
+    pat = _CODEBOOK_F64[codes]                # [B, 64, 4]
+    return (pat * d[:, None, None]).reshape(n, k)
+
+
+def dequant_bf16(packed: np.ndarray, n: int, k: int) -> np.ndarray:
+    """W^ as bf16 bits: bf16_RNE(fp32(d)) with the pattern's sign; zero lanes are +0.0."""
+    d_bits, codes = unpack_blocks(packed)
+    d32 = fp16_value(d_bits).astype(np.float32)
+    mag = bf16_bits_rne(d32)                  # d >= 0 for every encoder here; sign kept if not
+    pat = codebook()[codes]                   # [B, 64, 4]
+    magb = np.broadcast_to(mag[:, None, None], pat.shape)
+    out = np.where(pat == 0, np.uint16(0),
+                   np.where(pat < 0, magb ^ np.uint16(0x8000), magb)).astype(np.uint16)
+    return out.reshape(n, k)
+
+
+# ---------------------------------------------------------------------------
+# Contractions  [LEM "Runtime"]
+# ---------------------------------------------------------------------------
+
+
+def gemv(packed: np.ndarray, x_bits: np.ndarray, n: int, k: int) -> np.ndarray:
+    """y [b, n] = W^ x, fp64 (x: bf16 bits [b, k])."""
+    w = decode(packed, n, k)
+    x = bf16_to_f64(np.asarray(x_bits).reshape(-1, k))
+    return x @ w.T
+
+
+def gemv_abs(packed: np.ndarray, x_bits: np.ndarray, n: int, k: int) -> np.ndarray:
+    """sum_k |W^[j, k] x[t, k]|, the scale of the tolerance bound, fp64 [b, n]."""
+    w = np.abs(decode(packed, n, k))
+    x = np.abs(bf16_to_f64(np.asarray(x_bits).reshape(-1, k)))
+    return x @ w.T
+
+
+def tolerance(abs_sum: np.ndarray) -> np.ndarray:
+    """|y_gpu - y_oracle| <= 1e-3 * sum|W x| + 1e-6."""
+    return 1e-3 * abs_sum + 1e-6
+
+
+def route_pairs(ids: np.ndarray, n_experts: int):
+    """Token-slot pairs grouped by expert: (counts [E], offsets [E + 1], pairs sorted by
+    (expert, pair index)).  Pair index p = t * topk + s."""
+    ids = np.asarray(ids, dtype=np.int64)
+    if np.any(ids < 0) or np.any(ids >= n_experts):
+        raise OracleValueError("expert id out of range")
+    flat = ids.reshape(-1)
+    counts = np.bincount(flat, minlength=n_experts)
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    order = np.argsort(flat, kind="stable")
+    return counts, offsets, order
+
+
+def moe_gateup(expert_packed, x_bits: np.ndarray, ids: np.ndarray, weights: np.ndarray,
+               n: int, k: int, flags: int = 0, abs_sum: bool = False):
+    """y [T, topk, n] with y[t, s] = W^_{ids[t, s]} x_t (fp64).
+
+    ``expert_packed(e)`` returns expert e's bytes (or pass a list/array indexed by e).
+    Flag bit 0 scales the up half (rows n/2 .. n-1) by weights[t, s].
+    With ``abs_sum=True`` also returns sum_k |W^ x| for the tolerance.
+    """
+    ids = np.asarray(ids)
+    T, topk = ids.shape
+    get = expert_packed if callable(expert_packed) else (lambda e: expert_packed[e])
+    x = bf16_to_f64(np.asarray(x_bits).reshape(T, k))
+    y = np.zeros((T, topk, n))
+    ya = np.zeros((T, topk, n)) if abs_sum else None
+    for e in np.unique(ids):
+        tt, ss = np.nonzero(ids == e)
+        w = decode(get(int(e)), n, k)
+        y[tt, ss] = x[tt] @ w.T
+        if abs_sum:
+            ya[tt, ss] = np.abs(x[tt]) @ np.abs(w).T
+    if flags & FLAG_WEIGHT_UP:
+        wt = np.asarray(weights, dtype=np.float32).astype(np.float64)[:, :, None]
+        y[:, :, n // 2:] *= wt
+        if abs_sum:
+            ya[:, :, n // 2:] *= np.abs(wt)
+    return (y, ya) if abs_sum else y
+
+
+def half_from_struct(x: float) -> int:
+    """IEEE binary16 bits of x via Python's struct (round-half-even), for cross-checks."""
+    return struct.unpack("<H", struct.pack("<e", x))[0]
