@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark of the STQ1_0 decode GEMV (and MoE gate/up) on B200.
+
+Default (N = 1) workload: decode GEMV on expert-shaped STQ1_0 matrices,
+[4096, 7168] (fused gate+up of 2 x 2048 rows over hidden 7168), encoded by the
+WLS / weighted-zero-placement encoder with importance from 512 synthetic
+calibration vectors; bf16 activations, batch 1, fp32 accumulation.
+
+One step = one decode pass over a stack of L = 64 distinct such matrices
+(308 MB of packed weights, more than twice the 126 MB L2), i.e. 64 GEMV
+launches replayed from a CUDA graph, the same activation vector each time.
+``value`` = packed weight bytes streamed per second (GB/s) over the timed
+steps.  Extra keys report the same GEMV at batch 2/4/8 and the MoE decode
+gate/up workload (16 tokens, top-8 of 256 experts) in tokens/s.
+
+Multi-GPU: every rank runs the same per-rank workload (weak scaling, no
+collective on the data path); the time is the max over ranks.
+
+``--impl reference`` times the CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("STQ1_0 GEMV packed-weight GB/s & % HBM roofline; MoE gate/up tokens/s (1×B200)")
+N_ROWS, K_COLS = 4096, 7168
+PACKED = N_ROWS * (K_COLS // 256) * 42          # 4,816,896 bytes per matrix
+STACK = 64                                      # matrices per step
+HBM_NOMINAL_GBS = 8000.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("bf16_tflops", 1672.0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, sampled from a thread)
+# ---------------------------------------------------------------------------
+
+
+class ClockSampler:
+    REASONS = {
+        "hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+        "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# workload construction
+# ---------------------------------------------------------------------------
+
+
+def build_stack(torch, stq1, device):
+    """L distinct encoded matrices on the device: the WLS-encoded decode matrix and
+    copies whose block order is rotated (same statistics, distinct bytes)."""
+    import workloads
+    w, h, x = workloads.decode_gemv_inputs()
+    packed = stq1.quantize_ref(w, h, mode="sherry", rounds=3)
+    base = torch.from_numpy(packed).to(device)
+    blocks = base.view(-1, 42)
+    nblk = blocks.shape[0]
+    stack = torch.empty((STACK, PACKED), dtype=torch.uint8, device=device)
+    for i in range(STACK):
+        shift = (i * 7919) % nblk
+        stack[i].view(-1, 42).copy_(torch.roll(blocks, shifts=shift, dims=0))
+    return packed, stack, x
+
+
+def time_graph(torch, fn, steps, warmup, stream):
+    """Captures one step into a CUDA graph, runs `warmup` replays, then times `steps`."""
+    with torch.cuda.stream(stream):
+        fn()                                  # configure kernels before capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    return g
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import sub_bit_sparse_b200 as stq1
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device)
+    hbm_peak, bf16_peak, peak_kind = _peaks()
+
+    packed, stack, x_bits = build_stack(torch, stq1, device)
+    xs = torch.from_numpy(x_bits.view(np.int16)).to(device).view(torch.bfloat16)   # [8, K]
+    y_all = torch.empty((STACK, 8, N_ROWS), dtype=torch.float32, device=device)
+    ws = stq1.workspace(max(stq1.LIB.stq1_gemv_workspace(N_ROWS, K_COLS, b) for b in (1, 2, 4, 8)), device)
+
+    def make_step(b):
+        xb = xs[:b].contiguous()
+        def step():
+            for i in range(STACK):
+                stq1.gemv(stack[i], xb, N_ROWS, K_COLS, out=y_all[i, :b], ws=ws)
+        return step
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(g, steps):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(steps):
+                g.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        ms = start.elapsed_time(end)
+        barrier()
+        if world > 1:
+            t = torch.tensor([ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    # --- headline: batch 1 ---
+    g1 = time_graph(torch, make_step(1), args.steps, args.warmup, stream)
+    with ClockSampler(local) as clk:
+        ms = timed(g1, args.steps)
+    ms_step = ms / args.steps
+    launch_ms = ms_step / STACK
+    bytes_step = STACK * PACKED
+    value = world * bytes_step * args.steps / (ms * 1e-3) / 1e9
+    achieved = PACKED / (launch_ms * 1e-3) / 1e9
+
+    # --- the same GEMV at larger batches ---
+    batches = {}
+    for b in (2, 4, 8):
+        gb = time_graph(torch, make_step(b), max(1, args.steps // 4), 3, stream)
+        msb = timed(gb, max(1, args.steps // 4)) / max(1, args.steps // 4)
+        batches[str(b)] = {"gbs": round(bytes_step / (msb * 1e-3) / 1e9, 1),
+                           "ms_per_step": round(msb, 4)}
+        del gb
+
+    # --- MoE decode gate/up (16 tokens, top-8 of 256 experts) ---
+    moe = run_moe(torch, stq1, device, stream, args, world, timed)
+
+    # --- end to end through the public API with host buffers ---
+    e2e = run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier)
+
+    # --- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only) ---
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(packed, x_bits, seconds=args.cpu_seconds)
+
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        try:
+            with open(prof) as f:
+                traffic = json.load(f).get("lut_gemv_kernel_bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": "STQ1_0 decode GEMV, W [4096, 7168] WLS-encoded (1.3125 bpw), x bf16 batch 1, "
+                        "fp32 accumulation; one step = 64 distinct matrices (308 MB packed)",
+            "global_batch": 1, "l2": "inputs larger than L2 (64 x 4.8 MB packed matrices rotate)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "launch": "CUDA graph of 64 GEMV launches per step",
+        },
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                     "peak_kind": peak_kind, "frac_of_nominal_8tbs": round(achieved / HBM_NOMINAL_GBS, 4),
+                     "kernel": "lut_gemv_kernel<1>", "algorithmic_bytes_per_launch": PACKED},
+        "gemv_batches": batches,
+        "moe_decode": moe,
+        "e2e": e2e,
+        "gpu_launches": args.steps * STACK,
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g1
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_moe(torch, stq1, device, stream, args, world, timed):
+    import workloads
+    E, n, k = 256, N_ROWS, K_COLS
+    eb = PACKED
+    flat = torch.empty(E * eb, dtype=torch.uint8, device=device)
+    g = torch.Generator(device=device)
+    g.manual_seed(2024)
+    flat.copy_(torch.randint(0, 256, (E * eb,), dtype=torch.uint8, device=device, generator=g))
+    blk = flat.view(-1, 42)
+    d = (0.058 * (1 + 0.1 * torch.randn(blk.shape[0], device=device, generator=g))).to(torch.float16)
+    blk[:, 0:2].copy_(d.view(torch.uint8).view(-1, 2))
+    x, ids, wts = workloads.moe_decode_inputs()
+    xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    idd = torch.from_numpy(ids).to(device)
+    wd = torch.from_numpy(wts).to(device)
+    y = torch.empty((16, 8, n), dtype=torch.float32, device=device)
+    ws = stq1.workspace(stq1.LIB.stq1_moe_workspace(16, 8, E, n, k, 0), device, kind="moe")
+
+    def step():
+        stq1.moe_gateup(flat, xd, idd, wd, n, k, E, out=y, ws=ws)
+
+    steps = max(1, args.steps // 8)
+    gm = time_graph(torch, step, steps, 3, stream)
+    ms = timed(gm, steps) / steps
+    uniq = len(np.unique(ids))
+    del gm
+    return {"tokens_per_s": round(world * 16 / (ms * 1e-3), 1), "ms_per_call": round(ms, 4),
+            "unique_experts": int(uniq), "expert_bytes_read": int(uniq * eb),
+            "gbs": round(uniq * eb / (ms * 1e-3) / 1e9, 1),
+            "config": "256 experts x [4096, 7168] STQ1_0, 16 tokens, Zipf(1.1) top-8, unweighted"}
+
+
+def run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier):
+    """Public API, host buffers: per step copy x in from pinned memory, run the 64
+    GEMVs, read all outputs back to pinned memory."""
+    xh = torch.empty((1, K_COLS), dtype=torch.bfloat16).pin_memory()
+    xh.copy_(xs[:1].cpu())
+    yh = torch.empty((STACK, 1, N_ROWS), dtype=torch.float32).pin_memory()
+    xd = torch.empty((1, K_COLS), dtype=torch.bfloat16, device=device)
+    yd = torch.empty((STACK, 1, N_ROWS), dtype=torch.float32, device=device)
+    steps = max(1, args.steps // 10)
+
+    def one():
+        xd.copy_(xh, non_blocking=True)
+        for i in range(STACK):
+            stq1.gemv(stack[i], xd, N_ROWS, K_COLS, out=yd[i], ws=ws)
+        yh.copy_(yd, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            one()
+    torch.cuda.synchronize()
+    barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(steps):
+            one()
+        end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(world * STACK * PACKED * steps / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": K_COLS * 2, "d2h_bytes_per_step": STACK * N_ROWS * 4,
+            "steps": steps, "ms_per_step": round(ms / steps, 4)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+# ---------------------------------------------------------------------------
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        return 1
+
+
+def _oracle_sample(packed, x_bits, rows):
+    import oracle
+    rb = (K_COLS // 256) * 42
+    sub = packed[: rows * rb]
+    return oracle.gemv(sub, x_bits[:1], rows, K_COLS)
+
+
+def cpu_baseline(packed, x_bits, seconds=10.0):
+    """The oracle (decode + fp64 matmul) on row samples of the decode matrix."""
+    rows = 256
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < seconds:
+        _oracle_sample(packed, x_bits, rows)
+        n += 1
+    dt = time.perf_counter() - t0
+    rb = (K_COLS // 256) * 42
+    return {"value": round(n * rows * rb / dt / 1e9, 6), "unit": "GB/s", "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} oracle GEMVs of {rows} x {K_COLS} rows of the WLS-encoded decode matrix, "
+                      f"batch 1, {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm, on a bounded sample per step (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import workloads
+    import oracle
+    w, h, x = workloads.decode_gemv_inputs()
+    rows = 32
+    packed = oracle.encode_sherry(w[:rows], h, rounds=3)
+    rb = (K_COLS // 256) * 42
+    for _ in range(args.warmup):
+        oracle.gemv(packed, x[:1], rows, K_COLS)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.gemv(packed, x[:1], rows, K_COLS)
+    dt = time.perf_counter() - t0
+    value = args.steps * rows * rb / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "CPU oracle: decode + fp64 GEMV of a 32-row sample of the "
+                               "WLS-encoded [4096, 7168] decode matrix per step, batch 1"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": _blas_threads(),
+                         "kind": "oracle", "sample": f"{rows} rows x {K_COLS} per step"},
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def profile_case(args):
+    """Small launch sequence for ncu captures: the decode GEMV on 64 distinct
+    [4096, 7168] matrices (308 MB, larger than L2), 32 launches, batch 1
+    (or the MoE decode call with --profile-case moe)."""
+    import torch
+    import sub_bit_sparse_b200 as stq1
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    if args.profile_case == "moe":
+        stream = torch.cuda.current_stream()
+        out = run_moe(torch, stq1, device, stream, argparse.Namespace(steps=8), 1,
+                      lambda g, steps: 0.0)
+        print(json.dumps(out))
+        return
+    _, stack, x_bits = build_stack(torch, stq1, device)
+    xs = torch.from_numpy(x_bits.view(np.int16)).to(device).view(torch.bfloat16)
+    y = torch.empty((1, N_ROWS), dtype=torch.float32, device=device)
+    ws = stq1.workspace(stq1.LIB.stq1_gemv_workspace(N_ROWS, K_COLS, 1), device)
+    for i in range(32):
+        stq1.gemv(stack[i % STACK], xs[:1], N_ROWS, K_COLS, out=y, ws=ws)
+    torch.cuda.synchronize()
+    print("profile case done", float(y.abs().sum()))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", default=None, choices=["gemv", "moe"])
+    args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args)
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+/*
+ * stq1.h -- C ABI of the STQ1_0 quantized-matmul library (libstq1.so), sm_100a.
+ *
+ * STQ1_0 stores weights in groups of four lanes whose values are {-d, 0, +d}
+ * with exactly one zero lane; the 32 possible patterns are a 5-bit code, and
+ * one fp16 scale d is shared by 256 weights (lemmy.durstig.online post 66506,
+ * "Four weights, five bits").  Each group's code is a 4-bit code plus a 1-bit
+ * table-select into a 32-entry codebook; a 256-weight block is 42 bytes,
+ * 1.3125 bits per weight ("AngelSlim Shrinks Tencent's 1.5TB Hy4-Preview to
+ * 214 GiB at 6x Compression", "How STQ1_0 works").
+ *
+ * Block layout (the pages fix the semantics, not the bits; this library fixes
+ * them as follows), little-endian, 42 bytes, no padding:
+ *   bytes  0..1   d, IEEE binary16
+ *   bytes  2..33  qs[32]: the 4-bit code n of group g is
+ *                 (qs[g >> 1] >> (4 * (g & 1))) & 0xF
+ *   bytes 34..41  qh[8]:  the select bit t of group g is
+ *                 (qh[g >> 3] >> (g & 7)) & 1
+ * Group g (0..63) holds columns 256*b + 4*g + l, l = 0..3.  Codebook: the zero
+ * lane is z = n >> 2; the other lanes, in ascending order a < b < c, carry
+ * +1, (bit 1 of n ? -1 : +1), (bit 0 of n ? -1 : +1); t = 1 negates all
+ * three.  Decoded weight = pattern value * d.
+ * Matrix layout: an [N, K] matrix (K % 256 == 0) is N*K/256 blocks stored
+ * row-major; block (j, b) starts at byte (j * K/256 + b) * 42.
+ *
+ * Conventions for every call:
+ *   - Return value: STQ1_OK (0) or a negative STQ1_ERR_* code.  Nothing
+ *     throws across this boundary; arguments are checked on the host before
+ *     any work is enqueued, and a failed check enqueues nothing.
+ *   - Device pointers are raw CUDA device addresses owned by the caller; the
+ *     library never allocates, frees or retains them after the call returns
+ *     (work enqueued on the stream still reads them until it completes).
+ *   - Device calls are asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  Errors found on the device (for example an
+ *     expert id outside [0, E)) do not trap: the kernel records a code in a
+ *     device error word, skips the bad item and finishes; stq1_status()
+ *     reads and clears that word.
+ *   - bf16 and fp16 values are passed as uint16_t bit patterns.
+ */
+#ifndef STQ1_H
+#define STQ1_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define STQ1_OK 0
+#define STQ1_ERR_SHAPE (-1)       /* K % 256 != 0, a non-positive size, too large a size */
+#define STQ1_ERR_NULL (-2)        /* a required pointer is NULL */
+#define STQ1_ERR_CUDA (-3)        /* a CUDA runtime call failed (launch error etc.) */
+#define STQ1_ERR_DEVICE (-4)      /* (stq1_status) the device error word was set */
+#define STQ1_ERR_VALUE (-5)       /* NaN/Inf weight, negative or non-finite importance */
+#define STQ1_ERR_ALIGN (-6)       /* a pointer is not 16-byte aligned */
+#define STQ1_ERR_WORKSPACE (-7)   /* workspace NULL or smaller than the query says */
+#define STQ1_ERR_ARG (-8)         /* an invalid mode, flag or option */
+
+/* Device error word bits (reported through stq1_status). */
+#define STQ1_DEV_BAD_EXPERT 1     /* a topk id was outside [0, E); its slot was skipped */
+#define STQ1_DEV_WAIT_LIMIT 2     /* a bounded wait inside a kernel gave up */
+
+/* Encoder modes for stq1_quantize_ref. */
+#define STQ1_ENC_PLAIN 0          /* amax scale, smallest-|w| lane zeroed */
+#define STQ1_ENC_SHERRY 1         /* alternating WLS scale / weighted zero placement */
+
+/* stq1_moe_gateup flags. */
+#define STQ1_MOE_WEIGHT_UP 1      /* multiply rows N/2..N-1 (the up half) by the routing weight */
+#define STQ1_MOE_FP8 2            /* large-token path: e4m3 activations (error reported, not gated) */
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int stq1_version(void);
+
+/*
+ * stq1_quantize_ref -- host encoder (CPU only, deterministic, multi-threaded).
+ *
+ * Plain mode (amax encoder: "AngelSlim Shrinks ...", bullet list): per block
+ * d = fp16(max |w|) rounded to nearest-even and saturated at 65504; in each
+ * group the lane of least |w| is zero (ties: lowest lane) and the others take
+ * the sign of w (-0.0 counts as positive).
+ * Sherry mode (lemmy.durstig.online post 66506, "Scale and zero position are
+ * fit together"): start from the plain zero lanes; `rounds` times fit
+ * d = sum h|w| / sum h over the non-zero lanes (weighted least squares), then
+ * re-pick each group's zero lane as the one minimising h_l*d*(2|w_l| - d), the
+ * extra weighted error of zeroing it (ties: lowest lane); finally refit d for
+ * the final lanes and round it to fp16.  Arithmetic is IEEE fp64 with sums in
+ * ascending column order; a block whose importance is all zero uses h = 1, a
+ * fit whose denominator is zero uses h = 1.
+ *
+ *   W       [N, K] fp32, row-major, host memory (read only).
+ *   h       [K] fp32 per-column importance (diagonal imatrix), host memory;
+ *           NULL means h = 1.  Ignored in plain mode.
+ *   mode    STQ1_ENC_PLAIN or STQ1_ENC_SHERRY.
+ *   rounds  number of alternating rounds for Sherry mode (>= 0; the pages use 3).
+ *   out     host buffer of N*K/256*42 bytes, written completely.
+ *   threads worker threads (<= 0: use the hardware concurrency).
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE (K % 256, N <= 0), STQ1_ERR_VALUE
+ * (non-finite weight, negative or non-finite h), STQ1_ERR_ARG (mode, rounds).
+ * On error `out` may be partly written.
+ */
+int stq1_quantize_ref(const float* W, const float* h, int64_t N, int64_t K, int mode,
+                      int rounds, uint8_t* out, int threads);
+
+/*
+ * stq1_dequant -- decoded weights as bf16 (device).
+ * W_bf16[j, k] = bf16_rne(fp32(d)) with the pattern's sign, zero lanes +0.0.
+ *   W_packed  device, N*K/256*42 bytes, 16-byte aligned.
+ *   W_bf16    device, [N, K] uint16 (bf16 bits), 16-byte aligned.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_ALIGN, STQ1_ERR_CUDA.
+ */
+int stq1_dequant(const void* W_packed, uint16_t* W_bf16, int64_t N, int64_t K, void* stream);
+
+/*
+ * stq1_gemv_workspace -- bytes of device workspace stq1_gemv needs for this
+ * shape (0 if none).  Layout: the first 2048 bytes hold split-K arrival
+ * counters, the rest partial sums.  The counter bytes must be zero before the
+ * first call; every call that completes leaves them zero again, whatever the
+ * shape, so one workspace can serve calls of different shapes (not
+ * concurrently).  Do not share it with stq1_moe_gateup.
+ */
+size_t stq1_gemv_workspace(int64_t N, int64_t K, int batch);
+
+/*
+ * stq1_gemv -- y[t, j] = sum_k W^[j, k] x[t, k], fp32 accumulation.
+ * The decoded weight is never materialised: codes are expanded through a
+ * per-group lookup table of the activation sums, so the weight side has no
+ * multiplies ("Runtime" section of the lemmy post: STQ1_0 CUDA kernels).
+ * Small batches use the lookup-table kernel; larger batches the tensor-core
+ * tile kernel.
+ *   W_packed   device, [N, K] STQ1_0 blocks, 16-byte aligned.
+ *   x          device, [batch, K] bf16 bits, row-major, 16-byte aligned.
+ *   y          device, [batch, N] fp32, row-major (fully overwritten).
+ *   batch      1 .. 65535.
+ *   workspace  device, at least stq1_gemv_workspace(N, K, batch) bytes,
+ *              16-byte aligned (may be NULL when that is 0).
+ * Accuracy: |y - y_exact| <= 1e-3 * sum_k |W^[j,k] x[t,k]| + 1e-6.
+ * Calls that share a workspace must not run concurrently.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_ALIGN, STQ1_ERR_WORKSPACE,
+ * STQ1_ERR_CUDA.
+ */
+int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int64_t N, int64_t K,
+              int batch, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * stq1_moe_workspace -- bytes of device workspace stq1_moe_gateup needs
+ * (routing tables; no zero-fill needed).  Calls sharing it must not overlap.
+ */
+size_t stq1_moe_workspace(int T, int topk, int E, int64_t N, int64_t K, int flags);
+
+/*
+ * stq1_moe_gateup -- routed expert gate/up projections for top-k MoE.
+ * y[t, s, :] = W^_{e} x[t, :] with e = topk_ids[t, s] (unweighted), for the
+ * fused gate (rows 0..N/2-1) + up (rows N/2..N-1) matrix of each expert.
+ * Token-slot pairs are grouped by expert on the device and only the routed
+ * experts' blocks are read (256 routed experts, top-8: lemmy post,
+ * "Precision follows weight sensitivity").
+ *   expert_blocks  device, E consecutive [N, K] STQ1_0 matrices, 16-byte aligned.
+ *   x              device, [T, K] bf16 bits, 16-byte aligned.
+ *   topk_ids       device, [T, topk] int32.
+ *   topk_weights   device, [T, topk] fp32; read only with STQ1_MOE_WEIGHT_UP
+ *                  (may be NULL otherwise).
+ *   y              device, [T, topk, N] fp32 (fully overwritten; a slot whose
+ *                  id is out of range is set to 0 and flagged in the error word).
+ *   flags          STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8.
+ *   ws, ws_bytes   device workspace, at least stq1_moe_workspace(...) bytes.
+ * Requires N even, K % 256 == 0, 1 <= topk <= E.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_ALIGN, STQ1_ERR_WORKSPACE,
+ * STQ1_ERR_ARG, STQ1_ERR_CUDA.
+ */
+int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, const int32_t* topk_ids,
+                    const float* topk_weights, float* y, int T, int topk, int E, int64_t N,
+                    int64_t K, int flags, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * stq1_status -- synchronise `stream`, return STQ1_OK if no device error was
+ * recorded since the last call, else STQ1_ERR_DEVICE with the bits in
+ * *device_err (may be NULL).  Clears the word.  STQ1_ERR_CUDA if the
+ * synchronisation itself fails.
+ */
+int stq1_status(void* stream, int* device_err);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STQ1_H */

@@ -1,0 +1,219 @@
+"""Python binding of libstq1.so, the STQ1_0 quantized-matmul library for B200 (sm_100a).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels (or, for ``quantize_ref``, its C++ host encoder).
+PyTorch supplies device memory and the current CUDA stream.  There is no CPU
+fallback: if the compiled library is missing, importing this package raises.
+
+The functions mirror the C ABI declared in ``include/stq1.h``:
+``quantize_ref``, ``dequant``, ``gemv``, ``moe_gateup``, ``status``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libstq1.so")
+
+OK = 0
+ERRORS = {
+    -1: "STQ1_ERR_SHAPE", -2: "STQ1_ERR_NULL", -3: "STQ1_ERR_CUDA", -4: "STQ1_ERR_DEVICE",
+    -5: "STQ1_ERR_VALUE", -6: "STQ1_ERR_ALIGN", -7: "STQ1_ERR_WORKSPACE", -8: "STQ1_ERR_ARG",
+}
+DEV_BAD_EXPERT = 1
+DEV_WAIT_LIMIT = 2
+ENC_PLAIN = 0
+ENC_SHERRY = 1
+MOE_WEIGHT_UP = 1
+MOE_FP8 = 2
+BLOCK_BYTES = 42
+BLOCK_WEIGHTS = 256
+
+# Every symbol include/stq1.h declares: name -> (restype, argtypes)
+_c = ctypes
+SIGNATURES = {
+    "stq1_version": (_c.c_int, []),
+    "stq1_quantize_ref": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int,
+                                     _c.c_int, _c.c_void_p, _c.c_int]),
+    "stq1_dequant": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p]),
+    "stq1_gemv_workspace": (_c.c_size_t, [_c.c_int64, _c.c_int64, _c.c_int]),
+    "stq1_gemv": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int,
+                             _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "stq1_moe_workspace": (_c.c_size_t, [_c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int]),
+    "stq1_moe_gateup": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                   _c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
+                                   _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "stq1_status": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
+}
+
+
+class Stq1Error(RuntimeError):
+    def __init__(self, func: str, code: int, device_err: int = 0):
+        self.code = code
+        self.device_err = device_err
+        super().__init__(f"{func} returned {ERRORS.get(code, code)}"
+                         + (f" (device error bits {device_err:#x})" if device_err else ""))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libstq1.so not found at {LIB_PATH}; build it with "
+            "`python -m sub_bit_sparse_b200.build` (needs the CUDA toolkit)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+def _check(func: str, rc: int):
+    if rc != OK:
+        raise Stq1Error(func, rc)
+
+
+def packed_bytes(n: int, k: int) -> int:
+    """Size in bytes of an [n, k] STQ1_0 matrix."""
+    return n * (k // BLOCK_WEIGHTS) * BLOCK_BYTES
+
+
+# ---------------------------------------------------------------------------
+# Host encoder
+# ---------------------------------------------------------------------------
+
+
+def quantize_ref(w: np.ndarray, h: np.ndarray | None = None, mode: str = "plain", rounds: int = 3,
+                 threads: int = 0) -> np.ndarray:
+    """Encodes fp32 weights [N, K] with the host encoder; returns N*K/256*42 bytes (uint8)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    if w.ndim != 2:
+        raise ValueError("w must be [N, K]")
+    n, k = w.shape
+    hh = None if h is None else np.ascontiguousarray(h, dtype=np.float32)
+    out = np.empty(max(packed_bytes(n, k), 1), dtype=np.uint8)
+    m = {"plain": ENC_PLAIN, "sherry": ENC_SHERRY}[mode]
+    rc = LIB.stq1_quantize_ref(w.ctypes.data, None if hh is None else hh.ctypes.data, n, k, m, rounds,
+                               out.ctypes.data, threads)
+    _check("stq1_quantize_ref", rc)
+    return out[: packed_bytes(n, k)]
+
+
+# ---------------------------------------------------------------------------
+# Device calls
+# ---------------------------------------------------------------------------
+
+_ws_lock = threading.Lock()
+_ws_cache: dict = {}
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def workspace(nbytes: int, device, kind: str = "gemv") -> "torch.Tensor | None":
+    """A cached, zero-filled device workspace of at least ``nbytes`` for one kind of call
+    ("gemv" or "moe"); the GEMV kind keeps its counter bytes zero between calls."""
+    if nbytes == 0:
+        return None
+    torch = _torch()
+    dev = torch.device(device)
+    idx = dev.index if dev.index is not None else torch.cuda.current_device()
+    key = (idx, kind)
+    with _ws_lock:
+        buf = _ws_cache.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=f"cuda:{idx}")
+            _ws_cache[key] = buf
+        return buf
+
+
+def _stream(t):
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _require(t, dtype, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def dequant(w_packed, n: int, k: int, out=None):
+    """Decoded weights [n, k] as bf16."""
+    torch = _torch()
+    _require(w_packed, torch.uint8, "w_packed")
+    if out is None:
+        out = torch.empty((n, k), dtype=torch.bfloat16, device=w_packed.device)
+    _require(out, torch.bfloat16, "out")
+    rc = LIB.stq1_dequant(w_packed.data_ptr(), out.data_ptr(), n, k, _stream(w_packed))
+    _check("stq1_dequant", rc)
+    return out
+
+
+def gemv(w_packed, x, n: int, k: int, out=None, ws=None):
+    """y [b, n] fp32 = W^ x for x [b, k] bf16."""
+    torch = _torch()
+    _require(w_packed, torch.uint8, "w_packed")
+    _require(x, torch.bfloat16, "x")
+    b = x.shape[0] if x.dim() == 2 else 1
+    if out is None:
+        out = torch.empty((b, n), dtype=torch.float32, device=x.device)
+    _require(out, torch.float32, "out")
+    need = LIB.stq1_gemv_workspace(n, k, b)
+    if ws is None:
+        ws = workspace(need, x.device)
+    rc = LIB.stq1_gemv(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b,
+                       None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
+                       _stream(x))
+    _check("stq1_gemv", rc)
+    return out
+
+
+def moe_gateup(expert_blocks, x, topk_ids, topk_weights, n: int, k: int, n_experts: int, flags: int = 0,
+               out=None, ws=None):
+    """y [T, topk, n] fp32: each token's routed experts' fused gate/up projections."""
+    torch = _torch()
+    _require(expert_blocks, torch.uint8, "expert_blocks")
+    _require(x, torch.bfloat16, "x")
+    _require(topk_ids, torch.int32, "topk_ids")
+    if topk_weights is not None:
+        _require(topk_weights, torch.float32, "topk_weights")
+    t, topk = topk_ids.shape
+    if out is None:
+        out = torch.empty((t, topk, n), dtype=torch.float32, device=x.device)
+    _require(out, torch.float32, "out")
+    need = LIB.stq1_moe_workspace(t, topk, n_experts, n, k, flags)
+    if ws is None:
+        ws = workspace(need, x.device, kind="moe")
+    rc = LIB.stq1_moe_gateup(expert_blocks.data_ptr(), x.data_ptr(), topk_ids.data_ptr(),
+                             None if topk_weights is None else topk_weights.data_ptr(), out.data_ptr(),
+                             t, topk, n_experts, n, k, flags,
+                             None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
+                             _stream(x))
+    _check("stq1_moe_gateup", rc)
+    return out
+
+
+def status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error word; raises on errors."""
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    err = ctypes.c_int(0)
+    rc = LIB.stq1_status(ctypes.c_void_p(s.cuda_stream), ctypes.byref(err))
+    if rc not in (OK, -4):
+        raise Stq1Error("stq1_status", rc)
+    return err.value

@@ -1,0 +1,126 @@
+// Device helpers shared by the STQ1_0 kernels: block-format constants, the
+// codebook, and thin wrappers around the sm_90+/sm_100 PTX the kernels use
+// (mbarriers, 1-D bulk copies, shared-memory loads with immediate offsets).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/stq1.h"
+
+namespace stq1 {
+
+// ---- STQ1_0 block format ("How STQ1_0 works": 42 bytes per 256 weights) ----
+constexpr int kBlockWeights = 256;
+constexpr int kGroupsPerBlock = 64;
+constexpr int kBlockBytes = 42;
+constexpr int kOffD = 0;    // fp16 scale
+constexpr int kOffQs = 2;   // 32 bytes of 4-bit codes, even group in the low nibble
+constexpr int kOffQh = 34;  // 8 bytes of select bits, group g at bit g & 7 of byte g >> 3
+
+// Device error word, read and cleared by stq1_status().
+__device__ int g_dev_err;
+
+__device__ __forceinline__ void flag_error(int bits) { atomicOr(&g_dev_err, bits); }
+
+// Codebook: code = t << 4 | n; zero lane z = n >> 2; non-zero lanes a < b < c
+// carry +1, -(bit1 of n), -(bit0 of n); t = 1 negates them.  Returns the
+// lane values in {-1, 0, +1} (lemmy.durstig.online post 66506, "Four weights,
+// five bits"; the lane order and table split are this library's layout).
+__device__ __forceinline__ void code_pattern(unsigned code, int v[4]) {
+  const unsigned n = code & 15u, t = (code >> 4) & 1u;
+  const unsigned z = n >> 2;
+  const int s = t ? -1 : 1;
+  const int la = (z == 0) ? 1 : 0;
+  const int lb = (z <= 1) ? 2 : 1;
+  const int lc = (z == 3) ? 2 : 3;
+  v[0] = v[1] = v[2] = v[3] = 0;
+  v[la] = s;
+  v[lb] = ((n >> 1) & 1u) ? -s : s;
+  v[lc] = (n & 1u) ? -s : s;
+}
+
+// ---- PTX wrappers ----
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait on an mbarrier phase.  Each try_wait may suspend the thread for
+// a hardware-defined interval; the iteration cap bounds the total to well
+// under a second on any sane clock.  Returns false (and flags the device
+// error word) if the phase did not complete.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  for (uint32_t i = 0; i < (1u << 22); ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  flag_error(STQ1_DEV_WAIT_LIMIT);
+  return false;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completion counted in bytes
+// on `bar`.  dst, src and bytes must all be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+template <int OFF>
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(OFF));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts_v4f(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) {
+  return __uint_as_float(b << 16);
+}
+
+}  // namespace stq1

@@ -1,0 +1,173 @@
+// Routing sort, dequantization and the direct (generic-shape) GEMV.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace stq1 {
+
+// ---------------------------------------------------------------------------
+// Routing: group token-slot pairs by expert (top-k of E routed experts, lemmy
+// post "Precision follows weight sensitivity": 256 routed experts, top-8).
+// One CTA: histogram of ids, exclusive scans of pair counts and of tile
+// counts, tile table, then a scatter of pair ids into per-expert segments.
+// A pair p = t * topk + s.  Pairs with an id outside [0, E) get y = 0 and set
+// STQ1_DEV_BAD_EXPERT.  Order inside a segment is unspecified (it does not
+// change any result: every output row is computed on its own).
+// tile_info[4 * i] = expert, first pair offset, pair count (<= tile_tokens), 0.
+// ---------------------------------------------------------------------------
+constexpr int kRouteThreads = 1024;
+
+__global__ void __launch_bounds__(kRouteThreads)
+route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_tokens,
+             int* __restrict__ pairs_out, int* __restrict__ tile_info, int* __restrict__ n_tiles,
+             float* __restrict__ y, int N) {
+  extern __shared__ int sm[];
+  int* cnt = sm;            // [E]
+  int* off = sm + E;        // [E]
+  int* tst = sm + 2 * E;    // [E]
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
+    const int e = ids[p];
+    if (e < 0 || e >= E) {
+      flag_error(STQ1_DEV_BAD_EXPERT);
+      float* yr = y + static_cast<long long>(p) * N;
+      for (int j = 0; j < N; ++j) yr[j] = 0.f;
+    } else {
+      atomicAdd(&cnt[e], 1);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = (E + 31) / 32;
+    const int lo = min(E, lane * per), hi = min(E, lo + per);
+    int s1 = 0, s2 = 0;
+    for (int e = lo; e < hi; ++e) {
+      s1 += cnt[e];
+      s2 += (cnt[e] + tile_tokens - 1) / tile_tokens;
+    }
+    int i1 = s1, i2 = s2;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v1 = __shfl_up_sync(0xffffffffu, i1, d);
+      const int v2 = __shfl_up_sync(0xffffffffu, i2, d);
+      if (lane >= d) { i1 += v1; i2 += v2; }
+    }
+    int r1 = i1 - s1, r2 = i2 - s2;
+    for (int e = lo; e < hi; ++e) {
+      off[e] = r1;
+      tst[e] = r2;
+      r1 += cnt[e];
+      r2 += (cnt[e] + tile_tokens - 1) / tile_tokens;
+    }
+    if (lane == 31) *n_tiles = i2;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int c = cnt[e];
+    const int nt = (c + tile_tokens - 1) / tile_tokens;
+    for (int k = 0; k < nt; ++k) {
+      int* ti = tile_info + 4 * (tst[e] + k);
+      ti[0] = e;
+      ti[1] = off[e] + k * tile_tokens;
+      ti[2] = min(tile_tokens, c - k * tile_tokens);
+      ti[3] = 0;
+    }
+  }
+  __syncthreads();
+  for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
+    const int e = ids[p];
+    if (e < 0 || e >= E) continue;
+    const int pos = atomicSub(&cnt[e], 1) - 1;
+    pairs_out[off[e] + pos] = p;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Dequantization: one thread per group of four weights, 8-byte stores.
+// W^ = bf16_rne(fp32(d)) with the pattern's sign; zero lanes are +0.0.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+dequant_kernel(const uint8_t* __restrict__ W, uint16_t* __restrict__ out, long long n_groups) {
+  for (long long gid = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; gid < n_groups;
+       gid += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long blk = gid >> 6;
+    const int g = static_cast<int>(gid & 63);
+    const uint8_t* B = W + blk * kBlockBytes;
+    const unsigned short dbits = static_cast<unsigned short>(B[kOffD] | (B[kOffD + 1] << 8));
+    const unsigned n = (B[kOffQs + (g >> 1)] >> (4 * (g & 1))) & 15u;
+    const unsigned t = (B[kOffQh + (g >> 3)] >> (g & 7)) & 1u;
+    const __nv_bfloat16 db = __float2bfloat16_rn(__half2float(__ushort_as_half(dbits)));
+    const uint32_t mag = __bfloat16_as_ushort(db);
+    int v[4];
+    code_pattern(n | (t << 4), v);
+    uint32_t o[4];
+#pragma unroll
+    for (int l = 0; l < 4; ++l) o[l] = v[l] == 0 ? 0u : (v[l] > 0 ? mag : (mag ^ 0x8000u));
+    uint2 pk;
+    pk.x = o[0] | (o[1] << 16);
+    pk.y = o[2] | (o[3] << 16);
+    *reinterpret_cast<uint2*>(out + (blk << 8) + 4 * g) = pk;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Direct GEMV for shapes the table kernel does not take (an odd number of
+// blocks per row): one warp per output element, lanes stride over blocks and
+// decode each group arithmetically.  Correct for any K % 256 == 0; slow.
+// MoE use: ids != nullptr, pair p reads expert ids[p] and token p / topk.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+direct_gemv_kernel(const uint8_t* __restrict__ W, long long expert_bytes, int E,
+                   const uint16_t* __restrict__ x, const int32_t* __restrict__ ids, int topk,
+                   const float* __restrict__ route_w, int flags, float* __restrict__ y, int N,
+                   int K, int rows_out) {
+  const int nb = K / kBlockWeights;
+  const long long gw = blockIdx.x * 8LL + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= static_cast<long long>(rows_out) * N) return;
+  const int p = static_cast<int>(gw / N);
+  const int j = static_cast<int>(gw % N);
+  int e = 0;
+  if (ids) {
+    e = ids[p];
+    if (e < 0 || e >= E) {
+      if (lane == 0) {
+        y[static_cast<long long>(p) * N + j] = 0.f;
+        flag_error(STQ1_DEV_BAD_EXPERT);
+      }
+      return;
+    }
+  }
+  const int tok = ids ? p / topk : p;
+  const uint8_t* Wr = W + e * expert_bytes + static_cast<long long>(j) * nb * kBlockBytes;
+  const uint16_t* xr = x + static_cast<long long>(tok) * K;
+  float acc = 0.f;
+  for (int b = lane; b < nb; b += 32) {
+    const uint8_t* B = Wr + static_cast<long long>(b) * kBlockBytes;
+    const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(B[0] | (B[1] << 8))));
+    float s = 0.f;
+    for (int g = 0; g < kGroupsPerBlock; ++g) {
+      const unsigned n = (B[kOffQs + (g >> 1)] >> (4 * (g & 1))) & 15u;
+      const unsigned t = (B[kOffQh + (g >> 3)] >> (g & 7)) & 1u;
+      int v[4];
+      code_pattern(n | (t << 4), v);
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        const float xv = bf16_bits_to_f32(xr[b * kBlockWeights + 4 * g + l]);
+        if (v[l] > 0) s += xv;
+        else if (v[l] < 0) s -= xv;
+      }
+    }
+    acc = fmaf(d, s, acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
+    if ((flags & STQ1_MOE_WEIGHT_UP) && j >= N / 2 && route_w) acc *= route_w[p];
+    y[static_cast<long long>(p) * N + j] = acc;
+  }
+}
+
+}  // namespace stq1

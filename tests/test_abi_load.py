@@ -1,0 +1,52 @@
+"""The C-ABI library loads without a GPU and exports every symbol include/stq1.h declares."""
+
+import ctypes
+import os
+import re
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "stq1.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(stq1_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    import sub_bit_sparse_b200 as m
+    lib = ctypes.CDLL(m.LIB_PATH)
+    names = _declared_functions()
+    assert len(names) >= 8
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(m.SIGNATURES)
+    assert m.LIB.stq1_version() >= 100
+
+
+def test_error_codes_are_distinct_and_negative():
+    src = open(os.path.join(ROOT, "include", "stq1.h")).read()
+    codes = dict(re.findall(r"#define (STQ1_ERR_\w+) \((-\d+)\)", src))
+    vals = [int(v) for v in codes.values()]
+    assert len(vals) == len(set(vals)) and all(v < 0 for v in vals)
+    import sub_bit_sparse_b200 as m
+    assert {int(v): k for k, v in codes.items()} == m.ERRORS
+
+
+def test_host_side_argument_checks_need_no_gpu():
+    # Shape checks run before anything touches the device.
+    import sub_bit_sparse_b200 as m
+    L = m.LIB
+    assert L.stq1_gemv(None, None, None, 16, 256, 1, None, 0, None) == -2
+    assert L.stq1_gemv(1 << 20, 1 << 20, 1 << 20, 16, 300, 1, None, 0, None) == -1
+    assert L.stq1_gemv(1 << 20, 1 << 20, 1 << 20, 16, 256, 0, None, 0, None) == -1
+    assert L.stq1_gemv((1 << 20) + 8, 1 << 20, 1 << 20, 16, 256, 1, None, 0, None) == -6
+    assert L.stq1_dequant(None, None, 1, 256, None) == -2
+    assert L.stq1_dequant(1 << 20, 1 << 20, 1, 255, None) == -1
+    assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 8, 4, 64, 256, 0, None, 0, None) == -1
+    assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 63, 256, 0, None, 0, None) == -1
+    assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 1, None, 0, None) == -2
+    assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 8, None, 0, None) == -8
+    assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 0, None, 0, None) == -7
+    assert L.stq1_gemv_workspace(16, 300, 1) == 0
+    assert L.stq1_moe_workspace(16, 8, 256, 4096, 7168, 0) > 0
