@@ -216,6 +216,12 @@ def run_gpu(args):
     # --- MoE decode gate/up (16 tokens, top-8 of 256 experts) ---
     moe = run_moe(torch, stq1, device, stream, args, world, timed)
 
+    # --- MoE prefill gate/up on the tensor-core tile path (4096 tokens) ---
+    try:
+        prefill = run_prefill(torch, stq1, device, stream, args, world, timed, bf16_peak)
+    except Exception as exc:  # reported, never hidden
+        prefill = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     # --- end to end through the public API with host buffers ---
     e2e = run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier)
 
@@ -251,6 +257,7 @@ def run_gpu(args):
                      "kernel": "lut_gemv_kernel<1>", "algorithmic_bytes_per_launch": PACKED},
         "gemv_batches": batches,
         "moe_decode": moe,
+        "moe_prefill": prefill,
         "e2e": e2e,
         "gpu_launches": args.steps * STACK,
         "clocks": clk.summary(),
@@ -268,13 +275,7 @@ def run_moe(torch, stq1, device, stream, args, world, timed):
     import workloads
     E, n, k = 256, N_ROWS, K_COLS
     eb = PACKED
-    flat = torch.empty(E * eb, dtype=torch.uint8, device=device)
-    g = torch.Generator(device=device)
-    g.manual_seed(2024)
-    flat.copy_(torch.randint(0, 256, (E * eb,), dtype=torch.uint8, device=device, generator=g))
-    blk = flat.view(-1, 42)
-    d = (0.058 * (1 + 0.1 * torch.randn(blk.shape[0], device=device, generator=g))).to(torch.float16)
-    blk[:, 0:2].copy_(d.view(torch.uint8).view(-1, 2))
+    flat = _random_expert_bank(torch, device, E, 2024)
     x, ids, wts = workloads.moe_decode_inputs()
     xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
     idd = torch.from_numpy(ids).to(device)
@@ -294,6 +295,88 @@ def run_moe(torch, stq1, device, stream, args, world, timed):
             "unique_experts": int(uniq), "expert_bytes_read": int(uniq * eb),
             "gbs": round(uniq * eb / (ms * 1e-3) / 1e9, 1),
             "config": "256 experts x [4096, 7168] STQ1_0, 16 tokens, Zipf(1.1) top-8, unweighted"}
+
+
+def _random_expert_bank(torch, device, E, seed):
+    """E random but valid [4096, 7168] STQ1_0 matrices on the device: uniform code
+    bytes, fp16 scales near 0.058 (the amax of 256 N(0, 0.02^2) weights)."""
+    flat = torch.empty(E * PACKED, dtype=torch.uint8, device=device)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    flat.copy_(torch.randint(0, 256, (E * PACKED,), dtype=torch.uint8, device=device, generator=g))
+    blk = flat.view(-1, 42)
+    d = (0.058 * (1 + 0.1 * torch.randn(blk.shape[0], device=device, generator=g))).to(torch.float16)
+    blk[:, 0:2].copy_(d.view(torch.uint8).view(-1, 2))
+    return flat
+
+
+def run_prefill(torch, stq1, device, stream, args, world, timed, bf16_peak):
+    """MoE prefill gate/up: 4096 tokens x top-8 of 256 experts (32,768 pairs)."""
+    import workloads
+    E, n, k = 256, N_ROWS, K_COLS
+    flat = _random_expert_bank(torch, device, E, 4096)
+    x, ids, _ = workloads.moe_prefill_inputs()
+    xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    idd = torch.from_numpy(ids).to(device)
+    y = torch.empty((4096, 8, n), dtype=torch.float32, device=device)
+    ws = stq1.workspace(stq1.LIB.stq1_moe_workspace(4096, 8, E, n, k, 0), device, kind="moe")
+
+    def step():
+        stq1.moe_gateup(flat, xd, idd, None, n, k, E, out=y, ws=ws)
+
+    steps = max(2, args.steps // 40)
+    gp = time_graph(torch, step, steps, 3, stream)
+    ms = timed(gp, steps) / steps
+    del gp
+    flops = 2.0 * 4096 * 8 * n * k
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"tokens_per_s": round(world * 4096 / (ms * 1e-3), 1), "ms_per_call": round(ms, 4),
+            "tflops_dense_equiv": round(tflops, 1), "bf16_peak_tflops": bf16_peak,
+            "tensor_frac": round(tflops / bf16_peak, 4),
+            "config": "256 experts x [4096, 7168] STQ1_0, 4096 tokens, Zipf(1.1) top-8 (32,768 pairs), "
+                      "tcgen05 kind::f16 tiles, A = decoded +/-1 bf16 in TMEM, fp32 per-slab scale"}
+
+
+def run_sweep(args):
+    """Crossover sweep: one [18432, 7168] matrix, batch 1..1024, both kernels."""
+    import torch
+    import workloads
+    import sub_bit_sparse_b200 as stq1
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w, h, x = workloads.crossover_inputs()
+    n, k = w.shape
+    packed = stq1.quantize_ref(w, h, mode="sherry")
+    pb = packed.size
+    copies = max(2, (300 * 1024 * 1024) // pb + 1)          # rotate > 2 x L2
+    wd = torch.from_numpy(packed).to(device)
+    stack = torch.stack([torch.roll(wd.view(-1, 42), shifts=i * 7919, dims=0).reshape(-1) for i in range(copies)])
+    xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    y = torch.empty((1024, n), dtype=torch.float32, device=device)
+    ws = stq1.workspace(max(stq1.LIB.stq1_gemv_workspace(n, k, b) for b in (1, 4, 16, 64, 256, 1024)), device)
+    out = []
+    for b in (1, 4, 16, 64, 256, 1024):
+        row = {"batch": b}
+        for name, path in (("table", stq1.PATH_TABLE), ("tiles", stq1.PATH_TILES)):
+            stq1.set_path(path)
+            xb = xd[:b].contiguous()
+            for i in range(3):
+                stq1.gemv(stack[i % copies], xb, n, k, out=y[:b], ws=ws)
+            torch.cuda.synchronize()
+            reps = max(3, min(50, 2000 // b))
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            for i in range(reps):
+                stq1.gemv(stack[i % copies], xb, n, k, out=y[:b], ws=ws)
+            s1.record()
+            torch.cuda.synchronize()
+            ms = s0.elapsed_time(s1) / reps
+            row[name] = {"ms": round(ms, 4), "gbs": round(pb / (ms * 1e-3) / 1e9, 1),
+                         "tflops": round(2.0 * b * n * k / (ms * 1e-3) / 1e12, 2)}
+        stq1.set_path(stq1.PATH_AUTO)
+        out.append(row)
+        print(json.dumps(row), flush=True)
+    print(json.dumps({"sweep": "crossover", "matrix": [n, k], "packed_bytes": int(pb), "rows": out}))
 
 
 def run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier):
@@ -412,10 +495,11 @@ def profile_case(args):
     import sub_bit_sparse_b200 as stq1
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    if args.profile_case == "moe":
-        stream = torch.cuda.current_stream()
-        out = run_moe(torch, stq1, device, stream, argparse.Namespace(steps=8), 1,
-                      lambda g, steps: 0.0)
+    if args.profile_case in ("moe", "prefill"):
+        stream = torch.cuda.Stream(device)
+        fn = run_moe if args.profile_case == "moe" else run_prefill
+        extra = () if args.profile_case == "moe" else (1672.0,)
+        out = fn(torch, stq1, device, stream, argparse.Namespace(steps=80), 1, lambda g, steps: 1.0, *extra)
         print(json.dumps(out))
         return
     _, stack, x_bits = build_stack(torch, stq1, device)
@@ -436,8 +520,12 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", default=None, choices=["gemv", "moe"])
+    ap.add_argument("--profile-case", default=None, choices=["gemv", "moe", "prefill"])
+    ap.add_argument("--sweep", action="store_true", help="crossover sweep (18432 x 7168, batch 1..1024)")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.profile_case:
         profile_case(args)
         return

@@ -173,6 +173,16 @@ int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, const int32_t*
                     int64_t K, int flags, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * stq1_set_path -- process-wide choice between the two matmul kernels, for
+ * testing and crossover measurements: 0 = by size (default: batches of 16 or
+ * more tokens, and MoE calls averaging 16 or more pairs per routed expert, use
+ * the tensor-core tile kernel), 1 = always the lookup-table kernel, 2 = the tile
+ * kernel whenever the shape allows it (K / 256 even).  Not thread-safe with
+ * concurrent calls.  Errors: STQ1_ERR_ARG.
+ */
+int stq1_set_path(int path);
+
+/*
  * stq1_status -- synchronise `stream`, return STQ1_OK if no device error was
  * recorded since the last call, else STQ1_ERR_DEVICE with the bits in
  * *device_err (may be NULL).  Clears the word.  STQ1_ERR_CUDA if the

@@ -49,6 +49,7 @@ SIGNATURES = {
                                    _c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
                                    _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "stq1_status": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
+    "stq1_set_path": (_c.c_int, [_c.c_int]),
 }
 
 
@@ -60,20 +61,34 @@ class Stq1Error(RuntimeError):
                          + (f" (device error bits {device_err:#x})" if device_err else ""))
 
 
+_lib = None
+_lib_lock = threading.Lock()
+
+
 def _load():
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(
-            f"libstq1.so not found at {LIB_PATH}; build it with "
-            "`python -m sub_bit_sparse_b200.build` (needs the CUDA toolkit)")
-    lib = ctypes.CDLL(LIB_PATH)
-    for name, (res, args) in SIGNATURES.items():
-        fn = getattr(lib, name)
-        fn.restype = res
-        fn.argtypes = args
-    return lib
+    """Loads libstq1.so once; raises ImportError if it is missing (no CPU fallback)."""
+    global _lib
+    with _lib_lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"libstq1.so not found at {LIB_PATH}; build it with "
+                    "`python -m sub_bit_sparse_b200.build` (needs the CUDA toolkit)")
+            lib = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
 
 
-LIB = _load()
+def __getattr__(name):
+    # ``sub_bit_sparse_b200.LIB`` loads the library on first access, so the build
+    # module can be imported before the library exists.
+    if name == "LIB":
+        return _load()
+    raise AttributeError(name)
 
 
 def _check(func: str, rc: int):
@@ -101,7 +116,7 @@ def quantize_ref(w: np.ndarray, h: np.ndarray | None = None, mode: str = "plain"
     hh = None if h is None else np.ascontiguousarray(h, dtype=np.float32)
     out = np.empty(max(packed_bytes(n, k), 1), dtype=np.uint8)
     m = {"plain": ENC_PLAIN, "sherry": ENC_SHERRY}[mode]
-    rc = LIB.stq1_quantize_ref(w.ctypes.data, None if hh is None else hh.ctypes.data, n, k, m, rounds,
+    rc = _load().stq1_quantize_ref(w.ctypes.data, None if hh is None else hh.ctypes.data, n, k, m, rounds,
                                out.ctypes.data, threads)
     _check("stq1_quantize_ref", rc)
     return out[: packed_bytes(n, k)]
@@ -159,7 +174,7 @@ def dequant(w_packed, n: int, k: int, out=None):
     if out is None:
         out = torch.empty((n, k), dtype=torch.bfloat16, device=w_packed.device)
     _require(out, torch.bfloat16, "out")
-    rc = LIB.stq1_dequant(w_packed.data_ptr(), out.data_ptr(), n, k, _stream(w_packed))
+    rc = _load().stq1_dequant(w_packed.data_ptr(), out.data_ptr(), n, k, _stream(w_packed))
     _check("stq1_dequant", rc)
     return out
 
@@ -173,10 +188,10 @@ def gemv(w_packed, x, n: int, k: int, out=None, ws=None):
     if out is None:
         out = torch.empty((b, n), dtype=torch.float32, device=x.device)
     _require(out, torch.float32, "out")
-    need = LIB.stq1_gemv_workspace(n, k, b)
+    need = _load().stq1_gemv_workspace(n, k, b)
     if ws is None:
         ws = workspace(need, x.device)
-    rc = LIB.stq1_gemv(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b,
+    rc = _load().stq1_gemv(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b,
                        None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
                        _stream(x))
     _check("stq1_gemv", rc)
@@ -196,10 +211,10 @@ def moe_gateup(expert_blocks, x, topk_ids, topk_weights, n: int, k: int, n_exper
     if out is None:
         out = torch.empty((t, topk, n), dtype=torch.float32, device=x.device)
     _require(out, torch.float32, "out")
-    need = LIB.stq1_moe_workspace(t, topk, n_experts, n, k, flags)
+    need = _load().stq1_moe_workspace(t, topk, n_experts, n, k, flags)
     if ws is None:
         ws = workspace(need, x.device, kind="moe")
-    rc = LIB.stq1_moe_gateup(expert_blocks.data_ptr(), x.data_ptr(), topk_ids.data_ptr(),
+    rc = _load().stq1_moe_gateup(expert_blocks.data_ptr(), x.data_ptr(), topk_ids.data_ptr(),
                              None if topk_weights is None else topk_weights.data_ptr(), out.data_ptr(),
                              t, topk, n_experts, n, k, flags,
                              None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
@@ -208,12 +223,20 @@ def moe_gateup(expert_blocks, x, topk_ids, topk_weights, n: int, k: int, n_exper
     return out
 
 
+PATH_AUTO, PATH_TABLE, PATH_TILES = 0, 1, 2
+
+
+def set_path(path: int) -> None:
+    """Selects the matmul kernel process-wide (0 by size, 1 table kernel, 2 tile kernel)."""
+    _check("stq1_set_path", _load().stq1_set_path(path))
+
+
 def status(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device error word; raises on errors."""
     torch = _torch()
     s = torch.cuda.current_stream() if stream is None else stream
     err = ctypes.c_int(0)
-    rc = LIB.stq1_status(ctypes.c_void_p(s.cuda_stream), ctypes.byref(err))
+    rc = _load().stq1_status(ctypes.c_void_p(s.cuda_stream), ctypes.byref(err))
     if rc not in (OK, -4):
         raise Stq1Error("stq1_status", rc)
     return err.value

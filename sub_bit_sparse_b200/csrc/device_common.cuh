@@ -98,6 +98,16 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
+// Programmatic dependent launch: wait for the preceding kernel in the stream
+// (no-op when the launch did not ask for overlap), and let the next kernel
+// start launching.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 template <int OFF>
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
   float v;

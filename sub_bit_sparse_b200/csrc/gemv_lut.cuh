@@ -144,18 +144,24 @@ __device__ __forceinline__ void lut_row_chunk(uint32_t slot, uint32_t lut,
   }
 }
 
+// Activations of this thread's group for chunk `chunk`, TT tokens (8 bytes each).
+template <int TT>
+__device__ __forceinline__ void lut_load_x(const LutArgs& a, int chunk, const int* xrow, uint2 (&xv)[kLutMaxTT]) {
+  const int col = chunk * (kLutKC * kBlockWeights) + 4 * static_cast<int>(threadIdx.x);
+#pragma unroll
+  for (int t = 0; t < TT; ++t)
+    xv[t] = __ldg(reinterpret_cast<const uint2*>(a.x + static_cast<long long>(xrow[t]) * a.K + col));
+}
+
 // Tables for one chunk: thread g builds the 32 entries of group g for each token.
 // Entry c (code) = (-1)^t * (x_a + (-1)^beta x_b + (-1)^gamma x_c).
 template <int TT>
-__device__ __forceinline__ void lut_build(const LutArgs& a, int chunk, const int* xrow,
-                                          uint32_t lut) {
+__device__ __forceinline__ void lut_build(const uint2 (&xv)[kLutMaxTT], uint32_t lut) {
   const int g = threadIdx.x;                       // 0 .. 127 = kLutChunkGroups - 1
-  const int col = chunk * (kLutKC * kBlockWeights) + 4 * g;
 #pragma unroll
   for (int t = 0; t < TT; ++t) {
-    const uint2 xv = *reinterpret_cast<const uint2*>(a.x + static_cast<long long>(xrow[t]) * a.K + col);
-    const float x0 = bf16_bits_to_f32(xv.x & 0xFFFFu), x1 = bf16_bits_to_f32(xv.x >> 16);
-    const float x2 = bf16_bits_to_f32(xv.y & 0xFFFFu), x3 = bf16_bits_to_f32(xv.y >> 16);
+    const float x0 = bf16_bits_to_f32(xv[t].x & 0xFFFFu), x1 = bf16_bits_to_f32(xv[t].x >> 16);
+    const float x2 = bf16_bits_to_f32(xv[t].y & 0xFFFFu), x3 = bf16_bits_to_f32(xv[t].y >> 16);
     const uint32_t gb = lut + static_cast<uint32_t>(t * kLutTokenBytes + g * kLutGroupBytes);
     // z = 0: a=1 b=2 c=3 ; z = 1: a=0 b=2 c=3 ; z = 2: a=0 b=1 c=3 ; z = 3: a=0 b=1 c=2
     const float xa[4] = {x1, x0, x0, x0};
@@ -230,12 +236,26 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
   const long long row0 = static_cast<long long>(slab) * kLutRows + (warp % P) + 32 * P * (warp / P);
   const uintptr_t wbase = reinterpret_cast<uintptr_t>(Wm) + static_cast<uintptr_t>(row0 * a.rowbytes);
 
-  if (c0 < c1) issue(c0, 0);
+  // Weights do not depend on the previous kernel in the stream: start their
+  // copies before waiting for it (programmatic dependent launch), unless the
+  // unit itself came from a routing kernel.
+  if (a.tile_info == nullptr) {
+    if (c0 < c1) issue(c0, 0);
+    if (c0 + 1 < c1) issue(c0 + 1, 1);
+  }
+  griddep_wait();
+  if (a.tile_info != nullptr) {
+    if (c0 < c1) issue(c0, 0);
+    if (c0 + 1 < c1) issue(c0 + 1, 1);
+  }
+  griddep_launch_dependents();
+  uint2 xv[kLutMaxTT];
+  if (c0 < c1) lut_load_x<TT>(a, c0, xrow, xv);
   for (int c = c0; c < c1; ++c) {
     const int it = c - c0;
     const int st = it & 1;
-    if (c + 1 < c1) issue(c + 1, st ^ 1);
-    lut_build<TT>(a, c, xrow, lut);
+    lut_build<TT>(xv, lut);
+    if (c + 1 < c1) lut_load_x<TT>(a, c + 1, xrow, xv);   // prefetch the next chunk's activations
     const bool landed = mbar_wait_bounded(bar0 + 8u * st, (it >> 1) & 1);
     // one barrier: tables built, copies landed (agreed by every thread)
     if (!__syncthreads_and(landed)) {
@@ -256,8 +276,8 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
       }
     }
     __syncthreads();
+    if (c + 2 < c1) issue(c + 2, st);                      // this stage is free again
   }
-
   if (a.S == 1) {
     if (row_ok) {
 #pragma unroll
@@ -270,22 +290,24 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
     return;
   }
 
-  // split K: publish partials, the last unit of this (tile, slab) reduces
+  // split K: publish partials, the last unit of this (tile, slab) reduces.
+  // One thread fences after the barrier: the barrier orders the other threads'
+  // stores before it, and the gpu-scope fence is cumulative.
   if (row_ok) {
 #pragma unroll
     for (int t = 0; t < TT; ++t)
       a.partial[(static_cast<long long>(split) * a.rows_out + orow[t]) * a.N + row] = acc[t];
   }
   __shared__ int s_last;
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
+    __threadfence();
     const int old = atomicAdd(&a.counters[tile_id * a.n_slabs + slab], 1);
     s_last = (old == a.S - 1);
+    if (s_last) __threadfence();
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   if (row_ok) {
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
@@ -309,6 +331,7 @@ __global__ void __launch_bounds__(kLutThreads) lut_gemv_kernel(const LutArgs a) 
   const int slab = rest % a.n_slabs;
   const int tile = rest / a.n_slabs;
   if (a.tile_info) {
+    griddep_wait();                                  // the tile table comes from the routing kernel
     if (tile >= *a.n_tiles_dev) return;
     if (threadIdx.x == 0) {
       const int e = a.tile_info[4 * tile + 0];

@@ -14,6 +14,7 @@ namespace stq1 {
 // STQ1_DEV_BAD_EXPERT.  Order inside a segment is unspecified (it does not
 // change any result: every output row is computed on its own).
 // tile_info[4 * i] = expert, first pair offset, pair count (<= tile_tokens), 0.
+// n_tiles[0] = number of tiles, n_tiles[1] = number of pairs with a valid id.
 // ---------------------------------------------------------------------------
 constexpr int kRouteThreads = 1024;
 
@@ -22,6 +23,8 @@ route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_token
              int* __restrict__ pairs_out, int* __restrict__ tile_info, int* __restrict__ n_tiles,
              float* __restrict__ y, int N) {
   extern __shared__ int sm[];
+  griddep_wait();           // ids may come from the previous kernel in the stream
+  griddep_launch_dependents();
   int* cnt = sm;            // [E]
   int* off = sm + E;        // [E]
   int* tst = sm + 2 * E;    // [E]
@@ -61,7 +64,10 @@ route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_token
       r1 += cnt[e];
       r2 += (cnt[e] + tile_tokens - 1) / tile_tokens;
     }
-    if (lane == 31) *n_tiles = i2;
+    if (lane == 31) {
+      n_tiles[0] = i2;       // tiles
+      n_tiles[1] = i1;       // pairs with a valid expert id
+    }
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {

@@ -3,10 +3,14 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstdio>
+#include <utility>
+
+#include <cudaTypedefs.h>
 
 #include "device_common.cuh"
 #include "gemv_lut.cuh"
 #include "small_kernels.cuh"
+#include "tc_gemm.cuh"
 
 namespace stq1 {
 namespace {
@@ -22,6 +26,51 @@ static_assert(kTargetUnits * sizeof(int) <= kCounterBytes, "counter region too s
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Path selection: 0 = by size, 1 = table kernel, 2 = tensor-core tile kernel.
+int g_path = 0;
+constexpr int kTcMinBatch = 16;       // stq1_gemv: batches from here use the tile kernel
+constexpr int kTcMinPairsPerExpert = 16;
+constexpr int kMoeTableTokens = 2;    // MoE decode tiles: pairs per table-kernel unit
+
+int sm_count() {
+  static int cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (!cache[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = v > 0 ? v : 148;
+  }
+  return cache[dev];
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major bf16 matrix [rows, K]; box = 64 columns x kTcN rows,
+// 128-byte swizzle, out-of-range rows read as zero.
+bool make_b_map(CUtensorMap* map, const void* base, long long rows, long long K) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcKC), static_cast<cuuint32_t>(kTcN)};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int current_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -36,10 +85,14 @@ int ensure_configured() {
   if (done[dev]) return STQ1_OK;
   if (cudaFuncSetAttribute(lut_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(lut_smem_bytes(1))) != cudaSuccess ||
+      cudaFuncSetAttribute(lut_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(lut_smem_bytes(2))) != cudaSuccess ||
       cudaFuncSetAttribute(lut_gemv_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(lut_smem_bytes(4))) != cudaSuccess ||
       cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           3 * kMaxExperts * 4) != cudaSuccess)
+                           3 * kMaxExperts * 4) != cudaSuccess ||
+      cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kTcSmemBytes) != cudaSuccess)
     return STQ1_ERR_CUDA;
   done[dev] = true;
   return STQ1_OK;
@@ -47,6 +100,26 @@ int ensure_configured() {
 
 int launch_status() {
   return cudaGetLastError() == cudaSuccess ? STQ1_OK : STQ1_ERR_CUDA;
+}
+
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel in the stream drains; it calls griddepcontrol.wait before
+// touching anything that kernel may write.
+template <typename... Params, typename... Args>
+int launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+               Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? STQ1_OK
+                                                                                      : STQ1_ERR_CUDA;
 }
 
 int residue_period(long long rowbytes) {
@@ -58,12 +131,21 @@ int residue_period(long long rowbytes) {
 struct GemvPlan {
   int n_tiles, n_slabs, S, n_chunks;
   size_t partial_bytes, counter_bytes;
-  bool table_path;
+  bool table_path, tile_path;
 };
+
+bool want_tiles(long long nb, long long units) {
+  if (nb % 2 != 0) return false;          // the tile kernel needs 4-byte-aligned rows
+  if (g_path == 1) return false;
+  if (g_path == 2) return true;
+  return units >= kTcMinBatch;
+}
 
 GemvPlan plan_gemv(long long N, long long K, int batch) {
   GemvPlan p{};
   const long long nb = K / kBlockWeights;
+  p.tile_path = want_tiles(nb, batch);
+  if (p.tile_path) return p;
   p.table_path = (nb % 2 == 0);
   p.n_tiles = (batch + kLutMaxTT - 1) / kLutMaxTT;
   p.n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
@@ -121,6 +203,31 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long nb = K / kBlockWeights;
   const long long rowbytes = nb * kBlockBytes;
+  if (p.tile_path) {
+    CUtensorMap map;
+    if (!make_b_map(&map, x, batch, K)) return STQ1_ERR_CUDA;
+    TcArgs t{};
+    t.W = static_cast<const uint8_t*>(W_packed);
+    t.W_end = t.W + N * rowbytes;
+    t.expert_bytes = 0;
+    t.rowbytes = rowbytes;
+    t.y = y;
+    t.tile_info = nullptr;
+    t.n_tiles_dev = nullptr;
+    t.pairs = nullptr;
+    t.route_w = nullptr;
+    t.n_tiles = (batch + kTcN - 1) / kTcN;
+    t.N = static_cast<int>(N);
+    t.K = static_cast<int>(K);
+    t.nb = static_cast<int>(nb);
+    t.n_mtiles = static_cast<int>((N + kTcM - 1) / kTcM);
+    t.batch = batch;
+    t.P = residue_period(rowbytes);
+    t.flags = 0;
+    const long long items = static_cast<long long>(t.n_tiles) * t.n_mtiles;
+    const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
+    return launch_pdl(tc_gemm_kernel, grid, kTcThreads, kTcSmemBytes, s, map, t);
+  }
   if (!p.table_path) {
     const long long warps = static_cast<long long>(batch) * N;
     direct_gemv_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(
@@ -150,24 +257,28 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
   a.P = residue_period(rowbytes);
   a.flags = 0;
   const long long grid = static_cast<long long>(p.n_tiles) * p.n_slabs * p.S;
-  if (batch == 1) {
-    lut_gemv_kernel<1><<<static_cast<unsigned>(grid), kLutThreads, lut_smem_bytes(1), s>>>(a);
-  } else {
-    lut_gemv_kernel<4><<<static_cast<unsigned>(grid), kLutThreads, lut_smem_bytes(4), s>>>(a);
-  }
-  return launch_status();
+  if (batch == 1)
+    return launch_pdl(lut_gemv_kernel<1>, static_cast<unsigned>(grid), kLutThreads, lut_smem_bytes(1), s, a);
+  if (batch == 2)
+    return launch_pdl(lut_gemv_kernel<2>, static_cast<unsigned>(grid), kLutThreads, lut_smem_bytes(2), s, a);
+  return launch_pdl(lut_gemv_kernel<4>, static_cast<unsigned>(grid), kLutThreads, lut_smem_bytes(4), s, a);
 }
 
 namespace stq1 {
 namespace {
 struct MoePlan {
-  size_t pairs_off, tiles_off, ntiles_off, total;
-  int max_tiles;
+  size_t pairs_off, tiles_off, ntiles_off, xperm_off, total;
+  int max_tiles, tile_tokens;
+  bool tiles;
 };
-MoePlan plan_moe(int T, int topk, int E) {
+MoePlan plan_moe(int T, int topk, int E, long long K) {
   MoePlan m{};
   const long long n_pairs = static_cast<long long>(T) * topk;
-  m.max_tiles = static_cast<int>(std::min<long long>(n_pairs, n_pairs / kLutMaxTT + std::min<long long>(E, n_pairs)));
+  const long long nb = K / kBlockWeights;
+  const long long active = std::min<long long>(E, n_pairs);
+  m.tiles = want_tiles(nb, n_pairs >= kTcMinPairsPerExpert * active ? kTcMinBatch : 0);
+  m.tile_tokens = m.tiles ? kTcN : kMoeTableTokens;
+  m.max_tiles = static_cast<int>(std::min<long long>(n_pairs, n_pairs / m.tile_tokens + active));
   size_t off = 0;
   m.pairs_off = off;
   off += round16(n_pairs * sizeof(int));
@@ -175,6 +286,8 @@ MoePlan plan_moe(int T, int topk, int E) {
   off += round16(static_cast<size_t>(m.max_tiles) * 4 * sizeof(int));
   m.ntiles_off = off;
   off += 16;
+  m.xperm_off = off;
+  if (m.tiles) off += round16(static_cast<size_t>(n_pairs) * K * 2);
   m.total = off;
   return m;
 }
@@ -183,10 +296,9 @@ MoePlan plan_moe(int T, int topk, int E) {
 
 extern "C" size_t stq1_moe_workspace(int T, int topk, int E, int64_t N, int64_t K, int flags) {
   (void)N;
-  (void)K;
   (void)flags;
-  if (T <= 0 || topk <= 0 || E <= 0) return 0;
-  return plan_moe(T, topk, E).total;
+  if (T <= 0 || topk <= 0 || E <= 0 || K <= 0 || K % kBlockWeights) return 0;
+  return plan_moe(T, topk, E, K).total;
 }
 
 extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, const int32_t* topk_ids,
@@ -200,7 +312,7 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
       static_cast<long long>(T) * topk > (1LL << 30))
     return STQ1_ERR_SHAPE;
   if (!aligned16(expert_blocks) || !aligned16(x)) return STQ1_ERR_ALIGN;
-  const MoePlan m = plan_moe(T, topk, E);
+  const MoePlan m = plan_moe(T, topk, E, K);
   if (!ws || ws_bytes < m.total) return STQ1_ERR_WORKSPACE;
   if (!aligned16(ws)) return STQ1_ERR_ALIGN;
   int rc = ensure_configured();
@@ -222,10 +334,39 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
     return launch_status();
   }
 
-  route_kernel<<<1, kRouteThreads, 3 * E * sizeof(int), s>>>(topk_ids, n_pairs, E, kLutMaxTT, pairs,
-                                                             tiles, ntiles, y, static_cast<int>(N));
-  rc = launch_status();
+  rc = launch_pdl(route_kernel, 1, kRouteThreads, 3 * E * sizeof(int), s, topk_ids, n_pairs, E, m.tile_tokens,
+                  pairs, tiles, ntiles, y, static_cast<int>(N));
   if (rc != STQ1_OK) return rc;
+  if (m.tiles) {
+    uint16_t* xperm = reinterpret_cast<uint16_t*>(wsb + m.xperm_off);
+    rc = launch_pdl(gather_rows_kernel, static_cast<unsigned>(n_pairs), 256, 0, s, x,
+                    static_cast<const int*>(pairs), static_cast<const int*>(ntiles + 1), n_pairs, topk,
+                    static_cast<int>(K), xperm);
+    if (rc != STQ1_OK) return rc;
+    CUtensorMap map;
+    if (!make_b_map(&map, xperm, n_pairs, K)) return STQ1_ERR_CUDA;
+    TcArgs t{};
+    t.W = static_cast<const uint8_t*>(expert_blocks);
+    t.W_end = t.W + static_cast<long long>(E) * N * rowbytes;
+    t.expert_bytes = N * rowbytes;
+    t.rowbytes = rowbytes;
+    t.y = y;
+    t.tile_info = tiles;
+    t.n_tiles_dev = ntiles;
+    t.pairs = pairs;
+    t.route_w = topk_weights;
+    t.n_tiles = m.max_tiles;
+    t.N = static_cast<int>(N);
+    t.K = static_cast<int>(K);
+    t.nb = static_cast<int>(nb);
+    t.n_mtiles = static_cast<int>((N + kTcM - 1) / kTcM);
+    t.batch = 0;
+    t.P = residue_period(rowbytes);
+    t.flags = flags;
+    const long long items = static_cast<long long>(m.max_tiles) * t.n_mtiles;
+    const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
+    return launch_pdl(tc_gemm_kernel, grid, kTcThreads, kTcSmemBytes, s, map, t);
+  }
   LutArgs a{};
   a.W = static_cast<const uint8_t*>(expert_blocks);
   a.W_end = a.W + static_cast<long long>(E) * N * rowbytes;
@@ -252,8 +393,14 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   a.P = residue_period(rowbytes);
   a.flags = flags;
   const long long grid = static_cast<long long>(m.max_tiles) * a.n_slabs;
-  lut_gemv_kernel<4><<<static_cast<unsigned>(grid), kLutThreads, lut_smem_bytes(4), s>>>(a);
-  return launch_status();
+  return launch_pdl(lut_gemv_kernel<kMoeTableTokens>, static_cast<unsigned>(grid), kLutThreads,
+                    lut_smem_bytes(kMoeTableTokens), s, a);
+}
+
+extern "C" int stq1_set_path(int path) {
+  if (path < 0 || path > 2) return STQ1_ERR_ARG;
+  g_path = path;
+  return STQ1_OK;
 }
 
 extern "C" int stq1_status(void* stream, int* device_err) {

@@ -1,0 +1,494 @@
+// Tensor-core tile path for STQ1_0 at large token counts (sm_100a, tcgen05).
+//
+// y[p, j] = sum_k W^[j, k] x[tok(p), k] for all pairs p of an expert (or all
+// tokens of a plain matmul).  Per 256-column block the weights are
+// d_{j,b} * s_{jk} with s in {-1, 0, +1} ("How STQ1_0 works"); s is exact in
+// bf16, d is not.  So each tile contracts the +/-1 pattern against bf16
+// activations on the tensor cores, one 256-column slab at a time into a TMEM
+// accumulator, and CUDA cores add d_{j,b} * slab into an fp32 register
+// accumulator (a5 of the hot path, done once per row, slab and token).
+//
+// Tile: M = 128 weight rows x N = 128 tokens, K in 64-column stages.
+//   warp 0      TMA producer: x tiles (bf16, 128-byte swizzle) into a 4-stage
+//               shared ring (one 2-D tensor copy per stage, no multicast).
+//   warp 1      TMEM allocator and the single MMA-issuing thread:
+//               tcgen05.mma.cta_group::1.kind::f16, A from TMEM, B from shared.
+//   warps 2-5   decoders: one thread per weight row reads the row's 42-byte
+//               block for the slab, expands each group's 5-bit code to four
+//               bf16 values through a 32-entry table and stores 64 columns per
+//               stage into TMEM (tcgen05.st), the A operand.
+//   warps 6-9   epilogue: per slab, tcgen05.ld of the slab accumulator, fp32
+//               FMA with the row's d, release of the TMEM buffer; at the end
+//               of the tile, coalesced stores of y.
+// TMEM (512 columns allocated, one CTA per SM): slab accumulators 2 x 128
+// columns, A stages 4 x 32 columns.
+// All waits are bounded; a timeout sets the device error word and makes every
+// role stop at its next wait, so the CTA always reaches the final barrier and
+// frees its TMEM.
+#pragma once
+
+#include <cuda.h>
+
+#include "device_common.cuh"
+
+namespace stq1 {
+
+constexpr int kTcM = 128;
+constexpr int kTcN = 128;
+constexpr int kTcKC = 64;                     // K per stage (128 bytes of bf16)
+constexpr int kTcStages = 4;
+constexpr int kTcSlabChunks = kBlockWeights / kTcKC;    // 4 stages per scale block
+constexpr int kTcThreads = 320;
+constexpr uint32_t kTcTmemCols = 512;
+constexpr uint32_t kTcColD = 0;               // 2 x 128
+constexpr uint32_t kTcColA = 256;             // 4 x 32
+constexpr int kTcBStageBytes = kTcN * kTcKC * 2;   // 16 KB
+// shared layout (offsets from a 1024-aligned base)
+constexpr int kTcOffB = 0;
+constexpr int kTcOffTable = kTcStages * kTcBStageBytes;            // 65536: 2 x 128 B decode tables
+constexpr int kTcOffBar = kTcOffTable + 256;
+constexpr int kTcOffPairs = kTcOffBar + 256;                       // kTcN ints
+constexpr int kTcOffMisc = kTcOffPairs + kTcN * 4;
+constexpr int kTcSmemBytes = 1024 + kTcOffMisc + 64 + 100 * 1024;  // padded: one CTA per SM
+
+struct TcArgs {
+  const uint8_t* W;          // matrix or expert 0
+  const uint8_t* W_end;
+  long long expert_bytes;
+  long long rowbytes;
+  float* y;                  // [rows_out, N]
+  const int* tile_info;      // [tiles, 4] expert, first B row, count, pad (nullptr: plain)
+  const int* n_tiles_dev;    // device tile count (MoE) or nullptr
+  const int* pairs;          // output row of each B row (MoE) or nullptr (identity)
+  const float* route_w;
+  int n_tiles;               // plain: token tiles
+  int N, K, nb;
+  int n_mtiles;
+  int batch;                 // plain: tokens
+  int P;                     // residue period of row offsets mod 16
+  int flags;
+};
+
+// ---- tcgen05 / TMA wrappers ----
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem desc]
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+#define STQ1_TMEM_ST32(taddr, v)                                                                  \
+  asm volatile(                                                                                   \
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),   \
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),    \
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),          \
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),        \
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),        \
+      "r"(v[29]), "r"(v[30]), "r"(v[31])                                                         \
+      : "memory")
+
+#define STQ1_TMEM_LD32(taddr, v)                                                                  \
+  asm volatile(                                                                                   \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"              \
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),      \
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),  \
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),            \
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),            \
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])             \
+      : "r"(taddr)                                                                                \
+      : "memory")
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), version 1 (sm_100).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+// Instruction descriptor: D f32, A bf16, B bf16, both K-major, M = 128, N = kTcN.
+constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                              (static_cast<uint32_t>(kTcN >> 3) << 17) |
+                              (static_cast<uint32_t>(kTcM >> 4) << 24);
+
+// bf16 bit patterns of the 32 codes: lanes 0,1 (word 0) and lanes 2,3 (word 1).
+__device__ __forceinline__ void tc_fill_tables(uint32_t* t0, uint32_t* t1) {
+  const int c = threadIdx.x;
+  if (c < 32) {
+    int v[4];
+    code_pattern(static_cast<unsigned>(c), v);
+    uint32_t h[4];
+#pragma unroll
+    for (int l = 0; l < 4; ++l) h[l] = v[l] == 0 ? 0u : (v[l] > 0 ? 0x3F80u : 0xBF80u);
+    t0[c] = h[0] | (h[1] << 16);
+    t1[c] = h[2] | (h[3] << 16);
+  }
+}
+
+// Loads the 42-byte block at A (16-byte-aligned window of 64 bytes starting at
+// A & ~15) without reading past `end`.
+__device__ __forceinline__ void load_block_window(const uint8_t* A, const uint8_t* end,
+                                                  uint32_t (&w)[16]) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(A) & ~static_cast<uintptr_t>(15);
+  const uintptr_t need_end = reinterpret_cast<uintptr_t>(A) + kBlockBytes;
+  const uintptr_t e = reinterpret_cast<uintptr_t>(end);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uintptr_t q = lo + 16u * c;
+    if (q + 16 <= e && q < need_end) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(q));
+      w[4 * c] = v.x;
+      w[4 * c + 1] = v.y;
+      w[4 * c + 2] = v.z;
+      w[4 * c + 3] = v.w;
+    } else {
+      uint32_t tmp[4] = {0u, 0u, 0u, 0u};
+      for (int b = 0; b < 16; ++b)
+        if (q + b < e && q + b < need_end)
+          tmp[b >> 2] |= static_cast<uint32_t>(*reinterpret_cast<const uint8_t*>(q + b)) << (8 * (b & 3));
+      w[4 * c] = tmp[0];
+      w[4 * c + 1] = tmp[1];
+      w[4 * c + 2] = tmp[2];
+      w[4 * c + 3] = tmp[3];
+    }
+  }
+}
+
+// Decodes the block's four 64-column chunks; for each chunk waits for the
+// A stage to be free, stores 32 TMEM columns and signals the MMA thread.
+template <int BASE>
+__device__ __forceinline__ bool tc_decode_slab(const uint32_t (&w)[16], uint32_t tables,
+                                               uint32_t tmem_a_lane, uint32_t bar_full_a,
+                                               uint32_t bar_empty, uint32_t& it, volatile int* abort) {
+  uint32_t Q[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int p = BASE + kOffQs + 4 * i;
+    Q[i] = (p & 3) ? __funnelshift_r(w[p >> 2], w[(p >> 2) + 1], 8 * (p & 3)) : w[p >> 2];
+  }
+  const int ph = BASE + kOffQh;
+  const uint32_t H0 = (ph & 3) ? __funnelshift_r(w[ph >> 2], w[(ph >> 2) + 1], 8 * (ph & 3)) : w[ph >> 2];
+  const int ph1 = ph + 4;
+  const uint32_t H1 = (ph1 & 3) ? __funnelshift_r(w[ph1 >> 2], w[(ph1 >> 2) + 1], 8 * (ph1 & 3)) : w[ph1 >> 2];
+#pragma unroll
+  for (int q = 0; q < kTcSlabChunks; ++q) {          // 16 groups per chunk
+    uint32_t v[32];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = 2 * q + h;                       // qs word: groups 8i .. 8i+7
+      const uint32_t hb = (i < 4 ? H0 : H1) >> (8 * (i & 3));
+      const uint32_t ce = ((Q[i] << 2) & 0x3C3C3C3Cu) | (((hb & 0x55u) * 0x01041040u) & 0x40404040u);
+      const uint32_t co = ((Q[i] >> 2) & 0x3C3C3C3Cu) | ((((hb >> 1) & 0x55u) * 0x01041040u) & 0x40404040u);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        // code * 4 is in bits 2..6: shift right by 2 gives the code; table base
+        // is 256-aligned so the byte splices directly into the address
+        const uint32_t ae = __byte_perm(ce, tables, 0x7650u | m);
+        const uint32_t ao = __byte_perm(co, tables, 0x7650u | m);
+        uint32_t x0, x1, y0, y1;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(x0) : "r"(ae));
+        asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(x1) : "r"(ae));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(y0) : "r"(ao));
+        asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(y1) : "r"(ao));
+        const int g = 8 * h + 2 * m;                 // group within the chunk (0..15)
+        v[2 * g] = x0;
+        v[2 * g + 1] = x1;
+        v[2 * g + 2] = y0;
+        v[2 * g + 3] = y1;
+      }
+    }
+    const uint32_t s = it % kTcStages;
+    const uint32_t use = it / kTcStages;
+    if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) {
+      *abort = 1;
+      return false;
+    }
+    tc_fence_after();
+    STQ1_TMEM_ST32(tmem_a_lane + kTcColA + 32 * s, v);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(bar_full_a + 8 * s);
+    ++it;
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sbase = (sraw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - sraw);
+  const uint32_t sB = sbase + kTcOffB;
+  const uint32_t sTab = sbase + kTcOffTable;
+  const uint32_t bar = sbase + kTcOffBar;
+  // barriers: full_b[4] @0, full_a[4] @32, empty[4] @64, d_full[2] @96, d_empty[2] @112, drain @128
+  const uint32_t bar_full_b = bar, bar_full_a = bar + 32, bar_empty = bar + 64;
+  const uint32_t bar_d_full = bar + 96, bar_d_empty = bar + 112;
+  int* s_pairs = reinterpret_cast<int*>(sgen + kTcOffPairs);
+  volatile int* s_misc = reinterpret_cast<volatile int*>(sgen + kTcOffMisc);   // [0] tmem base, [1] abort
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(bar_full_b + 8 * i, 1);
+      mbar_init(bar_full_a + 8 * i, 128);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_d_full + 8 * i, 1);
+      mbar_init(bar_d_empty + 8 * i, 128);
+    }
+    mbar_init(bar + 128, 1);                         // drain barrier (abort path)
+    s_misc[1] = 0;
+    fence_mbar_init();
+  }
+  tc_fill_tables(reinterpret_cast<uint32_t*>(sgen + kTcOffTable),
+                 reinterpret_cast<uint32_t*>(sgen + kTcOffTable + 128));
+  if (warp == 1) {
+    tmem_alloc(sbase + kTcOffMisc, kTcTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(s_misc[0]);
+  volatile int* abort = s_misc + 1;
+  griddep_wait();                                    // inputs may come from the previous kernel
+  griddep_launch_dependents();
+
+  const int n_tiles = a.n_tiles_dev ? *a.n_tiles_dev : a.n_tiles;
+  const long long n_items = static_cast<long long>(n_tiles) * a.n_mtiles;
+  const int n_chunks = a.K / kTcKC;
+  const int n_slabs = a.nb;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
+        const int tile = static_cast<int>(item / a.n_mtiles);
+        const int b_row = a.tile_info ? a.tile_info[4 * tile + 1] : tile * kTcN;
+        for (int kc = 0; kc < n_chunks; ++kc, ++it) {
+          const uint32_t s = it % kTcStages, use = it / kTcStages;
+          if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) { *abort = 1; break; }
+          mbar_arrive_expect_tx(bar_full_b + 8 * s, kTcBStageBytes);
+          tma_load_2d(sB + s * kTcBStageBytes, &tmap_b, kc * kTcKC, b_row, bar_full_b + 8 * s);
+        }
+      }
+      if (*abort) {
+        // let the last tensor copies land before the CTA can exit (bounded)
+        for (uint32_t j = it > kTcStages ? it - kTcStages : 0; j < it; ++j)
+          mbar_wait_bounded(bar_full_b + 8 * (j % kTcStages), (j / kTcStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      uint32_t it = 0, sc = 0;
+      for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
+        for (int slab = 0; slab < n_slabs && !*abort; ++slab, ++sc) {
+          const uint32_t p = sc & 1, puse = sc >> 1;
+          if (!mbar_wait_bounded(bar_d_empty + 8 * p, (puse & 1) ^ 1)) { *abort = 1; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + kTcColD + p * kTcN;
+          for (int q = 0; q < kTcSlabChunks; ++q, ++it) {
+            const uint32_t s = it % kTcStages, use = it / kTcStages;
+            if (!mbar_wait_bounded(bar_full_b + 8 * s, use & 1) ||
+                !mbar_wait_bounded(bar_full_a + 8 * s, use & 1)) { *abort = 1; break; }
+            tc_fence_after();
+            const uint64_t bdesc = smem_desc_sw128(sB + s * kTcBStageBytes);
+#pragma unroll
+            for (int kk = 0; kk < kTcKC / 16; ++kk) {
+              tc_mma_ts(d_tmem, tmem + kTcColA + 32 * s + 8 * kk, bdesc + 2 * kk, kTcIdesc,
+                        (q > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(bar_empty + 8 * s);
+          }
+          if (*abort) break;
+          tc_commit(bar_d_full + 8 * p);
+        }
+      }
+      if (*abort) {
+        // all MMAs this thread issued must finish before TMEM is freed (bounded)
+        tc_commit(bar + 128);
+        mbar_wait_bounded(bar + 128, 0);
+      }
+    }
+  } else if (warp < 6) {
+    // ---------------- decoders ----------------
+    const int quad = warp & 3;                       // TMEM lane quadrant of this warp
+    const int P = a.P;
+    const int rho = P * lane + (quad % P) + 32 * P * (quad / P);   // row within the tile
+    const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(32 * quad) << 16);
+    uint32_t it = 0;
+    for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
+      const int tile = static_cast<int>(item / a.n_mtiles);
+      const int mt = static_cast<int>(item % a.n_mtiles);
+      const int e = a.tile_info ? a.tile_info[4 * tile + 0] : 0;
+      const int row = mt * kTcM + rho;
+      const bool row_ok = row < a.N;
+      const uint8_t* rbase = a.W + e * a.expert_bytes + static_cast<long long>(row_ok ? row : 0) * a.rowbytes;
+      // every lane of the warp has the same block offset mod 16 (rows of one residue class)
+      const uint8_t* r0 = a.W + e * a.expert_bytes +
+                          static_cast<long long>(mt * kTcM + (quad % P) + 32 * P * (quad / P)) * a.rowbytes;
+      for (int slab = 0; slab < n_slabs; ++slab) {
+        uint32_t w[16];
+        if (row_ok) {
+          load_block_window(rbase + static_cast<long long>(slab) * kBlockBytes, a.W_end, w);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = 0u;     // rows past N: computed, never stored
+        }
+        const int base = static_cast<int>((reinterpret_cast<uintptr_t>(r0) + static_cast<uintptr_t>(slab) * kBlockBytes) & 15);
+        bool ok;
+        switch (base) {
+          case 0: ok = tc_decode_slab<0>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
+          case 2: ok = tc_decode_slab<2>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
+          case 4: ok = tc_decode_slab<4>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
+          case 6: ok = tc_decode_slab<6>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
+          case 8: ok = tc_decode_slab<8>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
+          case 10: ok = tc_decode_slab<10>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
+          case 12: ok = tc_decode_slab<12>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
+          default: ok = tc_decode_slab<14>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
+        }
+        if (!ok) break;
+      }
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int quad = warp & 3;
+    const int P = a.P;
+    const int rho = P * lane + (quad % P) + 32 * P * (quad / P);
+    const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(32 * quad) << 16);
+    const int et = threadIdx.x - 192;                // 0..127
+    uint32_t sc = 0;
+    for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
+      const int tile = static_cast<int>(item / a.n_mtiles);
+      const int mt = static_cast<int>(item % a.n_mtiles);
+      const int e = a.tile_info ? a.tile_info[4 * tile + 0] : 0;
+      const int b_row = a.tile_info ? a.tile_info[4 * tile + 1] : tile * kTcN;
+      const int cnt = a.tile_info ? a.tile_info[4 * tile + 2] : min(kTcN, a.batch - tile * kTcN);
+      named_bar(1, 128);                             // previous tile's stores are done
+      if (et < kTcN) s_pairs[et] = et < cnt ? (a.pairs ? a.pairs[b_row + et] : b_row + et) : -1;
+      named_bar(1, 128);
+      const int row = mt * kTcM + rho;
+      const bool row_ok = row < a.N;
+      const uint8_t* rbase = a.W + e * a.expert_bytes + static_cast<long long>(row_ok ? row : 0) * a.rowbytes;
+      float acc[kTcN];
+#pragma unroll
+      for (int j = 0; j < kTcN; ++j) acc[j] = 0.f;
+      bool ok = true;
+      for (int slab = 0; slab < n_slabs; ++slab, ++sc) {
+        const uint8_t* B = rbase + static_cast<long long>(slab) * kBlockBytes;
+        const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(B[0] | (B[1] << 8))));
+        const uint32_t p = sc & 1, puse = sc >> 1;
+        if (!mbar_wait_bounded(bar_d_full + 8 * p, puse & 1)) { *abort = 1; ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kTcN / 32; ++c) {
+          uint32_t v[32];
+          STQ1_TMEM_LD32(tmem_lane + kTcColD + p * kTcN + 32 * c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[32 * c + i] = fmaf(d, __uint_as_float(v[i]), acc[32 * c + i]);
+        }
+        tc_fence_before();
+        mbar_arrive(bar_d_empty + 8 * p);
+      }
+      if (!ok) break;
+      if (row_ok) {
+        const bool up = (a.flags & STQ1_MOE_WEIGHT_UP) && row >= a.N / 2;
+#pragma unroll
+        for (int j = 0; j < kTcN; ++j) {
+          const int pr = s_pairs[j];
+          if (pr >= 0) {
+            float v = acc[j];
+            if (up) v *= a.route_w[pr];
+            a.y[static_cast<long long>(pr) * a.N + row] = v;
+          }
+        }
+      }
+    }
+  }
+
+  // all roles meet here (every wait above is bounded)
+  tc_fence_before();
+  __syncthreads();
+  if (*abort && threadIdx.x == 0) flag_error(STQ1_DEV_WAIT_LIMIT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTcTmemCols);
+  }
+}
+
+// x rows gathered into expert order for the tile path's TMA tiles.
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint16_t* __restrict__ x, const int* __restrict__ pairs, const int* __restrict__ n_valid,
+                   int n_rows, int topk, int K, uint16_t* __restrict__ out) {
+  const int r = blockIdx.x;
+  griddep_wait();
+  griddep_launch_dependents();
+  if (r >= n_rows) return;
+  const int nv = n_valid ? *n_valid : n_rows;
+  uint4* dst = reinterpret_cast<uint4*>(out + static_cast<long long>(r) * K);
+  if (r >= nv) {
+    for (int i = threadIdx.x; i < K / 8; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  const int tok = pairs[r] / topk;
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<long long>(tok) * K);
+  for (int i = threadIdx.x; i < K / 8; i += blockDim.x) dst[i] = src[i];
+}
+
+}  // namespace stq1

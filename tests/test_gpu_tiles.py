@@ -1,0 +1,108 @@
+"""Tensor-core tile path (tcgen05) vs the CPU oracle, through the C ABI (needs a B200)."""
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import sub_bit_sparse_b200 as stq1
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _bf16(xbits):
+    return _dev(xbits.astype(np.uint16).view(np.int16)).view(torch.bfloat16)
+
+
+def _assert_close(y_gpu, y_or, bound, what=""):
+    err = np.abs(y_gpu.astype(np.float64) - y_or)
+    tol = oracle.tolerance(bound)
+    bad = err > tol
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside tolerance; worst {(err / tol).max():.3g}"
+
+
+@pytest.fixture
+def tiles_path():
+    stq1.set_path(stq1.PATH_TILES)
+    yield
+    stq1.set_path(stq1.PATH_AUTO)
+
+
+@pytest.mark.parametrize("n,k,b", [(128, 512, 1), (128, 512, 16), (256, 1024, 128), (130, 512, 3),
+                                   (512, 2048, 129), (4096, 7168, 64), (384, 7168, 300), (1000, 1536, 40)])
+def test_tiles_gemv(tiles_path, n, k, b):
+    rng = np.random.default_rng(n + k + b)
+    w = (rng.standard_normal((n, k)) * rng.uniform(0.005, 0.05, (n, 1))).astype(np.float32)
+    packed = stq1.quantize_ref(w)
+    x = workloads.activations_bf16(b, k, seed=b)
+    y = stq1.gemv(_dev(packed), _bf16(x), n, k).cpu().numpy()
+    _assert_close(y, oracle.gemv(packed, x, n, k), oracle.gemv_abs(packed, x, n, k), f"tiles n={n} k={k} b={b}")
+    assert stq1.status() == 0
+
+
+def test_tiles_gemv_special_scales(tiles_path):
+    n, k = 128, 512
+    codes = (np.arange(n * 2 * 64) % 32).astype(np.uint8).reshape(n * 2, 64)
+    d = np.tile([0.0, 65504.0, 1.0, 2.0 ** -24, 0.5, 3.0e-3, 7.0, 1.0 / 3], n * 2 // 8)
+    packed = oracle.pack_blocks(oracle.fp16_bits(d), codes)
+    x = workloads.activations_bf16(20, k, seed=5)
+    y = stq1.gemv(_dev(packed), _bf16(x), n, k).cpu().numpy()
+    _assert_close(y, oracle.gemv(packed, x, n, k), oracle.gemv_abs(packed, x, n, k), "special scales")
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+def test_tiles_moe_small(tiles_path, flags):
+    n, k, E, T, topk = 256, 1024, 6, 70, 3
+    experts = np.concatenate([stq1.quantize_ref(workloads.gaussian_matrix(n, k, 0.02, seed=300 + e)) for e in range(E)])
+    x = workloads.activations_bf16(T, k, seed=31)
+    ids = workloads.zipf_topk_ids(T, E, topk, seed=32)
+    wts = workloads.softmax_route_weights(T, topk, seed=33)
+    y = stq1.moe_gateup(_dev(experts), _bf16(x), _dev(ids), _dev(wts), n, k, E, flags=flags).cpu().numpy()
+    eb = oracle.packed_size(n, k)
+    yr, ya = oracle.moe_gateup(lambda e: experts[e * eb:(e + 1) * eb], x, ids, wts, n, k, flags=flags, abs_sum=True)
+    _assert_close(y, yr, ya, f"tiles moe flags={flags}")
+
+
+def test_prefill_workload_sampled_experts():
+    # 256 experts x [4096, 7168], 4096 tokens, Zipf(1.1) top-8: 32,768 pairs on the
+    # tile path (chosen by size).  The oracle recomputes every output of a sample
+    # of experts: the most loaded one and a spread of small ones.
+    n, k, E = 4096, 7168, 256
+    eb = oracle.packed_size(n, k)
+    flat = workloads.random_packed_blocks(E * eb // 42, seed=4096)
+    x, ids, wts = workloads.moe_prefill_inputs()
+    y = stq1.moe_gateup(_dev(flat), _bf16(x), _dev(ids), _dev(wts), n, k, E).cpu().numpy()
+    assert stq1.status() == 0
+    xf = oracle.bf16_to_f64(x)
+    counts = np.bincount(ids.reshape(-1), minlength=E)
+    sample = [int(np.argmax(counts))] + [int(e) for e in np.argsort(counts)[::37][:6]]
+    for e in sample:
+        w = oracle.decode(flat[e * eb:(e + 1) * eb], n, k)
+        tt, ss = np.nonzero(ids == e)
+        ref = xf[tt] @ w.T
+        bound = np.abs(xf[tt]) @ np.abs(w).T
+        _assert_close(y[tt, ss], ref, bound, f"prefill expert {e} ({len(tt)} pairs)")
+
+
+def test_table_and_tile_paths_agree_on_decode_matrix():
+    w, h, x = workloads.decode_gemv_inputs()
+    packed = stq1.quantize_ref(w, h, mode="sherry")
+    wd, xd = _dev(packed), _bf16(x)
+    stq1.set_path(stq1.PATH_TABLE)
+    try:
+        y_table = stq1.gemv(wd, xd, 4096, 7168).cpu().numpy()
+        stq1.set_path(stq1.PATH_TILES)
+        y_tiles = stq1.gemv(wd, xd, 4096, 7168).cpu().numpy()
+    finally:
+        stq1.set_path(stq1.PATH_AUTO)
+    bound = oracle.gemv_abs(packed, x, 4096, 7168)
+    ref = oracle.gemv(packed, x, 4096, 7168)
+    _assert_close(y_table, ref, bound, "table")
+    _assert_close(y_tiles, ref, bound, "tiles")
