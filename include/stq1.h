@@ -56,6 +56,7 @@ extern "C" {
 #define STQ1_ERR_ALIGN (-6)       /* a pointer is not 16-byte aligned */
 #define STQ1_ERR_WORKSPACE (-7)   /* workspace NULL or smaller than the query says */
 #define STQ1_ERR_ARG (-8)         /* an invalid mode, flag or option */
+#define STQ1_ERR_SCRATCH (-9)     /* (stq1_gemv_noalloc) the shape needs more than the built-in scratch */
 
 /* Device error word bits (reported through stq1_status). */
 #define STQ1_DEV_BAD_EXPERT 1     /* a topk id was outside [0, E); its slot was skipped */
@@ -171,6 +172,32 @@ size_t stq1_moe_workspace(int T, int topk, int E, int64_t N, int64_t K, int flag
 int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, const int32_t* topk_ids,
                     const float* topk_weights, float* y, int T, int topk, int E, int64_t N,
                     int64_t K, int flags, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * stq1_gemv_noalloc -- stq1_gemv without a caller workspace and without any
+ * allocation.  The source pages have no counterpart; this entry point exists
+ * for callers that cannot allocate device memory or keep a workspace: hosts
+ * and plugin frameworks that own all device memory and pass only input and
+ * output buffers, and latency-critical code that must not call cudaMalloc
+ * (it can synchronize the device).
+ *   Same arguments, layouts and accuracy as stq1_gemv, minus the workspace.
+ *   Always uses the lookup-table kernel.  Its split-K scratch (2 KiB of
+ *   arrival counters plus the partial sums) lives in a 1 MiB buffer compiled
+ *   into the library, which every GPU that loads the library holds until the
+ *   process exits.  A shape needing more (2048 + S*batch*N*4 bytes, with S the
+ *   split count; [4096, 7168] at batch 8 needs 919,552) returns
+ *   STQ1_ERR_SCRATCH and enqueues nothing.
+ *   The first call on a device looks up that buffer's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Each call clears the counters on `stream` before its kernel.  All calls
+ *   in the process share the one buffer and it keeps the last call's contents:
+ *   calls that may overlap on the GPU (different streams, or concurrent host
+ *   threads) race on it and must be serialized by the caller.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_ALIGN, STQ1_ERR_SCRATCH,
+ * STQ1_ERR_CUDA.
+ */
+int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float* y, int64_t N, int64_t K,
+                      int batch, void* stream);
 
 /*
  * stq1_set_path -- process-wide choice between the two matmul kernels, for

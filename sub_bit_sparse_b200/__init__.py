@@ -24,6 +24,7 @@ OK = 0
 ERRORS = {
     -1: "STQ1_ERR_SHAPE", -2: "STQ1_ERR_NULL", -3: "STQ1_ERR_CUDA", -4: "STQ1_ERR_DEVICE",
     -5: "STQ1_ERR_VALUE", -6: "STQ1_ERR_ALIGN", -7: "STQ1_ERR_WORKSPACE", -8: "STQ1_ERR_ARG",
+    -9: "STQ1_ERR_SCRATCH",
 }
 DEV_BAD_EXPERT = 1
 DEV_WAIT_LIMIT = 2
@@ -50,6 +51,8 @@ SIGNATURES = {
                                    _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "stq1_status": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
     "stq1_set_path": (_c.c_int, [_c.c_int]),
+    "stq1_gemv_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int,
+                                     _c.c_void_p]),
 }
 
 
@@ -195,6 +198,22 @@ def gemv(w_packed, x, n: int, k: int, out=None, ws=None):
                        None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
                        _stream(x))
     _check("stq1_gemv", rc)
+    return out
+
+
+def gemv_noalloc(w_packed, x, n: int, k: int, out=None):
+    """Like ``gemv`` but the library allocates nothing and takes no workspace: for
+    callers that cannot allocate device memory.  Its built-in scratch is shared by
+    all calls in the process, so calls must not overlap on the GPU."""
+    torch = _torch()
+    _require(w_packed, torch.uint8, "w_packed")
+    _require(x, torch.bfloat16, "x")
+    b = x.shape[0] if x.dim() == 2 else 1
+    if out is None:
+        out = torch.empty((b, n), dtype=torch.float32, device=x.device)
+    _require(out, torch.float32, "out")
+    rc = _load().stq1_gemv_noalloc(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b, _stream(x))
+    _check("stq1_gemv_noalloc", rc)
     return out
 
 

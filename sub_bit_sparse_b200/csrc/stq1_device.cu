@@ -414,3 +414,110 @@ extern "C" int stq1_status(void* stream, int* device_err) {
   if (device_err) *device_err = v;
   return v ? STQ1_ERR_DEVICE : STQ1_OK;
 }
+
+// ---------------------------------------------------------------------------
+// GEMV that allocates nothing (no counterpart on the source pages).
+//
+// Some callers cannot hand this library a workspace: frameworks and plugin
+// hosts that own all device memory and pass in only the input and output
+// buffers, and latency-critical code that must not call cudaMalloc, which can
+// synchronize the whole device.  For them, stq1_gemv_noalloc runs the table
+// GEMV with its split-K scratch (arrival counters and partial sums) in a
+// fixed buffer compiled into the library.
+// ---------------------------------------------------------------------------
+namespace stq1 {
+namespace {
+
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(1) << 20;   // 1 MiB
+
+// Loaded with the library on every GPU that uses it and kept until the process
+// exits.  Host code must not use this name as a device address: it only
+// stands in for the symbol; the device address comes from
+// cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+uint8_t* g_static_scratch_ptr[kMaxDevices] = {};
+
+// One-time set-up per device, with that device current.
+int static_scratch(uint8_t** out) {
+  const int dev = current_device();
+  if (dev < 0) return STQ1_ERR_CUDA;
+  if (!g_static_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || ptr == nullptr)
+      return STQ1_ERR_CUDA;
+    g_static_scratch_ptr[dev] = static_cast<uint8_t*>(ptr);
+  }
+  *out = g_static_scratch_ptr[dev];
+  return STQ1_OK;
+}
+
+}  // namespace
+}  // namespace stq1
+
+extern "C" int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float* y, int64_t N,
+                                 int64_t K, int batch, void* stream) {
+  if (!W_packed || !x || !y) return STQ1_ERR_NULL;
+  if (N <= 0 || K <= 0 || K % kBlockWeights || batch <= 0 || batch > 65535 ||
+      N > (1LL << 31) - 1 || K > (1LL << 31) - 1)
+    return STQ1_ERR_SHAPE;
+  if (!aligned16(W_packed) || !aligned16(x)) return STQ1_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long nb = K / kBlockWeights;
+  const long long rowbytes = nb * kBlockBytes;
+  int rc = ensure_configured();
+  if (rc != STQ1_OK) return rc;
+  if (nb % 2 != 0) {
+    // rows with an odd number of blocks use the direct kernel, which needs no scratch
+    const long long warps = static_cast<long long>(batch) * N;
+    direct_gemv_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(
+        static_cast<const uint8_t*>(W_packed), 0, 1, x, nullptr, 1, nullptr, 0, y,
+        static_cast<int>(N), static_cast<int>(K), batch);
+    return launch_status();
+  }
+  // Same work split as the table path of stq1_gemv.
+  const int n_tiles = (batch + kLutMaxTT - 1) / kLutMaxTT;
+  const int n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
+  const int n_chunks = static_cast<int>(nb / kLutKC);
+  const long long units0 = static_cast<long long>(n_tiles) * n_slabs;
+  const int S = static_cast<int>(std::max<long long>(
+      1, std::min<long long>((kTargetUnits + units0 - 1) / units0, std::max(1, n_chunks))));
+  const size_t need = S > 1 ? kCounterBytes + static_cast<size_t>(S) * batch * N * sizeof(float) : 0;
+  if (need > kStaticScratchBytes) return STQ1_ERR_SCRATCH;
+  uint8_t* scratch = nullptr;
+  if (S > 1) {
+    rc = static_scratch(&scratch);
+    if (rc != STQ1_OK) return rc;
+    // the array keeps the previous call's contents: the counters must start at zero
+    if (cudaMemsetAsync(scratch, 0, kCounterBytes, s) != cudaSuccess) return STQ1_ERR_CUDA;
+  }
+  LutArgs a{};
+  a.W = static_cast<const uint8_t*>(W_packed);
+  a.W_end = a.W + N * rowbytes;
+  a.expert_bytes = 0;
+  a.rowbytes = rowbytes;
+  a.x = x;
+  a.y = y;
+  a.counters = S > 1 ? reinterpret_cast<int*>(scratch) : nullptr;
+  a.partial = S > 1 ? reinterpret_cast<float*>(scratch + kCounterBytes) : nullptr;
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.nb = static_cast<int>(nb);
+  a.topk = 1;
+  a.batch = batch;
+  a.rows_out = batch;
+  a.n_tiles = n_tiles;
+  a.n_slabs = n_slabs;
+  a.S = S;
+  a.n_chunks = n_chunks;
+  a.P = residue_period(rowbytes);
+  a.flags = 0;
+  const unsigned grid = static_cast<unsigned>(static_cast<long long>(n_tiles) * n_slabs * S);
+  if (batch == 1)
+    lut_gemv_kernel<1><<<grid, kLutThreads, lut_smem_bytes(1), s>>>(a);
+  else if (batch == 2)
+    lut_gemv_kernel<2><<<grid, kLutThreads, lut_smem_bytes(2), s>>>(a);
+  else
+    lut_gemv_kernel<4><<<grid, kLutThreads, lut_smem_bytes(4), s>>>(a);
+  return launch_status();
+}
