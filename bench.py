@@ -54,6 +54,27 @@ def _peaks():
 
 
 # ---------------------------------------------------------------------------
+# multi-rank aggregation (weak scaling: every rank runs the per-rank workload)
+# ---------------------------------------------------------------------------
+
+
+def max_over_ranks(ms: float, device=None) -> float:
+    """The slowest rank's elapsed time (all ranks take part; no-op at world 1)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
+# ---------------------------------------------------------------------------
 # clocks during the timed region (NVML, sampled from a thread)
 # ---------------------------------------------------------------------------
 
@@ -188,11 +209,7 @@ def run_gpu(args):
         torch.cuda.synchronize()
         ms = start.elapsed_time(end)
         barrier()
-        if world > 1:
-            t = torch.tensor([ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(ms, device)
 
     # --- headline: batch 1 ---
     g1 = time_graph(torch, make_step(1), args.steps, args.warmup, stream)
@@ -201,7 +218,7 @@ def run_gpu(args):
     ms_step = ms / args.steps
     launch_ms = ms_step / STACK
     bytes_step = STACK * PACKED
-    value = world * bytes_step * args.steps / (ms * 1e-3) / 1e9
+    value = whole_job_rate(bytes_step * args.steps, world, ms) / 1e9
     achieved = PACKED / (launch_ms * 1e-3) / 1e9
 
     # --- the same GEMV at larger batches ---
@@ -355,22 +372,27 @@ def run_sweep(args):
     y = torch.empty((1024, n), dtype=torch.float32, device=device)
     ws = stq1.workspace(max(stq1.LIB.stq1_gemv_workspace(n, k, b) for b in (1, 4, 16, 64, 256, 1024)), device)
     out = []
+    stream = torch.cuda.Stream(device)
     for b in (1, 4, 16, 64, 256, 1024):
         row = {"batch": b}
         for name, path in (("table", stq1.PATH_TABLE), ("tiles", stq1.PATH_TILES)):
             stq1.set_path(path)
             xb = xd[:b].contiguous()
-            for i in range(3):
-                stq1.gemv(stack[i % copies], xb, n, k, out=y[:b], ws=ws)
-            torch.cuda.synchronize()
-            reps = max(3, min(50, 2000 // b))
+            reps = max(2, min(copies, 4096 // b))
+
+            def step():
+                for i in range(reps):
+                    stq1.gemv(stack[i % copies], xb, n, k, out=y[:b], ws=ws)
+
+            g = time_graph(torch, step, 1, 3, stream)
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s0.record()
-            for i in range(reps):
-                stq1.gemv(stack[i % copies], xb, n, k, out=y[:b], ws=ws)
-            s1.record()
+            with torch.cuda.stream(stream):
+                s0.record(stream)
+                g.replay()
+                s1.record(stream)
             torch.cuda.synchronize()
             ms = s0.elapsed_time(s1) / reps
+            del g
             row[name] = {"ms": round(ms, 4), "gbs": round(pb / (ms * 1e-3) / 1e9, 1),
                          "tflops": round(2.0 * b * n * k / (ms * 1e-3) / 1e12, 2)}
         stq1.set_path(stq1.PATH_AUTO)
@@ -407,13 +429,8 @@ def run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier):
             one()
         end.record(stream)
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(world * STACK * PACKED * steps / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+    ms = max_over_ranks(start.elapsed_time(end), device)
+    return {"value": round(whole_job_rate(STACK * PACKED * steps, world, ms) / 1e9, 1), "unit": "GB/s",
             "h2d_bytes_per_step": K_COLS * 2, "d2h_bytes_per_step": STACK * N_ROWS * 4,
             "steps": steps, "ms_per_step": round(ms / steps, 4)}
 

@@ -68,7 +68,7 @@ extern "C" {
 
 /* stq1_moe_gateup flags. */
 #define STQ1_MOE_WEIGHT_UP 1      /* multiply rows N/2..N-1 (the up half) by the routing weight */
-#define STQ1_MOE_FP8 2            /* large-token path: e4m3 activations (error reported, not gated) */
+#define STQ1_MOE_FP8 2            /* reserved for an e4m3 tile variant; currently STQ1_ERR_ARG */
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 int stq1_version(void);

@@ -18,10 +18,16 @@
 // which lets each warp decode with compile-time byte offsets and
 // conflict-free 16-byte shared loads.
 //
-// Split K: with few rows the K range is divided into S contiguous pieces; each
-// unit stores its partial sums and the last unit to finish a (tile, slab)
-// adds them in order 0..S-1 (deterministic) and writes y.
+// Split K: with few rows the K range is divided into S contiguous pieces.  The
+// S units of a (tile, slab) normally form one thread-block cluster: each keeps
+// its partial sums in its own shared memory and, after a cluster barrier, each
+// adds a slice of the rows from all S peers (distributed shared memory) in
+// order 0..S-1 and writes y.  Without clusters (a caller-provided scratch
+// buffer instead), each unit stores its partials in global memory and the last
+// unit to finish adds them in the same order.  Both are deterministic.
 #pragma once
+
+#include <utility>
 
 #include "device_common.cuh"
 
@@ -60,6 +66,7 @@ struct LutArgs {
   int n_chunks;
   int P;                     // rows per residue class of (row * rowbytes) mod 16
   int flags;
+  int cluster;               // 1: the S splits of a (tile, slab) form one thread-block cluster
 };
 
 __device__ __forceinline__ uint32_t win_word(const uint32_t* w, int p) {
@@ -78,70 +85,91 @@ __device__ __forceinline__ float lds_f32_addr(uint32_t addr) {
   return v;
 }
 
-// Decode the chunk's KC blocks of this lane's row against TT tokens' tables.
-// O = byte offset of the row's span inside its 16-byte-aligned slot.
-template <int TT, int O>
-__device__ __forceinline__ void lut_row_chunk(uint32_t slot, uint32_t lut,
-                                              float (&acc)[kLutMaxTT]) {
+// Code words of one block, extracted from a 16-byte-aligned register window:
+// d (fp32), qs as 8 little-endian words, qh as 2 words.
+struct BlockCodes {
+  float d;
+  uint32_t Q[8];
+  uint32_t H0, H1;
+};
+
+// Loads the block starting at byte B0 of a slot (B0 compile-time) with 16-byte
+// shared loads and extracts its fields.
+template <int B0>
+__device__ __forceinline__ void load_block_codes(uint32_t slot, BlockCodes& bc) {
+  constexpr int C0 = B0 >> 4;
+  constexpr int C1 = (B0 + kBlockBytes - 1) >> 4;
+  uint32_t w[16];
 #pragma unroll
-  for (int j = 0; j < kLutKC; ++j) {
-    const int B0 = O + kBlockBytes * j;            // block start inside the slot
-    const int C0 = B0 >> 4;
-    const int C1 = (B0 + kBlockBytes - 1) >> 4;
-    uint32_t w[16];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (C0 + c <= C1) {
-        const uint4 v = lds_v4(slot + 16u * (C0 + c));
-        w[4 * c + 0] = v.x;
-        w[4 * c + 1] = v.y;
-        w[4 * c + 2] = v.z;
-        w[4 * c + 3] = v.w;
-      } else {
-        w[4 * c + 0] = w[4 * c + 1] = w[4 * c + 2] = w[4 * c + 3] = 0u;
-      }
-    }
-    const int base = B0 - 16 * C0;                 // block start inside the window (even)
-    const uint32_t dword = w[base >> 2] >> (8 * (base & 3));
-    const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(dword & 0xFFFFu)));
-    const uint32_t H0 = win_word(w, base + kOffQh);
-    const uint32_t H1 = win_word(w, base + kOffQh + 4);
-    float2 s0[TT], s1[TT];
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      s0[t] = make_float2(0.f, 0.f);
-      s1[t] = make_float2(0.f, 0.f);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {                  // qs word i: groups 8i .. 8i+7
-      const uint32_t Q = win_word(w, base + kOffQs + 4 * i);
-      const uint32_t hb = (i < 4 ? H0 : H1) >> (8 * (i & 3));
-      // table byte offsets (t << 6 | n << 2) of the 4 even / 4 odd groups
-      const uint32_t ce = ((Q << 2) & 0x3C3C3C3Cu) | spread_even_bits(hb);
-      const uint32_t co = ((Q >> 2) & 0x3C3C3C3Cu) | spread_even_bits(hb >> 1);
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const uint32_t ae = __byte_perm(ce, lut, 0x7650u | m);   // lut is 256-aligned
-        const uint32_t ao = __byte_perm(co, lut, 0x7650u | m);
-        const int ge = 64 * j + 8 * i + 2 * m;    // even group's index in the chunk
-#pragma unroll
-        for (int t = 0; t < TT; ++t) {
-          const uint32_t off = static_cast<uint32_t>(t * kLutTokenBytes + ge * kLutGroupBytes);
-          const float ve = lds_f32_addr(ae + off);
-          const float vo = lds_f32_addr(ao + off + kLutGroupBytes);
-          if (m & 1)
-            s1[t] = __fadd2_rn(s1[t], make_float2(ve, vo));
-          else
-            s0[t] = __fadd2_rn(s0[t], make_float2(ve, vo));
-        }
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      const float sum = (s0[t].x + s0[t].y) + (s1[t].x + s1[t].y);
-      acc[t] = fmaf(d, sum, acc[t]);
+  for (int c = 0; c < 4; ++c) {
+    if (C0 + c <= C1) {
+      const uint4 v = lds_v4(slot + 16u * (C0 + c));
+      w[4 * c + 0] = v.x;
+      w[4 * c + 1] = v.y;
+      w[4 * c + 2] = v.z;
+      w[4 * c + 3] = v.w;
+    } else {
+      w[4 * c + 0] = w[4 * c + 1] = w[4 * c + 2] = w[4 * c + 3] = 0u;
     }
   }
+  constexpr int base = B0 - 16 * C0;                // even
+  const uint32_t dword = w[base >> 2] >> (8 * (base & 3));
+  bc.d = __half2float(__ushort_as_half(static_cast<unsigned short>(dword & 0xFFFFu)));
+  bc.H0 = win_word(w, base + kOffQh);
+  bc.H1 = win_word(w, base + kOffQh + 4);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) bc.Q[i] = win_word(w, base + kOffQs + 4 * i);
+}
+
+// Compile-time loop helper.
+template <int I>
+struct IntC {
+  static constexpr int value = I;
+};
+template <typename F, int... Is>
+__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, Is...>) {
+  (f(IntC<Is>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+// Table lookups of one block's 64 groups for TT tokens; `lut` is the 256-aligned
+// base of this block's tables, every offset below it is an immediate of the
+// shared load, and the group's code byte is spliced into the base with one
+// byte permute.
+template <int TT>
+__device__ __forceinline__ void lut_block_body(const BlockCodes& bc, uint32_t lut, float (&acc)[kLutMaxTT]) {
+  float s[TT][4];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) s[t][0] = s[t][1] = s[t][2] = s[t][3] = 0.f;
+  static_for<8>([&](auto IC) {                       // qs word i: groups 8i .. 8i+7
+    constexpr int i = decltype(IC)::value;
+    const uint32_t Q = bc.Q[i];
+    const uint32_t hb = (i < 4 ? bc.H0 : bc.H1) >> (8 * (i & 3));
+    // table byte offsets (t << 6 | n << 2) of the 4 even / 4 odd groups
+    const uint32_t ce = ((Q << 2) & 0x3C3C3C3Cu) | (((hb & 0x55u) * 0x01041040u) & 0x40404040u);
+    const uint32_t co = ((Q >> 2) & 0x3C3C3C3Cu) | (((hb & 0xAAu) * 0x00820820u) & 0x40404040u);
+    static_for<4>([&](auto MC) {
+      constexpr int m = decltype(MC)::value;
+      constexpr int ge = 8 * i + 2 * m;              // even group's index in the block
+      const uint32_t ae = __byte_perm(ce, lut, 0x7650u | m);
+      const uint32_t ao = __byte_perm(co, lut, 0x7650u | m);
+      s[0][m] += lds_f32<ge * kLutGroupBytes>(ae) + lds_f32<(ge + 1) * kLutGroupBytes>(ao);
+      if constexpr (TT > 1)
+        s[1][m] += lds_f32<kLutTokenBytes + ge * kLutGroupBytes>(ae) +
+                   lds_f32<kLutTokenBytes + (ge + 1) * kLutGroupBytes>(ao);
+      if constexpr (TT > 2)
+        s[2][m] += lds_f32<2 * kLutTokenBytes + ge * kLutGroupBytes>(ae) +
+                   lds_f32<2 * kLutTokenBytes + (ge + 1) * kLutGroupBytes>(ao);
+      if constexpr (TT > 3)
+        s[3][m] += lds_f32<3 * kLutTokenBytes + ge * kLutGroupBytes>(ae) +
+                   lds_f32<3 * kLutTokenBytes + (ge + 1) * kLutGroupBytes>(ao);
+    });
+  });
+#pragma unroll
+  for (int t = 0; t < TT; ++t) acc[t] = fmaf(bc.d, (s[t][0] + s[t][1]) + (s[t][2] + s[t][3]), acc[t]);
 }
 
 // Activations of this thread's group for chunk `chunk`, TT tokens (8 bytes each).
@@ -164,16 +192,16 @@ __device__ __forceinline__ void lut_build(const uint2 (&xv)[kLutMaxTT], uint32_t
     const float x2 = bf16_bits_to_f32(xv[t].y & 0xFFFFu), x3 = bf16_bits_to_f32(xv[t].y >> 16);
     const uint32_t gb = lut + static_cast<uint32_t>(t * kLutTokenBytes + g * kLutGroupBytes);
     // z = 0: a=1 b=2 c=3 ; z = 1: a=0 b=2 c=3 ; z = 2: a=0 b=1 c=3 ; z = 3: a=0 b=1 c=2
-    const float xa[4] = {x1, x0, x0, x0};
-    const float xb[4] = {x2, x2, x1, x1};
-    const float xc[4] = {x3, x3, x3, x2};
-#pragma unroll
-    for (int z = 0; z < 4; ++z) {
-      const float p = xa[z] + xb[z], q = xa[z] - xb[z];
-      const float e0 = p + xc[z], e1 = p - xc[z], e2 = q + xc[z], e3 = q - xc[z];
+    auto put = [&](int z, float xa, float xb, float xc) {
+      const float p = xa + xb, q = xa - xb;
+      const float e0 = p + xc, e1 = p - xc, e2 = q + xc, e3 = q - xc;
       sts_v4f(gb + 16u * z, e0, e1, e2, e3);
       sts_v4f(gb + 64u + 16u * z, -e0, -e1, -e2, -e3);
-    }
+    };
+    put(0, x1, x2, x3);
+    put(1, x0, x2, x3);
+    put(2, x0, x1, x3);
+    put(3, x0, x1, x2);
   }
 }
 
@@ -182,8 +210,9 @@ template <int TT>
 __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int split, int tile_id,
                          const int* xrow, const int* orow, uint8_t* smem) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rg = warp;                                           // 32-row group
   const int P = a.P;
-  const int rho = P * lane + (warp % P) + 32 * P * (warp / P);   // row within the slab
+  const int rho = P * lane + (rg % P) + 32 * P * (rg / P);       // row within the slab
   const long long row = static_cast<long long>(slab) * kLutRows + rho;
   const bool row_ok = row < a.N;
   const int c0 = static_cast<int>(static_cast<long long>(split) * a.n_chunks / a.S);
@@ -191,9 +220,9 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t lut = (sbase + 255u) & ~255u;
-  const uint32_t stage0 = lut + TT * kLutTokenBytes;
-  const uint32_t bar0 = stage0 + 2 * kLutStageBytes;
-  const uint32_t my_slot_off = static_cast<uint32_t>(threadIdx.x) * kLutSlotBytes;
+  const uint32_t bar0 = lut + TT * kLutTokenBytes;   // 2 mbarriers, then the stages
+  const uint32_t stage0 = bar0 + 16;
+  const uint32_t my_slot_off = static_cast<uint32_t>(rg * 32 + lane) * kLutSlotBytes;
 
   if (threadIdx.x == 0) {
     mbar_init(bar0, kLutThreads);
@@ -233,7 +262,7 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
   for (int t = 0; t < kLutMaxTT; ++t) acc[t] = 0.f;
 
   // offset of the warp's spans inside their 16-byte slots (same for every lane)
-  const long long row0 = static_cast<long long>(slab) * kLutRows + (warp % P) + 32 * P * (warp / P);
+  const long long row0 = static_cast<long long>(slab) * kLutRows + (rg % P) + 32 * P * (rg / P);
   const uintptr_t wbase = reinterpret_cast<uintptr_t>(Wm) + static_cast<uintptr_t>(row0 * a.rowbytes);
 
   // Weights do not depend on the previous kernel in the stream: start their
@@ -251,6 +280,7 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
   griddep_launch_dependents();
   uint2 xv[kLutMaxTT];
   if (c0 < c1) lut_load_x<TT>(a, c0, xrow, xv);
+  bool failed = false;
   for (int c = c0; c < c1; ++c) {
     const int it = c - c0;
     const int st = it & 1;
@@ -259,38 +289,70 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
     const bool landed = mbar_wait_bounded(bar0 + 8u * st, (it >> 1) & 1);
     // one barrier: tables built, copies landed (agreed by every thread)
     if (!__syncthreads_and(landed)) {
-      // A copy did not complete within the bound.  Wait (bounded) for the copy
-      // already issued into the other stage, so no bulk copy is still writing
-      // this CTA's shared memory when it exits; the error word is set.
+      // A copy did not complete within the bound (the error word is set).
+      // Wait (bounded) for the copy already issued into the other stage, so no
+      // bulk copy is still writing this CTA's shared memory when it exits.
       if (c + 1 < c1) mbar_wait_bounded(bar0 + 8u * (st ^ 1), ((it + 1) >> 1) & 1);
-      return;
+      failed = true;
+      break;
     }
     if (row_ok) {
       const uint32_t slot = stage0 + st * kLutStageBytes + my_slot_off;
       const int o = static_cast<int>((wbase + static_cast<uintptr_t>(c) * (kLutKC * kBlockBytes)) & 15);
+      // only the extraction depends on the warp's offset; one copy of the body follows
+      BlockCodes b0, b1;
       switch (o) {
-        case 0: lut_row_chunk<TT, 0>(slot, lut, acc); break;
-        case 4: lut_row_chunk<TT, 4>(slot, lut, acc); break;
-        case 8: lut_row_chunk<TT, 8>(slot, lut, acc); break;
-        default: lut_row_chunk<TT, 12>(slot, lut, acc); break;
+        case 0: load_block_codes<0>(slot, b0); load_block_codes<0 + kBlockBytes>(slot, b1); break;
+        case 4: load_block_codes<4>(slot, b0); load_block_codes<4 + kBlockBytes>(slot, b1); break;
+        case 8: load_block_codes<8>(slot, b0); load_block_codes<8 + kBlockBytes>(slot, b1); break;
+        default: load_block_codes<12>(slot, b0); load_block_codes<12 + kBlockBytes>(slot, b1); break;
       }
+      // the second block's tables start 64 groups into the chunk's (256-aligned)
+      lut_block_body<TT>(b0, lut, acc);
+      lut_block_body<TT>(b1, lut + static_cast<uint32_t>(kGroupsPerBlock * kLutGroupBytes), acc);
     }
     __syncthreads();
     if (c + 2 < c1) issue(c + 2, st);                      // this stage is free again
   }
+  const bool up = (a.flags & STQ1_MOE_WEIGHT_UP) && row >= a.N / 2;
   if (a.S == 1) {
-    if (row_ok) {
+    if (row_ok && !failed) {
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
         float v = acc[t];
-        if ((a.flags & STQ1_MOE_WEIGHT_UP) && row >= a.N / 2) v *= a.route_w[orow[t]];
+        if (up) v *= a.route_w[orow[t]];
         a.y[static_cast<long long>(orow[t]) * a.N + row] = v;
       }
     }
     return;
   }
 
-  // split K: publish partials, the last unit of this (tile, slab) reduces.
+  if (a.cluster) {
+    // Every CTA of the cluster reaches both cluster barriers, failed or not.
+    const uint32_t red = lut;                          // tables are no longer needed
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(red + 4u * (t * kLutRows + rho)), "f"(acc[t]) : "memory");
+    cluster_sync_all();
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int lo = rank * kLutRows / a.S, hi = (rank + 1) * kLutRows / a.S;
+    const int nr = hi - lo;
+    for (int idx = threadIdx.x; idx < nr * TT; idx += kLutThreads) {
+      const int t = idx / nr, rr = lo + idx % nr;
+      float v = 0.f;
+      for (int sp = 0; sp < a.S; ++sp) v += ld_peer_f32(red + 4u * (t * kLutRows + rr), sp);
+      const long long rrow = static_cast<long long>(slab) * kLutRows + rr;
+      if (rrow < a.N) {
+        if ((a.flags & STQ1_MOE_WEIGHT_UP) && rrow >= a.N / 2) v *= a.route_w[orow[t]];
+        a.y[static_cast<long long>(orow[t]) * a.N + rrow] = v;
+      }
+    }
+    cluster_sync_all();                                // peers may still read this CTA's partials
+    return;
+  }
+  if (failed) return;
+
+  // Scratch mode: publish partials, the last unit of this (tile, slab) reduces.
   // One thread fences after the barrier: the barrier orders the other threads'
   // stores before it, and the gpu-scope fence is cumulative.
   if (row_ok) {
@@ -312,9 +374,9 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
       float v = 0.f;
-      for (int s = 0; s < a.S; ++s)
-        v += __ldcg(&a.partial[(static_cast<long long>(s) * a.rows_out + orow[t]) * a.N + row]);
-      if ((a.flags & STQ1_MOE_WEIGHT_UP) && row >= a.N / 2) v *= a.route_w[orow[t]];
+      for (int sp = 0; sp < a.S; ++sp)
+        v += __ldcg(&a.partial[(static_cast<long long>(sp) * a.rows_out + orow[t]) * a.N + row]);
+      if (up) v *= a.route_w[orow[t]];
       a.y[static_cast<long long>(orow[t]) * a.N + row] = v;
     }
   }
@@ -371,8 +433,8 @@ __global__ void __launch_bounds__(kLutThreads) lut_gemv_kernel(const LutArgs a) 
   }
 }
 
-inline size_t lut_smem_bytes(int ttmax) {
-  return 256 + static_cast<size_t>(ttmax) * kLutTokenBytes + 2 * kLutStageBytes + 16;
+inline size_t lut_smem_bytes(int ttmax, int stages = 2) {
+  return 256 + static_cast<size_t>(ttmax) * kLutTokenBytes + 16 + static_cast<size_t>(stages) * kLutStageBytes;
 }
 
 }  // namespace stq1

@@ -31,6 +31,7 @@ int g_path = 0;
 constexpr int kTcMinBatch = 16;       // stq1_gemv: batches from here use the tile kernel
 constexpr int kTcMinPairsPerExpert = 16;
 constexpr int kMoeTableTokens = 2;    // MoE decode tiles: pairs per table-kernel unit
+constexpr int kMaxClusterSplit = 16;  // largest (non-portable) cluster used for split K
 
 int sm_count() {
   static int cache[kMaxDevices] = {};
@@ -94,6 +95,12 @@ int ensure_configured() {
       cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kTcSmemBytes) != cudaSuccess)
     return STQ1_ERR_CUDA;
+  // split-K clusters of up to 16 CTAs (above the portable 8); a refusal only
+  // disables the cluster path
+  cudaFuncSetAttribute(lut_gemv_kernel<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaFuncSetAttribute(lut_gemv_kernel<2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaFuncSetAttribute(lut_gemv_kernel<4>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaGetLastError();
   done[dev] = true;
   return STQ1_OK;
 }
@@ -106,20 +113,35 @@ int launch_status() {
 // previous kernel in the stream drains; it calls griddepcontrol.wait before
 // touching anything that kernel may write.
 template <typename... Params, typename... Args>
-int launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
-               Args&&... args) {
+int launch_pdl_cluster(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                       unsigned cluster, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? STQ1_OK
-                                                                                      : STQ1_ERR_CUDA;
+  cfg.numAttrs = n;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess) return STQ1_OK;
+  cudaGetLastError();   // clear a refused launch so the caller can fall back
+  return STQ1_ERR_CUDA;
+}
+
+template <typename... Params, typename... Args>
+int launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+               Args&&... args) {
+  return launch_pdl_cluster(kernel, grid, block, smem, s, 1u, std::forward<Args>(args)...);
 }
 
 int residue_period(long long rowbytes) {
@@ -257,11 +279,23 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
   a.P = residue_period(rowbytes);
   a.flags = 0;
   const long long grid = static_cast<long long>(p.n_tiles) * p.n_slabs * p.S;
-  if (batch == 1)
-    return launch_pdl(lut_gemv_kernel<1>, static_cast<unsigned>(grid), kLutThreads, lut_smem_bytes(1), s, a);
-  if (batch == 2)
-    return launch_pdl(lut_gemv_kernel<2>, static_cast<unsigned>(grid), kLutThreads, lut_smem_bytes(2), s, a);
-  return launch_pdl(lut_gemv_kernel<4>, static_cast<unsigned>(grid), kLutThreads, lut_smem_bytes(4), s, a);
+  // one shared stage is enough when every unit holds a single chunk
+  const int stages = (p.n_chunks + p.S - 1) / p.S >= 2 ? 2 : 1;
+  const int tt = batch == 1 ? 1 : (batch == 2 ? 2 : 4);
+  auto go = [&](int cluster) {
+    a.cluster = cluster > 1 ? 1 : 0;
+    const size_t smem = lut_smem_bytes(tt, stages);
+    if (tt == 1)
+      return launch_pdl_cluster(lut_gemv_kernel<1>, static_cast<unsigned>(grid), kLutThreads, smem, s, cluster, a);
+    if (tt == 2)
+      return launch_pdl_cluster(lut_gemv_kernel<2>, static_cast<unsigned>(grid), kLutThreads, smem, s, cluster, a);
+    return launch_pdl_cluster(lut_gemv_kernel<4>, static_cast<unsigned>(grid), kLutThreads, smem, s, cluster, a);
+  };
+  // split K reduces through distributed shared memory inside a cluster of the
+  // S units of a slab; if the device refuses such a cluster, through the
+  // caller's scratch buffer
+  if (p.S > 1 && p.S <= kMaxClusterSplit && go(p.S) == STQ1_OK) return STQ1_OK;
+  return go(1);
 }
 
 namespace stq1 {
@@ -307,6 +341,7 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   if (!expert_blocks || !x || !topk_ids || !y) return STQ1_ERR_NULL;
   if ((flags & STQ1_MOE_WEIGHT_UP) && !topk_weights) return STQ1_ERR_NULL;
   if (flags & ~(STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8)) return STQ1_ERR_ARG;
+  if (flags & STQ1_MOE_FP8) return STQ1_ERR_ARG;   // the e4m3 tile variant is not built yet
   if (T <= 0 || topk <= 0 || E <= 0 || topk > E || E > kMaxExperts || N <= 0 || (N & 1) || K <= 0 ||
       K % kBlockWeights || N > (1LL << 30) || K > (1LL << 30) ||
       static_cast<long long>(T) * topk > (1LL << 30))

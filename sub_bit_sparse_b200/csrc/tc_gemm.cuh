@@ -13,15 +13,17 @@
 //               shared ring (one 2-D tensor copy per stage, no multicast).
 //   warp 1      TMEM allocator and the single MMA-issuing thread:
 //               tcgen05.mma.cta_group::1.kind::f16, A from TMEM, B from shared.
-//   warps 2-5   decoders: one thread per weight row reads the row's 42-byte
-//               block for the slab, expands each group's 5-bit code to four
-//               bf16 values through a 32-entry table and stores 64 columns per
-//               stage into TMEM (tcgen05.st), the A operand.
-//   warps 6-9   epilogue: per slab, tcgen05.ld of the slab accumulator, fp32
-//               FMA with the row's d, release of the TMEM buffer; at the end
-//               of the tile, coalesced stores of y.
+//   warps 2-9   decoders, two per TMEM lane quadrant: a thread owns one weight
+//               row, reads the row's 42-byte block for the slab (one slab
+//               ahead), expands each group's 5-bit code to four bf16 values
+//               through a 32-entry table and stores its half of each stage's
+//               64 columns into TMEM (tcgen05.st), the A operand.
+//   warps 10-17 epilogue, two per quadrant (64 token columns each): per slab,
+//               tcgen05.ld of the slab accumulator, fp32 FMA with the row's d,
+//               release of the TMEM buffer; at the end of the tile, coalesced
+//               stores of y.
 // TMEM (512 columns allocated, one CTA per SM): slab accumulators 2 x 128
-// columns, A stages 4 x 32 columns.
+// columns, A stages 8 x 32 columns.  Shared memory: 8 x-tile stages of 16 KB.
 // All waits are bounded; a timeout sets the device error word and makes every
 // role stop at its next wait, so the CTA always reaches the final barrier and
 // frees its TMEM.
@@ -36,20 +38,22 @@ namespace stq1 {
 constexpr int kTcM = 128;
 constexpr int kTcN = 128;
 constexpr int kTcKC = 64;                     // K per stage (128 bytes of bf16)
-constexpr int kTcStages = 4;
+constexpr int kTcStages = 8;
 constexpr int kTcSlabChunks = kBlockWeights / kTcKC;    // 4 stages per scale block
-constexpr int kTcThreads = 320;
+constexpr int kTcThreads = 576;
+constexpr int kTcDecoders = 256;                 // threads: 8 warps
+constexpr int kTcEpilogue = 256;                 // threads: 8 warps
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcColD = 0;               // 2 x 128
-constexpr uint32_t kTcColA = 256;             // 4 x 32
+constexpr uint32_t kTcColA = 256;             // kTcStages x 32
 constexpr int kTcBStageBytes = kTcN * kTcKC * 2;   // 16 KB
 // shared layout (offsets from a 1024-aligned base)
 constexpr int kTcOffB = 0;
-constexpr int kTcOffTable = kTcStages * kTcBStageBytes;            // 65536: 2 x 128 B decode tables
+constexpr int kTcOffTable = kTcStages * kTcBStageBytes;            // 131072: 2 x 128 B decode tables
 constexpr int kTcOffBar = kTcOffTable + 256;
 constexpr int kTcOffPairs = kTcOffBar + 256;                       // kTcN ints
 constexpr int kTcOffMisc = kTcOffPairs + kTcN * 4;
-constexpr int kTcSmemBytes = 1024 + kTcOffMisc + 64 + 100 * 1024;  // padded: one CTA per SM
+constexpr int kTcSmemBytes = 1024 + kTcOffMisc + 64;   // > 114 KB: one CTA per SM
 
 struct TcArgs {
   const uint8_t* W;          // matrix or expert 0
@@ -135,6 +139,25 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "r"(taddr)                                                                                \
       : "memory")
 
+#define STQ1_TMEM_LD16(taddr, v)                                                                  \
+  asm volatile(                                                                                   \
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+      "%15}, [%16];"                                                                               \
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),      \
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),  \
+        "=r"(v[14]), "=r"(v[15])                                                                   \
+      : "r"(taddr)                                                                                \
+      : "memory")
+
+#define STQ1_TMEM_ST16(taddr, v)                                                                  \
+  asm volatile(                                                                                   \
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+      "%15,%16};" ::"r"(taddr),                                                                    \
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),    \
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),          \
+      "r"(v[15])                                                                                   \
+      : "memory")
+
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -204,57 +227,55 @@ __device__ __forceinline__ void load_block_window(const uint8_t* A, const uint8_
   }
 }
 
-// Decodes the block's four 64-column chunks; for each chunk waits for the
-// A stage to be free, stores 32 TMEM columns and signals the MMA thread.
+// qs (8 words) and qh (2 words) of the block starting at window byte BASE.
 template <int BASE>
-__device__ __forceinline__ bool tc_decode_slab(const uint32_t (&w)[16], uint32_t tables,
-                                               uint32_t tmem_a_lane, uint32_t bar_full_a,
-                                               uint32_t bar_empty, uint32_t& it, volatile int* abort) {
-  uint32_t Q[8];
+__device__ __forceinline__ void tc_extract(const uint32_t (&w)[16], uint32_t (&Q)[8], uint32_t& H0,
+                                           uint32_t& H1) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int p = BASE + kOffQs + 4 * i;
     Q[i] = (p & 3) ? __funnelshift_r(w[p >> 2], w[(p >> 2) + 1], 8 * (p & 3)) : w[p >> 2];
   }
-  const int ph = BASE + kOffQh;
-  const uint32_t H0 = (ph & 3) ? __funnelshift_r(w[ph >> 2], w[(ph >> 2) + 1], 8 * (ph & 3)) : w[ph >> 2];
-  const int ph1 = ph + 4;
-  const uint32_t H1 = (ph1 & 3) ? __funnelshift_r(w[ph1 >> 2], w[(ph1 >> 2) + 1], 8 * (ph1 & 3)) : w[ph1 >> 2];
+  constexpr int ph = BASE + kOffQh;
+  H0 = (ph & 3) ? __funnelshift_r(w[ph >> 2], w[(ph >> 2) + 1], 8 * (ph & 3)) : w[ph >> 2];
+  constexpr int ph1 = ph + 4;
+  H1 = (ph1 & 3) ? __funnelshift_r(w[ph1 >> 2], w[(ph1 >> 2) + 1], 8 * (ph1 & 3)) : w[ph1 >> 2];
+}
+
+// Expands this thread's half (8 groups = 16 TMEM columns) of each of the
+// block's four 64-column chunks; for each chunk waits for the A stage to be
+// free, stores its columns and signals the MMA thread.
+template <int HALF>
+__device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t H0, uint32_t H1,
+                                               uint32_t tables, uint32_t tmem_a_lane, uint32_t bar_full_a,
+                                               uint32_t bar_empty, uint32_t& it) {
 #pragma unroll
-  for (int q = 0; q < kTcSlabChunks; ++q) {          // 16 groups per chunk
-    uint32_t v[32];
+  for (int q = 0; q < kTcSlabChunks; ++q) {
+    uint32_t v[16];
+    const int i = 2 * q + HALF;                      // qs word: groups 8i .. 8i+7
+    const uint32_t hb = (i < 4 ? H0 : H1) >> (8 * (i & 3));
+    const uint32_t ce = ((Q[i] << 2) & 0x3C3C3C3Cu) | (((hb & 0x55u) * 0x01041040u) & 0x40404040u);
+    const uint32_t co = ((Q[i] >> 2) & 0x3C3C3C3Cu) | (((hb & 0xAAu) * 0x00820820u) & 0x40404040u);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = 2 * q + h;                       // qs word: groups 8i .. 8i+7
-      const uint32_t hb = (i < 4 ? H0 : H1) >> (8 * (i & 3));
-      const uint32_t ce = ((Q[i] << 2) & 0x3C3C3C3Cu) | (((hb & 0x55u) * 0x01041040u) & 0x40404040u);
-      const uint32_t co = ((Q[i] >> 2) & 0x3C3C3C3Cu) | ((((hb >> 1) & 0x55u) * 0x01041040u) & 0x40404040u);
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        // code * 4 is in bits 2..6: shift right by 2 gives the code; table base
-        // is 256-aligned so the byte splices directly into the address
-        const uint32_t ae = __byte_perm(ce, tables, 0x7650u | m);
-        const uint32_t ao = __byte_perm(co, tables, 0x7650u | m);
-        uint32_t x0, x1, y0, y1;
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(x0) : "r"(ae));
-        asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(x1) : "r"(ae));
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(y0) : "r"(ao));
-        asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(y1) : "r"(ao));
-        const int g = 8 * h + 2 * m;                 // group within the chunk (0..15)
-        v[2 * g] = x0;
-        v[2 * g + 1] = x1;
-        v[2 * g + 2] = y0;
-        v[2 * g + 3] = y1;
-      }
+    for (int m = 0; m < 4; ++m) {
+      // the group's (code * 4) byte spliced into the 256-aligned table base
+      const uint32_t ae = __byte_perm(ce, tables, 0x7650u | m);
+      const uint32_t ao = __byte_perm(co, tables, 0x7650u | m);
+      uint32_t x0, x1, y0, y1;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(x0) : "r"(ae));
+      asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(x1) : "r"(ae));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(y0) : "r"(ao));
+      asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(y1) : "r"(ao));
+      v[4 * m] = x0;
+      v[4 * m + 1] = x1;
+      v[4 * m + 2] = y0;
+      v[4 * m + 3] = y1;
     }
     const uint32_t s = it % kTcStages;
     const uint32_t use = it / kTcStages;
-    if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) {
-      *abort = 1;
-      return false;
-    }
+    if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) return false;
     tc_fence_after();
-    STQ1_TMEM_ST32(tmem_a_lane + kTcColA + 32 * s, v);
+    STQ1_TMEM_ST16(tmem_a_lane + kTcColA + 32 * s + 16 * HALF, v);
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(bar_full_a + 8 * s);
@@ -272,9 +293,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
   const uint32_t sB = sbase + kTcOffB;
   const uint32_t sTab = sbase + kTcOffTable;
   const uint32_t bar = sbase + kTcOffBar;
-  // barriers: full_b[4] @0, full_a[4] @32, empty[4] @64, d_full[2] @96, d_empty[2] @112, drain @128
-  const uint32_t bar_full_b = bar, bar_full_a = bar + 32, bar_empty = bar + 64;
-  const uint32_t bar_d_full = bar + 96, bar_d_empty = bar + 112;
+  // barriers: full_b[8] @0, full_a[8] @64, empty[8] @128, d_full[2] @192, d_empty[2] @208, drain @224
+  const uint32_t bar_full_b = bar, bar_full_a = bar + 64, bar_empty = bar + 128;
+  const uint32_t bar_d_full = bar + 192, bar_d_empty = bar + 208;
+  const uint32_t bar_drain = bar + 224;
   int* s_pairs = reinterpret_cast<int*>(sgen + kTcOffPairs);
   volatile int* s_misc = reinterpret_cast<volatile int*>(sgen + kTcOffMisc);   // [0] tmem base, [1] abort
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -282,14 +304,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < kTcStages; ++i) {
       mbar_init(bar_full_b + 8 * i, 1);
-      mbar_init(bar_full_a + 8 * i, 128);
+      mbar_init(bar_full_a + 8 * i, kTcDecoders);
       mbar_init(bar_empty + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_d_full + 8 * i, 1);
-      mbar_init(bar_d_empty + 8 * i, 128);
+      mbar_init(bar_d_empty + 8 * i, kTcEpilogue);
     }
-    mbar_init(bar + 128, 1);                         // drain barrier (abort path)
+    mbar_init(bar_drain, 1);                         // drain barrier (abort path)
     s_misc[1] = 0;
     fence_mbar_init();
   }
@@ -361,18 +383,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
       }
       if (*abort) {
         // all MMAs this thread issued must finish before TMEM is freed (bounded)
-        tc_commit(bar + 128);
-        mbar_wait_bounded(bar + 128, 0);
+        tc_commit(bar_drain);
+        mbar_wait_bounded(bar_drain, 0);
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 10) {
     // ---------------- decoders ----------------
+    const int half = (warp - 2) >> 2;               // which 8 of each chunk's 16 groups
     const int quad = warp & 3;                       // TMEM lane quadrant of this warp
     const int P = a.P;
     const int rho = P * lane + (quad % P) + 32 * P * (quad / P);   // row within the tile
     const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(32 * quad) << 16);
     uint32_t it = 0;
-    for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
+    bool ok = true;
+    for (long long item = blockIdx.x; item < n_items && ok && !*abort; item += gridDim.x) {
       const int tile = static_cast<int>(item / a.n_mtiles);
       const int mt = static_cast<int>(item % a.n_mtiles);
       const int e = a.tile_info ? a.tile_info[4 * tile + 0] : 0;
@@ -382,36 +406,54 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
       // every lane of the warp has the same block offset mod 16 (rows of one residue class)
       const uint8_t* r0 = a.W + e * a.expert_bytes +
                           static_cast<long long>(mt * kTcM + (quad % P) + 32 * P * (quad / P)) * a.rowbytes;
+      // packed windows of the next two slabs, loaded ahead (rows past N decode
+      // zeros: computed, never stored)
+      uint32_t wn[16], wn2[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) wn[i] = wn2[i] = 0u;
+      if (row_ok) {
+        load_block_window(rbase, a.W_end, wn);
+        if (n_slabs > 1) load_block_window(rbase + kBlockBytes, a.W_end, wn2);
+      }
       for (int slab = 0; slab < n_slabs; ++slab) {
         uint32_t w[16];
-        if (row_ok) {
-          load_block_window(rbase + static_cast<long long>(slab) * kBlockBytes, a.W_end, w);
-        } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) w[i] = 0u;     // rows past N: computed, never stored
+        for (int i = 0; i < 16; ++i) {
+          w[i] = wn[i];
+          wn[i] = wn2[i];
         }
+        if (row_ok && slab + 2 < n_slabs)
+          load_block_window(rbase + static_cast<long long>(slab + 2) * kBlockBytes, a.W_end, wn2);
         const int base = static_cast<int>((reinterpret_cast<uintptr_t>(r0) + static_cast<uintptr_t>(slab) * kBlockBytes) & 15);
-        bool ok;
-        switch (base) {
-          case 0: ok = tc_decode_slab<0>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
-          case 2: ok = tc_decode_slab<2>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
-          case 4: ok = tc_decode_slab<4>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
-          case 6: ok = tc_decode_slab<6>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
-          case 8: ok = tc_decode_slab<8>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
-          case 10: ok = tc_decode_slab<10>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
-          case 12: ok = tc_decode_slab<12>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
-          default: ok = tc_decode_slab<14>(w, sTab, tmem_lane, bar_full_a, bar_empty, it, abort); break;
+        uint32_t Q[8], H0, H1;
+        switch (base) {                              // only the extraction depends on the offset
+          case 0: tc_extract<0>(w, Q, H0, H1); break;
+          case 2: tc_extract<2>(w, Q, H0, H1); break;
+          case 4: tc_extract<4>(w, Q, H0, H1); break;
+          case 6: tc_extract<6>(w, Q, H0, H1); break;
+          case 8: tc_extract<8>(w, Q, H0, H1); break;
+          case 10: tc_extract<10>(w, Q, H0, H1); break;
+          case 12: tc_extract<12>(w, Q, H0, H1); break;
+          default: tc_extract<14>(w, Q, H0, H1); break;
         }
-        if (!ok) break;
+        const bool okd = half == 0 ? tc_decode_slab<0>(Q, H0, H1, sTab, tmem_lane, bar_full_a, bar_empty, it)
+                                   : tc_decode_slab<1>(Q, H0, H1, sTab, tmem_lane, bar_full_a, bar_empty, it);
+        if (!okd) {
+          *abort = 1;
+          ok = false;
+          break;
+        }
       }
     }
   } else {
     // ---------------- epilogue ----------------
     const int quad = warp & 3;
+    const int chalf = (warp - 10) >> 2;              // token columns [64 * chalf, 64 * chalf + 64)
     const int P = a.P;
     const int rho = P * lane + (quad % P) + 32 * P * (quad / P);
     const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(32 * quad) << 16);
-    const int et = threadIdx.x - 192;                // 0..127
+    const int et = threadIdx.x - 320;                // 0..255
+    constexpr int kCols = kTcN / 2;
     uint32_t sc = 0;
     for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
       const int tile = static_cast<int>(item / a.n_mtiles);
@@ -419,29 +461,31 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
       const int e = a.tile_info ? a.tile_info[4 * tile + 0] : 0;
       const int b_row = a.tile_info ? a.tile_info[4 * tile + 1] : tile * kTcN;
       const int cnt = a.tile_info ? a.tile_info[4 * tile + 2] : min(kTcN, a.batch - tile * kTcN);
-      named_bar(1, 128);                             // previous tile's stores are done
+      named_bar(1, kTcEpilogue);                     // previous tile's stores are done
       if (et < kTcN) s_pairs[et] = et < cnt ? (a.pairs ? a.pairs[b_row + et] : b_row + et) : -1;
-      named_bar(1, 128);
+      named_bar(1, kTcEpilogue);
       const int row = mt * kTcM + rho;
       const bool row_ok = row < a.N;
       const uint8_t* rbase = a.W + e * a.expert_bytes + static_cast<long long>(row_ok ? row : 0) * a.rowbytes;
-      float acc[kTcN];
+      float acc[kCols];
 #pragma unroll
-      for (int j = 0; j < kTcN; ++j) acc[j] = 0.f;
+      for (int j = 0; j < kCols; ++j) acc[j] = 0.f;
       bool ok = true;
+      unsigned short dn = __ldg(reinterpret_cast<const unsigned short*>(rbase));   // d of slab 0
       for (int slab = 0; slab < n_slabs; ++slab, ++sc) {
-        const uint8_t* B = rbase + static_cast<long long>(slab) * kBlockBytes;
-        const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(B[0] | (B[1] << 8))));
+        const float d = __half2float(__ushort_as_half(dn));
+        if (slab + 1 < n_slabs)                      // prefetch the next slab's scale
+          dn = __ldg(reinterpret_cast<const unsigned short*>(rbase + static_cast<long long>(slab + 1) * kBlockBytes));
         const uint32_t p = sc & 1, puse = sc >> 1;
         if (!mbar_wait_bounded(bar_d_full + 8 * p, puse & 1)) { *abort = 1; ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kTcN / 32; ++c) {
-          uint32_t v[32];
-          STQ1_TMEM_LD32(tmem_lane + kTcColD + p * kTcN + 32 * c, v);
+        for (int c = 0; c < kCols / 16; ++c) {
+          uint32_t v[16];
+          STQ1_TMEM_LD16(tmem_lane + kTcColD + p * kTcN + kCols * chalf + 16 * c, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[32 * c + i] = fmaf(d, __uint_as_float(v[i]), acc[32 * c + i]);
+          for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(d, __uint_as_float(v[i]), acc[16 * c + i]);
         }
         tc_fence_before();
         mbar_arrive(bar_d_empty + 8 * p);
@@ -450,8 +494,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
       if (row_ok) {
         const bool up = (a.flags & STQ1_MOE_WEIGHT_UP) && row >= a.N / 2;
 #pragma unroll
-        for (int j = 0; j < kTcN; ++j) {
-          const int pr = s_pairs[j];
+        for (int j = 0; j < kCols; ++j) {
+          const int pr = s_pairs[kCols * chalf + j];
           if (pr >= 0) {
             float v = acc[j];
             if (up) v *= a.route_w[pr];

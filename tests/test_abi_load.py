@@ -47,6 +47,7 @@ def test_host_side_argument_checks_need_no_gpu():
     assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 63, 256, 0, None, 0, None) == -1
     assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 1, None, 0, None) == -2
     assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 8, None, 0, None) == -8
+    assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 2, None, 0, None) == -8
     assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 0, None, 0, None) == -7
     assert L.stq1_gemv_workspace(16, 300, 1) == 0
     assert L.stq1_moe_workspace(16, 8, 256, 4096, 7168, 0) > 0
