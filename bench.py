@@ -23,6 +23,7 @@ workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -247,15 +248,7 @@ def run_gpu(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(packed, x_bits, seconds=args.cpu_seconds)
 
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof):
-        try:
-            with open(prof) as f:
-                traffic = json.load(f).get("lut_gemv_kernel_bytes_per_launch")
-        except Exception:
-            traffic = None
-
+    traffic = kernel_traffic("lut_gemv_kernel<1>")
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -502,6 +495,31 @@ def run_reference(args):
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def kernel_source_digest():
+    """SHA-256 over the table kernel's sources: a DRAM-traffic figure recorded
+    for an older version of the kernel no longer applies."""
+    h = hashlib.sha256()
+    for rel in ("sub_bit_sparse_b200/csrc/gemv_lut.cuh", "sub_bit_sparse_b200/csrc/device_common.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def kernel_traffic(kernel):
+    """DRAM bytes (read + write) per launch of `kernel` from the ncu summary in
+    profiles/traffic.json, or None when it was taken on other sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(kernel)
+    if not ent or ent.get("source_sha256") != kernel_source_digest():
+        return None
+    return ent.get("dram_bytes_per_launch")
 
 
 def profile_case(args):

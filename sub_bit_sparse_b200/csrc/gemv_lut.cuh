@@ -11,12 +11,18 @@
 // Work unit = (token tile, 128-row slab, K split).  One lane owns one weight row,
 // so all 32 lanes of a warp read the same group's table at the same time and
 // the 32 distinct codes hit 32 distinct banks.  Weight rows are streamed in
-// chunks of two blocks (512 columns, 84 bytes per row) by 1-D bulk copies into
-// a two-stage shared-memory ring; one copy per row fetches the 16-byte-aligned
-// superset of the row's 84 bytes.  Rows are assigned to lanes so that the
-// copied span starts at the same offset (mod 16) for every lane of a warp,
-// which lets each warp decode with compile-time byte offsets and
-// conflict-free 16-byte shared loads.
+// chunks of two blocks (512 columns, 84 bytes per row) into a shared-memory
+// ring by 2-D tensor copies (TMA).  A row's 84 bytes rarely start on the
+// 16-byte boundary a tensor copy needs, and a row's stride (K / 256 * 42
+// bytes) is rarely a multiple of 16, so the packed buffer is viewed as
+// "super-rows" of P consecutive rows, P = 16 / gcd(rowbytes, 16) in {1, 2, 4},
+// whose stride P * rowbytes is.  Rows of the same residue r = row mod P start
+// their chunk at the same offset mod 16; one copy per residue fetches a
+// 112-byte window (the chunk plus lead-in, rounded to 16) of every super-row
+// of the slab.  Each warp holds rows of one residue, so it decodes with
+// compile-time byte offsets and conflict-free 16-byte shared loads (the
+// 112-byte pitch is an odd multiple of 16).  The last rows of the buffer, when
+// they do not fill a super-row, come through a second, 1-D tensor map.
 //
 // Split K: with few rows the K range is divided into S contiguous pieces.  The
 // S units of a (tile, slab) normally form one thread-block cluster: each keeps
@@ -29,42 +35,47 @@
 
 #include <utility>
 
+#include <cudaTypedefs.h>
+
 #include "device_common.cuh"
 
 namespace stq1 {
 
-constexpr int kLutRows = 128;                 // rows per unit = threads per CTA
-constexpr int kLutThreads = 128;
+constexpr int kLutRows = 128;                 // rows per unit
+constexpr int kLutThreads = 256;              // two threads per row: one per block of a chunk
 constexpr int kLutKC = 2;                     // blocks per chunk
+constexpr int kLutChunkBytes = kLutKC * kBlockBytes;         // 84 bytes of a row per chunk
 constexpr int kLutChunkGroups = kGroupsPerBlock * kLutKC;    // 128
 constexpr int kLutGroupBytes = 144;           // 32 fp32 entries + 16-byte pad
 constexpr int kLutTokenBytes = kLutChunkGroups * kLutGroupBytes;   // 18432 = 72 * 256
-constexpr int kLutSlotBytes = 112;            // 84-byte span + alignment slack, 7 x 16 B
-constexpr int kLutStageBytes = kLutRows * kLutSlotBytes;     // 14336
+constexpr int kLutSlotBytes = 112;            // tensor-copy box width: 84-byte span + lead-in, 7 x 16 B
+constexpr int kLutTailSlots = 3;              // rows of a partial last super-row (P - 1 at most)
+constexpr int kLutTailSlotBytes = 128;
 constexpr int kLutMaxTT = 4;                  // tokens per tile
 
 struct LutArgs {
-  const uint8_t* W;          // matrix, or expert 0 of a contiguous expert array
-  const uint8_t* W_end;      // one past the last byte of the packed buffer
-  long long expert_bytes;    // bytes per expert matrix (N * rowbytes)
-  long long rowbytes;        // K / 256 * 42
   const uint16_t* x;         // [T, K] bf16 bits
   float* y;                  // [rows_out, N]
-  float* partial;            // [S, rows_out, N] (S > 1)
-  int* counters;             // [n_tiles, n_slabs] (S > 1), zero between calls
+  float* partial;            // [S, rows_out, N] (S > 1, no cluster)
+  int* counters;             // [n_units] (S > 1, no cluster), zero between calls
   const int* tile_info;      // MoE: [n_tiles_max, 4] = expert, pair offset, count, pad
   const int* n_tiles_dev;    // MoE: number of valid tiles
   const int* pairs;          // MoE: pair ids grouped by expert
   const float* route_w;      // [rows_out] routing weight per pair (flag WEIGHT_UP)
-  int N, K, nb;
+  long long rowbytes;        // K / 256 * 42
+  long long tail_row0;       // first buffer row fetched through the tail map
+  long long rows_total;      // rows in the packed buffer (N, or E * N)
+  int main_srows;            // super-rows in the main map (tail_row0 / P)
+  int N, K;
   int topk;                  // pairs per token (1 for a plain GEMV)
   int batch;                 // plain GEMV: tokens
   int rows_out;              // rows of y
-  int n_tiles;               // tiles in the grid
   int n_slabs;
-  int S;
-  int n_chunks;
-  int P;                     // rows per residue class of (row * rowbytes) mod 16
+  int S, cq, cr;             // K splits; split s has cq chunks, plus one if s < cr
+  int logP;                  // rows per super-row = 1 << logP
+  int box_h;                 // super-rows per box: 128 / P, plus one when N % P != 0
+  int buf_bytes;             // shared bytes per residue buffer (box_h * 112, 128-aligned)
+  int stage_bytes;           // P * buf_bytes + tail slots
   int flags;
   int cluster;               // 1: the S splits of a (tile, slab) form one thread-block cluster
 };
@@ -174,18 +185,19 @@ __device__ __forceinline__ void lut_block_body(const BlockCodes& bc, uint32_t lu
 
 // Activations of this thread's group for chunk `chunk`, TT tokens (8 bytes each).
 template <int TT>
-__device__ __forceinline__ void lut_load_x(const LutArgs& a, int chunk, const int* xrow, uint2 (&xv)[kLutMaxTT]) {
-  const int col = chunk * (kLutKC * kBlockWeights) + 4 * static_cast<int>(threadIdx.x);
+__device__ __forceinline__ void lut_load_x(const uint16_t* const (&xr)[kLutMaxTT], int chunk, uint2 (&xv)[kLutMaxTT]) {
+  const int col = chunk * (kLutKC * kBlockWeights) + 4 * static_cast<int>(threadIdx.x & (kLutChunkGroups - 1));
 #pragma unroll
-  for (int t = 0; t < TT; ++t)
-    xv[t] = __ldg(reinterpret_cast<const uint2*>(a.x + static_cast<long long>(xrow[t]) * a.K + col));
+  for (int t = 0; t < TT; ++t) xv[t] = __ldg(reinterpret_cast<const uint2*>(xr[t] + col));
 }
 
-// Tables for one chunk: thread g builds the 32 entries of group g for each token.
+// Tables for one chunk: threads g and g + 128 build the 32 entries of group g
+// for each token (zero lane 0, 1 and zero lane 2, 3 respectively).
 // Entry c (code) = (-1)^t * (x_a + (-1)^beta x_b + (-1)^gamma x_c).
 template <int TT>
 __device__ __forceinline__ void lut_build(const uint2 (&xv)[kLutMaxTT], uint32_t lut) {
-  const int g = threadIdx.x;                       // 0 .. 127 = kLutChunkGroups - 1
+  const int g = threadIdx.x & (kLutChunkGroups - 1);
+  const bool hi = threadIdx.x >= kLutChunkGroups;   // uniform over a warp
 #pragma unroll
   for (int t = 0; t < TT; ++t) {
     const float x0 = bf16_bits_to_f32(xv[t].x & 0xFFFFu), x1 = bf16_bits_to_f32(xv[t].x >> 16);
@@ -198,125 +210,197 @@ __device__ __forceinline__ void lut_build(const uint2 (&xv)[kLutMaxTT], uint32_t
       sts_v4f(gb + 16u * z, e0, e1, e2, e3);
       sts_v4f(gb + 64u + 16u * z, -e0, -e1, -e2, -e3);
     };
-    put(0, x1, x2, x3);
-    put(1, x0, x2, x3);
-    put(2, x0, x1, x3);
-    put(3, x0, x1, x2);
+    if (!hi) {
+      put(0, x1, x2, x3);
+      put(1, x0, x2, x3);
+    } else {
+      put(2, x0, x1, x3);
+      put(3, x0, x1, x2);
+    }
   }
 }
 
-// One work unit with TT tokens.
+__device__ __forceinline__ void tma_load_w2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_w1d(uint32_t dst, const CUtensorMap* map, int x, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.1d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2}], [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(bar)
+      : "memory");
+}
+
+// One work unit with TT tokens.  R0 = first packed-buffer row of the slab
+// (expert * N + slab * 128); xr / orow = activation row pointers and output
+// rows of the tile's tokens.  Threads q and q + 128 own the same row; the
+// first decodes the chunk's first block, the second its second block.
 template <int TT>
-__device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int split, int tile_id,
-                         const int* xrow, const int* orow, uint8_t* smem) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rg = warp;                                           // 32-row group
-  const int P = a.P;
-  const int rho = P * lane + (rg % P) + 32 * P * (rg / P);       // row within the slab
-  const long long row = static_cast<long long>(slab) * kLutRows + rho;
+__device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wmap, const CUtensorMap* tmap, long long R0,
+                         int slab, int split, int unit, const uint16_t* const (&xr)[kLutMaxTT],
+                         const int (&orow)[kLutMaxTT], uint8_t* smem) {
+  const int c0 = split * a.cq + min(split, a.cr);
+  const int c1 = c0 + a.cq + (split < a.cr ? 1 : 0);
+  const int half = threadIdx.x >> 7;               // block of the chunk this thread decodes
+  const int q = threadIdx.x & (kLutRows - 1);
+
+  // ---- this thread's row and window (slots in residue-major order) ----
+  const int shift = 7 - a.logP;                    // log2(rows of one residue per slab)
+  const int res = q >> shift;                      // residue, uniform over a warp
+  const int kk = q & ((1 << shift) - 1);
+  const int R0mod = static_cast<int>(R0 & ((1 << a.logP) - 1));
+  const int br = res < R0mod ? 1 : 0;              // residues below R0's start one super-row later
+  const long long sr0 = R0 >> a.logP;
+  const long long R = ((sr0 + br + kk) << a.logP) + res;
+  const int rho = static_cast<int>(R - R0);        // row within the slab, 0..127
+  const int row = slab * kLutRows + rho;           // output row
   const bool row_ok = row < a.N;
-  const int c0 = static_cast<int>(static_cast<long long>(split) * a.n_chunks / a.S);
-  const int c1 = static_cast<int>(static_cast<long long>(split + 1) * a.n_chunks / a.S);
+  const uint32_t my_slot = R >= a.tail_row0
+      ? static_cast<uint32_t>((1 << a.logP) * a.buf_bytes) +
+            static_cast<uint32_t>(R - a.tail_row0) * kLutTailSlotBytes
+      : static_cast<uint32_t>(res * a.buf_bytes + (br + kk) * kLutSlotBytes);
 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t lut = (sbase + 255u) & ~255u;
-  const uint32_t bar0 = lut + TT * kLutTokenBytes;   // 2 mbarriers, then the stages
-  const uint32_t stage0 = bar0 + 16;
-  const uint32_t my_slot_off = static_cast<uint32_t>(rg * 32 + lane) * kLutSlotBytes;
+  const uint32_t bar0 = lut + TT * kLutTokenBytes;   // 2 mbarriers
+  const uint32_t stage0 = bar0 + 128;                // 128-aligned tensor-copy destinations
+  const int NS = (c1 - c0 >= 2) ? 2 : 1;
+  // split-K partials pushed by the cluster, at the same offset in every CTA of it
+  const uint32_t red = stage0 + ((a.cq + (a.cr > 0 ? 1 : 0)) >= 2 ? 2 : 1) * a.stage_bytes;
+  const bool push = a.cluster && a.S > 1;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar0, kLutThreads);
-    mbar_init(bar0 + 8, kLutThreads);
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
     fence_mbar_init();
   }
+  // Peers may write this CTA's shared memory only once it runs: announce it
+  // now, and wait for every peer's announcement before the first push.
+  if (push) cluster_arrive_relaxed();
   __syncthreads();
 
-  // Bulk copy of this lane's row span for chunk c into stage st.
+  // Tensor copies of chunk c into stage st (thread 0 only): one box per residue
+  // over the slab's super-rows, plus the slab's rows of a partial last super-row.
   auto issue = [&](int c, int st) {
     const uint32_t bar = bar0 + 8u * st;
-    if (!row_ok) {
-      mbar_arrive(bar);
-      return;
+    const uint32_t dst = stage0 + st * a.stage_bytes;
+    const int P = 1 << a.logP;
+    const int xc = c * kLutChunkBytes;
+    const bool main = sr0 < a.main_srows;
+    int ntail = 0;
+    const long long t0 = a.tail_row0 > R0 ? a.tail_row0 : R0;
+    const long long t1 = a.rows_total < R0 + kLutRows ? a.rows_total : R0 + kLutRows;
+    if (t1 > t0) ntail = static_cast<int>(t1 - t0);
+    mbar_arrive_expect_tx(bar, (main ? P * a.box_h * kLutSlotBytes : 0) + ntail * kLutSlotBytes);
+    if (main)
+      for (int r = 0; r < P; ++r)
+        tma_load_w2d(dst + r * a.buf_bytes, wmap, (static_cast<int>(r * a.rowbytes) + xc) & ~15,
+                     static_cast<int>(sr0), bar);
+    for (int i = 0; i < ntail; ++i) {
+      const int t = static_cast<int>(t0 - a.tail_row0) + i;
+      tma_load_w1d(dst + P * a.buf_bytes + t * kLutTailSlotBytes, tmap,
+                   (static_cast<int>(t * a.rowbytes) + xc) & ~15, bar);
     }
-    const uint8_t* A = Wm + row * a.rowbytes + static_cast<long long>(c) * (kLutKC * kBlockBytes);
-    const uintptr_t lo = reinterpret_cast<uintptr_t>(A) & ~static_cast<uintptr_t>(15);
-    uintptr_t hi = (reinterpret_cast<uintptr_t>(A) + kLutKC * kBlockBytes + 15) & ~static_cast<uintptr_t>(15);
-    const uintptr_t end = reinterpret_cast<uintptr_t>(a.W_end);
-    const uint32_t dst = stage0 + st * kLutStageBytes + my_slot_off;
-    if (hi > end) {
-      // the last row of an unaligned buffer: bulk-copy the aligned part, plain-copy the tail
-      const uintptr_t end16 = end & ~static_cast<uintptr_t>(15);
-      for (uintptr_t q = end16; q < end; ++q) {
-        const uint8_t v = *reinterpret_cast<const uint8_t*>(q);
-        asm volatile("st.shared.u8 [%0], %1;" ::"r"(dst + static_cast<uint32_t>(q - lo)), "r"(static_cast<uint32_t>(v)) : "memory");
-      }
-      hi = end16;
-    }
-    const uint32_t bytes = static_cast<uint32_t>(hi - lo);
-    mbar_arrive_expect_tx(bar, bytes);
-    if (bytes) bulk_g2s(dst, reinterpret_cast<const void*>(lo), bytes, bar);
   };
 
   float acc[kLutMaxTT];
 #pragma unroll
   for (int t = 0; t < kLutMaxTT; ++t) acc[t] = 0.f;
 
-  // offset of the warp's spans inside their 16-byte slots (same for every lane)
-  const long long row0 = static_cast<long long>(slab) * kLutRows + (rg % P) + 32 * P * (rg / P);
-  const uintptr_t wbase = reinterpret_cast<uintptr_t>(Wm) + static_cast<uintptr_t>(row0 * a.rowbytes);
-
   // Weights do not depend on the previous kernel in the stream: start their
   // copies before waiting for it (programmatic dependent launch), unless the
-  // unit itself came from a routing kernel.
-  if (a.tile_info == nullptr) {
-    if (c0 < c1) issue(c0, 0);
-    if (c0 + 1 < c1) issue(c0 + 1, 1);
+  // unit itself came from a routing kernel (which already waited).
+  if (threadIdx.x == 0) {
+    issue(c0, 0);
+    if (NS == 2) issue(c0 + 1, 1);
   }
-  griddep_wait();
-  if (a.tile_info != nullptr) {
-    if (c0 < c1) issue(c0, 0);
-    if (c0 + 1 < c1) issue(c0 + 1, 1);
-  }
+  if (a.tile_info == nullptr) griddep_wait();
   griddep_launch_dependents();
   uint2 xv[kLutMaxTT];
-  if (c0 < c1) lut_load_x<TT>(a, c0, xrow, xv);
+  lut_load_x<TT>(xr, c0, xv);
+  // offset (mod 16) of the thread's block inside its window, before the chunk term
+  const int obase = (static_cast<int>(res * a.rowbytes) & 15) + half * kBlockBytes;
+  const uint32_t lut_half = lut + static_cast<uint32_t>(half * kGroupsPerBlock * kLutGroupBytes);
   bool failed = false;
   for (int c = c0; c < c1; ++c) {
     const int it = c - c0;
-    const int st = it & 1;
+    const int st = NS == 2 ? (it & 1) : 0;
+    const uint32_t parity = static_cast<uint32_t>(NS == 2 ? (it >> 1) : it) & 1u;
     lut_build<TT>(xv, lut);
-    if (c + 1 < c1) lut_load_x<TT>(a, c + 1, xrow, xv);   // prefetch the next chunk's activations
-    const bool landed = mbar_wait_bounded(bar0 + 8u * st, (it >> 1) & 1);
+    if (c + 1 < c1) lut_load_x<TT>(xr, c + 1, xv);   // prefetch the next chunk's activations
+    const bool landed = mbar_wait_bounded(bar0 + 8u * st, parity);
     // one barrier: tables built, copies landed (agreed by every thread)
     if (!__syncthreads_and(landed)) {
       // A copy did not complete within the bound (the error word is set).
-      // Wait (bounded) for the copy already issued into the other stage, so no
-      // bulk copy is still writing this CTA's shared memory when it exits.
-      if (c + 1 < c1) mbar_wait_bounded(bar0 + 8u * (st ^ 1), ((it + 1) >> 1) & 1);
+      // Wait (bounded) for the copies already issued into the other stage, so
+      // no tensor copy is still writing this CTA's shared memory when it exits.
+      if (NS == 2 && c + 1 < c1) mbar_wait_bounded(bar0 + 8u * (st ^ 1), static_cast<uint32_t>((it + 1) >> 1) & 1u);
       failed = true;
       break;
     }
     if (row_ok) {
-      const uint32_t slot = stage0 + st * kLutStageBytes + my_slot_off;
-      const int o = static_cast<int>((wbase + static_cast<uintptr_t>(c) * (kLutKC * kBlockBytes)) & 15);
-      // only the extraction depends on the warp's offset; one copy of the body follows
-      BlockCodes b0, b1;
-      switch (o) {
-        case 0: load_block_codes<0>(slot, b0); load_block_codes<0 + kBlockBytes>(slot, b1); break;
-        case 4: load_block_codes<4>(slot, b0); load_block_codes<4 + kBlockBytes>(slot, b1); break;
-        case 8: load_block_codes<8>(slot, b0); load_block_codes<8 + kBlockBytes>(slot, b1); break;
-        default: load_block_codes<12>(slot, b0); load_block_codes<12 + kBlockBytes>(slot, b1); break;
+      const uint32_t slot = stage0 + st * a.stage_bytes + my_slot;
+      // only the extraction depends on the block's offset; one copy of the body follows
+      BlockCodes b;
+      switch ((obase + c * kLutChunkBytes) & 15 | (half << 4)) {
+        case 0: load_block_codes<0>(slot, b); break;
+        case 4: load_block_codes<4>(slot, b); break;
+        case 8: load_block_codes<8>(slot, b); break;
+        case 12: load_block_codes<12>(slot, b); break;
+        case 16 | 10: load_block_codes<0 + kBlockBytes>(slot, b); break;    // 42 = 2 (mod 16)
+        case 16 | 14: load_block_codes<4 + kBlockBytes>(slot, b); break;
+        case 16 | 2: load_block_codes<8 + kBlockBytes>(slot, b); break;
+        default: load_block_codes<12 + kBlockBytes>(slot, b); break;         // 16 | 6
       }
-      // the second block's tables start 64 groups into the chunk's (256-aligned)
-      lut_block_body<TT>(b0, lut, acc);
-      lut_block_body<TT>(b1, lut + static_cast<uint32_t>(kGroupsPerBlock * kLutGroupBytes), acc);
+      lut_block_body<TT>(b, lut_half, acc);
     }
     __syncthreads();
-    if (c + 2 < c1) issue(c + 2, st);                      // this stage is free again
+    if (threadIdx.x == 0 && c + NS < c1) issue(c + NS, st);   // this stage is free again
+  }
+
+  if (push) {
+    // Push both halves' partials into the shared memory of the CTA that owns
+    // the row (cluster rank (row * S) / 128, the rank equal to its split),
+    // then one cluster barrier; every CTA reaches it, failed or not.
+    cluster_wait();
+    const int owner = (rho * a.S) >> 7;
+    // the owner's rows are ceil(128 r / S) .. ceil(128 (r + 1) / S) - 1
+    const int local = rho - (owner * kLutRows + a.S - 1) / a.S;
+    const int per = (kLutRows + a.S - 1) / a.S;      // rows per owner, at most
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+      st_peer_f32(red + 4u * (((t * 2 * a.S) + 2 * split + half) * per + local), owner, acc[t]);
+    cluster_sync_all();
+    if (half == 0 && owner == split && row_ok) {
+      const bool up = (a.flags & STQ1_MOE_WEIGHT_UP) && row >= a.N / 2;
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        float v = 0.f;
+        for (int i = 0; i < 2 * a.S; ++i) v += lds_f32_addr(red + 4u * ((t * 2 * a.S + i) * per + local));
+        if (up) v *= a.route_w[orow[t]];
+        a.y[static_cast<long long>(orow[t]) * a.N + row] = v;
+      }
+    }
+    return;
+  }
+
+  // Add the second half into the first through shared memory (the tables are
+  // free after the loop's last barrier).
+  if (half == 1) {
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(lut + 4u * (t * kLutRows + rho)), "f"(acc[t]) : "memory");
+  }
+  __syncthreads();
+  if (half == 0) {
+#pragma unroll
+    for (int t = 0; t < TT; ++t) acc[t] += lds_f32_addr(lut + 4u * (t * kLutRows + rho));
   }
   const bool up = (a.flags & STQ1_MOE_WEIGHT_UP) && row >= a.N / 2;
   if (a.S == 1) {
-    if (row_ok && !failed) {
+    if (half == 0 && row_ok && !failed) {
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
         float v = acc[t];
@@ -326,36 +410,12 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
     }
     return;
   }
-
-  if (a.cluster) {
-    // Every CTA of the cluster reaches both cluster barriers, failed or not.
-    const uint32_t red = lut;                          // tables are no longer needed
-#pragma unroll
-    for (int t = 0; t < TT; ++t)
-      asm volatile("st.shared.f32 [%0], %1;" ::"r"(red + 4u * (t * kLutRows + rho)), "f"(acc[t]) : "memory");
-    cluster_sync_all();
-    const int rank = static_cast<int>(cluster_ctarank());
-    const int lo = rank * kLutRows / a.S, hi = (rank + 1) * kLutRows / a.S;
-    const int nr = hi - lo;
-    for (int idx = threadIdx.x; idx < nr * TT; idx += kLutThreads) {
-      const int t = idx / nr, rr = lo + idx % nr;
-      float v = 0.f;
-      for (int sp = 0; sp < a.S; ++sp) v += ld_peer_f32(red + 4u * (t * kLutRows + rr), sp);
-      const long long rrow = static_cast<long long>(slab) * kLutRows + rr;
-      if (rrow < a.N) {
-        if ((a.flags & STQ1_MOE_WEIGHT_UP) && rrow >= a.N / 2) v *= a.route_w[orow[t]];
-        a.y[static_cast<long long>(orow[t]) * a.N + rrow] = v;
-      }
-    }
-    cluster_sync_all();                                // peers may still read this CTA's partials
-    return;
-  }
   if (failed) return;
 
   // Scratch mode: publish partials, the last unit of this (tile, slab) reduces.
   // One thread fences after the barrier: the barrier orders the other threads'
   // stores before it, and the gpu-scope fence is cumulative.
-  if (row_ok) {
+  if (half == 0 && row_ok) {
 #pragma unroll
     for (int t = 0; t < TT; ++t)
       a.partial[(static_cast<long long>(split) * a.rows_out + orow[t]) * a.N + row] = acc[t];
@@ -364,13 +424,13 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
-    const int old = atomicAdd(&a.counters[tile_id * a.n_slabs + slab], 1);
+    const int old = atomicAdd(&a.counters[unit], 1);
     s_last = (old == a.S - 1);
     if (s_last) __threadfence();
   }
   __syncthreads();
   if (!s_last) return;
-  if (row_ok) {
+  if (half == 0 && row_ok) {
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
       float v = 0.f;
@@ -380,61 +440,84 @@ __device__ void lut_unit(const LutArgs& a, const uint8_t* Wm, int slab, int spli
       a.y[static_cast<long long>(orow[t]) * a.N + row] = v;
     }
   }
-  if (threadIdx.x == 0) a.counters[tile_id * a.n_slabs + slab] = 0;
+  if (threadIdx.x == 0) a.counters[unit] = 0;
 }
 
+// CTAs per SM the register budget must allow (the host's work split assumes it).
+constexpr int lut_min_blocks(int ttmax) { return ttmax == 1 ? 4 : (ttmax == 2 ? 3 : 2); }
+
+// Grid: x = unit = tile * n_slabs + slab, y = K split; clusters of (1, S, 1).
 template <int TTMAX>
-__global__ void __launch_bounds__(kLutThreads) lut_gemv_kernel(const LutArgs a) {
+__global__ void __launch_bounds__(kLutThreads, lut_min_blocks(TTMAX))
+lut_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap tmap, const LutArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
-  __shared__ int s_xrow[kLutMaxTT], s_orow[kLutMaxTT], s_cnt, s_expert;
-  const int u = blockIdx.x;
-  const int split = u % a.S;
-  const int rest = u / a.S;
-  const int slab = rest % a.n_slabs;
-  const int tile = rest / a.n_slabs;
+  const int unit = blockIdx.x;
+  const int split = blockIdx.y;
+  const int tile = unit / a.n_slabs;
+  const int slab = unit - tile * a.n_slabs;
+  const uint16_t* xr[kLutMaxTT];
+  int orow[kLutMaxTT];
+  int cnt, expert = 0;
   if (a.tile_info) {
     griddep_wait();                                  // the tile table comes from the routing kernel
-    if (tile >= *a.n_tiles_dev) return;
-    if (threadIdx.x == 0) {
-      const int e = a.tile_info[4 * tile + 0];
-      const int off = a.tile_info[4 * tile + 1];
-      const int cnt = a.tile_info[4 * tile + 2];
-      s_expert = e;
-      s_cnt = cnt;
-      for (int t = 0; t < kLutMaxTT; ++t) {
-        const int p = a.pairs[off + (t < cnt ? t : 0)];
-        s_orow[t] = p;
-        s_xrow[t] = p / a.topk;
-      }
+    if (tile >= *a.n_tiles_dev) return;              // whole clusters leave together (same tile)
+    expert = a.tile_info[4 * tile + 0];
+    const int off = a.tile_info[4 * tile + 1];
+    cnt = a.tile_info[4 * tile + 2];
+#pragma unroll
+    for (int t = 0; t < kLutMaxTT; ++t) {
+      const int p = a.pairs[off + (t < cnt ? t : 0)];
+      orow[t] = p;
+      xr[t] = a.x + static_cast<long long>(p / a.topk) * a.K;
     }
   } else {
-    if (threadIdx.x == 0) {
-      const int t0 = tile * kLutMaxTT;
-      const int cnt = min(kLutMaxTT, a.batch - t0);
-      s_expert = 0;
-      s_cnt = cnt;
-      for (int t = 0; t < kLutMaxTT; ++t) {
-        s_orow[t] = t0 + (t < cnt ? t : 0);
-        s_xrow[t] = s_orow[t];
-      }
+    const int t0 = tile * kLutMaxTT;
+    cnt = min(kLutMaxTT, a.batch - t0);
+#pragma unroll
+    for (int t = 0; t < kLutMaxTT; ++t) {
+      orow[t] = t0 + (t < cnt ? t : 0);
+      xr[t] = a.x + static_cast<long long>(orow[t]) * a.K;
     }
   }
-  __syncthreads();
-  const uint8_t* Wm = a.W + static_cast<long long>(s_expert) * a.expert_bytes;
-  const int cnt = s_cnt;
-  if (TTMAX >= 4 && cnt >= 4) {
-    lut_unit<(TTMAX >= 4 ? 4 : 1)>(a, Wm, slab, split, tile, s_xrow, s_orow, smem);
-  } else if (TTMAX >= 3 && cnt == 3) {
-    lut_unit<(TTMAX >= 3 ? 3 : 1)>(a, Wm, slab, split, tile, s_xrow, s_orow, smem);
-  } else if (TTMAX >= 2 && cnt == 2) {
-    lut_unit<(TTMAX >= 2 ? 2 : 1)>(a, Wm, slab, split, tile, s_xrow, s_orow, smem);
-  } else {
-    lut_unit<1>(a, Wm, slab, split, tile, s_xrow, s_orow, smem);
+  const long long R0 = static_cast<long long>(expert) * a.N + static_cast<long long>(slab) * kLutRows;
+  if constexpr (TTMAX >= 4) {
+    if (cnt >= 4) {
+      lut_unit<4>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, smem);
+      return;
+    }
   }
+  if constexpr (TTMAX >= 3) {
+    if (cnt == 3) {
+      lut_unit<3>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, smem);
+      return;
+    }
+  }
+  if constexpr (TTMAX >= 2) {
+    if (cnt == 2) {
+      lut_unit<2>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, smem);
+      return;
+    }
+  }
+  lut_unit<1>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, smem);
 }
 
-inline size_t lut_smem_bytes(int ttmax, int stages = 2) {
-  return 256 + static_cast<size_t>(ttmax) * kLutTokenBytes + 16 + static_cast<size_t>(stages) * kLutStageBytes;
+// Shared bytes of one stage for super-rows of 2^logP rows and boxes of box_h super-rows.
+inline int lut_buf_bytes(int box_h) { return (box_h * kLutSlotBytes + 127) & ~127; }
+inline int lut_stage_bytes(int logP, int box_h) {
+  return (1 << logP) * lut_buf_bytes(box_h) + kLutTailSlots * kLutTailSlotBytes;
+}
+
+// Dynamic shared memory: tables, barriers, stages and (cluster split K) the
+// partials pushed by the S CTAs of the cluster into the CTA that owns a row:
+// two per split, token and owned row (ceil(128 / S) rows).
+inline size_t lut_smem_bytes(int ttmax, int stages, int stage_bytes, int cluster_S) {
+  const size_t per = cluster_S > 1 ? static_cast<size_t>((kLutRows + cluster_S - 1) / cluster_S) : 0;
+  return 256 + static_cast<size_t>(ttmax) * kLutTokenBytes + 128 + static_cast<size_t>(stages) * stage_bytes +
+         static_cast<size_t>(ttmax) * 2 * cluster_S * per * 4;
+}
+// Upper bound over every geometry (P = 4 with the extra super-row is the largest stage).
+inline size_t lut_smem_bytes_max(int ttmax) {
+  return lut_smem_bytes(ttmax, 2, lut_stage_bytes(2, 33), kMaxClusterRanks);
 }
 
 }  // namespace stq1

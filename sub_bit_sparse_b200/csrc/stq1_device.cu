@@ -31,7 +31,6 @@ int g_path = 0;
 constexpr int kTcMinBatch = 16;       // stq1_gemv: batches from here use the tile kernel
 constexpr int kTcMinPairsPerExpert = 16;
 constexpr int kMoeTableTokens = 2;    // MoE decode tiles: pairs per table-kernel unit
-constexpr int kMaxClusterSplit = 16;  // largest (non-portable) cluster used for split K
 
 int sm_count() {
   static int cache[kMaxDevices] = {};
@@ -85,11 +84,11 @@ int ensure_configured() {
   if (dev < 0) return STQ1_ERR_CUDA;
   if (done[dev]) return STQ1_OK;
   if (cudaFuncSetAttribute(lut_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(lut_smem_bytes(1))) != cudaSuccess ||
+                           static_cast<int>(lut_smem_bytes_max(1))) != cudaSuccess ||
       cudaFuncSetAttribute(lut_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(lut_smem_bytes(2))) != cudaSuccess ||
+                           static_cast<int>(lut_smem_bytes_max(2))) != cudaSuccess ||
       cudaFuncSetAttribute(lut_gemv_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(lut_smem_bytes(4))) != cudaSuccess ||
+                           static_cast<int>(lut_smem_bytes_max(4))) != cudaSuccess ||
       cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            3 * kMaxExperts * 4) != cudaSuccess ||
       cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -111,12 +110,12 @@ int launch_status() {
 
 // Launch with programmatic stream serialization: the kernel may start while the
 // previous kernel in the stream drains; it calls griddepcontrol.wait before
-// touching anything that kernel may write.
+// touching anything that kernel may write.  cluster_y > 1 groups CTAs along y.
 template <typename... Params, typename... Args>
-int launch_pdl_cluster(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
-                       unsigned cluster, Args&&... args) {
+int launch_pdl_cluster(void (*kernel)(Params...), dim3 grid, unsigned block, size_t smem, cudaStream_t s,
+                       unsigned cluster_y, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = grid;
   cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -124,10 +123,10 @@ int launch_pdl_cluster(void (*kernel)(Params...), unsigned grid, unsigned block,
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   int n = 1;
-  if (cluster > 1) {
+  if (cluster_y > 1) {
     attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = cluster;
-    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = cluster_y;
     attr[1].val.clusterDim.z = 1;
     n = 2;
   }
@@ -141,7 +140,7 @@ int launch_pdl_cluster(void (*kernel)(Params...), unsigned grid, unsigned block,
 template <typename... Params, typename... Args>
 int launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
                Args&&... args) {
-  return launch_pdl_cluster(kernel, grid, block, smem, s, 1u, std::forward<Args>(args)...);
+  return launch_pdl_cluster(kernel, dim3(grid), block, smem, s, 1u, std::forward<Args>(args)...);
 }
 
 int residue_period(long long rowbytes) {
@@ -150,8 +149,72 @@ int residue_period(long long rowbytes) {
   return static_cast<int>(16 / g);
 }
 
+// Tensor maps of the table kernel over a packed buffer of rows_total rows:
+// the main map views it as super-rows of P = 2^logP rows (stride P * rowbytes,
+// a multiple of 16) and copies boxes of 112 bytes x box_h super-rows; the tail
+// map (1-D) covers the last rows_total mod P rows.  extra_srow: slabs may start
+// inside a super-row (MoE experts with N % P != 0), so boxes take one more.
+struct LutMaps {
+  CUtensorMap w, t;
+};
+
+int make_lut_maps(LutMaps* m, LutArgs* a, const uint8_t* W, long long rows_total, long long rowbytes,
+                  bool extra_srow) {
+  auto fn = encode_fn();
+  if (!fn) return STQ1_ERR_CUDA;
+  const int P = residue_period(rowbytes);
+  const int logP = P == 1 ? 0 : (P == 2 ? 1 : 2);
+  const long long srow_bytes = P * rowbytes;
+  const long long main_srows = rows_total >> logP;
+  if (main_srows >= (1LL << 31) || srow_bytes + kLutSlotBytes >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  a->rowbytes = rowbytes;
+  a->rows_total = rows_total;
+  a->tail_row0 = main_srows << logP;
+  a->main_srows = static_cast<int>(main_srows);
+  a->logP = logP;
+  a->box_h = (kLutRows >> logP) + (extra_srow ? 1 : 0);
+  a->buf_bytes = lut_buf_bytes(a->box_h);
+  a->stage_bytes = lut_stage_bytes(logP, a->box_h);
+  cuuint32_t es[2] = {1, 1};
+  {
+    // a map that is never read (no full super-row) still has to be valid
+    const bool any = main_srows > 0;
+    cuuint64_t gdim[2] = {static_cast<cuuint64_t>(any ? srow_bytes : 16),
+                          static_cast<cuuint64_t>(any ? main_srows : 1)};
+    cuuint64_t gstride[1] = {static_cast<cuuint64_t>(any ? srow_bytes : 16)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(any ? kLutSlotBytes : 16),
+                         static_cast<cuuint32_t>(any ? a->box_h : 1)};
+    if (fn(&m->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(W), gdim, gstride, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return STQ1_ERR_CUDA;
+  }
+  {
+    const long long nt = rows_total - a->tail_row0;
+    const uint8_t* base = nt > 0 ? W + a->tail_row0 * rowbytes : W;
+    cuuint64_t gdim[1] = {static_cast<cuuint64_t>(nt > 0 ? nt * rowbytes : 16)};
+    cuuint64_t gstride[1] = {0};
+    cuuint32_t box[1] = {static_cast<cuuint32_t>(nt > 0 ? kLutSlotBytes : 16)};
+    if (fn(&m->t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, const_cast<uint8_t*>(base), gdim, gstride, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return STQ1_ERR_CUDA;
+  }
+  return STQ1_OK;
+}
+
+// K split of n_chunks chunks into S pieces (split s: cq chunks, one more if s < cr).
+void set_split(LutArgs* a, int n_chunks, int S) {
+  a->S = S;
+  a->cq = n_chunks / S;
+  a->cr = n_chunks % S;
+}
+
+// Shared-memory stages: two when some split holds at least two chunks.
+int lut_stages(const LutArgs& a) { return a.cq + (a.cr > 0 ? 1 : 0) >= 2 ? 2 : 1; }
+
 struct GemvPlan {
-  int n_tiles, n_slabs, S, n_chunks;
+  int n_tiles, n_slabs, S, n_chunks, tt;
   size_t partial_bytes, counter_bytes;
   bool table_path, tile_path;
 };
@@ -163,19 +226,56 @@ bool want_tiles(long long nb, long long units) {
   return units >= kTcMinBatch;
 }
 
+int smem_per_sm() {
+  static int cache[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return 228 * 1024;
+  if (!cache[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    cache[dev] = v > 0 ? v : 228 * 1024;
+  }
+  return cache[dev];
+}
+
+// Work split of the table kernel: (token tile, 128-row slab) units, each cut
+// into S pieces of K so that there are about kTargetUnits CTAs and, with
+// one_wave, no more than fit on the device at once.
+void plan_table(GemvPlan* p, long long N, long long K, int batch, bool one_wave) {
+  const long long nb = K / kBlockWeights;
+  p->tt = batch == 1 ? 1 : (batch == 2 ? 2 : 4);
+  p->n_tiles = (batch + kLutMaxTT - 1) / kLutMaxTT;
+  p->n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
+  p->n_chunks = static_cast<int>(nb / kLutKC);
+  const long long units0 = static_cast<long long>(p->n_tiles) * p->n_slabs;
+  long long S = (kTargetUnits + units0 - 1) / units0;
+  S = std::max<long long>(1, std::min<long long>(S, std::max(1, p->n_chunks)));
+  const int P = residue_period(nb * kBlockBytes);
+  const int logP = P == 1 ? 0 : (P == 2 ? 1 : 2);
+  const int stage = lut_stage_bytes(logP, kLutRows >> logP);
+  const long long slots_sm = smem_per_sm();
+  for (; one_wave && S > 1; --S) {
+    const int cq = static_cast<int>(p->n_chunks / S), cr = static_cast<int>(p->n_chunks % S);
+    const int stages = cq + (cr > 0 ? 1 : 0) >= 2 ? 2 : 1;
+    const long long smem = static_cast<long long>(lut_smem_bytes(p->tt, stages, stage, static_cast<int>(S))) + 1024;
+    const long long per_sm = std::min<long long>(lut_min_blocks(p->tt), slots_sm / smem);
+    if (units0 * S <= per_sm * sm_count()) break;
+  }
+  // the fewest splits that keep the longest split as short: n_chunks = 14 and
+  // at most 13 splits gives 7 splits of 2 chunks, not 13 with one of 2
+  const long long longest = (p->n_chunks + S - 1) / S;
+  if (longest > 0) S = (p->n_chunks + longest - 1) / longest;
+  p->S = static_cast<int>(std::max<long long>(1, S));
+}
+
 GemvPlan plan_gemv(long long N, long long K, int batch) {
   GemvPlan p{};
   const long long nb = K / kBlockWeights;
   p.tile_path = want_tiles(nb, batch);
   if (p.tile_path) return p;
   p.table_path = (nb % 2 == 0);
-  p.n_tiles = (batch + kLutMaxTT - 1) / kLutMaxTT;
-  p.n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
-  p.n_chunks = static_cast<int>(nb / kLutKC);
-  const long long units0 = static_cast<long long>(p.n_tiles) * p.n_slabs;
-  long long S = (kTargetUnits + units0 - 1) / units0;
-  S = std::max<long long>(1, std::min<long long>(S, std::max(1, p.n_chunks)));
-  p.S = p.table_path ? static_cast<int>(S) : 1;
+  plan_table(&p, N, K, batch, true);
+  if (!p.table_path) p.S = 1;
   if (p.table_path && p.S > 1) {
     p.partial_bytes = static_cast<size_t>(p.S) * batch * N * sizeof(float);
     p.counter_bytes = kCounterBytes;
@@ -258,43 +358,37 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
     return launch_status();
   }
   LutArgs a{};
-  a.W = static_cast<const uint8_t*>(W_packed);
-  a.W_end = a.W + N * rowbytes;
-  a.expert_bytes = 0;
-  a.rowbytes = rowbytes;
+  LutMaps maps;
+  rc = make_lut_maps(&maps, &a, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
+  if (rc != STQ1_OK) return rc;
   a.x = x;
   a.y = y;
   a.counters = p.S > 1 ? static_cast<int*>(workspace) : nullptr;
   a.partial = p.S > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes) : nullptr;
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
-  a.nb = static_cast<int>(nb);
   a.topk = 1;
   a.batch = batch;
   a.rows_out = batch;
-  a.n_tiles = p.n_tiles;
   a.n_slabs = p.n_slabs;
-  a.S = p.S;
-  a.n_chunks = p.n_chunks;
-  a.P = residue_period(rowbytes);
+  set_split(&a, p.n_chunks, p.S);
   a.flags = 0;
-  const long long grid = static_cast<long long>(p.n_tiles) * p.n_slabs * p.S;
-  // one shared stage is enough when every unit holds a single chunk
-  const int stages = (p.n_chunks + p.S - 1) / p.S >= 2 ? 2 : 1;
-  const int tt = batch == 1 ? 1 : (batch == 2 ? 2 : 4);
+  const long long units = static_cast<long long>(p.n_tiles) * p.n_slabs;
+  if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  const dim3 grid(static_cast<unsigned>(units), static_cast<unsigned>(p.S));
   auto go = [&](int cluster) {
     a.cluster = cluster > 1 ? 1 : 0;
-    const size_t smem = lut_smem_bytes(tt, stages);
-    if (tt == 1)
-      return launch_pdl_cluster(lut_gemv_kernel<1>, static_cast<unsigned>(grid), kLutThreads, smem, s, cluster, a);
-    if (tt == 2)
-      return launch_pdl_cluster(lut_gemv_kernel<2>, static_cast<unsigned>(grid), kLutThreads, smem, s, cluster, a);
-    return launch_pdl_cluster(lut_gemv_kernel<4>, static_cast<unsigned>(grid), kLutThreads, smem, s, cluster, a);
+    const size_t smem = lut_smem_bytes(p.tt, lut_stages(a), a.stage_bytes, cluster);
+    if (p.tt == 1)
+      return launch_pdl_cluster(lut_gemv_kernel<1>, grid, kLutThreads, smem, s, cluster, maps.w, maps.t, a);
+    if (p.tt == 2)
+      return launch_pdl_cluster(lut_gemv_kernel<2>, grid, kLutThreads, smem, s, cluster, maps.w, maps.t, a);
+    return launch_pdl_cluster(lut_gemv_kernel<4>, grid, kLutThreads, smem, s, cluster, maps.w, maps.t, a);
   };
   // split K reduces through distributed shared memory inside a cluster of the
   // S units of a slab; if the device refuses such a cluster, through the
   // caller's scratch buffer
-  if (p.S > 1 && p.S <= kMaxClusterSplit && go(p.S) == STQ1_OK) return STQ1_OK;
+  if (p.S > 1 && p.S <= kMaxClusterRanks && go(p.S) == STQ1_OK) return STQ1_OK;
   return go(1);
 }
 
@@ -403,10 +497,11 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
     return launch_pdl(tc_gemm_kernel, grid, kTcThreads, kTcSmemBytes, s, map, t);
   }
   LutArgs a{};
-  a.W = static_cast<const uint8_t*>(expert_blocks);
-  a.W_end = a.W + static_cast<long long>(E) * N * rowbytes;
-  a.expert_bytes = N * rowbytes;
-  a.rowbytes = rowbytes;
+  LutMaps maps;
+  const int P = residue_period(rowbytes);
+  rc = make_lut_maps(&maps, &a, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
+                     rowbytes, N % P != 0);
+  if (rc != STQ1_OK) return rc;
   a.x = x;
   a.y = y;
   a.partial = nullptr;
@@ -417,19 +512,18 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   a.route_w = topk_weights;
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
-  a.nb = static_cast<int>(nb);
   a.topk = topk;
   a.batch = 0;
   a.rows_out = n_pairs;
-  a.n_tiles = m.max_tiles;
   a.n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
-  a.S = 1;
-  a.n_chunks = static_cast<int>(nb / kLutKC);
-  a.P = residue_period(rowbytes);
+  set_split(&a, static_cast<int>(nb / kLutKC), 1);
   a.flags = flags;
-  const long long grid = static_cast<long long>(m.max_tiles) * a.n_slabs;
-  return launch_pdl(lut_gemv_kernel<kMoeTableTokens>, static_cast<unsigned>(grid), kLutThreads,
-                    lut_smem_bytes(kMoeTableTokens), s, a);
+  a.cluster = 0;
+  const long long units = static_cast<long long>(m.max_tiles) * a.n_slabs;
+  if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  return launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(units)), kLutThreads,
+                            lut_smem_bytes(kMoeTableTokens, lut_stages(a), a.stage_bytes, 1), s, 1u, maps.w, maps.t,
+                            a);
 }
 
 extern "C" int stq1_set_path(int path) {
@@ -510,13 +604,12 @@ extern "C" int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float*
         static_cast<int>(N), static_cast<int>(K), batch);
     return launch_status();
   }
-  // Same work split as the table path of stq1_gemv.
-  const int n_tiles = (batch + kLutMaxTT - 1) / kLutMaxTT;
-  const int n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
-  const int n_chunks = static_cast<int>(nb / kLutKC);
+  // The table path's work split, without its one-wave cap on the K split (a
+  // plain launch reduces through the scratch buffer, whatever the split).
+  GemvPlan p{};
+  plan_table(&p, N, K, batch, false);
+  const int n_tiles = p.n_tiles, n_slabs = p.n_slabs, n_chunks = p.n_chunks, S = p.S;
   const long long units0 = static_cast<long long>(n_tiles) * n_slabs;
-  const int S = static_cast<int>(std::max<long long>(
-      1, std::min<long long>((kTargetUnits + units0 - 1) / units0, std::max(1, n_chunks))));
   const size_t need = S > 1 ? kCounterBytes + static_cast<size_t>(S) * batch * N * sizeof(float) : 0;
   if (need > kStaticScratchBytes) return STQ1_ERR_SCRATCH;
   uint8_t* scratch = nullptr;
@@ -527,32 +620,30 @@ extern "C" int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float*
     if (cudaMemsetAsync(scratch, 0, kCounterBytes, s) != cudaSuccess) return STQ1_ERR_CUDA;
   }
   LutArgs a{};
-  a.W = static_cast<const uint8_t*>(W_packed);
-  a.W_end = a.W + N * rowbytes;
-  a.expert_bytes = 0;
-  a.rowbytes = rowbytes;
+  LutMaps maps;
+  rc = make_lut_maps(&maps, &a, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
+  if (rc != STQ1_OK) return rc;
   a.x = x;
   a.y = y;
   a.counters = S > 1 ? reinterpret_cast<int*>(scratch) : nullptr;
   a.partial = S > 1 ? reinterpret_cast<float*>(scratch + kCounterBytes) : nullptr;
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
-  a.nb = static_cast<int>(nb);
   a.topk = 1;
   a.batch = batch;
   a.rows_out = batch;
-  a.n_tiles = n_tiles;
   a.n_slabs = n_slabs;
-  a.S = S;
-  a.n_chunks = n_chunks;
-  a.P = residue_period(rowbytes);
+  set_split(&a, n_chunks, S);
   a.flags = 0;
-  const unsigned grid = static_cast<unsigned>(static_cast<long long>(n_tiles) * n_slabs * S);
+  a.cluster = 0;
+  if (units0 >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  const dim3 grid(static_cast<unsigned>(units0), static_cast<unsigned>(S));
+  const size_t smem = lut_smem_bytes(batch == 1 ? 1 : (batch == 2 ? 2 : 4), lut_stages(a), a.stage_bytes, 1);
   if (batch == 1)
-    lut_gemv_kernel<1><<<grid, kLutThreads, lut_smem_bytes(1), s>>>(a);
+    lut_gemv_kernel<1><<<grid, kLutThreads, smem, s>>>(maps.w, maps.t, a);
   else if (batch == 2)
-    lut_gemv_kernel<2><<<grid, kLutThreads, lut_smem_bytes(2), s>>>(a);
+    lut_gemv_kernel<2><<<grid, kLutThreads, smem, s>>>(maps.w, maps.t, a);
   else
-    lut_gemv_kernel<4><<<grid, kLutThreads, lut_smem_bytes(4), s>>>(a);
+    lut_gemv_kernel<4><<<grid, kLutThreads, smem, s>>>(maps.w, maps.t, a);
   return launch_status();
 }

@@ -176,6 +176,19 @@ def test_moe_skewed_and_duplicate_ids():
     _moe_check(experts, x, ids, wts, n, k, E, flags=1)
 
 
+@pytest.mark.parametrize("n,k,E", [(130, 512, 5), (6, 1536, 3), (258, 1024, 3)])
+def test_moe_expert_rows_straddle_super_rows(n, k, E):
+    # With 84 * m bytes per row (m odd: P = 4 rows per 16-byte-aligned super-row;
+    # m = 2 mod 4: P = 2) and N not a multiple of P, experts start inside a
+    # super-row and the buffer ends in a partial one.
+    T, topk = 7, 2
+    experts = [stq1.quantize_ref(workloads.gaussian_matrix(n, k, 0.02, seed=500 + e)) for e in range(E)]
+    x = workloads.activations_bf16(T, k, seed=21)
+    ids = workloads.zipf_topk_ids(T, E, topk, seed=22)
+    wts = workloads.softmax_route_weights(T, topk, seed=23)
+    _moe_check(experts, x, ids, wts, n, k, E, flags=1)
+
+
 def test_moe_decode_workload_full():
     # 256 experts x [4096, 7168] (1.23 GB packed), 16 tokens, Zipf(1.1) top-8.
     # Expert bytes are random valid blocks: every 5-bit code is legal, and the
