@@ -60,6 +60,14 @@ design notes):
 6. Matmul: y[t, j] = sum_k W^[j, k] x[t, k] with W^ = pattern * fp32(d).
    MoE gate/up: y[t, s, :] = W^_{ids[t, s]} x_t, unweighted unless flag bit 0
    asks to scale the up half (rows N/2..N-1) by the routing weight.
+7. fp8 variant of the tile path (the pages have no fp8 step; the reading is
+   this library's): each token row x_t is scaled by one fp32 factor to the
+   e4m3 range, inv_t = 448 / amax_t and s_t = amax_t / 448 (both fp32
+   divisions; 0 for an all-zero row), each element becomes the e4m3 code of
+   the fp32 product x * inv_t, rounded to nearest with ties to the even code
+   and saturated at +/-448 (OCP FP8 E4M3: no infinities, 0x7F / 0xFF NaN),
+   and y = s_t * W^ q_t with q_t the codes' values.  Weights stay exact
+   (+/-1 and 0 are e4m3 values, d is applied in fp32).
 """
 
 from __future__ import annotations
@@ -418,10 +426,15 @@ def moe_gateup(expert_packed, x_bits: np.ndarray, ids: np.ndarray, weights: np.n
     Flag bit 0 scales the up half (rows n/2 .. n-1) by weights[t, s].
     With ``abs_sum=True`` also returns sum_k |W^ x| for the tolerance.
     """
+    x = bf16_to_f64(np.asarray(x_bits).reshape(np.asarray(ids).shape[0], k))
+    return _moe_from_f64(expert_packed, x, ids, weights, n, k, flags, abs_sum)
+
+
+def _moe_from_f64(expert_packed, x: np.ndarray, ids, weights, n: int, k: int, flags: int, abs_sum: bool):
+    """MoE gate/up on fp64 activations x [T, k]."""
     ids = np.asarray(ids)
     T, topk = ids.shape
     get = expert_packed if callable(expert_packed) else (lambda e: expert_packed[e])
-    x = bf16_to_f64(np.asarray(x_bits).reshape(T, k))
     y = np.zeros((T, topk, n))
     ya = np.zeros((T, topk, n)) if abs_sum else None
     for e in np.unique(ids):
@@ -436,6 +449,66 @@ def moe_gateup(expert_packed, x_bits: np.ndarray, ids: np.ndarray, weights: np.n
         if abs_sum:
             ya[:, :, n // 2:] *= np.abs(wt)
     return (y, ya) if abs_sum else y
+
+
+# ---------------------------------------------------------------------------
+# fp8 (e4m3) activations for the fp8 tile variant (reading 7)
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """OCP FP8 E4M3 code -> fp64: sign bit 7, exponent bits 3-6 (bias 7), mantissa bits 0-2;
+    exponent 0 is subnormal (m / 8 * 2^-6); codes 0x7F and 0xFF are NaN."""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & ((c & 0x7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_round(v) -> np.ndarray:
+    """fp32 values -> E4M3 codes: nearest value, ties to the even code, magnitudes above 448
+    saturate to 448; the sign bit follows the input's (so -0.0 -> 0x80).  Finite inputs."""
+    v = np.asarray(v, dtype=np.float32).astype(np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(a)                       # a = f * 2^ex with f in [0.5, 1), or a = 0
+    e = np.maximum(ex - 1, -6)                # a in [2^e, 2^(e+1)); below 2^-6 one subnormal step
+    step = np.exp2(e - 3.0)                   # 8 values per binade
+    r = np.rint(a / step)                     # ties to the even multiple = the even mantissa
+    q = np.minimum(r * step, E4M3_MAX)
+    # q is an E4M3 magnitude: encode it
+    _, qx = np.frexp(q)
+    qe = qx - 1                               # q in [2^qe, 2^(qe+1)) for q > 0
+    normal = q >= 2.0 ** -6
+    exp_field = np.where(normal, qe + 7, 0)
+    man = np.where(normal, q / np.exp2(qe.astype(np.float64)) * 8.0 - 8.0, q / 2.0 ** -9)
+    code = (exp_field.astype(np.int64) << 3) | np.rint(man).astype(np.int64)
+    code = np.where(q == 0, 0, code)
+    return (code | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8)
+
+
+def quantize_x_e4m3(x_bits: np.ndarray):
+    """bf16 rows [T, K] -> (E4M3 codes uint8 [T, K], scales fp32 [T]) per reading 7."""
+    x = bf16_to_f64(np.asarray(x_bits)).astype(np.float32)
+    x = x.reshape(x.shape[0], -1)
+    amax = np.max(np.abs(x), axis=1)
+    with np.errstate(divide="ignore"):
+        inv = np.where(amax > 0, np.float32(E4M3_MAX) / amax, np.float32(0.0)).astype(np.float32)
+    s = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    v = (x * inv[:, None]).astype(np.float32)
+    return e4m3_round(v), s
+
+
+def moe_gateup_fp8(expert_packed, x_bits: np.ndarray, ids: np.ndarray, weights: np.ndarray,
+                   n: int, k: int, flags: int = 0, abs_sum: bool = False):
+    """The fp8 variant of ``moe_gateup``: x_t replaced by s_t * q_t (reading 7), fp64."""
+    codes, s = quantize_x_e4m3(np.asarray(x_bits).reshape(-1, k))
+    xq = e4m3_value(codes) * s.astype(np.float64)[:, None]
+    return _moe_from_f64(expert_packed, xq, ids, weights, n, k, flags, abs_sum)
 
 
 def half_from_struct(x: float) -> int:

@@ -391,6 +391,114 @@ def test_route_pairs_is_a_grouping():
 
 
 # ---------------------------------------------------------------------------
+# fp8 activations (E4M3) for the fp8 tile variant
+# ---------------------------------------------------------------------------
+
+
+def test_e4m3_code_table_landmarks():
+    # OCP FP8 E4M3 (no infinities): fixed points of the published format
+    v = oracle.e4m3_value(np.arange(256))
+    assert v[0x00] == 0.0 and v[0x01] == 2.0 ** -9 and v[0x07] == 7 * 2.0 ** -9
+    assert v[0x08] == 2.0 ** -6 and v[0x38] == 1.0 and v[0x39] == 1.125 and v[0x7E] == 448.0
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF])
+    assert np.all(np.diff(v[0x00:0x7F]) > 0)                 # 127 ordered non-negative values
+    assert np.array_equal(v[0x80:0xFF], -v[0x00:0x7F])       # sign bit mirrors
+
+
+def _e4m3_brute_force(vals):
+    # nearest of the 127 non-negative finite values, ties to the even code,
+    # saturating; the sign bit follows the input
+    grid = oracle.e4m3_value(np.arange(0x7F))
+    out = []
+    for x in np.asarray(vals, np.float32).astype(np.float64):
+        a = min(abs(x), 448.0)
+        dist = np.abs(grid - a)
+        best = np.flatnonzero(dist == dist.min())
+        code = int(best[0]) if len(best) == 1 else int([c for c in best if c % 2 == 0][0])
+        out.append(code | (0x80 if np.signbit(x) else 0))
+    return np.array(out, np.uint8)
+
+
+def test_e4m3_round_is_nearest_with_ties_to_even():
+    rng = np.random.default_rng(88)
+    grid = oracle.e4m3_value(np.arange(0x7F))
+    mids = (grid[:-1] + grid[1:]) / 2                        # exact ties (fp32-representable)
+    vals = np.concatenate([
+        rng.standard_normal(3000) * 30, rng.uniform(-2.0 ** -6, 2.0 ** -6, 1000),
+        rng.uniform(-500, 500, 1000), mids, -mids, grid, [0.0, -0.0, 448.0, 464.0, 465.0, -1e6, 1e-30]])
+    vals = vals.astype(np.float32)
+    assert np.array_equal(oracle.e4m3_round(vals), _e4m3_brute_force(vals))
+
+
+def test_e4m3_round_matches_torch_cast():
+    torch = pytest.importorskip("torch")
+    if not hasattr(torch, "float8_e4m3fn"):
+        pytest.skip("torch without float8")
+    rng = np.random.default_rng(89)
+    vals = np.concatenate([rng.standard_normal(20000) * 40, rng.uniform(-0.02, 0.02, 5000)]).astype(np.float32)
+    vals = np.clip(vals, -448, 448)
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_round(vals), ref)
+
+
+def test_quantize_x_e4m3_scales_each_row_to_the_range():
+    x = workloads.activations_bf16(6, 512, seed=90)
+    x[3] = 0                                                  # an all-zero row
+    x[4, ::7] = 0x8000                                        # some -0.0
+    codes, s = oracle.quantize_x_e4m3(x)
+    xf = oracle.bf16_to_f64(x)
+    for t in range(6):
+        amax = np.max(np.abs(xf[t]))
+        if amax == 0:
+            assert s[t] == 0 and np.all((codes[t] & 0x7F) == 0)
+            continue
+        assert np.max(codes[t] & 0x7F) == 0x7E                 # the largest element lands on 448
+        assert s[t] == np.float32(np.float32(amax) / np.float32(448))
+        back = oracle.e4m3_value(codes[t]) * np.float64(s[t])
+        # E4M3 has 3 mantissa bits: relative error <= 2^-4 above the subnormal range
+        big = np.abs(xf[t]) > amax * 2.0 ** -6
+        assert np.all(np.abs(back[big] - xf[t][big]) <= 2.0 ** -4 * np.abs(xf[t][big]) * 1.001)
+
+
+def test_moe_fp8_is_exact_when_x_is_representable():
+    # rows whose values are E4M3 values and whose amax is 448 quantize to themselves
+    n, k, E, T, topk = 64, 512, 3, 4, 2
+    experts = [oracle.encode_plain(workloads.gaussian_matrix(n, k, 0.02, seed=400 + e)) for e in range(E)]
+    rng = np.random.default_rng(91)
+    vals = oracle.e4m3_value(rng.integers(0, 0x7F, (T, k)) | (rng.integers(0, 2, (T, k)) << 7))
+    vals[:, 0] = 448.0
+    x = oracle.bf16_bits_rne(vals.astype(np.float32))
+    assert np.array_equal(oracle.bf16_to_f64(x), vals)
+    ids = workloads.zipf_topk_ids(T, E, topk, seed=92)
+    y8 = oracle.moe_gateup_fp8(experts, x, ids, None, n, k)
+    y = oracle.moe_gateup(experts, x, ids, None, n, k)
+    assert np.array_equal(y8, y)
+
+
+@pytest.mark.parametrize("mistake", ["ties_away", "no_saturation", "subnormal_step"])
+def test_planted_fp8_mistakes_are_caught(monkeypatch, mistake):
+    import oracle.stq1 as o
+    grid = oracle.e4m3_value(np.arange(0x7F))
+    vals = np.concatenate([grid, (grid[:-1] + grid[1:]) / 2,
+                           [470.0, 500.0, 3 * 2.0 ** -10, 5 * 2.0 ** -11]]).astype(np.float32)
+    assert np.array_equal(o.e4m3_round(vals), _e4m3_brute_force(vals))
+    orig_rint, orig_min, orig_max = np.rint, np.minimum, np.maximum
+    if mistake == "ties_away":
+        monkeypatch.setattr(o.np, "rint", lambda a: np.floor(np.asarray(a) + 0.5))
+    elif mistake == "no_saturation":
+        monkeypatch.setattr(o, "E4M3_MAX", 480.0)
+    elif mistake == "subnormal_step":
+        # the step of the lowest normal binade extended one binade too far up
+        monkeypatch.setattr(o.np, "maximum", lambda a, b: orig_max(a, b + 1) if np.isscalar(b) and b == -6 else orig_max(a, b))
+    try:
+        got = o.e4m3_round(vals)
+    finally:
+        monkeypatch.undo()
+    assert not np.array_equal(got, _e4m3_brute_force(vals))
+    assert orig_rint is np.rint and orig_min is np.minimum
+
+
+# ---------------------------------------------------------------------------
 # The pins catch planted mistakes
 # ---------------------------------------------------------------------------
 
