@@ -41,6 +41,7 @@ METRIC = ("STQ1_0 GEMV packed-weight GB/s & % HBM roofline; MoE gate/up tokens/s
 N_ROWS, K_COLS = 4096, 7168
 PACKED = N_ROWS * (K_COLS // 256) * 42          # 4,816,896 bytes per matrix
 STACK = 64                                      # matrices per step
+FP8_OVER_BF16 = 2.0                        # nominal dense fp8 / bf16 tensor rate on B200
 HBM_NOMINAL_GBS = 8000.0
 
 
@@ -321,30 +322,50 @@ def _random_expert_bank(torch, device, E, seed):
 
 
 def run_prefill(torch, stq1, device, stream, args, world, timed, bf16_peak):
-    """MoE prefill gate/up: 4096 tokens x top-8 of 256 experts (32,768 pairs)."""
+    """MoE prefill gate/up: 4096 tokens x top-8 of 256 experts (32,768 pairs), on
+    the bf16 tile path and on its fp8 variant.  The fp8 error is measured
+    against the bf16 result (itself within 1e-3 * sum|W x| of the exact one)."""
     import workloads
     E, n, k = 256, N_ROWS, K_COLS
     flat = _random_expert_bank(torch, device, E, 4096)
     x, ids, _ = workloads.moe_prefill_inputs()
     xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
     idd = torch.from_numpy(ids).to(device)
-    y = torch.empty((4096, 8, n), dtype=torch.float32, device=device)
-    ws = stq1.workspace(stq1.LIB.stq1_moe_workspace(4096, 8, E, n, k, 0), device, kind="moe")
-
-    def step():
-        stq1.moe_gateup(flat, xd, idd, None, n, k, E, out=y, ws=ws)
-
-    steps = max(2, args.steps // 40)
-    gp = time_graph(torch, step, steps, 3, stream)
-    ms = timed(gp, steps) / steps
-    del gp
     flops = 2.0 * 4096 * 8 * n * k
-    tflops = flops / (ms * 1e-3) / 1e12
-    return {"tokens_per_s": round(world * 4096 / (ms * 1e-3), 1), "ms_per_call": round(ms, 4),
-            "tflops_dense_equiv": round(tflops, 1), "bf16_peak_tflops": bf16_peak,
-            "tensor_frac": round(tflops / bf16_peak, 4),
-            "config": "256 experts x [4096, 7168] STQ1_0, 4096 tokens, Zipf(1.1) top-8 (32,768 pairs), "
-                      "tcgen05 kind::f16 tiles, A = decoded +/-1 bf16 in TMEM, fp32 per-slab scale"}
+    out = {}
+    ys = {}
+    for name, flags, peak in (("bf16", 0, bf16_peak), ("fp8", stq1.MOE_FP8, bf16_peak * FP8_OVER_BF16)):
+        y = torch.empty((4096, 8, n), dtype=torch.float32, device=device)
+        ws = stq1.workspace(stq1.LIB.stq1_moe_workspace(4096, 8, E, n, k, flags), device, kind="moe")
+
+        def step():
+            stq1.moe_gateup(flat, xd, idd, None, n, k, E, flags=flags, out=y, ws=ws)
+
+        steps = max(2, args.steps // 40)
+        gp = time_graph(torch, step, steps, 3, stream)
+        ms = timed(gp, steps) / steps
+        del gp
+        tflops = flops / (ms * 1e-3) / 1e12
+        out[name] = {"tokens_per_s": round(world * 4096 / (ms * 1e-3), 1), "ms_per_call": round(ms, 4),
+                     "tflops_dense_equiv": round(tflops, 1), "peak_tflops": round(peak, 1),
+                     "tensor_frac": round(tflops / peak, 4)}
+        ys[name] = y
+        del ws
+    d = (ys["fp8"] - ys["bf16"]).abs_()
+    ref = ys["bf16"].abs()
+    scale = float(ref.mean())
+    out["fp8"]["error_vs_bf16"] = {
+        "mean_abs_over_mean_abs_y": round(float(d.mean()) / scale, 6),
+        "max_abs_over_mean_abs_y": round(float(d.max()) / scale, 6),
+        "rel_l2": round(float(torch.linalg.vector_norm(d) / torch.linalg.vector_norm(ys["bf16"])), 6)}
+    del ys, d, ref
+    res = out["bf16"]
+    res["bf16_peak_tflops"] = bf16_peak
+    res["fp8"] = out["fp8"]
+    res["config"] = ("256 experts x [4096, 7168] STQ1_0, 4096 tokens, Zipf(1.1) top-8 (32,768 pairs), "
+                     "tcgen05 tiles, A = decoded +/-1 in TMEM (bf16, kind::f16; fp8: E4M3, kind::f8f6f4 with "
+                     "per-token E4M3 activations), fp32 per-block scale; fp8 peak = measured bf16 x 2 (nominal ratio)")
+    return res
 
 
 def run_sweep(args):

@@ -68,7 +68,7 @@ extern "C" {
 
 /* stq1_moe_gateup flags. */
 #define STQ1_MOE_WEIGHT_UP 1      /* multiply rows N/2..N-1 (the up half) by the routing weight */
-#define STQ1_MOE_FP8 2            /* reserved for an e4m3 tile variant; currently STQ1_ERR_ARG */
+#define STQ1_MOE_FP8 2            /* tile path: E4M3 activations (per-token fp32 scale), fp8 MMAs */
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 int stq1_version(void);
@@ -164,14 +164,42 @@ size_t stq1_moe_workspace(int T, int topk, int E, int64_t N, int64_t K, int flag
  *   y              device, [T, topk, N] fp32 (fully overwritten; a slot whose
  *                  id is out of range is set to 0 and flagged in the error word).
  *   flags          STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8.
- *   ws, ws_bytes   device workspace, at least stq1_moe_workspace(...) bytes.
+ *   ws, ws_bytes   device workspace, at least stq1_moe_workspace(...) bytes
+ *                  (computed with the same flags).
  * Requires N even, K % 256 == 0, 1 <= topk <= E.
+ * Paths: with few token-slot pairs per routed expert (decode) the lookup-table
+ * kernel runs; with many (prefill) the tensor-core tile kernel.
+ * STQ1_MOE_FP8 applies to the tile kernel only: each token row of x is
+ * quantized to E4M3 as by stq1_quantize_x_e4m3, the +/-1 weight patterns are
+ * E4M3 too, the MMAs run in fp8 with fp32 accumulation and y is multiplied by
+ * the row's scale.  The weights stay exact; the activations carry E4M3's
+ * relative error (up to 2^-4), so this variant is outside the accuracy bound
+ * below and its error is measured, not bounded.  The table kernel ignores the
+ * flag.
+ * Accuracy (without STQ1_MOE_FP8): as stq1_gemv, per output.
  * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_ALIGN, STQ1_ERR_WORKSPACE,
  * STQ1_ERR_ARG, STQ1_ERR_CUDA.
  */
 int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, const int32_t* topk_ids,
                     const float* topk_weights, float* y, int T, int topk, int E, int64_t N,
                     int64_t K, int flags, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * stq1_quantize_x_e4m3 -- the activation quantization of the fp8 tile variant
+ * (the pages have no fp8 step; this is the library's choice).  Per row t of
+ * x: amax = max |x[t, k]|, inv = 448 / amax and scales[t] = amax / 448 (IEEE
+ * fp32 divisions; both 0 for an all-zero row), q[t, k] = the OCP FP8 E4M3 code
+ * of the fp32 product x[t, k] * inv, rounded to nearest with ties to even and
+ * saturated at +/-448 (the sign of zero is kept).  x[t, k] ~= scales[t] *
+ * value(q[t, k]).
+ *   x       device, [T, K] bf16 bits (finite), 16-byte aligned.
+ *   q       device, [T, K] bytes, 16-byte aligned (fully overwritten).
+ *   scales  device, [T] fp32.
+ * Requires K % 16 == 0.  Asynchronous on `stream`.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_ALIGN, STQ1_ERR_CUDA.
+ */
+int stq1_quantize_x_e4m3(const uint16_t* x, int64_t T, int64_t K, uint8_t* q, float* scales,
+                         void* stream);
 
 /*
  * stq1_gemv_noalloc -- stq1_gemv without a caller workspace and without any

@@ -53,6 +53,8 @@ SIGNATURES = {
     "stq1_set_path": (_c.c_int, [_c.c_int]),
     "stq1_gemv_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int,
                                      _c.c_void_p]),
+    "stq1_quantize_x_e4m3": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p, _c.c_void_p,
+                                        _c.c_void_p]),
 }
 
 
@@ -240,6 +242,22 @@ def moe_gateup(expert_blocks, x, topk_ids, topk_weights, n: int, k: int, n_exper
                              _stream(x))
     _check("stq1_moe_gateup", rc)
     return out
+
+
+def quantize_x_e4m3(x, out=None, scales=None):
+    """bf16 [T, K] -> (E4M3 codes uint8 [T, K], fp32 scales [T]), as the fp8 tile variant does."""
+    torch = _torch()
+    _require(x, torch.bfloat16, "x")
+    t, k = x.shape
+    if out is None:
+        out = torch.empty((t, k), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((t,), dtype=torch.float32, device=x.device)
+    _require(out, torch.uint8, "out")
+    _require(scales, torch.float32, "scales")
+    rc = _load().stq1_quantize_x_e4m3(x.data_ptr(), t, k, out.data_ptr(), scales.data_ptr(), _stream(x))
+    _check("stq1_quantize_x_e4m3", rc)
+    return out, scales
 
 
 PATH_AUTO, PATH_TABLE, PATH_TILES = 0, 1, 2

@@ -57,18 +57,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D map over a row-major bf16 matrix [rows, K]; box = 64 columns x kTcN rows,
-// 128-byte swizzle, out-of-range rows read as zero.
-bool make_b_map(CUtensorMap* map, const void* base, long long rows, long long K) {
+// 2-D map over a row-major activation matrix [rows, K] of bf16 (or, fp8, of
+// E4M3 bytes); box = 128 bytes of columns x kTcN rows, 128-byte swizzle,
+// out-of-range rows read as zero.
+bool make_b_map(CUtensorMap* map, const void* base, long long rows, long long K, bool fp8) {
   auto fn = encode_fn();
   if (!fn) return false;
+  const int esize = fp8 ? 1 : 2;
   cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcKC), static_cast<cuuint32_t>(kTcN)};
+  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * esize};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcStageBytesK / esize), static_cast<cuuint32_t>(kTcN)};
   cuuint32_t estride[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
-            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int current_device() {
@@ -91,7 +94,9 @@ int ensure_configured() {
                            static_cast<int>(lut_smem_bytes_max(4))) != cudaSuccess ||
       cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            3 * kMaxExperts * 4) != cudaSuccess ||
-      cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(tc_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kTcSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kTcSmemBytes) != cudaSuccess)
     return STQ1_ERR_CUDA;
   // split-K clusters of up to 16 CTAs (above the portable 8); a refusal only
@@ -327,7 +332,7 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
   const long long rowbytes = nb * kBlockBytes;
   if (p.tile_path) {
     CUtensorMap map;
-    if (!make_b_map(&map, x, batch, K)) return STQ1_ERR_CUDA;
+    if (!make_b_map(&map, x, batch, K, false)) return STQ1_ERR_CUDA;
     TcArgs t{};
     t.W = static_cast<const uint8_t*>(W_packed);
     t.W_end = t.W + N * rowbytes;
@@ -338,6 +343,7 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
     t.n_tiles_dev = nullptr;
     t.pairs = nullptr;
     t.route_w = nullptr;
+    t.xscale = nullptr;
     t.n_tiles = (batch + kTcN - 1) / kTcN;
     t.N = static_cast<int>(N);
     t.K = static_cast<int>(K);
@@ -348,7 +354,7 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
     t.flags = 0;
     const long long items = static_cast<long long>(t.n_tiles) * t.n_mtiles;
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
-    return launch_pdl(tc_gemm_kernel, grid, kTcThreads, kTcSmemBytes, s, map, t);
+    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, t);
   }
   if (!p.table_path) {
     const long long warps = static_cast<long long>(batch) * N;
@@ -395,11 +401,11 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
 namespace stq1 {
 namespace {
 struct MoePlan {
-  size_t pairs_off, tiles_off, ntiles_off, xperm_off, total;
+  size_t pairs_off, tiles_off, ntiles_off, xperm_off, xq_off, sq_off, sperm_off, total;
   int max_tiles, tile_tokens;
-  bool tiles;
+  bool tiles, fp8;
 };
-MoePlan plan_moe(int T, int topk, int E, long long K) {
+MoePlan plan_moe(int T, int topk, int E, long long K, int flags) {
   MoePlan m{};
   const long long n_pairs = static_cast<long long>(T) * topk;
   const long long nb = K / kBlockWeights;
@@ -414,8 +420,18 @@ MoePlan plan_moe(int T, int topk, int E, long long K) {
   off += round16(static_cast<size_t>(m.max_tiles) * 4 * sizeof(int));
   m.ntiles_off = off;
   off += 16;
+  m.fp8 = m.tiles && (flags & STQ1_MOE_FP8);
   m.xperm_off = off;
-  if (m.tiles) off += round16(static_cast<size_t>(n_pairs) * K * 2);
+  if (m.tiles) off += round16(static_cast<size_t>(n_pairs) * K * (m.fp8 ? 1 : 2));
+  m.xq_off = m.sq_off = m.sperm_off = off;
+  if (m.fp8) {
+    m.xq_off = off;
+    off += round16(static_cast<size_t>(T) * K);
+    m.sq_off = off;
+    off += round16(static_cast<size_t>(T) * sizeof(float));
+    m.sperm_off = off;
+    off += round16(static_cast<size_t>(n_pairs) * sizeof(float));
+  }
   m.total = off;
   return m;
 }
@@ -424,9 +440,8 @@ MoePlan plan_moe(int T, int topk, int E, long long K) {
 
 extern "C" size_t stq1_moe_workspace(int T, int topk, int E, int64_t N, int64_t K, int flags) {
   (void)N;
-  (void)flags;
   if (T <= 0 || topk <= 0 || E <= 0 || K <= 0 || K % kBlockWeights) return 0;
-  return plan_moe(T, topk, E, K).total;
+  return plan_moe(T, topk, E, K, flags).total;
 }
 
 extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, const int32_t* topk_ids,
@@ -435,13 +450,12 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   if (!expert_blocks || !x || !topk_ids || !y) return STQ1_ERR_NULL;
   if ((flags & STQ1_MOE_WEIGHT_UP) && !topk_weights) return STQ1_ERR_NULL;
   if (flags & ~(STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8)) return STQ1_ERR_ARG;
-  if (flags & STQ1_MOE_FP8) return STQ1_ERR_ARG;   // the e4m3 tile variant is not built yet
   if (T <= 0 || topk <= 0 || E <= 0 || topk > E || E > kMaxExperts || N <= 0 || (N & 1) || K <= 0 ||
       K % kBlockWeights || N > (1LL << 30) || K > (1LL << 30) ||
       static_cast<long long>(T) * topk > (1LL << 30))
     return STQ1_ERR_SHAPE;
   if (!aligned16(expert_blocks) || !aligned16(x)) return STQ1_ERR_ALIGN;
-  const MoePlan m = plan_moe(T, topk, E, K);
+  const MoePlan m = plan_moe(T, topk, E, K, flags);
   if (!ws || ws_bytes < m.total) return STQ1_ERR_WORKSPACE;
   if (!aligned16(ws)) return STQ1_ERR_ALIGN;
   int rc = ensure_configured();
@@ -467,13 +481,26 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
                   pairs, tiles, ntiles, y, static_cast<int>(N));
   if (rc != STQ1_OK) return rc;
   if (m.tiles) {
-    uint16_t* xperm = reinterpret_cast<uint16_t*>(wsb + m.xperm_off);
-    rc = launch_pdl(gather_rows_kernel, static_cast<unsigned>(n_pairs), 256, 0, s, x,
-                    static_cast<const int*>(pairs), static_cast<const int*>(ntiles + 1), n_pairs, topk,
-                    static_cast<int>(K), xperm);
+    void* xperm = wsb + m.xperm_off;
+    float* sperm = reinterpret_cast<float*>(wsb + m.sperm_off);
+    if (m.fp8) {
+      uint8_t* xq = wsb + m.xq_off;
+      float* sq = reinterpret_cast<float*>(wsb + m.sq_off);
+      rc = launch_pdl(quant_e4m3_kernel, static_cast<unsigned>(T), kQuantThreads, 0, s, x, static_cast<int>(K), xq,
+                      sq);
+      if (rc != STQ1_OK) return rc;
+      rc = launch_pdl(gather_rows8_kernel, static_cast<unsigned>(n_pairs), 256, 0, s,
+                      static_cast<const uint8_t*>(xq), static_cast<const float*>(sq), static_cast<const int*>(pairs),
+                      static_cast<const int*>(ntiles + 1), n_pairs, topk, static_cast<int>(K),
+                      static_cast<uint8_t*>(xperm), sperm);
+    } else {
+      rc = launch_pdl(gather_rows_kernel, static_cast<unsigned>(n_pairs), 256, 0, s, x,
+                      static_cast<const int*>(pairs), static_cast<const int*>(ntiles + 1), n_pairs, topk,
+                      static_cast<int>(K), static_cast<uint16_t*>(xperm));
+    }
     if (rc != STQ1_OK) return rc;
     CUtensorMap map;
-    if (!make_b_map(&map, xperm, n_pairs, K)) return STQ1_ERR_CUDA;
+    if (!make_b_map(&map, xperm, n_pairs, K, m.fp8)) return STQ1_ERR_CUDA;
     TcArgs t{};
     t.W = static_cast<const uint8_t*>(expert_blocks);
     t.W_end = t.W + static_cast<long long>(E) * N * rowbytes;
@@ -484,6 +511,7 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
     t.n_tiles_dev = ntiles;
     t.pairs = pairs;
     t.route_w = topk_weights;
+    t.xscale = m.fp8 ? sperm : nullptr;
     t.n_tiles = m.max_tiles;
     t.N = static_cast<int>(N);
     t.K = static_cast<int>(K);
@@ -494,7 +522,8 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
     t.flags = flags;
     const long long items = static_cast<long long>(m.max_tiles) * t.n_mtiles;
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
-    return launch_pdl(tc_gemm_kernel, grid, kTcThreads, kTcSmemBytes, s, map, t);
+    if (m.fp8) return launch_pdl(tc_gemm_kernel<true>, grid, kTcThreads, kTcSmemBytes, s, map, t);
+    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, t);
   }
   LutArgs a{};
   LutMaps maps;
@@ -524,6 +553,17 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   return launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(units)), kLutThreads,
                             lut_smem_bytes(kMoeTableTokens, lut_stages(a), a.stage_bytes, 1), s, 1u, maps.w, maps.t,
                             a);
+}
+
+extern "C" int stq1_quantize_x_e4m3(const uint16_t* x, int64_t T, int64_t K, uint8_t* q, float* scales,
+                                    void* stream) {
+  if (!x || !q || !scales) return STQ1_ERR_NULL;
+  if (T <= 0 || K <= 0 || K % 16 || T > (1LL << 31) - 1) return STQ1_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(q)) return STQ1_ERR_ALIGN;
+  int rc = ensure_configured();
+  if (rc != STQ1_OK) return rc;
+  return launch_pdl(quant_e4m3_kernel, static_cast<unsigned>(T), kQuantThreads, 0, static_cast<cudaStream_t>(stream),
+                    x, static_cast<int>(K), q, scales);
 }
 
 extern "C" int stq1_set_path(int path) {

@@ -27,9 +27,17 @@
 // All waits are bounded; a timeout sets the device error word and makes every
 // role stop at its next wait, so the CTA always reaches the final barrier and
 // frees its TMEM.
+//
+// fp8 variant (FP8 = true): x rows arrive as E4M3 codes with one fp32 scale
+// per row, the pattern is expanded to E4M3 +/-1 and 0 (one byte per weight,
+// a 32-bit word per group), the MMA is kind::f8f6f4, and a stage covers 128
+// columns (128 bytes, the same 32 TMEM columns and 16 KB x tile as a bf16
+// stage of 64 columns), so a scale block takes two stages instead of four.
+// The row's scale multiplies the finished sum.
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp8.h>
 
 #include "device_common.cuh"
 
@@ -37,22 +45,28 @@ namespace stq1 {
 
 constexpr int kTcM = 128;
 constexpr int kTcN = 128;
-constexpr int kTcKC = 64;                     // K per stage (128 bytes of bf16)
+constexpr int kTcStageBytesK = 128;           // bytes of x per row and stage
+constexpr int kTcKC = 64;                     // K per stage, bf16 (128 bytes)
+constexpr int kTcKC8 = 128;                   // K per stage, fp8 (128 bytes)
 constexpr int kTcStages = 8;
-constexpr int kTcSlabChunks = kBlockWeights / kTcKC;    // 4 stages per scale block
+template <bool FP8>
+constexpr int tc_kc() { return FP8 ? kTcKC8 : kTcKC; }
+template <bool FP8>
+constexpr int tc_slab_chunks() { return kBlockWeights / tc_kc<FP8>(); }   // 4 (bf16) or 2 (fp8)
 constexpr int kTcThreads = 576;
 constexpr int kTcDecoders = 256;                 // threads: 8 warps
 constexpr int kTcEpilogue = 256;                 // threads: 8 warps
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcColD = 0;               // 2 x 128
 constexpr uint32_t kTcColA = 256;             // kTcStages x 32
-constexpr int kTcBStageBytes = kTcN * kTcKC * 2;   // 16 KB
+constexpr int kTcBStageBytes = kTcN * kTcStageBytesK;   // 16 KB
 // shared layout (offsets from a 1024-aligned base)
 constexpr int kTcOffB = 0;
 constexpr int kTcOffTable = kTcStages * kTcBStageBytes;            // 131072: 2 x 128 B decode tables
 constexpr int kTcOffBar = kTcOffTable + 256;
 constexpr int kTcOffPairs = kTcOffBar + 256;                       // kTcN ints
-constexpr int kTcOffMisc = kTcOffPairs + kTcN * 4;
+constexpr int kTcOffScale = kTcOffPairs + kTcN * 4;                // kTcN floats (fp8)
+constexpr int kTcOffMisc = kTcOffScale + kTcN * 4;
 constexpr int kTcSmemBytes = 1024 + kTcOffMisc + 64;   // > 114 KB: one CTA per SM
 
 struct TcArgs {
@@ -65,6 +79,7 @@ struct TcArgs {
   const int* n_tiles_dev;    // device tile count (MoE) or nullptr
   const int* pairs;          // output row of each B row (MoE) or nullptr (identity)
   const float* route_w;
+  const float* xscale;       // fp8: scale of each B row, nullptr otherwise
   int n_tiles;               // plain: token tiles
   int N, K, nb;
   int n_mtiles;
@@ -97,15 +112,25 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                    bar)
                : "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem desc]
+// D[tmem] (+)= A[tmem] * B[smem desc]: bf16 x bf16 (kind::f16) or E4M3 x E4M3 (kind::f8f6f4)
+template <bool FP8>
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if constexpr (FP8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {
@@ -179,22 +204,36 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
          (static_cast<uint64_t>(2) << 61);
 }
 
-// Instruction descriptor: D f32, A bf16, B bf16, both K-major, M = 128, N = kTcN.
-constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                              (static_cast<uint32_t>(kTcN >> 3) << 17) |
-                              (static_cast<uint32_t>(kTcM >> 4) << 24);
+// Instruction descriptor: D f32 (bits 4-5 = 1), A and B types (bits 7-9,
+// 10-12: bf16 = 1 for kind::f16, E4M3 = 0 for kind::f8f6f4), both K-major,
+// N >> 3 at bit 17, M >> 4 at bit 24.
+template <bool FP8>
+constexpr uint32_t tc_idesc() {
+  return (1u << 4) | (FP8 ? 0u : ((1u << 7) | (1u << 10))) | (static_cast<uint32_t>(kTcN >> 3) << 17) |
+         (static_cast<uint32_t>(kTcM >> 4) << 24);
+}
 
-// bf16 bit patterns of the 32 codes: lanes 0,1 (word 0) and lanes 2,3 (word 1).
+// bf16 bit patterns of the 32 codes: lanes 0,1 (word 0) and lanes 2,3 (word 1);
+// for fp8 one word per code, lane l in byte l (E4M3 +1 = 0x38, -1 = 0xB8).
+template <bool FP8>
 __device__ __forceinline__ void tc_fill_tables(uint32_t* t0, uint32_t* t1) {
   const int c = threadIdx.x;
   if (c < 32) {
     int v[4];
     code_pattern(static_cast<unsigned>(c), v);
-    uint32_t h[4];
+    if constexpr (FP8) {
+      uint32_t w = 0;
 #pragma unroll
-    for (int l = 0; l < 4; ++l) h[l] = v[l] == 0 ? 0u : (v[l] > 0 ? 0x3F80u : 0xBF80u);
-    t0[c] = h[0] | (h[1] << 16);
-    t1[c] = h[2] | (h[3] << 16);
+      for (int l = 0; l < 4; ++l) w |= (v[l] == 0 ? 0u : (v[l] > 0 ? 0x38u : 0xB8u)) << (8 * l);
+      t0[c] = w;
+      t1[c] = 0u;
+    } else {
+      uint32_t h[4];
+#pragma unroll
+      for (int l = 0; l < 4; ++l) h[l] = v[l] == 0 ? 0u : (v[l] > 0 ? 0x3F80u : 0xBF80u);
+      t0[c] = h[0] | (h[1] << 16);
+      t1[c] = h[2] | (h[3] << 16);
+    }
   }
 }
 
@@ -242,34 +281,47 @@ __device__ __forceinline__ void tc_extract(const uint32_t (&w)[16], uint32_t (&Q
   H1 = (ph1 & 3) ? __funnelshift_r(w[ph1 >> 2], w[(ph1 >> 2) + 1], 8 * (ph1 & 3)) : w[ph1 >> 2];
 }
 
-// Expands this thread's half (8 groups = 16 TMEM columns) of each of the
-// block's four 64-column chunks; for each chunk waits for the A stage to be
-// free, stores its columns and signals the MMA thread.
-template <int HALF>
+// Expands this thread's half of each of the block's stages into 16 TMEM
+// columns (bf16: 8 groups x 2 words of each 64-column stage; fp8: 16 groups
+// x 1 word of each 128-column stage); for each stage waits for the A stage
+// to be free, stores its columns and signals the MMA thread.
+template <bool FP8, int HALF>
 __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t H0, uint32_t H1,
                                                uint32_t tables, uint32_t tmem_a_lane, uint32_t bar_full_a,
                                                uint32_t bar_empty, uint32_t& it) {
 #pragma unroll
-  for (int q = 0; q < kTcSlabChunks; ++q) {
+  for (int q = 0; q < tc_slab_chunks<FP8>(); ++q) {
     uint32_t v[16];
-    const int i = 2 * q + HALF;                      // qs word: groups 8i .. 8i+7
-    const uint32_t hb = (i < 4 ? H0 : H1) >> (8 * (i & 3));
-    const uint32_t ce = ((Q[i] << 2) & 0x3C3C3C3Cu) | (((hb & 0x55u) * 0x01041040u) & 0x40404040u);
-    const uint32_t co = ((Q[i] >> 2) & 0x3C3C3C3Cu) | (((hb & 0xAAu) * 0x00820820u) & 0x40404040u);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      // the group's (code * 4) byte spliced into the 256-aligned table base
-      const uint32_t ae = __byte_perm(ce, tables, 0x7650u | m);
-      const uint32_t ao = __byte_perm(co, tables, 0x7650u | m);
-      uint32_t x0, x1, y0, y1;
-      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(x0) : "r"(ae));
-      asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(x1) : "r"(ae));
-      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(y0) : "r"(ao));
-      asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(y1) : "r"(ao));
-      v[4 * m] = x0;
-      v[4 * m + 1] = x1;
-      v[4 * m + 2] = y0;
-      v[4 * m + 3] = y1;
+    for (int w = 0; w < (FP8 ? 2 : 1); ++w) {
+      // qs word i: groups 8i .. 8i+7
+      const int i = FP8 ? 4 * q + 2 * HALF + w : 2 * q + HALF;
+      const uint32_t hb = (i < 4 ? H0 : H1) >> (8 * (i & 3));
+      const uint32_t ce = ((Q[i] << 2) & 0x3C3C3C3Cu) | (((hb & 0x55u) * 0x01041040u) & 0x40404040u);
+      const uint32_t co = ((Q[i] >> 2) & 0x3C3C3C3Cu) | (((hb & 0xAAu) * 0x00820820u) & 0x40404040u);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        // the group's (code * 4) byte spliced into the 256-aligned table base
+        const uint32_t ae = __byte_perm(ce, tables, 0x7650u | m);
+        const uint32_t ao = __byte_perm(co, tables, 0x7650u | m);
+        if constexpr (FP8) {
+          uint32_t x0, y0;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(x0) : "r"(ae));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(y0) : "r"(ao));
+          v[8 * w + 2 * m] = x0;
+          v[8 * w + 2 * m + 1] = y0;
+        } else {
+          uint32_t x0, x1, y0, y1;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(x0) : "r"(ae));
+          asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(x1) : "r"(ae));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(y0) : "r"(ao));
+          asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(y1) : "r"(ao));
+          v[4 * m] = x0;
+          v[4 * m + 1] = x1;
+          v[4 * m + 2] = y0;
+          v[4 * m + 3] = y1;
+        }
+      }
     }
     const uint32_t s = it % kTcStages;
     const uint32_t use = it / kTcStages;
@@ -284,8 +336,11 @@ __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t 
   return true;
 }
 
+template <bool FP8>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
+  constexpr int KC = tc_kc<FP8>();
+  constexpr int kSlabChunks = tc_slab_chunks<FP8>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
@@ -298,6 +353,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
   const uint32_t bar_d_full = bar + 192, bar_d_empty = bar + 208;
   const uint32_t bar_drain = bar + 224;
   int* s_pairs = reinterpret_cast<int*>(sgen + kTcOffPairs);
+  float* s_scale = reinterpret_cast<float*>(sgen + kTcOffScale);
   volatile int* s_misc = reinterpret_cast<volatile int*>(sgen + kTcOffMisc);   // [0] tmem base, [1] abort
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -315,8 +371,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
     s_misc[1] = 0;
     fence_mbar_init();
   }
-  tc_fill_tables(reinterpret_cast<uint32_t*>(sgen + kTcOffTable),
-                 reinterpret_cast<uint32_t*>(sgen + kTcOffTable + 128));
+  tc_fill_tables<FP8>(reinterpret_cast<uint32_t*>(sgen + kTcOffTable),
+                      reinterpret_cast<uint32_t*>(sgen + kTcOffTable + 128));
   if (warp == 1) {
     tmem_alloc(sbase + kTcOffMisc, kTcTmemCols);
     tmem_relinquish();
@@ -331,7 +387,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
 
   const int n_tiles = a.n_tiles_dev ? *a.n_tiles_dev : a.n_tiles;
   const long long n_items = static_cast<long long>(n_tiles) * a.n_mtiles;
-  const int n_chunks = a.K / kTcKC;
+  const int n_chunks = a.K / KC;
   const int n_slabs = a.nb;
 
   if (warp == 0) {
@@ -345,7 +401,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
           const uint32_t s = it % kTcStages, use = it / kTcStages;
           if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) { *abort = 1; break; }
           mbar_arrive_expect_tx(bar_full_b + 8 * s, kTcBStageBytes);
-          tma_load_2d(sB + s * kTcBStageBytes, &tmap_b, kc * kTcKC, b_row, bar_full_b + 8 * s);
+          tma_load_2d(sB + s * kTcBStageBytes, &tmap_b, kc * KC, b_row, bar_full_b + 8 * s);
         }
       }
       if (*abort) {
@@ -364,16 +420,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
           if (!mbar_wait_bounded(bar_d_empty + 8 * p, (puse & 1) ^ 1)) { *abort = 1; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem + kTcColD + p * kTcN;
-          for (int q = 0; q < kTcSlabChunks; ++q, ++it) {
+          for (int q = 0; q < kSlabChunks; ++q, ++it) {
             const uint32_t s = it % kTcStages, use = it / kTcStages;
             if (!mbar_wait_bounded(bar_full_b + 8 * s, use & 1) ||
                 !mbar_wait_bounded(bar_full_a + 8 * s, use & 1)) { *abort = 1; break; }
             tc_fence_after();
             const uint64_t bdesc = smem_desc_sw128(sB + s * kTcBStageBytes);
 #pragma unroll
-            for (int kk = 0; kk < kTcKC / 16; ++kk) {
-              tc_mma_ts(d_tmem, tmem + kTcColA + 32 * s + 8 * kk, bdesc + 2 * kk, kTcIdesc,
-                        (q > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kTcStageBytesK / 32; ++kk) {   // 32 bytes of K per MMA
+              tc_mma_ts<FP8>(d_tmem, tmem + kTcColA + 32 * s + 8 * kk, bdesc + 2 * kk, tc_idesc<FP8>(),
+                             (q > 0 || kk > 0) ? 1u : 0u);
             }
             tc_commit(bar_empty + 8 * s);
           }
@@ -436,8 +492,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
           case 12: tc_extract<12>(w, Q, H0, H1); break;
           default: tc_extract<14>(w, Q, H0, H1); break;
         }
-        const bool okd = half == 0 ? tc_decode_slab<0>(Q, H0, H1, sTab, tmem_lane, bar_full_a, bar_empty, it)
-                                   : tc_decode_slab<1>(Q, H0, H1, sTab, tmem_lane, bar_full_a, bar_empty, it);
+        const bool okd = half == 0 ? tc_decode_slab<FP8, 0>(Q, H0, H1, sTab, tmem_lane, bar_full_a, bar_empty, it)
+                                   : tc_decode_slab<FP8, 1>(Q, H0, H1, sTab, tmem_lane, bar_full_a, bar_empty, it);
         if (!okd) {
           *abort = 1;
           ok = false;
@@ -462,7 +518,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
       const int b_row = a.tile_info ? a.tile_info[4 * tile + 1] : tile * kTcN;
       const int cnt = a.tile_info ? a.tile_info[4 * tile + 2] : min(kTcN, a.batch - tile * kTcN);
       named_bar(1, kTcEpilogue);                     // previous tile's stores are done
-      if (et < kTcN) s_pairs[et] = et < cnt ? (a.pairs ? a.pairs[b_row + et] : b_row + et) : -1;
+      if (et < kTcN) {
+        s_pairs[et] = et < cnt ? (a.pairs ? a.pairs[b_row + et] : b_row + et) : -1;
+        if constexpr (FP8) s_scale[et] = et < cnt ? a.xscale[b_row + et] : 0.f;
+      }
       named_bar(1, kTcEpilogue);
       const int row = mt * kTcM + rho;
       const bool row_ok = row < a.N;
@@ -498,6 +557,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
           const int pr = s_pairs[kCols * chalf + j];
           if (pr >= 0) {
             float v = acc[j];
+            if constexpr (FP8) v *= s_scale[kCols * chalf + j];
             if (up) v *= a.route_w[pr];
             a.y[static_cast<long long>(pr) * a.N + row] = v;
           }
@@ -533,6 +593,71 @@ gather_rows_kernel(const uint16_t* __restrict__ x, const int* __restrict__ pairs
   const int tok = pairs[r] / topk;
   const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<long long>(tok) * K);
   for (int i = threadIdx.x; i < K / 8; i += blockDim.x) dst[i] = src[i];
+}
+
+// E4M3 codes of x rows with one fp32 scale per row (fp8 variant): inv = 448 /
+// amax and s = amax / 448 (IEEE divisions; 0 for an all-zero row), code =
+// round-to-nearest-even, saturating, of the fp32 product x * inv.
+constexpr int kQuantThreads = 256;
+__global__ void __launch_bounds__(kQuantThreads)
+quant_e4m3_kernel(const uint16_t* __restrict__ x, int K, uint8_t* __restrict__ q, float* __restrict__ s) {
+  __shared__ float s_red[kQuantThreads / 32];
+  const long long r = blockIdx.x;
+  griddep_wait();
+  griddep_launch_dependents();
+  const uint16_t* xr = x + r * K;
+  float m = 0.f;
+  for (int i = threadIdx.x; i < K / 8; i += kQuantThreads) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr) + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[j] >> 16))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < kQuantThreads / 32; ++i) amax = fmaxf(amax, s_red[i]);
+  const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+  if (threadIdx.x == 0) s[r] = __fdiv_rn(amax, 448.f);
+  uint8_t* qr = q + r * K;
+  for (int i = threadIdx.x; i < K / 8; i += kQuantThreads) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr) + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = __nv_cvt_float_to_fp8(__fmul_rn(bf16_bits_to_f32(w[j] & 0xFFFFu), inv), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float_to_fp8(__fmul_rn(bf16_bits_to_f32(w[j] >> 16), inv), __NV_SATFINITE, __NV_E4M3);
+      o[j >> 1] |= (lo | (hi << 8)) << (16 * (j & 1));
+    }
+    reinterpret_cast<uint2*>(qr)[i] = make_uint2(o[0], o[1]);
+  }
+}
+
+// E4M3 rows and their scales gathered into expert order (fp8 variant).
+__global__ void __launch_bounds__(256)
+gather_rows8_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s, const int* __restrict__ pairs,
+                    const int* __restrict__ n_valid, int n_rows, int topk, int K, uint8_t* __restrict__ out,
+                    float* __restrict__ s_out) {
+  const int r = blockIdx.x;
+  griddep_wait();
+  griddep_launch_dependents();
+  if (r >= n_rows) return;
+  const int nv = n_valid ? *n_valid : n_rows;
+  uint4* dst = reinterpret_cast<uint4*>(out + static_cast<long long>(r) * K);
+  if (r >= nv) {
+    for (int i = threadIdx.x; i < K / 16; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x == 0) s_out[r] = 0.f;
+    return;
+  }
+  const int tok = pairs[r] / topk;
+  const uint4* src = reinterpret_cast<const uint4*>(q + static_cast<long long>(tok) * K);
+  for (int i = threadIdx.x; i < K / 16; i += blockDim.x) dst[i] = src[i];
+  if (threadIdx.x == 0) s_out[r] = s[tok];
 }
 
 }  // namespace stq1

@@ -47,7 +47,16 @@ def test_host_side_argument_checks_need_no_gpu():
     assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 63, 256, 0, None, 0, None) == -1
     assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 1, None, 0, None) == -2
     assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 8, None, 0, None) == -8
-    assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 2, None, 0, None) == -8
+    # the fp8 variant is a supported flag: without a workspace it is the workspace error
+    assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 2, None, 0, None) == -7
     assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 4, 2, 4, 64, 256, 0, None, 0, None) == -7
     assert L.stq1_gemv_workspace(16, 300, 1) == 0
     assert L.stq1_moe_workspace(16, 8, 256, 4096, 7168, 0) > 0
+    # prefill-sized calls: the fp8 variant stages E4M3 rows (1 byte per element
+    # instead of 2) plus the per-token copy and the scales
+    bf, f8 = L.stq1_moe_workspace(4096, 8, 256, 4096, 7168, 0), L.stq1_moe_workspace(4096, 8, 256, 4096, 7168, 2)
+    assert f8 == bf - 32768 * 7168 + 4096 * 7168 + 4096 * 4 + 32768 * 4
+    assert L.stq1_quantize_x_e4m3(None, 4, 256, 1 << 20, 1 << 20, None) == -2
+    assert L.stq1_quantize_x_e4m3(1 << 20, 4, 250, 1 << 20, 1 << 20, None) == -1
+    assert L.stq1_quantize_x_e4m3(1 << 20, 0, 256, 1 << 20, 1 << 20, None) == -1
+    assert L.stq1_quantize_x_e4m3((1 << 20) + 2, 4, 256, 1 << 20, 1 << 20, None) == -6
