@@ -369,7 +369,8 @@ def run_prefill(torch, stq1, device, stream, args, world, timed, bf16_peak):
 
 
 def run_sweep(args):
-    """Crossover sweep: one [18432, 7168] matrix, batch 1..1024, both kernels."""
+    """Crossover sweep: one [18432, 7168] matrix, batch 1..1024 (the stated
+    1, 4, 16, 64, 256, 1024 plus 2, 8 and 32 around the crossover), both kernels."""
     import torch
     import workloads
     import sub_bit_sparse_b200 as stq1
@@ -384,10 +385,11 @@ def run_sweep(args):
     stack = torch.stack([torch.roll(wd.view(-1, 42), shifts=i * 7919, dims=0).reshape(-1) for i in range(copies)])
     xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
     y = torch.empty((1024, n), dtype=torch.float32, device=device)
-    ws = stq1.workspace(max(stq1.LIB.stq1_gemv_workspace(n, k, b) for b in (1, 4, 16, 64, 256, 1024)), device)
+    batches = (1, 2, 4, 8, 16, 32, 64, 256, 1024)
+    ws = stq1.workspace(max(stq1.LIB.stq1_gemv_workspace(n, k, b) for b in batches), device)
     out = []
     stream = torch.cuda.Stream(device)
-    for b in (1, 4, 16, 64, 256, 1024):
+    for b in batches:
         row = {"batch": b}
         for name, path in (("table", stq1.PATH_TABLE), ("tiles", stq1.PATH_TILES)):
             stq1.set_path(path)

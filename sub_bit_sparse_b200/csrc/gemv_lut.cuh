@@ -33,24 +33,17 @@
 // unit to finish adds them in the same order.  Both are deterministic.
 #pragma once
 
-#include <utility>
-
-#include <cudaTypedefs.h>
-
 #include "device_common.cuh"
+#include "packed_copy.cuh"
 
 namespace stq1 {
 
-constexpr int kLutRows = 128;                 // rows per unit
+constexpr int kLutRows = kSlabRows;           // rows per unit
 constexpr int kLutThreads = 256;              // two threads per row: one per block of a chunk
-constexpr int kLutKC = 2;                     // blocks per chunk
-constexpr int kLutChunkBytes = kLutKC * kBlockBytes;         // 84 bytes of a row per chunk
+constexpr int kLutKC = kChunkBlocks;          // blocks per chunk
 constexpr int kLutChunkGroups = kGroupsPerBlock * kLutKC;    // 128
 constexpr int kLutGroupBytes = 144;           // 32 fp32 entries + 16-byte pad
 constexpr int kLutTokenBytes = kLutChunkGroups * kLutGroupBytes;   // 18432 = 72 * 256
-constexpr int kLutSlotBytes = 112;            // tensor-copy box width: 84-byte span + lead-in, 7 x 16 B
-constexpr int kLutTailSlots = 3;              // rows of a partial last super-row (P - 1 at most)
-constexpr int kLutTailSlotBytes = 128;
 constexpr int kLutMaxTT = 4;                  // tokens per tile
 
 struct LutArgs {
@@ -62,28 +55,16 @@ struct LutArgs {
   const int* n_tiles_dev;    // MoE: number of valid tiles
   const int* pairs;          // MoE: pair ids grouped by expert
   const float* route_w;      // [rows_out] routing weight per pair (flag WEIGHT_UP)
-  long long rowbytes;        // K / 256 * 42
-  long long tail_row0;       // first buffer row fetched through the tail map
-  long long rows_total;      // rows in the packed buffer (N, or E * N)
-  int main_srows;            // super-rows in the main map (tail_row0 / P)
+  PackedGeom g;              // tensor maps' view of the packed buffer
   int N, K;
   int topk;                  // pairs per token (1 for a plain GEMV)
   int batch;                 // plain GEMV: tokens
   int rows_out;              // rows of y
   int n_slabs;
   int S, cq, cr;             // K splits; split s has cq chunks, plus one if s < cr
-  int logP;                  // rows per super-row = 1 << logP
-  int box_h;                 // super-rows per box: 128 / P, plus one when N % P != 0
-  int buf_bytes;             // shared bytes per residue buffer (box_h * 112, 128-aligned)
-  int stage_bytes;           // P * buf_bytes + tail slots
   int flags;
   int cluster;               // 1: the S splits of a (tile, slab) form one thread-block cluster
 };
-
-__device__ __forceinline__ uint32_t win_word(const uint32_t* w, int p) {
-  // p is a compile-time constant after unrolling
-  return (p & 3) ? __funnelshift_r(w[p >> 2], w[(p >> 2) + 1], 8 * (p & 3)) : w[p >> 2];
-}
 
 // Spread bits 0, 2, 4, 6 of x to bit 6 of bytes 0..3 (other bits cleared).
 __device__ __forceinline__ uint32_t spread_even_bits(uint32_t x) {
@@ -94,56 +75,6 @@ __device__ __forceinline__ float lds_f32_addr(uint32_t addr) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
   return v;
-}
-
-// Code words of one block, extracted from a 16-byte-aligned register window:
-// d (fp32), qs as 8 little-endian words, qh as 2 words.
-struct BlockCodes {
-  float d;
-  uint32_t Q[8];
-  uint32_t H0, H1;
-};
-
-// Loads the block starting at byte B0 of a slot (B0 compile-time) with 16-byte
-// shared loads and extracts its fields.
-template <int B0>
-__device__ __forceinline__ void load_block_codes(uint32_t slot, BlockCodes& bc) {
-  constexpr int C0 = B0 >> 4;
-  constexpr int C1 = (B0 + kBlockBytes - 1) >> 4;
-  uint32_t w[16];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    if (C0 + c <= C1) {
-      const uint4 v = lds_v4(slot + 16u * (C0 + c));
-      w[4 * c + 0] = v.x;
-      w[4 * c + 1] = v.y;
-      w[4 * c + 2] = v.z;
-      w[4 * c + 3] = v.w;
-    } else {
-      w[4 * c + 0] = w[4 * c + 1] = w[4 * c + 2] = w[4 * c + 3] = 0u;
-    }
-  }
-  constexpr int base = B0 - 16 * C0;                // even
-  const uint32_t dword = w[base >> 2] >> (8 * (base & 3));
-  bc.d = __half2float(__ushort_as_half(static_cast<unsigned short>(dword & 0xFFFFu)));
-  bc.H0 = win_word(w, base + kOffQh);
-  bc.H1 = win_word(w, base + kOffQh + 4);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) bc.Q[i] = win_word(w, base + kOffQs + 4 * i);
-}
-
-// Compile-time loop helper.
-template <int I>
-struct IntC {
-  static constexpr int value = I;
-};
-template <typename F, int... Is>
-__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, Is...>) {
-  (f(IntC<Is>{}), ...);
-}
-template <int N, typename F>
-__device__ __forceinline__ void static_for(F&& f) {
-  static_for_impl(f, std::make_integer_sequence<int, N>{});
 }
 
 // Table lookups of one block's 64 groups for TT tokens; `lut` is the 256-aligned
@@ -220,19 +151,6 @@ __device__ __forceinline__ void lut_build(const uint2 (&xv)[kLutMaxTT], uint32_t
   }
 }
 
-__device__ __forceinline__ void tma_load_w2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_w1d(uint32_t dst, const CUtensorMap* map, int x, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.1d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2}], [%3];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(bar)
-      : "memory");
-}
-
 // One work unit with TT tokens.  R0 = first packed-buffer row of the slab
 // (expert * N + slab * 128); xr / orow = activation row pointers and output
 // rows of the tile's tokens.  Threads q and q + 128 own the same row; the
@@ -247,20 +165,12 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
   const int q = threadIdx.x & (kLutRows - 1);
 
   // ---- this thread's row and window (slots in residue-major order) ----
-  const int shift = 7 - a.logP;                    // log2(rows of one residue per slab)
-  const int res = q >> shift;                      // residue, uniform over a warp
-  const int kk = q & ((1 << shift) - 1);
-  const int R0mod = static_cast<int>(R0 & ((1 << a.logP) - 1));
-  const int br = res < R0mod ? 1 : 0;              // residues below R0's start one super-row later
-  const long long sr0 = R0 >> a.logP;
-  const long long R = ((sr0 + br + kk) << a.logP) + res;
-  const int rho = static_cast<int>(R - R0);        // row within the slab, 0..127
+  const PackedRow pr = packed_row(a.g, R0, q);
+  const int res = pr.res;                          // residue, uniform over a warp
+  const int rho = pr.rho;                          // row within the slab, 0..127
   const int row = slab * kLutRows + rho;           // output row
   const bool row_ok = row < a.N;
-  const uint32_t my_slot = R >= a.tail_row0
-      ? static_cast<uint32_t>((1 << a.logP) * a.buf_bytes) +
-            static_cast<uint32_t>(R - a.tail_row0) * kLutTailSlotBytes
-      : static_cast<uint32_t>(res * a.buf_bytes + (br + kk) * kLutSlotBytes);
+  const uint32_t my_slot = pr.slot;
 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t lut = (sbase + 255u) & ~255u;
@@ -268,7 +178,7 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
   const uint32_t stage0 = bar0 + 128;                // 128-aligned tensor-copy destinations
   const int NS = (c1 - c0 >= 2) ? 2 : 1;
   // split-K partials pushed by the cluster, at the same offset in every CTA of it
-  const uint32_t red = stage0 + ((a.cq + (a.cr > 0 ? 1 : 0)) >= 2 ? 2 : 1) * a.stage_bytes;
+  const uint32_t red = stage0 + ((a.cq + (a.cr > 0 ? 1 : 0)) >= 2 ? 2 : 1) * a.g.stage_bytes;
   const bool push = a.cluster && a.S > 1;
 
   if (threadIdx.x == 0) {
@@ -281,28 +191,9 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
   if (push) cluster_arrive_relaxed();
   __syncthreads();
 
-  // Tensor copies of chunk c into stage st (thread 0 only): one box per residue
-  // over the slab's super-rows, plus the slab's rows of a partial last super-row.
+  // Tensor copies of chunk c into stage st (thread 0 only).
   auto issue = [&](int c, int st) {
-    const uint32_t bar = bar0 + 8u * st;
-    const uint32_t dst = stage0 + st * a.stage_bytes;
-    const int P = 1 << a.logP;
-    const int xc = c * kLutChunkBytes;
-    const bool main = sr0 < a.main_srows;
-    int ntail = 0;
-    const long long t0 = a.tail_row0 > R0 ? a.tail_row0 : R0;
-    const long long t1 = a.rows_total < R0 + kLutRows ? a.rows_total : R0 + kLutRows;
-    if (t1 > t0) ntail = static_cast<int>(t1 - t0);
-    mbar_arrive_expect_tx(bar, (main ? P * a.box_h * kLutSlotBytes : 0) + ntail * kLutSlotBytes);
-    if (main)
-      for (int r = 0; r < P; ++r)
-        tma_load_w2d(dst + r * a.buf_bytes, wmap, (static_cast<int>(r * a.rowbytes) + xc) & ~15,
-                     static_cast<int>(sr0), bar);
-    for (int i = 0; i < ntail; ++i) {
-      const int t = static_cast<int>(t0 - a.tail_row0) + i;
-      tma_load_w1d(dst + P * a.buf_bytes + t * kLutTailSlotBytes, tmap,
-                   (static_cast<int>(t * a.rowbytes) + xc) & ~15, bar);
-    }
+    packed_issue_chunk(a.g, wmap, tmap, R0, c, stage0 + st * a.g.stage_bytes, bar0 + 8u * st);
   };
 
   float acc[kLutMaxTT];
@@ -320,8 +211,6 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
   griddep_launch_dependents();
   uint2 xv[kLutMaxTT];
   lut_load_x<TT>(xr, c0, xv);
-  // offset (mod 16) of the thread's block inside its window, before the chunk term
-  const int obase = (static_cast<int>(res * a.rowbytes) & 15) + half * kBlockBytes;
   const uint32_t lut_half = lut + static_cast<uint32_t>(half * kGroupsPerBlock * kLutGroupBytes);
   bool failed = false;
   for (int c = c0; c < c1; ++c) {
@@ -341,19 +230,9 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
       break;
     }
     if (row_ok) {
-      const uint32_t slot = stage0 + st * a.stage_bytes + my_slot;
       // only the extraction depends on the block's offset; one copy of the body follows
       BlockCodes b;
-      switch ((obase + c * kLutChunkBytes) & 15 | (half << 4)) {
-        case 0: load_block_codes<0>(slot, b); break;
-        case 4: load_block_codes<4>(slot, b); break;
-        case 8: load_block_codes<8>(slot, b); break;
-        case 12: load_block_codes<12>(slot, b); break;
-        case 16 | 10: load_block_codes<0 + kBlockBytes>(slot, b); break;    // 42 = 2 (mod 16)
-        case 16 | 14: load_block_codes<4 + kBlockBytes>(slot, b); break;
-        case 16 | 2: load_block_codes<8 + kBlockBytes>(slot, b); break;
-        default: load_block_codes<12 + kBlockBytes>(slot, b); break;         // 16 | 6
-      }
+      load_chunk_block(stage0 + st * a.g.stage_bytes + my_slot, packed_window_offset(a.g, res, c), half, b);
       lut_block_body<TT>(b, lut_half, acc);
     }
     __syncthreads();
@@ -501,12 +380,6 @@ lut_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
   lut_unit<1>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, smem);
 }
 
-// Shared bytes of one stage for super-rows of 2^logP rows and boxes of box_h super-rows.
-inline int lut_buf_bytes(int box_h) { return (box_h * kLutSlotBytes + 127) & ~127; }
-inline int lut_stage_bytes(int logP, int box_h) {
-  return (1 << logP) * lut_buf_bytes(box_h) + kLutTailSlots * kLutTailSlotBytes;
-}
-
 // Dynamic shared memory: tables, barriers, stages and (cluster split K) the
 // partials pushed by the S CTAs of the cluster into the CTA that owns a row:
 // two per split, token and owned row (ceil(128 / S) rows).
@@ -517,7 +390,7 @@ inline size_t lut_smem_bytes(int ttmax, int stages, int stage_bytes, int cluster
 }
 // Upper bound over every geometry (P = 4 with the extra super-row is the largest stage).
 inline size_t lut_smem_bytes_max(int ttmax) {
-  return lut_smem_bytes(ttmax, 2, lut_stage_bytes(2, 33), kMaxClusterRanks);
+  return lut_smem_bytes(ttmax, 2, kPackedStageMax, kMaxClusterRanks);
 }
 
 }  // namespace stq1

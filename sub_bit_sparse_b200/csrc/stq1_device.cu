@@ -154,32 +154,33 @@ int residue_period(long long rowbytes) {
   return static_cast<int>(16 / g);
 }
 
-// Tensor maps of the table kernel over a packed buffer of rows_total rows:
-// the main map views it as super-rows of P = 2^logP rows (stride P * rowbytes,
-// a multiple of 16) and copies boxes of 112 bytes x box_h super-rows; the tail
-// map (1-D) covers the last rows_total mod P rows.  extra_srow: slabs may start
-// inside a super-row (MoE experts with N % P != 0), so boxes take one more.
-struct LutMaps {
+// Tensor maps over a packed buffer of rows_total rows (table and tile
+// kernels): the main map views it as super-rows of P = 2^logP rows (stride
+// P * rowbytes, a multiple of 16) and copies boxes of 112 bytes x box_h
+// super-rows; the tail map (1-D) covers the last rows_total mod P rows.
+// extra_srow: slabs may start inside a super-row (MoE experts with N % P !=
+// 0), so boxes take one more.
+struct PackedMaps {
   CUtensorMap w, t;
 };
 
-int make_lut_maps(LutMaps* m, LutArgs* a, const uint8_t* W, long long rows_total, long long rowbytes,
-                  bool extra_srow) {
+int make_packed_maps(PackedMaps* m, PackedGeom* g, const uint8_t* W, long long rows_total, long long rowbytes,
+                     bool extra_srow) {
   auto fn = encode_fn();
   if (!fn) return STQ1_ERR_CUDA;
   const int P = residue_period(rowbytes);
   const int logP = P == 1 ? 0 : (P == 2 ? 1 : 2);
   const long long srow_bytes = P * rowbytes;
   const long long main_srows = rows_total >> logP;
-  if (main_srows >= (1LL << 31) || srow_bytes + kLutSlotBytes >= (1LL << 31)) return STQ1_ERR_SHAPE;
-  a->rowbytes = rowbytes;
-  a->rows_total = rows_total;
-  a->tail_row0 = main_srows << logP;
-  a->main_srows = static_cast<int>(main_srows);
-  a->logP = logP;
-  a->box_h = (kLutRows >> logP) + (extra_srow ? 1 : 0);
-  a->buf_bytes = lut_buf_bytes(a->box_h);
-  a->stage_bytes = lut_stage_bytes(logP, a->box_h);
+  if (main_srows >= (1LL << 31) || srow_bytes + kWindowBytes >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  g->rowbytes = rowbytes;
+  g->rows_total = rows_total;
+  g->tail_row0 = main_srows << logP;
+  g->main_srows = static_cast<int>(main_srows);
+  g->logP = logP;
+  g->box_h = (kSlabRows >> logP) + (extra_srow ? 1 : 0);
+  g->buf_bytes = packed_buf_bytes(g->box_h);
+  g->stage_bytes = packed_stage_bytes(logP, g->box_h);
   cuuint32_t es[2] = {1, 1};
   {
     // a map that is never read (no full super-row) still has to be valid
@@ -187,19 +188,19 @@ int make_lut_maps(LutMaps* m, LutArgs* a, const uint8_t* W, long long rows_total
     cuuint64_t gdim[2] = {static_cast<cuuint64_t>(any ? srow_bytes : 16),
                           static_cast<cuuint64_t>(any ? main_srows : 1)};
     cuuint64_t gstride[1] = {static_cast<cuuint64_t>(any ? srow_bytes : 16)};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(any ? kLutSlotBytes : 16),
-                         static_cast<cuuint32_t>(any ? a->box_h : 1)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(any ? kWindowBytes : 16),
+                         static_cast<cuuint32_t>(any ? g->box_h : 1)};
     if (fn(&m->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(W), gdim, gstride, box, es,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return STQ1_ERR_CUDA;
   }
   {
-    const long long nt = rows_total - a->tail_row0;
-    const uint8_t* base = nt > 0 ? W + a->tail_row0 * rowbytes : W;
+    const long long nt = rows_total - g->tail_row0;
+    const uint8_t* base = nt > 0 ? W + g->tail_row0 * rowbytes : W;
     cuuint64_t gdim[1] = {static_cast<cuuint64_t>(nt > 0 ? nt * rowbytes : 16)};
     cuuint64_t gstride[1] = {0};
-    cuuint32_t box[1] = {static_cast<cuuint32_t>(nt > 0 ? kLutSlotBytes : 16)};
+    cuuint32_t box[1] = {static_cast<cuuint32_t>(nt > 0 ? kWindowBytes : 16)};
     if (fn(&m->t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, const_cast<uint8_t*>(base), gdim, gstride, box, es,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -257,7 +258,7 @@ void plan_table(GemvPlan* p, long long N, long long K, int batch, bool one_wave)
   S = std::max<long long>(1, std::min<long long>(S, std::max(1, p->n_chunks)));
   const int P = residue_period(nb * kBlockBytes);
   const int logP = P == 1 ? 0 : (P == 2 ? 1 : 2);
-  const int stage = lut_stage_bytes(logP, kLutRows >> logP);
+  const int stage = packed_stage_bytes(logP, kLutRows >> logP);
   const long long slots_sm = smem_per_sm();
   for (; one_wave && S > 1; --S) {
     const int cq = static_cast<int>(p->n_chunks / S), cr = static_cast<int>(p->n_chunks % S);
@@ -334,10 +335,9 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
     CUtensorMap map;
     if (!make_b_map(&map, x, batch, K, false)) return STQ1_ERR_CUDA;
     TcArgs t{};
-    t.W = static_cast<const uint8_t*>(W_packed);
-    t.W_end = t.W + N * rowbytes;
-    t.expert_bytes = 0;
-    t.rowbytes = rowbytes;
+    PackedMaps pm;
+    rc = make_packed_maps(&pm, &t.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
+    if (rc != STQ1_OK) return rc;
     t.y = y;
     t.tile_info = nullptr;
     t.n_tiles_dev = nullptr;
@@ -350,11 +350,10 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
     t.nb = static_cast<int>(nb);
     t.n_mtiles = static_cast<int>((N + kTcM - 1) / kTcM);
     t.batch = batch;
-    t.P = residue_period(rowbytes);
     t.flags = 0;
     const long long items = static_cast<long long>(t.n_tiles) * t.n_mtiles;
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
-    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, t);
+    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
   }
   if (!p.table_path) {
     const long long warps = static_cast<long long>(batch) * N;
@@ -364,8 +363,8 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
     return launch_status();
   }
   LutArgs a{};
-  LutMaps maps;
-  rc = make_lut_maps(&maps, &a, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
+  PackedMaps maps;
+  rc = make_packed_maps(&maps, &a.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
   if (rc != STQ1_OK) return rc;
   a.x = x;
   a.y = y;
@@ -384,7 +383,7 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
   const dim3 grid(static_cast<unsigned>(units), static_cast<unsigned>(p.S));
   auto go = [&](int cluster) {
     a.cluster = cluster > 1 ? 1 : 0;
-    const size_t smem = lut_smem_bytes(p.tt, lut_stages(a), a.stage_bytes, cluster);
+    const size_t smem = lut_smem_bytes(p.tt, lut_stages(a), a.g.stage_bytes, cluster);
     if (p.tt == 1)
       return launch_pdl_cluster(lut_gemv_kernel<1>, grid, kLutThreads, smem, s, cluster, maps.w, maps.t, a);
     if (p.tt == 2)
@@ -502,10 +501,10 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
     CUtensorMap map;
     if (!make_b_map(&map, xperm, n_pairs, K, m.fp8)) return STQ1_ERR_CUDA;
     TcArgs t{};
-    t.W = static_cast<const uint8_t*>(expert_blocks);
-    t.W_end = t.W + static_cast<long long>(E) * N * rowbytes;
-    t.expert_bytes = N * rowbytes;
-    t.rowbytes = rowbytes;
+    PackedMaps pm;
+    rc = make_packed_maps(&pm, &t.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
+                          rowbytes, N % residue_period(rowbytes) != 0);
+    if (rc != STQ1_OK) return rc;
     t.y = y;
     t.tile_info = tiles;
     t.n_tiles_dev = ntiles;
@@ -518,17 +517,16 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
     t.nb = static_cast<int>(nb);
     t.n_mtiles = static_cast<int>((N + kTcM - 1) / kTcM);
     t.batch = 0;
-    t.P = residue_period(rowbytes);
     t.flags = flags;
     const long long items = static_cast<long long>(m.max_tiles) * t.n_mtiles;
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
-    if (m.fp8) return launch_pdl(tc_gemm_kernel<true>, grid, kTcThreads, kTcSmemBytes, s, map, t);
-    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, t);
+    if (m.fp8) return launch_pdl(tc_gemm_kernel<true>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
+    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
   }
   LutArgs a{};
-  LutMaps maps;
+  PackedMaps maps;
   const int P = residue_period(rowbytes);
-  rc = make_lut_maps(&maps, &a, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
+  rc = make_packed_maps(&maps, &a.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
                      rowbytes, N % P != 0);
   if (rc != STQ1_OK) return rc;
   a.x = x;
@@ -551,7 +549,7 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   const long long units = static_cast<long long>(m.max_tiles) * a.n_slabs;
   if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
   return launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(units)), kLutThreads,
-                            lut_smem_bytes(kMoeTableTokens, lut_stages(a), a.stage_bytes, 1), s, 1u, maps.w, maps.t,
+                            lut_smem_bytes(kMoeTableTokens, lut_stages(a), a.g.stage_bytes, 1), s, 1u, maps.w, maps.t,
                             a);
 }
 
@@ -660,8 +658,8 @@ extern "C" int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float*
     if (cudaMemsetAsync(scratch, 0, kCounterBytes, s) != cudaSuccess) return STQ1_ERR_CUDA;
   }
   LutArgs a{};
-  LutMaps maps;
-  rc = make_lut_maps(&maps, &a, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
+  PackedMaps maps;
+  rc = make_packed_maps(&maps, &a.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
   if (rc != STQ1_OK) return rc;
   a.x = x;
   a.y = y;
@@ -678,7 +676,7 @@ extern "C" int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float*
   a.cluster = 0;
   if (units0 >= (1LL << 31)) return STQ1_ERR_SHAPE;
   const dim3 grid(static_cast<unsigned>(units0), static_cast<unsigned>(S));
-  const size_t smem = lut_smem_bytes(batch == 1 ? 1 : (batch == 2 ? 2 : 4), lut_stages(a), a.stage_bytes, 1);
+  const size_t smem = lut_smem_bytes(batch == 1 ? 1 : (batch == 2 ? 2 : 4), lut_stages(a), a.g.stage_bytes, 1);
   if (batch == 1)
     lut_gemv_kernel<1><<<grid, kLutThreads, smem, s>>>(maps.w, maps.t, a);
   else if (batch == 2)

@@ -13,17 +13,23 @@
 //               shared ring (one 2-D tensor copy per stage, no multicast).
 //   warp 1      TMEM allocator and the single MMA-issuing thread:
 //               tcgen05.mma.cta_group::1.kind::f16, A from TMEM, B from shared.
+//   warp 18     TMA producer of the packed weights: per 128-row tile, chunks
+//               of two blocks (the super-row tensor copies of
+//               packed_copy.cuh) into a 4-stage shared ring.
 //   warps 2-9   decoders, two per TMEM lane quadrant: a thread owns one weight
-//               row, reads the row's 42-byte block for the slab (one slab
-//               ahead), expands each group's 5-bit code to four bf16 values
-//               through a 32-entry table and stores its half of each stage's
-//               64 columns into TMEM (tcgen05.st), the A operand.
+//               row (TMEM lane order = the ring's slot order), copies a
+//               chunk's two blocks of codes from shared memory into registers
+//               (releasing the stage), expands each group's 5-bit code to four
+//               bf16 values through a 32-entry table and stores its half of
+//               each stage's 64 columns into TMEM (tcgen05.st), the A operand.
 //   warps 10-17 epilogue, two per quadrant (64 token columns each): per slab,
-//               tcgen05.ld of the slab accumulator, fp32 FMA with the row's d,
+//               tcgen05.ld of the slab accumulator, fp32 FMA with the row's d
+//               (read from the packed ring),
 //               release of the TMEM buffer; at the end of the tile, coalesced
 //               stores of y.
 // TMEM (512 columns allocated, one CTA per SM): slab accumulators 2 x 128
-// columns, A stages 8 x 32 columns.  Shared memory: 8 x-tile stages of 16 KB.
+// columns, A stages 8 x 32 columns.  Shared memory: 8 x-tile stages of 16 KB
+// and 4 packed-weight stages of up to 15 KB.
 // All waits are bounded; a timeout sets the device error word and makes every
 // role stop at its next wait, so the CTA always reaches the final barrier and
 // frees its TMEM.
@@ -40,6 +46,7 @@
 #include <cuda_fp8.h>
 
 #include "device_common.cuh"
+#include "packed_copy.cuh"
 
 namespace stq1 {
 
@@ -53,7 +60,8 @@ template <bool FP8>
 constexpr int tc_kc() { return FP8 ? kTcKC8 : kTcKC; }
 template <bool FP8>
 constexpr int tc_slab_chunks() { return kBlockWeights / tc_kc<FP8>(); }   // 4 (bf16) or 2 (fp8)
-constexpr int kTcThreads = 576;
+constexpr int kTcThreads = 608;
+constexpr int kTcAStages = 4;                    // packed-weight chunks in flight
 constexpr int kTcDecoders = 256;                 // threads: 8 warps
 constexpr int kTcEpilogue = 256;                 // threads: 8 warps
 constexpr uint32_t kTcTmemCols = 512;
@@ -62,18 +70,17 @@ constexpr uint32_t kTcColA = 256;             // kTcStages x 32
 constexpr int kTcBStageBytes = kTcN * kTcStageBytesK;   // 16 KB
 // shared layout (offsets from a 1024-aligned base)
 constexpr int kTcOffB = 0;
-constexpr int kTcOffTable = kTcStages * kTcBStageBytes;            // 131072: 2 x 128 B decode tables
+constexpr int kTcOffA = kTcStages * kTcBStageBytes;                // 131072: packed-weight ring
+constexpr int kTcOffTable = kTcOffA + kTcAStages * kPackedStageMax; // 2 x 128 B decode tables
+static_assert(kTcOffTable % 256 == 0, "decode tables must be 256-aligned");
 constexpr int kTcOffBar = kTcOffTable + 256;
-constexpr int kTcOffPairs = kTcOffBar + 256;                       // kTcN ints
+constexpr int kTcOffPairs = kTcOffBar + 512;                       // kTcN ints
 constexpr int kTcOffScale = kTcOffPairs + kTcN * 4;                // kTcN floats (fp8)
 constexpr int kTcOffMisc = kTcOffScale + kTcN * 4;
 constexpr int kTcSmemBytes = 1024 + kTcOffMisc + 64;   // > 114 KB: one CTA per SM
 
 struct TcArgs {
-  const uint8_t* W;          // matrix or expert 0
-  const uint8_t* W_end;
-  long long expert_bytes;
-  long long rowbytes;
+  PackedGeom g;              // tensor maps' view of the packed weights
   float* y;                  // [rows_out, N]
   const int* tile_info;      // [tiles, 4] expert, first B row, count, pad (nullptr: plain)
   const int* n_tiles_dev;    // device tile count (MoE) or nullptr
@@ -84,7 +91,6 @@ struct TcArgs {
   int N, K, nb;
   int n_mtiles;
   int batch;                 // plain: tokens
-  int P;                     // residue period of row offsets mod 16
   int flags;
 };
 
@@ -237,50 +243,6 @@ __device__ __forceinline__ void tc_fill_tables(uint32_t* t0, uint32_t* t1) {
   }
 }
 
-// Loads the 42-byte block at A (16-byte-aligned window of 64 bytes starting at
-// A & ~15) without reading past `end`.
-__device__ __forceinline__ void load_block_window(const uint8_t* A, const uint8_t* end,
-                                                  uint32_t (&w)[16]) {
-  const uintptr_t lo = reinterpret_cast<uintptr_t>(A) & ~static_cast<uintptr_t>(15);
-  const uintptr_t need_end = reinterpret_cast<uintptr_t>(A) + kBlockBytes;
-  const uintptr_t e = reinterpret_cast<uintptr_t>(end);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uintptr_t q = lo + 16u * c;
-    if (q + 16 <= e && q < need_end) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(q));
-      w[4 * c] = v.x;
-      w[4 * c + 1] = v.y;
-      w[4 * c + 2] = v.z;
-      w[4 * c + 3] = v.w;
-    } else {
-      uint32_t tmp[4] = {0u, 0u, 0u, 0u};
-      for (int b = 0; b < 16; ++b)
-        if (q + b < e && q + b < need_end)
-          tmp[b >> 2] |= static_cast<uint32_t>(*reinterpret_cast<const uint8_t*>(q + b)) << (8 * (b & 3));
-      w[4 * c] = tmp[0];
-      w[4 * c + 1] = tmp[1];
-      w[4 * c + 2] = tmp[2];
-      w[4 * c + 3] = tmp[3];
-    }
-  }
-}
-
-// qs (8 words) and qh (2 words) of the block starting at window byte BASE.
-template <int BASE>
-__device__ __forceinline__ void tc_extract(const uint32_t (&w)[16], uint32_t (&Q)[8], uint32_t& H0,
-                                           uint32_t& H1) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int p = BASE + kOffQs + 4 * i;
-    Q[i] = (p & 3) ? __funnelshift_r(w[p >> 2], w[(p >> 2) + 1], 8 * (p & 3)) : w[p >> 2];
-  }
-  constexpr int ph = BASE + kOffQh;
-  H0 = (ph & 3) ? __funnelshift_r(w[ph >> 2], w[(ph >> 2) + 1], 8 * (ph & 3)) : w[ph >> 2];
-  constexpr int ph1 = ph + 4;
-  H1 = (ph1 & 3) ? __funnelshift_r(w[ph1 >> 2], w[(ph1 >> 2) + 1], 8 * (ph1 & 3)) : w[ph1 >> 2];
-}
-
 // Expands this thread's half of each of the block's stages into 16 TMEM
 // columns (bf16: 8 groups x 2 words of each 64-column stage; fp8: 16 groups
 // x 1 word of each 128-column stage); for each stage waits for the A stage
@@ -338,7 +300,8 @@ __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t 
 
 template <bool FP8>
 __global__ void __launch_bounds__(kTcThreads, 1)
-tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap wmap,
+               const __grid_constant__ CUtensorMap tmap_w, const TcArgs a) {
   constexpr int KC = tc_kc<FP8>();
   constexpr int kSlabChunks = tc_slab_chunks<FP8>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -346,12 +309,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - sraw);
   const uint32_t sB = sbase + kTcOffB;
+  const uint32_t sA = sbase + kTcOffA;
   const uint32_t sTab = sbase + kTcOffTable;
   const uint32_t bar = sbase + kTcOffBar;
-  // barriers: full_b[8] @0, full_a[8] @64, empty[8] @128, d_full[2] @192, d_empty[2] @208, drain @224
+  // barriers: full_b[8] @0, full_a[8] @64, empty[8] @128, d_full[2] @192, d_empty[2] @208, drain @224,
+  // packed ring full[4] @256, empty[4] @288
   const uint32_t bar_full_b = bar, bar_full_a = bar + 64, bar_empty = bar + 128;
   const uint32_t bar_d_full = bar + 192, bar_d_empty = bar + 208;
   const uint32_t bar_drain = bar + 224;
+  const uint32_t bar_pk_full = bar + 256, bar_pk_empty = bar + 288;
   int* s_pairs = reinterpret_cast<int*>(sgen + kTcOffPairs);
   float* s_scale = reinterpret_cast<float*>(sgen + kTcOffScale);
   volatile int* s_misc = reinterpret_cast<volatile int*>(sgen + kTcOffMisc);   // [0] tmem base, [1] abort
@@ -368,6 +334,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
       mbar_init(bar_d_empty + 8 * i, kTcEpilogue);
     }
     mbar_init(bar_drain, 1);                         // drain barrier (abort path)
+    for (int i = 0; i < kTcAStages; ++i) {
+      mbar_init(bar_pk_full + 8 * i, 1);
+      mbar_init(bar_pk_empty + 8 * i, kTcDecoders + kTcEpilogue);
+    }
     s_misc[1] = 0;
     fence_mbar_init();
   }
@@ -389,6 +359,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
   const long long n_items = static_cast<long long>(n_tiles) * a.n_mtiles;
   const int n_chunks = a.K / KC;
   const int n_slabs = a.nb;
+  const int n_pk = a.nb / kChunkBlocks;              // packed chunks per tile (two slabs each)
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -445,55 +416,35 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
     }
   } else if (warp < 10) {
     // ---------------- decoders ----------------
-    const int half = (warp - 2) >> 2;               // which 8 of each chunk's 16 groups
+    const int half = (warp - 2) >> 2;               // which half of each stage's groups
     const int quad = warp & 3;                       // TMEM lane quadrant of this warp
-    const int P = a.P;
-    const int rho = P * lane + (quad % P) + 32 * P * (quad / P);   // row within the tile
     const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(32 * quad) << 16);
-    uint32_t it = 0;
+    uint32_t it = 0, ca = 0;
     bool ok = true;
     for (long long item = blockIdx.x; item < n_items && ok && !*abort; item += gridDim.x) {
       const int tile = static_cast<int>(item / a.n_mtiles);
-      const int mt = static_cast<int>(item % a.n_mtiles);
+      const int mt = static_cast<int>(item - static_cast<long long>(tile) * a.n_mtiles);
       const int e = a.tile_info ? a.tile_info[4 * tile + 0] : 0;
-      const int row = mt * kTcM + rho;
-      const bool row_ok = row < a.N;
-      const uint8_t* rbase = a.W + e * a.expert_bytes + static_cast<long long>(row_ok ? row : 0) * a.rowbytes;
-      // every lane of the warp has the same block offset mod 16 (rows of one residue class)
-      const uint8_t* r0 = a.W + e * a.expert_bytes +
-                          static_cast<long long>(mt * kTcM + (quad % P) + 32 * P * (quad / P)) * a.rowbytes;
-      // packed windows of the next two slabs, loaded ahead (rows past N decode
-      // zeros: computed, never stored)
-      uint32_t wn[16], wn2[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) wn[i] = wn2[i] = 0u;
-      if (row_ok) {
-        load_block_window(rbase, a.W_end, wn);
-        if (n_slabs > 1) load_block_window(rbase + kBlockBytes, a.W_end, wn2);
-      }
-      for (int slab = 0; slab < n_slabs; ++slab) {
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          w[i] = wn[i];
-          wn[i] = wn2[i];
+      const long long R0 = static_cast<long long>(e) * a.N + static_cast<long long>(mt) * kTcM;
+      // TMEM lane 32 * quad + lane holds the row of slot 32 * quad + lane of the ring
+      const PackedRow pr = packed_row(a.g, R0, 32 * quad + lane);
+      const bool row_ok = mt * kTcM + pr.rho < a.N;   // rows past N decode zeros: computed, never stored
+      for (int c = 0; c < n_pk; ++c, ++ca) {
+        const uint32_t sa = ca % kTcAStages, ause = ca / kTcAStages;
+        if (!mbar_wait_bounded(bar_pk_full + 8 * sa, ause & 1)) { *abort = 1; ok = false; break; }
+        BlockCodes b0 = {}, b1 = {};
+        if (row_ok) {
+          const uint32_t slot = sA + sa * kPackedStageMax + pr.slot;
+          const int o = packed_window_offset(a.g, pr.res, c);
+          load_chunk_block(slot, o, 0, b0);
+          load_chunk_block(slot, o, 1, b1);
         }
-        if (row_ok && slab + 2 < n_slabs)
-          load_block_window(rbase + static_cast<long long>(slab + 2) * kBlockBytes, a.W_end, wn2);
-        const int base = static_cast<int>((reinterpret_cast<uintptr_t>(r0) + static_cast<uintptr_t>(slab) * kBlockBytes) & 15);
-        uint32_t Q[8], H0, H1;
-        switch (base) {                              // only the extraction depends on the offset
-          case 0: tc_extract<0>(w, Q, H0, H1); break;
-          case 2: tc_extract<2>(w, Q, H0, H1); break;
-          case 4: tc_extract<4>(w, Q, H0, H1); break;
-          case 6: tc_extract<6>(w, Q, H0, H1); break;
-          case 8: tc_extract<8>(w, Q, H0, H1); break;
-          case 10: tc_extract<10>(w, Q, H0, H1); break;
-          case 12: tc_extract<12>(w, Q, H0, H1); break;
-          default: tc_extract<14>(w, Q, H0, H1); break;
-        }
-        const bool okd = half == 0 ? tc_decode_slab<FP8, 0>(Q, H0, H1, sTab, tmem_lane, bar_full_a, bar_empty, it)
-                                   : tc_decode_slab<FP8, 1>(Q, H0, H1, sTab, tmem_lane, bar_full_a, bar_empty, it);
+        mbar_arrive(bar_pk_empty + 8 * sa);          // the codes are in registers now
+        const bool okd =
+            (half == 0 ? tc_decode_slab<FP8, 0>(b0.Q, b0.H0, b0.H1, sTab, tmem_lane, bar_full_a, bar_empty, it)
+                       : tc_decode_slab<FP8, 1>(b0.Q, b0.H0, b0.H1, sTab, tmem_lane, bar_full_a, bar_empty, it)) &&
+            (half == 0 ? tc_decode_slab<FP8, 0>(b1.Q, b1.H0, b1.H1, sTab, tmem_lane, bar_full_a, bar_empty, it)
+                       : tc_decode_slab<FP8, 1>(b1.Q, b1.H0, b1.H1, sTab, tmem_lane, bar_full_a, bar_empty, it));
         if (!okd) {
           *abort = 1;
           ok = false;
@@ -501,19 +452,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
         }
       }
     }
-  } else {
+  } else if (warp < 18) {
     // ---------------- epilogue ----------------
     const int quad = warp & 3;
     const int chalf = (warp - 10) >> 2;              // token columns [64 * chalf, 64 * chalf + 64)
-    const int P = a.P;
-    const int rho = P * lane + (quad % P) + 32 * P * (quad / P);
     const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(32 * quad) << 16);
     const int et = threadIdx.x - 320;                // 0..255
     constexpr int kCols = kTcN / 2;
-    uint32_t sc = 0;
+    uint32_t sc = 0, ca = 0;
     for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
       const int tile = static_cast<int>(item / a.n_mtiles);
-      const int mt = static_cast<int>(item % a.n_mtiles);
+      const int mt = static_cast<int>(item - static_cast<long long>(tile) * a.n_mtiles);
       const int e = a.tile_info ? a.tile_info[4 * tile + 0] : 0;
       const int b_row = a.tile_info ? a.tile_info[4 * tile + 1] : tile * kTcN;
       const int cnt = a.tile_info ? a.tile_info[4 * tile + 2] : min(kTcN, a.batch - tile * kTcN);
@@ -523,18 +472,33 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
         if constexpr (FP8) s_scale[et] = et < cnt ? a.xscale[b_row + et] : 0.f;
       }
       named_bar(1, kTcEpilogue);
-      const int row = mt * kTcM + rho;
+      const long long R0 = static_cast<long long>(e) * a.N + static_cast<long long>(mt) * kTcM;
+      const PackedRow pr = packed_row(a.g, R0, 32 * quad + lane);
+      const int row = mt * kTcM + pr.rho;
       const bool row_ok = row < a.N;
-      const uint8_t* rbase = a.W + e * a.expert_bytes + static_cast<long long>(row_ok ? row : 0) * a.rowbytes;
       float acc[kCols];
 #pragma unroll
       for (int j = 0; j < kCols; ++j) acc[j] = 0.f;
       bool ok = true;
-      unsigned short dn = __ldg(reinterpret_cast<const unsigned short*>(rbase));   // d of slab 0
+      float dpair[2] = {0.f, 0.f};
       for (int slab = 0; slab < n_slabs; ++slab, ++sc) {
-        const float d = __half2float(__ushort_as_half(dn));
-        if (slab + 1 < n_slabs)                      // prefetch the next slab's scale
-          dn = __ldg(reinterpret_cast<const unsigned short*>(rbase + static_cast<long long>(slab + 1) * kBlockBytes));
+        if ((slab & 1) == 0) {
+          // the scales of this chunk's two blocks, then release the ring stage
+          const uint32_t sa = ca % kTcAStages, ause = ca / kTcAStages;
+          if (!mbar_wait_bounded(bar_pk_full + 8 * sa, ause & 1)) { *abort = 1; ok = false; break; }
+          if (row_ok) {
+            const uint32_t w0 = sA + sa * kPackedStageMax + pr.slot +
+                                static_cast<uint32_t>(packed_window_offset(a.g, pr.res, slab >> 1));
+            unsigned short h0, h1;
+            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h0) : "r"(w0));
+            asm volatile("ld.shared.u16 %0, [%1+42];" : "=h"(h1) : "r"(w0));
+            dpair[0] = __half2float(__ushort_as_half(h0));
+            dpair[1] = __half2float(__ushort_as_half(h1));
+          }
+          mbar_arrive(bar_pk_empty + 8 * sa);
+          ++ca;
+        }
+        const float d = dpair[slab & 1];
         const uint32_t p = sc & 1, puse = sc >> 1;
         if (!mbar_wait_bounded(bar_d_full + 8 * p, puse & 1)) { *abort = 1; ok = false; break; }
         tc_fence_after();
@@ -554,14 +518,35 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
         const bool up = (a.flags & STQ1_MOE_WEIGHT_UP) && row >= a.N / 2;
 #pragma unroll
         for (int j = 0; j < kCols; ++j) {
-          const int pr = s_pairs[kCols * chalf + j];
-          if (pr >= 0) {
+          const int pair = s_pairs[kCols * chalf + j];
+          if (pair >= 0) {
             float v = acc[j];
             if constexpr (FP8) v *= s_scale[kCols * chalf + j];
-            if (up) v *= a.route_w[pr];
-            a.y[static_cast<long long>(pr) * a.N + row] = v;
+            if (up) v *= a.route_w[pair];
+            a.y[static_cast<long long>(pair) * a.N + row] = v;
           }
         }
+      }
+    }
+  } else {
+    // ---------------- TMA producer of the packed weights (warp 18) ----------------
+    if (lane == 0) {
+      uint32_t ca = 0;
+      for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
+        const int tile = static_cast<int>(item / a.n_mtiles);
+        const int mt = static_cast<int>(item - static_cast<long long>(tile) * a.n_mtiles);
+        const int e = a.tile_info ? a.tile_info[4 * tile + 0] : 0;
+        const long long R0 = static_cast<long long>(e) * a.N + static_cast<long long>(mt) * kTcM;
+        for (int c = 0; c < n_pk; ++c, ++ca) {
+          const uint32_t sa = ca % kTcAStages, ause = ca / kTcAStages;
+          if (!mbar_wait_bounded(bar_pk_empty + 8 * sa, (ause & 1) ^ 1)) { *abort = 1; break; }
+          packed_issue_chunk(a.g, &wmap, &tmap_w, R0, c, sA + sa * kPackedStageMax, bar_pk_full + 8 * sa);
+        }
+      }
+      if (*abort) {
+        // let the last chunk copies land before the CTA can exit (bounded)
+        for (uint32_t j = ca > kTcAStages ? ca - kTcAStages : 0; j < ca; ++j)
+          mbar_wait_bounded(bar_pk_full + 8 * (j % kTcAStages), (j / kTcAStages) & 1);
       }
     }
   }
