@@ -241,6 +241,12 @@ def run_gpu(args):
     except Exception as exc:  # reported, never hidden
         prefill = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
+    # --- encoders (GPU and host) ---
+    try:
+        encoder = run_encoder(torch, stq1, device, stream)
+    except Exception as exc:  # reported, never hidden
+        encoder = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     # --- end to end through the public API with host buffers ---
     e2e = run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier)
 
@@ -269,6 +275,7 @@ def run_gpu(args):
         "gemv_batches": batches,
         "moe_decode": moe,
         "moe_prefill": prefill,
+        "encoder": encoder,
         "e2e": e2e,
         "gpu_launches": args.steps * STACK,
         "clocks": clk.summary(),
@@ -365,6 +372,39 @@ def run_prefill(torch, stq1, device, stream, args, world, timed, bf16_peak):
     res["config"] = ("256 experts x [4096, 7168] STQ1_0, 4096 tokens, Zipf(1.1) top-8 (32,768 pairs), "
                      "tcgen05 tiles, A = decoded +/-1 in TMEM (bf16, kind::f16; fp8: E4M3, kind::f8f6f4 with "
                      "per-token E4M3 activations), fp32 per-block scale; fp8 peak = measured bf16 x 2 (nominal ratio)")
+    return res
+
+
+def run_encoder(torch, stq1, device, stream):
+    """Encoders on the decode matrix [4096, 7168]: GPU (stq1_quantize) and host
+    (stq1_quantize_ref, all cores), weights per second; the GPU and host bytes
+    are checked equal."""
+    import workloads
+    import time
+    w, h, _ = workloads.decode_gemv_inputs()
+    n, k = w.shape
+    wd = torch.from_numpy(w).to(device)
+    hd = torch.from_numpy(h).to(device)
+    res = {}
+    outs = {}
+    for mode, hh in (("plain", None), ("sherry", hd)):
+        with torch.cuda.stream(stream):
+            o = stq1.quantize_gpu(wd, hh, mode=mode)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 5
+            e0.record(stream)
+            for _ in range(reps):
+                stq1.quantize_gpu(wd, hh, mode=mode, out=o)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        res[f"gpu_{mode}_weights_per_s"] = round(n * k * reps / (e0.elapsed_time(e1) * 1e-3), 1)
+        outs[mode] = o.cpu().numpy()
+    t0 = time.perf_counter()
+    host = stq1.quantize_ref(w, h, mode="sherry")
+    res["host_sherry_weights_per_s"] = round(n * k / (time.perf_counter() - t0), 1)
+    res["host_threads"] = os.cpu_count()
+    res["gpu_equals_host"] = bool(np.array_equal(host, outs["sherry"]))
+    res["config"] = "decode matrix [4096, 7168], Sherry 3 rounds with calibration importance; plain = amax"
     return res
 
 

@@ -61,8 +61,9 @@ extern "C" {
 /* Device error word bits (reported through stq1_status). */
 #define STQ1_DEV_BAD_EXPERT 1     /* a topk id was outside [0, E); its slot was skipped */
 #define STQ1_DEV_WAIT_LIMIT 2     /* a bounded wait inside a kernel gave up */
+#define STQ1_DEV_BAD_VALUE 4      /* (stq1_quantize) NaN/Inf weight or negative/non-finite importance */
 
-/* Encoder modes for stq1_quantize_ref. */
+/* Encoder modes for stq1_quantize_ref and stq1_quantize. */
 #define STQ1_ENC_PLAIN 0          /* amax scale, smallest-|w| lane zeroed */
 #define STQ1_ENC_SHERRY 1         /* alternating WLS scale / weighted zero placement */
 
@@ -102,6 +103,24 @@ int stq1_version(void);
  */
 int stq1_quantize_ref(const float* W, const float* h, int64_t N, int64_t K, int mode,
                       int rounds, uint8_t* out, int threads);
+
+/*
+ * stq1_quantize -- the same encoders on the GPU, byte-identical to
+ * stq1_quantize_ref for every input that function accepts (one thread per
+ * 256-weight block, fp64 in the same order, no fused multiply-add).
+ *   W      device, [N, K] fp32 row-major, 16-byte aligned.
+ *   h      device, [K] fp32 importance (Sherry mode; NULL means h = 1;
+ *          ignored in plain mode).
+ *   out    device, N*K/256*42 bytes, 2-byte aligned (fully overwritten).
+ *   rounds Sherry rounds (0..1000; the pages use 3).
+ * Asynchronous on `stream`.  A NaN/Inf weight, or a negative or non-finite
+ * importance, sets STQ1_DEV_BAD_VALUE in the device error word (read it with
+ * stq1_status) and the affected blocks are written as zeros.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_ARG, STQ1_ERR_ALIGN,
+ * STQ1_ERR_CUDA.
+ */
+int stq1_quantize(const float* W, const float* h, int64_t N, int64_t K, int mode, int rounds,
+                  uint8_t* out, void* stream);
 
 /*
  * stq1_dequant -- decoded weights as bf16 (device).

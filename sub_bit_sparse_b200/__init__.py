@@ -28,6 +28,7 @@ ERRORS = {
 }
 DEV_BAD_EXPERT = 1
 DEV_WAIT_LIMIT = 2
+DEV_BAD_VALUE = 4
 ENC_PLAIN = 0
 ENC_SHERRY = 1
 MOE_WEIGHT_UP = 1
@@ -53,6 +54,8 @@ SIGNATURES = {
     "stq1_set_path": (_c.c_int, [_c.c_int]),
     "stq1_gemv_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int,
                                      _c.c_void_p]),
+    "stq1_quantize": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int, _c.c_int,
+                                 _c.c_void_p, _c.c_void_p]),
     "stq1_quantize_x_e4m3": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p, _c.c_void_p,
                                         _c.c_void_p]),
 }
@@ -241,6 +244,23 @@ def moe_gateup(expert_blocks, x, topk_ids, topk_weights, n: int, k: int, n_exper
                              None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
                              _stream(x))
     _check("stq1_moe_gateup", rc)
+    return out
+
+
+def quantize_gpu(w, h=None, mode: str = "plain", rounds: int = 3, out=None):
+    """fp32 [N, K] CUDA tensor -> packed STQ1_0 bytes (uint8 CUDA tensor), byte-identical to quantize_ref."""
+    torch = _torch()
+    _require(w, torch.float32, "w")
+    n, k = w.shape
+    if h is not None:
+        _require(h, torch.float32, "h")
+    if out is None:
+        out = torch.empty((n * (k // BLOCK_WEIGHTS) * BLOCK_BYTES,), dtype=torch.uint8, device=w.device)
+    _require(out, torch.uint8, "out")
+    m = ENC_SHERRY if mode == "sherry" else ENC_PLAIN
+    rc = _load().stq1_quantize(w.data_ptr(), None if h is None else h.data_ptr(), n, k, m, rounds, out.data_ptr(),
+                               _stream(w))
+    _check("stq1_quantize", rc)
     return out
 
 

@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 
 #include "device_common.cuh"
+#include "encode_device.cuh"
 #include "gemv_lut.cuh"
 #include "small_kernels.cuh"
 #include "tc_gemm.cuh"
@@ -97,7 +98,9 @@ int ensure_configured() {
       cudaFuncSetAttribute(tc_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kTcSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kTcSmemBytes) != cudaSuccess)
+                           kTcSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(encode_smem_bytes())) != cudaSuccess)
     return STQ1_ERR_CUDA;
   // split-K clusters of up to 16 CTAs (above the portable 8); a refusal only
   // disables the cluster path
@@ -551,6 +554,24 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   return launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(units)), kLutThreads,
                             lut_smem_bytes(kMoeTableTokens, lut_stages(a), a.g.stage_bytes, 1), s, 1u, maps.w, maps.t,
                             a);
+}
+
+extern "C" int stq1_quantize(const float* W, const float* h, int64_t N, int64_t K, int mode, int rounds,
+                             uint8_t* out, void* stream) {
+  if (!W || !out) return STQ1_ERR_NULL;
+  if (N <= 0 || K <= 0 || K % kBlockWeights) return STQ1_ERR_SHAPE;
+  if (mode != STQ1_ENC_PLAIN && mode != STQ1_ENC_SHERRY) return STQ1_ERR_ARG;
+  if (mode == STQ1_ENC_SHERRY && (rounds < 0 || rounds > 1000)) return STQ1_ERR_ARG;
+  if (N > (1LL << 40) / K) return STQ1_ERR_SHAPE;
+  if (!aligned16(W) || (reinterpret_cast<uintptr_t>(out) & 1)) return STQ1_ERR_ALIGN;
+  const long long n_blocks = N * (K / kBlockWeights);
+  const long long grid = (n_blocks + kEncThreads - 1) / kEncThreads;
+  if (grid >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  int rc = ensure_configured();
+  if (rc != STQ1_OK) return rc;
+  return launch_pdl(encode_kernel, static_cast<unsigned>(grid), kEncThreads, encode_smem_bytes(),
+                    static_cast<cudaStream_t>(stream), W, h, n_blocks, static_cast<int>(K / kBlockWeights), mode,
+                    rounds, out);
 }
 
 extern "C" int stq1_quantize_x_e4m3(const uint16_t* x, int64_t T, int64_t K, uint8_t* q, float* scales,

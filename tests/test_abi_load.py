@@ -56,6 +56,12 @@ def test_host_side_argument_checks_need_no_gpu():
     # instead of 2) plus the per-token copy and the scales
     bf, f8 = L.stq1_moe_workspace(4096, 8, 256, 4096, 7168, 0), L.stq1_moe_workspace(4096, 8, 256, 4096, 7168, 2)
     assert f8 == bf - 32768 * 7168 + 4096 * 7168 + 4096 * 4 + 32768 * 4
+    assert L.stq1_quantize(None, None, 4, 256, 0, 3, 1 << 20, None) == -2
+    assert L.stq1_quantize(1 << 20, None, 4, 300, 0, 3, 1 << 20, None) == -1
+    assert L.stq1_quantize(1 << 20, None, 4, 256, 7, 3, 1 << 20, None) == -8
+    assert L.stq1_quantize(1 << 20, None, 4, 256, 1, -1, 1 << 20, None) == -8
+    assert L.stq1_quantize((1 << 20) + 4, None, 4, 256, 0, 3, 1 << 20, None) == -6
+    assert L.stq1_quantize(1 << 20, None, 4, 256, 0, 3, (1 << 20) + 1, None) == -6
     assert L.stq1_quantize_x_e4m3(None, 4, 256, 1 << 20, 1 << 20, None) == -2
     assert L.stq1_quantize_x_e4m3(1 << 20, 4, 250, 1 << 20, 1 << 20, None) == -1
     assert L.stq1_quantize_x_e4m3(1 << 20, 0, 256, 1 << 20, 1 << 20, None) == -1
