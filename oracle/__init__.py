@@ -13,4 +13,5 @@ from .stq1 import (  # noqa: F401
     encode_plain, encode_sherry, wls_scale, zero_lane_choice, weighted_error,
     decode, dequant_bf16, gemv, gemv_abs, tolerance, route_pairs, moe_gateup,
     half_from_struct, E4M3_MAX, e4m3_value, e4m3_round, quantize_x_e4m3, moe_gateup_fp8,
+    bf16_bits_from_f64, silu, swiglu_bf16, moe_combine, moe_ffn,
 )

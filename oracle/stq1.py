@@ -68,6 +68,13 @@ design notes):
    and saturated at +/-448 (OCP FP8 E4M3: no infinities, 0x7F / 0xFF NaN),
    and y = s_t * W^ q_t with q_t the codes' values.  Weights stay exact
    (+/-1 and 0 are e4m3 values, d is applied in fp32).
+8. After gate/up (the pages stop there; the steps below are the plain reading
+   of a gated MoE feed-forward): act = SiLU(g) * u with g = y[:, :N/2],
+   u = y[:, N/2:] and SiLU(v) = v / (1 + e^-v), evaluated in fp64 and
+   rounded once to bf16 (nearest, ties to even) because it is the bf16 input
+   of the down projection; the down projection is the same STQ1_0 matmul per
+   routed (token, slot) pair; the combine is sum_s w[t, s] * y_down[t, s]
+   (or the plain sum when the weights were applied to the up half).
 """
 
 from __future__ import annotations
@@ -509,6 +516,79 @@ def moe_gateup_fp8(expert_packed, x_bits: np.ndarray, ids: np.ndarray, weights: 
     codes, s = quantize_x_e4m3(np.asarray(x_bits).reshape(-1, k))
     xq = e4m3_value(codes) * s.astype(np.float64)[:, None]
     return _moe_from_f64(expert_packed, xq, ids, weights, n, k, flags, abs_sum)
+
+
+# ---------------------------------------------------------------------------
+# After gate/up: SwiGLU, down projection, combine (reading 8)
+# ---------------------------------------------------------------------------
+
+
+def bf16_bits_from_f64(x) -> np.ndarray:
+    """fp64 -> bf16 bits directly (no fp32 step): nearest, ties to even; 8 significant
+    bits, exponent range of fp32, subnormal quantum 2^-133; overflow to +/-inf."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    sign = np.where(np.signbit(x), 0x8000, 0).astype(np.int64)
+    _, ex = np.frexp(a)
+    e = np.maximum(ex - 1, -126)               # a in [2^e, 2^(e+1)), subnormals share 2^-126's step
+    step = np.exp2(e - 7.0)
+    q = np.rint(a / step) * step               # ties to the even multiple
+    _, qx = np.frexp(q)
+    qe = qx - 1
+    normal = q >= 2.0 ** -126
+    man = np.where(normal, q / np.exp2(qe.astype(np.float64)) * 128.0 - 128.0, q / 2.0 ** -133)
+    bits = np.where(normal, ((qe + 127).astype(np.int64) << 7) | np.rint(man).astype(np.int64),
+                    np.rint(man).astype(np.int64))
+    bits = np.where(q == 0, 0, bits)
+    bits = np.where(q >= 2.0 ** 128, 0x7F80, bits)
+    return (bits | sign).astype(np.uint16)
+
+
+def silu(v) -> np.ndarray:
+    """SiLU(v) = v / (1 + e^-v) in fp64."""
+    v = np.asarray(v, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return v / (1.0 + np.exp(-v))
+
+
+def swiglu_bf16(y: np.ndarray, n: int) -> np.ndarray:
+    """Fused gate/up rows y [P, n] (fp64 or fp32) -> act bf16 bits [P, n/2] = bf16(SiLU(g) * u)."""
+    y = np.asarray(y, dtype=np.float64).reshape(-1, n)
+    g, u = y[:, : n // 2], y[:, n // 2:]
+    return bf16_bits_from_f64(silu(g) * u)
+
+
+def moe_combine(y_down: np.ndarray, weights) -> np.ndarray:
+    """[T, topk, H] -> [T, H]: sum over slots, weighted by weights[t, s] when given (fp64)."""
+    yd = np.asarray(y_down, dtype=np.float64)
+    if weights is None:
+        return yd.sum(axis=1)
+    w = np.asarray(weights, dtype=np.float32).astype(np.float64)
+    return np.einsum("ts,tsh->th", w, yd)
+
+
+def moe_ffn(gateup_packed, down_packed, x_bits, ids, weights, n: int, hidden: int, flags: int = 0,
+            abs_sum: bool = False):
+    """Routed MoE feed-forward: gate/up -> SwiGLU (bf16) -> down -> combine, fp64 (reading 8).
+
+    ``flags`` bit 0 applies the routing weight to the up half (and the combine is then a plain sum);
+    otherwise the combine applies it.  With ``abs_sum`` also returns sum|W_down act| * |w| summed
+    over slots, the scale of the tolerance for the final output.
+    """
+    ids = np.asarray(ids)
+    T, topk = ids.shape
+    y = moe_gateup(gateup_packed, x_bits, ids, weights, n, hidden, flags=flags)
+    act = swiglu_bf16(y.reshape(T * topk, n), n)             # [P, n/2] bf16 bits
+    flat_ids = ids.reshape(T * topk, 1)
+    yd, ya = moe_gateup(down_packed, act, flat_ids, None, hidden, n // 2, abs_sum=True)
+    yd = yd.reshape(T, topk, hidden)
+    ya = ya.reshape(T, topk, hidden)
+    w = None if flags & FLAG_WEIGHT_UP else weights
+    out = moe_combine(yd, w)
+    if not abs_sum:
+        return out
+    wa = np.ones((T, topk)) if w is None else np.abs(np.asarray(w, dtype=np.float32).astype(np.float64))
+    return out, np.einsum("ts,tsh->th", wa, ya)
 
 
 def half_from_struct(x: float) -> int:

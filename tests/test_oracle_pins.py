@@ -499,6 +499,121 @@ def test_planted_fp8_mistakes_are_caught(monkeypatch, mistake):
 
 
 # ---------------------------------------------------------------------------
+# After gate/up: SwiGLU, combine, the MoE feed-forward chain
+# ---------------------------------------------------------------------------
+
+
+def _bf16_val(bits):
+    # bf16 is the top half of an fp32 word (format definition)
+    return (np.asarray(bits, np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_bf16_from_f64_is_nearest_with_ties_to_even():
+    rng = np.random.default_rng(93)
+    base = np.concatenate([rng.standard_normal(4000) * 10.0 ** rng.integers(-30, 30, 4000),
+                           rng.uniform(-1e-38, 1e-38, 500)])
+    # exact ties between neighbouring bf16 values, and values a hair off them
+    b = rng.integers(0x0001, 0x7F7F, 500).astype(np.uint32)
+    mids = (_bf16_val(b) + _bf16_val(b + 1)) / 2
+    vals = np.concatenate([base, mids, -mids, np.nextafter(mids, 0), np.nextafter(mids, np.inf)])
+    bits = oracle.bf16_bits_from_f64(vals).astype(np.uint32)
+    mag = bits & 0x7FFF
+    here = np.abs(np.abs(vals) - _bf16_val(mag))
+    lo = np.abs(np.abs(vals) - _bf16_val(np.maximum(mag, 1) - 1))
+    hi = np.abs(np.abs(vals) - _bf16_val(mag + 1))
+    assert np.all(here <= lo) and np.all(here <= hi)
+    tie = (here == hi) | ((here == lo) & (mag > 0))
+    assert np.all(mag[tie] % 2 == 0)
+    assert np.array_equal(bits >> 15, np.signbit(vals).astype(np.uint32))
+    # agrees with the fp32 rounding routine wherever the value is an fp32
+    f32 = rng.standard_normal(5000).astype(np.float32)
+    assert np.array_equal(oracle.bf16_bits_from_f64(f32.astype(np.float64)), oracle.bf16_bits_rne(f32))
+
+
+def test_silu_against_logistic_and_identities():
+    special = pytest.importorskip("scipy.special")
+    v = np.linspace(-40, 40, 4001)
+    s = oracle.silu(v)
+    assert np.allclose(s, v * special.expit(v), rtol=1e-14, atol=1e-300)
+    assert oracle.silu(np.array([0.0]))[0] == 0.0
+    assert np.allclose(oracle.silu(-v), s - v, rtol=1e-12, atol=1e-12)   # SiLU(-v) = SiLU(v) - v
+    assert abs(oracle.silu(np.array([60.0]))[0] - 60.0) < 1e-20
+
+
+def test_swiglu_pairs_gate_with_up():
+    n = 8
+    y = np.zeros((2, n))
+    y[0, :4] = [0.0, 30.0, -30.0, 1.0]      # gates
+    y[0, 4:] = [5.0, 2.0, 3.0, 4.0]         # ups
+    y[1, :4] = 1.0
+    y[1, 4:] = [1.0, -1.0, 0.5, 0.0]
+    act = oracle.swiglu_bf16(y, n)
+    vals = _bf16_val(act)
+    s1 = 1.0 / (1.0 + np.exp(-1.0))
+    assert vals[0, 0] == 0.0 and vals[0, 1] == 60.0 and abs(vals[0, 2]) < 1e-9
+    assert vals[0, 3] == _bf16_val(oracle.bf16_bits_from_f64(np.array([4 * s1])))[0]
+    assert np.allclose(vals[1], [s1, -s1, s1 / 2, 0.0], rtol=2 ** -8)
+
+
+def test_moe_combine_weights_slots():
+    yd = np.arange(2 * 3 * 4, dtype=np.float64).reshape(2, 3, 4)
+    assert np.array_equal(oracle.moe_combine(yd, None), yd.sum(axis=1))
+    w = np.array([[0, 1, 0], [0.5, 0, 0.25]], np.float32)
+    got = oracle.moe_combine(yd, w)
+    assert np.array_equal(got[0], yd[0, 1]) and np.allclose(got[1], 0.5 * yd[1, 0] + 0.25 * yd[1, 2])
+
+
+def test_moe_ffn_equals_the_chain_of_single_matmuls():
+    # gate/up and down through oracle.gemv per (token, slot) pair instead of the grouped path
+    n, hidden, E, T, topk = 512, 256, 3, 3, 2
+    gu = [oracle.encode_plain(workloads.gaussian_matrix(n, hidden, 0.05, seed=600 + e)) for e in range(E)]
+    dn = [oracle.encode_plain(workloads.gaussian_matrix(hidden, n // 2, 0.05, seed=700 + e)) for e in range(E)]
+    x = workloads.activations_bf16(T, hidden, seed=94)
+    ids = workloads.zipf_topk_ids(T, E, topk, seed=95)
+    wts = workloads.softmax_route_weights(T, topk, seed=96)
+    out = oracle.moe_ffn(gu, dn, x, ids, wts, n, hidden)
+    ref = np.zeros((T, hidden))
+    for t in range(T):
+        for s in range(topk):
+            e = int(ids[t, s])
+            y = oracle.gemv(gu[e], x[t:t + 1], n, hidden)[0]
+            act = oracle.swiglu_bf16(y[None, :], n)
+            ref[t] += np.float64(np.float32(wts[t, s])) * oracle.gemv(dn[e], act, hidden, n // 2)[0]
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-12)
+    # weights on the up half instead: SiLU(g) * (w u) = w SiLU(g) u up to the bf16 rounding of act
+    # (bf16 rounding of act, up to 2^-9 relative per element, against sum |w W act|)
+    out_up = oracle.moe_ffn(gu, dn, x, ids, wts, n, hidden, flags=oracle.FLAG_WEIGHT_UP)
+    _, scale = oracle.moe_ffn(gu, dn, x, ids, wts, n, hidden, abs_sum=True)
+    assert np.all(np.abs(out_up - out) <= 2 ** -8 * scale + 1e-9)
+
+
+@pytest.mark.parametrize("mistake", ["swap_gate_up", "silu_sign", "combine_unweighted"])
+def test_planted_ffn_mistakes_are_caught(monkeypatch, mistake):
+    import oracle.stq1 as o
+    def passes():
+        try:
+            test_silu_against_logistic_and_identities()
+            test_swiglu_pairs_gate_with_up()
+            test_moe_combine_weights_slots()
+        except AssertionError:
+            return False
+        return True
+    assert passes()
+    def plant(name, fn):                     # in the module and in the package's re-export
+        monkeypatch.setattr(o, name, fn)
+        monkeypatch.setattr(oracle, name, fn)
+    if mistake == "swap_gate_up":
+        orig = o.swiglu_bf16
+        plant("swiglu_bf16", lambda y, n: orig(np.concatenate(
+            [np.asarray(y, np.float64).reshape(-1, n)[:, n // 2:], np.asarray(y, np.float64).reshape(-1, n)[:, :n // 2]], 1), n))
+    elif mistake == "silu_sign":
+        plant("silu", lambda v: np.asarray(v, np.float64) / (1.0 + np.exp(np.asarray(v, np.float64))))
+    elif mistake == "combine_unweighted":
+        plant("moe_combine", lambda yd, w: np.asarray(yd, np.float64).sum(axis=1))
+    assert not passes()
+
+
+# ---------------------------------------------------------------------------
 # The pins catch planted mistakes
 # ---------------------------------------------------------------------------
 
