@@ -235,6 +235,12 @@ def run_gpu(args):
     # --- MoE decode gate/up (16 tokens, top-8 of 256 experts) ---
     moe = run_moe(torch, stq1, device, stream, args, world, timed)
 
+    # --- a whole routed MoE feed-forward layer at decode ---
+    try:
+        ffn = run_moe_ffn(torch, stq1, device, stream, args, world, timed)
+    except Exception as exc:  # reported, never hidden
+        ffn = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     # --- MoE prefill gate/up on the tensor-core tile path (4096 tokens) ---
     try:
         prefill = run_prefill(torch, stq1, device, stream, args, world, timed, bf16_peak)
@@ -275,6 +281,7 @@ def run_gpu(args):
         "gemv_batches": batches,
         "moe_decode": moe,
         "moe_prefill": prefill,
+        "moe_ffn_decode": ffn,
         "encoder": encoder,
         "e2e": e2e,
         "gpu_launches": args.steps * STACK,
@@ -315,17 +322,49 @@ def run_moe(torch, stq1, device, stream, args, world, timed):
             "config": "256 experts x [4096, 7168] STQ1_0, 16 tokens, Zipf(1.1) top-8, unweighted"}
 
 
-def _random_expert_bank(torch, device, E, seed):
-    """E random but valid [4096, 7168] STQ1_0 matrices on the device: uniform code
-    bytes, fp16 scales near 0.058 (the amax of 256 N(0, 0.02^2) weights)."""
-    flat = torch.empty(E * PACKED, dtype=torch.uint8, device=device)
+def _random_expert_bank(torch, device, E, seed, packed=None, d_mean=0.058):
+    """E random but valid STQ1_0 matrices (default [4096, 7168]) on the device:
+    uniform code bytes, fp16 scales near d_mean (0.058 = the amax of 256
+    N(0, 0.02^2) weights)."""
+    packed = PACKED if packed is None else packed
+    flat = torch.empty(E * packed, dtype=torch.uint8, device=device)
     g = torch.Generator(device=device)
     g.manual_seed(seed)
-    flat.copy_(torch.randint(0, 256, (E * PACKED,), dtype=torch.uint8, device=device, generator=g))
+    flat.copy_(torch.randint(0, 256, (E * packed,), dtype=torch.uint8, device=device, generator=g))
     blk = flat.view(-1, 42)
-    d = (0.058 * (1 + 0.1 * torch.randn(blk.shape[0], device=device, generator=g))).to(torch.float16)
+    d = (d_mean * (1 + 0.1 * torch.randn(blk.shape[0], device=device, generator=g))).to(torch.float16)
     blk[:, 0:2].copy_(d.view(torch.uint8).view(-1, 2))
     return flat
+
+
+def run_moe_ffn(torch, stq1, device, stream, args, world, timed):
+    """A routed MoE feed-forward layer at decode: 16 tokens, top-8 of 256 experts,
+    gate/up [4096, 7168] -> SwiGLU -> down [7168, 2048] -> combine."""
+    import workloads
+    E, n, hidden = 256, N_ROWS, K_COLS
+    gu = _random_expert_bank(torch, device, E, 2024)
+    down_packed = hidden * (n // 2) // 256 * 42
+    dn = _random_expert_bank(torch, device, E, 2025, packed=down_packed, d_mean=0.004)
+    x, ids, wts = workloads.moe_decode_inputs()
+    xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    idd = torch.from_numpy(ids).to(device)
+    wd = torch.from_numpy(wts).to(device)
+    out = torch.empty((16, hidden), dtype=torch.float32, device=device)
+    ws = stq1.workspace(stq1.LIB.stq1_moe_ffn_workspace(16, 8, E, n, hidden, 0), device, kind="ffn")
+
+    def step():
+        stq1.moe_ffn(gu, dn, xd, idd, wd, n, hidden, E, out=out, ws=ws)
+
+    steps = max(1, args.steps // 8)
+    gm = time_graph(torch, step, steps, 3, stream)
+    ms = timed(gm, steps) / steps
+    uniq = len(np.unique(ids))
+    del gm
+    return {"tokens_per_s": round(world * 16 / (ms * 1e-3), 1), "ms_per_call": round(ms, 4),
+            "expert_bytes_read": int(uniq * (PACKED + down_packed)),
+            "gbs": round(uniq * (PACKED + down_packed) / (ms * 1e-3) / 1e9, 1),
+            "config": "256 experts, gate/up [4096, 7168] + down [7168, 2048] STQ1_0, 16 tokens, Zipf(1.1) "
+                      "top-8, SwiGLU (bf16) and routing-weighted combine"}
 
 
 def run_prefill(torch, stq1, device, stream, args, world, timed, bf16_peak):
@@ -564,7 +603,8 @@ def kernel_source_digest():
     """SHA-256 over the table kernel's sources: a DRAM-traffic figure recorded
     for an older version of the kernel no longer applies."""
     h = hashlib.sha256()
-    for rel in ("sub_bit_sparse_b200/csrc/gemv_lut.cuh", "sub_bit_sparse_b200/csrc/device_common.cuh"):
+    for rel in ("sub_bit_sparse_b200/csrc/gemv_lut.cuh", "sub_bit_sparse_b200/csrc/packed_copy.cuh",
+                "sub_bit_sparse_b200/csrc/device_common.cuh"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()

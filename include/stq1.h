@@ -204,6 +204,55 @@ int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, const int32_t*
                     int64_t K, int flags, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * stq1_swiglu -- the gated activation after a fused gate/up projection (the
+ * pages stop at gate/up; this is the plain reading of a gated MoE FFN):
+ * act[p, j] = bf16(SiLU(y[p, j]) * y[p, N/2 + j]), SiLU(v) = v / (1 + e^-v),
+ * evaluated in fp64 and rounded once to bf16 (nearest, ties to even), ready to
+ * be the bf16 input of the down projection.
+ *   y    device, [P, N] fp32 (gate rows 0..N/2-1, then up rows), e.g. the
+ *        [T, topk, N] output of stq1_moe_gateup with P = T * topk.
+ *   act  device, [P, N/2] bf16 bits (fully overwritten).
+ * Requires N even.  Asynchronous on `stream`.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_CUDA.
+ */
+int stq1_swiglu(const float* y, uint16_t* act, int64_t P, int64_t N, void* stream);
+
+/*
+ * stq1_moe_combine -- out[t, h] = sum_s w[t, s] * y[t, s, h] in fp32, slots in
+ * order (the plain sum when w is NULL, e.g. when the routing weight was
+ * applied to the up half with STQ1_MOE_WEIGHT_UP).
+ *   y    device, [T, topk, H] fp32;  w  device, [T, topk] fp32 or NULL;
+ *   out  device, [T, H] fp32 (fully overwritten).
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_CUDA.
+ */
+int stq1_moe_combine(const float* y, const float* w, float* out, int64_t T, int topk, int64_t H,
+                     void* stream);
+
+/*
+ * stq1_moe_ffn_workspace / stq1_moe_ffn -- a routed MoE feed-forward layer:
+ * gate/up (stq1_moe_gateup) -> SwiGLU (stq1_swiglu) -> down projection per
+ * routed (token, slot) pair (stq1_moe_gateup with each pair as its own token)
+ * -> combine (stq1_moe_combine), all on `stream`.
+ *   gateup_blocks  device, E consecutive [N, H] STQ1_0 matrices (gate rows
+ *                  0..N/2-1, up rows N/2..N-1).
+ *   down_blocks    device, E consecutive [H, N/2] STQ1_0 matrices.
+ *   x              device, [T, H] bf16 bits.  topk_ids [T, topk] int32.
+ *   topk_weights   device, [T, topk] fp32; with STQ1_MOE_WEIGHT_UP applied to
+ *                  the up half (combine = plain sum), otherwise in the combine;
+ *                  NULL (without that flag) gives the unweighted sum.
+ *   out            device, [T, H] fp32 (fully overwritten).
+ *   flags          STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8 (fp8 applies to the tile
+ *                  path of both projections).
+ *   ws, ws_bytes   at least stq1_moe_ffn_workspace(...) bytes, 16-byte aligned.
+ * Requires N even, H and N/2 multiples of 256.
+ * Errors: as stq1_moe_gateup.
+ */
+size_t stq1_moe_ffn_workspace(int T, int topk, int E, int64_t N, int64_t H, int flags);
+int stq1_moe_ffn(const void* gateup_blocks, const void* down_blocks, const uint16_t* x,
+                 const int32_t* topk_ids, const float* topk_weights, float* out, int T, int topk, int E,
+                 int64_t N, int64_t H, int flags, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * stq1_quantize_x_e4m3 -- the activation quantization of the fp8 tile variant
  * (the pages have no fp8 step; this is the library's choice).  Per row t of
  * x: amax = max |x[t, k]|, inv = 448 / amax and scales[t] = amax / 448 (IEEE

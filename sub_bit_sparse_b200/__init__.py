@@ -54,6 +54,13 @@ SIGNATURES = {
     "stq1_set_path": (_c.c_int, [_c.c_int]),
     "stq1_gemv_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int,
                                      _c.c_void_p]),
+    "stq1_swiglu": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p]),
+    "stq1_moe_combine": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int, _c.c_int64,
+                                    _c.c_void_p]),
+    "stq1_moe_ffn_workspace": (_c.c_size_t, [_c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int]),
+    "stq1_moe_ffn": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                _c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
+                                _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "stq1_quantize": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int, _c.c_int,
                                  _c.c_void_p, _c.c_void_p]),
     "stq1_quantize_x_e4m3": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p, _c.c_void_p,
@@ -244,6 +251,59 @@ def moe_gateup(expert_blocks, x, topk_ids, topk_weights, n: int, k: int, n_exper
                              None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
                              _stream(x))
     _check("stq1_moe_gateup", rc)
+    return out
+
+
+def swiglu(y, n: int, out=None):
+    """fp32 [P, n] fused gate/up rows -> bf16 [P, n/2] = SiLU(gate) * up."""
+    torch = _torch()
+    _require(y, torch.float32, "y")
+    p = y.numel() // n
+    if out is None:
+        out = torch.empty((p, n // 2), dtype=torch.bfloat16, device=y.device)
+    _require(out, torch.bfloat16, "out")
+    _check("stq1_swiglu", _load().stq1_swiglu(y.data_ptr(), out.data_ptr(), p, n, _stream(y)))
+    return out
+
+
+def moe_combine(y, weights=None, out=None):
+    """fp32 [T, topk, H] -> [T, H], routing-weighted sum over slots (plain sum without weights)."""
+    torch = _torch()
+    _require(y, torch.float32, "y")
+    t, topk, h = y.shape
+    if weights is not None:
+        _require(weights, torch.float32, "weights")
+    if out is None:
+        out = torch.empty((t, h), dtype=torch.float32, device=y.device)
+    _require(out, torch.float32, "out")
+    rc = _load().stq1_moe_combine(y.data_ptr(), None if weights is None else weights.data_ptr(), out.data_ptr(),
+                                  t, topk, h, _stream(y))
+    _check("stq1_moe_combine", rc)
+    return out
+
+
+def moe_ffn(gateup_blocks, down_blocks, x, topk_ids, topk_weights, n: int, hidden: int, n_experts: int,
+            flags: int = 0, out=None, ws=None):
+    """Routed MoE feed-forward: gate/up -> SwiGLU -> down -> combine; returns fp32 [T, hidden]."""
+    torch = _torch()
+    _require(gateup_blocks, torch.uint8, "gateup_blocks")
+    _require(down_blocks, torch.uint8, "down_blocks")
+    _require(x, torch.bfloat16, "x")
+    _require(topk_ids, torch.int32, "topk_ids")
+    if topk_weights is not None:
+        _require(topk_weights, torch.float32, "topk_weights")
+    t, topk = topk_ids.shape
+    if out is None:
+        out = torch.empty((t, hidden), dtype=torch.float32, device=x.device)
+    _require(out, torch.float32, "out")
+    need = _load().stq1_moe_ffn_workspace(t, topk, n_experts, n, hidden, flags)
+    if ws is None:
+        ws = workspace(need, x.device, kind="ffn")
+    rc = _load().stq1_moe_ffn(gateup_blocks.data_ptr(), down_blocks.data_ptr(), x.data_ptr(), topk_ids.data_ptr(),
+                              None if topk_weights is None else topk_weights.data_ptr(), out.data_ptr(), t, topk,
+                              n_experts, n, hidden, flags, None if ws is None else ws.data_ptr(),
+                              0 if ws is None else ws.numel(), _stream(x))
+    _check("stq1_moe_ffn", rc)
     return out
 
 

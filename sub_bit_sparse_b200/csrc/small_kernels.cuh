@@ -176,4 +176,66 @@ direct_gemv_kernel(const uint8_t* __restrict__ W, long long expert_bytes, int E,
   }
 }
 
+// ---------------------------------------------------------------------------
+// After gate/up: SwiGLU and the top-k combine.
+// ---------------------------------------------------------------------------
+
+// fp64 -> bf16 bits, one rounding (nearest, ties to even): 8 significant bits,
+// exponent bias 127, subnormal quantum 2^-133, overflow to infinity.  ldexp is
+// exact and rint rounds ties to even.
+__device__ __forceinline__ uint16_t bf16_bits_from_f64(double x) {
+  const uint16_t sign = signbit(x) ? 0x8000u : 0u;
+  const double a = fabs(x);
+  if (isnan(x)) return 0x7FC0u;
+  if (a == 0.0) return sign;
+  int e = 0;
+  frexp(a, &e);                                   // a = m * 2^e, m in [0.5, 1)
+  int ex = e - 1;
+  if (ex >= -126) {
+    double q = rint(ldexp(a, 7 - ex));            // in [128, 256]
+    if (q >= 256.0) {
+      q = 128.0;
+      ex += 1;
+    }
+    if (ex > 127) return sign | 0x7F80u;
+    return sign | static_cast<uint16_t>(((ex + 127) << 7) | (static_cast<int>(q) - 128));
+  }
+  return sign | static_cast<uint16_t>(rint(ldexp(a, 133)));
+}
+
+// act[p, j] = bf16(SiLU(g) * u), g = y[p, j], u = y[p, half + j], SiLU(v) =
+// v / (1 + e^-v), in fp64 (the down projection's bf16 input, rounded once).
+__global__ void __launch_bounds__(256)
+swiglu_kernel(const float* __restrict__ y, uint16_t* __restrict__ act, long long P, int half) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const long long total = P * half;
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += 256LL * gridDim.x) {
+    const long long p = i / half;
+    const int j = static_cast<int>(i - p * half);
+    const double g = y[p * 2 * half + j];
+    const double u = y[p * 2 * half + half + j];
+    const double s = g / (1.0 + exp(-g));
+    act[i] = bf16_bits_from_f64(s * u);
+  }
+}
+
+// out[t, h] = sum_s w[t, s] * y[t, s, h] (plain sum without w), fp32 in slot order.
+__global__ void __launch_bounds__(256)
+combine_kernel(const float* __restrict__ y, const float* __restrict__ w, float* __restrict__ out, long long T,
+               int topk, int H) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const long long total = T * H;
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += 256LL * gridDim.x) {
+    const long long t = i / H;
+    const int h = static_cast<int>(i - t * H);
+    const float* yt = y + t * topk * H + h;
+    float acc = 0.f;
+    for (int s = 0; s < topk; ++s) acc = w ? fmaf(w[t * topk + s], yt[static_cast<long long>(s) * H], acc)
+                                           : acc + yt[static_cast<long long>(s) * H];
+    out[i] = acc;
+  }
+}
+
 }  // namespace stq1

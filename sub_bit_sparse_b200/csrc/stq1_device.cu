@@ -585,6 +585,83 @@ extern "C" int stq1_quantize_x_e4m3(const uint16_t* x, int64_t T, int64_t K, uin
                     x, static_cast<int>(K), q, scales);
 }
 
+extern "C" int stq1_swiglu(const float* y, uint16_t* act, int64_t P, int64_t N, void* stream) {
+  if (!y || !act) return STQ1_ERR_NULL;
+  if (P <= 0 || N <= 0 || (N & 1) || N > (1LL << 31) - 1 || P > (1LL << 40) / N) return STQ1_ERR_SHAPE;
+  const long long total = P * (N / 2);
+  const long long grid = std::min<long long>((total + 255) / 256, 148LL * 16);
+  return launch_pdl(swiglu_kernel, static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream), y, act, P,
+                    static_cast<int>(N / 2));
+}
+
+extern "C" int stq1_moe_combine(const float* y, const float* w, float* out, int64_t T, int topk, int64_t H,
+                                void* stream) {
+  if (!y || !out) return STQ1_ERR_NULL;
+  if (T <= 0 || topk <= 0 || H <= 0 || H > (1LL << 31) - 1 || T > (1LL << 40) / (H * topk)) return STQ1_ERR_SHAPE;
+  const long long total = T * H;
+  const long long grid = std::min<long long>((total + 255) / 256, 148LL * 16);
+  return launch_pdl(combine_kernel, static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream), y, w, out,
+                    static_cast<long long>(T), topk, static_cast<int>(H));
+}
+
+namespace stq1 {
+namespace {
+struct FfnPlan {
+  size_t ygu_off, act_off, yd_off, moe_off, moe_bytes, total;
+};
+FfnPlan plan_ffn(int T, int topk, int E, long long N, long long H, int flags) {
+  FfnPlan f{};
+  const long long P = static_cast<long long>(T) * topk;
+  size_t off = 0;
+  f.ygu_off = off;
+  off += round16(static_cast<size_t>(P) * N * sizeof(float));
+  f.act_off = off;
+  off += round16(static_cast<size_t>(P) * (N / 2) * sizeof(uint16_t));
+  f.yd_off = off;
+  off += round16(static_cast<size_t>(P) * H * sizeof(float));
+  f.moe_off = off;
+  f.moe_bytes = std::max(plan_moe(T, topk, E, H, flags).total, plan_moe(static_cast<int>(P), 1, E, N / 2, flags).total);
+  f.total = off + f.moe_bytes;
+  return f;
+}
+}  // namespace
+}  // namespace stq1
+
+extern "C" size_t stq1_moe_ffn_workspace(int T, int topk, int E, int64_t N, int64_t H, int flags) {
+  if (T <= 0 || topk <= 0 || E <= 0 || N <= 0 || (N & 1) || H <= 0 || H % kBlockWeights || (N / 2) % kBlockWeights)
+    return 0;
+  return plan_ffn(T, topk, E, N, H, flags).total;
+}
+
+extern "C" int stq1_moe_ffn(const void* gateup_blocks, const void* down_blocks, const uint16_t* x,
+                            const int32_t* topk_ids, const float* topk_weights, float* out, int T, int topk, int E,
+                            int64_t N, int64_t H, int flags, void* ws, size_t ws_bytes, void* stream) {
+  if (!gateup_blocks || !down_blocks || !x || !topk_ids || !out) return STQ1_ERR_NULL;
+  if (flags & ~(STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8)) return STQ1_ERR_ARG;
+  if (T <= 0 || topk <= 0 || E <= 0 || N <= 0 || (N & 1) || H <= 0 || H % kBlockWeights || (N / 2) % kBlockWeights ||
+      (H & 1) || static_cast<long long>(T) * topk > (1LL << 30))
+    return STQ1_ERR_SHAPE;
+  const FfnPlan f = plan_ffn(T, topk, E, N, H, flags);
+  if (!ws || ws_bytes < f.total) return STQ1_ERR_WORKSPACE;
+  if (!aligned16(ws)) return STQ1_ERR_ALIGN;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* ygu = reinterpret_cast<float*>(wsb + f.ygu_off);
+  uint16_t* act = reinterpret_cast<uint16_t*>(wsb + f.act_off);
+  float* yd = reinterpret_cast<float*>(wsb + f.yd_off);
+  const int P = T * topk;
+  // gate/up per (token, slot) pair; the routing weight goes on the up half or into the combine
+  int rc = stq1_moe_gateup(gateup_blocks, x, topk_ids, topk_weights, ygu, T, topk, E, N, H, flags, wsb + f.moe_off,
+                           f.moe_bytes, stream);
+  if (rc != STQ1_OK) return rc;
+  rc = stq1_swiglu(ygu, act, P, N, stream);
+  if (rc != STQ1_OK) return rc;
+  // down projection: each pair is its own token (ids [T, topk] read as [P, 1])
+  rc = stq1_moe_gateup(down_blocks, act, topk_ids, nullptr, yd, P, 1, E, H, N / 2, flags & STQ1_MOE_FP8,
+                       wsb + f.moe_off, f.moe_bytes, stream);
+  if (rc != STQ1_OK) return rc;
+  return stq1_moe_combine(yd, (flags & STQ1_MOE_WEIGHT_UP) ? nullptr : topk_weights, out, T, topk, H, stream);
+}
+
 extern "C" int stq1_set_path(int path) {
   if (path < 0 || path > 2) return STQ1_ERR_ARG;
   g_path = path;

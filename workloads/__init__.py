@@ -199,3 +199,16 @@ def random_packed_blocks(n_blocks: int, seed: int, d_sigma: float = 0.058) -> np
     d = (d_sigma * (1.0 + 0.1 * rng.standard_normal(n_blocks))).astype(np.float16)
     blocks[:, 0:2] = d.view(np.uint8).reshape(n_blocks, 2)
     return blocks.reshape(-1)
+
+
+def gateup_outputs(p: int, n: int, seed: int) -> np.ndarray:
+    """fp32 [p, n] stand-ins for fused gate/up outputs: N(0, 1) scaled per row by
+    10^U(-3, 2), with a few entries at +/-1e3 (exp underflow / overflow in SiLU)
+    and some exact zeros."""
+    rng = np.random.default_rng(seed)
+    y = rng.standard_normal((p, n)) * 10.0 ** rng.uniform(-3, 2, (p, 1))
+    flat = y.reshape(-1)
+    idx = rng.choice(flat.size, size=max(1, flat.size // 500), replace=False)
+    flat[idx] = rng.choice([-1e3, 1e3, 0.0], size=idx.size)
+    return y.astype(np.float32)
+
