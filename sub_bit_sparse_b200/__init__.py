@@ -83,6 +83,8 @@ _lib_lock = threading.Lock()
 def _load():
     """Loads libstq1.so once; raises ImportError if it is missing (no CPU fallback)."""
     global _lib
+    if _lib is not None:
+        return _lib
     with _lib_lock:
         if _lib is None:
             if not os.path.exists(LIB_PATH):
@@ -145,9 +147,15 @@ _ws_lock = threading.Lock()
 _ws_cache: dict = {}
 
 
+_torch_mod = None
+
+
 def _torch():
-    import torch
-    return torch
+    global _torch_mod
+    if _torch_mod is None:
+        import torch
+        _torch_mod = torch
+    return _torch_mod
 
 
 def workspace(nbytes: int, device, kind: str = "gemv") -> "torch.Tensor | None":
@@ -167,19 +175,31 @@ def workspace(nbytes: int, device, kind: str = "gemv") -> "torch.Tensor | None":
         return buf
 
 
+_raw_stream = None
+
+
 def _stream(t):
+    """The current CUDA stream of t's device, as the handle the C ABI takes."""
+    global _raw_stream
     torch = _torch()
-    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+    if _raw_stream is None:
+        # torch's raw getter skips building a Stream object (about 2 us per call);
+        # fall back to the public call if this torch lacks it
+        getter = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        _raw_stream = getter if getter is not None else (
+            lambda idx: torch.cuda.current_stream(idx).cuda_stream)
+    return _raw_stream(t.get_device())
 
 
 def _require(t, dtype, name):
+    if getattr(t, "dtype", None) is dtype and t.is_cuda and t.is_contiguous():
+        return
     torch = _torch()
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
+    raise ValueError(f"{name} must be contiguous")
 
 
 def dequant(w_packed, n: int, k: int, out=None):
@@ -203,10 +223,10 @@ def gemv(w_packed, x, n: int, k: int, out=None, ws=None):
     if out is None:
         out = torch.empty((b, n), dtype=torch.float32, device=x.device)
     _require(out, torch.float32, "out")
-    need = _load().stq1_gemv_workspace(n, k, b)
+    lib = _load()
     if ws is None:
-        ws = workspace(need, x.device)
-    rc = _load().stq1_gemv(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b,
+        ws = workspace(lib.stq1_gemv_workspace(n, k, b), x.device)
+    rc = lib.stq1_gemv(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b,
                        None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
                        _stream(x))
     _check("stq1_gemv", rc)

@@ -3,6 +3,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 #include <utility>
 
 #include <cudaTypedefs.h>
@@ -212,6 +213,54 @@ int make_packed_maps(PackedMaps* m, PackedGeom* g, const uint8_t* W, long long r
   return STQ1_OK;
 }
 
+// Encoded maps are a pure function of (device, buffer address, rows, row bytes,
+// extra super-row): a direct-mapped cache saves re-encoding them on every call
+// (a call on the same matrix is the common case).  An entry stays correct even
+// if the buffer is freed and the address reused with the same shape, since a
+// map only describes an address and a shape.
+struct MapCacheEntry {
+  const void* base;
+  long long rows, rowbytes;
+  int dev;
+  bool extra, valid;
+  PackedMaps maps;
+  PackedGeom g;
+};
+constexpr int kMapCacheSize = 1024;
+MapCacheEntry g_map_cache[kMapCacheSize];
+std::mutex g_map_mutex;
+
+int packed_maps_cached(PackedMaps* m, PackedGeom* g, const uint8_t* W, long long rows_total, long long rowbytes,
+                       bool extra_srow) {
+  const int dev = current_device();
+  const uint64_t h = (reinterpret_cast<uintptr_t>(W) >> 4) * 0x9E3779B97F4A7C15ull ^
+                     static_cast<uint64_t>(rows_total) * 0xC2B2AE3D27D4EB4Full ^ static_cast<uint64_t>(rowbytes) ^
+                     (static_cast<uint64_t>(dev) << 1) ^ (extra_srow ? 1u : 0u);
+  MapCacheEntry& e = g_map_cache[(h >> 32) % kMapCacheSize];
+  {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    if (e.valid && e.base == W && e.rows == rows_total && e.rowbytes == rowbytes && e.dev == dev &&
+        e.extra == extra_srow) {
+      *m = e.maps;
+      *g = e.g;
+      return STQ1_OK;
+    }
+  }
+  const int rc = make_packed_maps(m, g, W, rows_total, rowbytes, extra_srow);
+  if (rc == STQ1_OK) {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    e.base = W;
+    e.rows = rows_total;
+    e.rowbytes = rowbytes;
+    e.dev = dev;
+    e.extra = extra_srow;
+    e.maps = *m;
+    e.g = *g;
+    e.valid = true;
+  }
+  return rc;
+}
+
 // K split of n_chunks chunks into S pieces (split s: cq chunks, one more if s < cr).
 void set_split(LutArgs* a, int n_chunks, int S) {
   a->S = S;
@@ -339,7 +388,7 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
     if (!make_b_map(&map, x, batch, K, false)) return STQ1_ERR_CUDA;
     TcArgs t{};
     PackedMaps pm;
-    rc = make_packed_maps(&pm, &t.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
+    rc = packed_maps_cached(&pm, &t.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
     if (rc != STQ1_OK) return rc;
     t.y = y;
     t.tile_info = nullptr;
@@ -367,7 +416,7 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
   }
   LutArgs a{};
   PackedMaps maps;
-  rc = make_packed_maps(&maps, &a.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
+  rc = packed_maps_cached(&maps, &a.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
   if (rc != STQ1_OK) return rc;
   a.x = x;
   a.y = y;
@@ -505,7 +554,7 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
     if (!make_b_map(&map, xperm, n_pairs, K, m.fp8)) return STQ1_ERR_CUDA;
     TcArgs t{};
     PackedMaps pm;
-    rc = make_packed_maps(&pm, &t.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
+    rc = packed_maps_cached(&pm, &t.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
                           rowbytes, N % residue_period(rowbytes) != 0);
     if (rc != STQ1_OK) return rc;
     t.y = y;
@@ -529,7 +578,7 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   LutArgs a{};
   PackedMaps maps;
   const int P = residue_period(rowbytes);
-  rc = make_packed_maps(&maps, &a.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
+  rc = packed_maps_cached(&maps, &a.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
                      rowbytes, N % P != 0);
   if (rc != STQ1_OK) return rc;
   a.x = x;
@@ -757,7 +806,7 @@ extern "C" int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float*
   }
   LutArgs a{};
   PackedMaps maps;
-  rc = make_packed_maps(&maps, &a.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
+  rc = packed_maps_cached(&maps, &a.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
   if (rc != STQ1_OK) return rc;
   a.x = x;
   a.y = y;
