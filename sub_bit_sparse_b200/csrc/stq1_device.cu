@@ -312,6 +312,8 @@ void plan_table(GemvPlan* p, long long N, long long K, int batch, bool one_wave)
   const int logP = P == 1 ? 0 : (P == 2 ? 1 : 2);
   const int stage = packed_stage_bytes(logP, kLutRows >> logP);
   const long long slots_sm = smem_per_sm();
+  // the split-K partials meet inside one thread-block cluster (at most 16 CTAs)
+  if (one_wave) S = std::min<long long>(S, kMaxClusterRanks);
   for (; one_wave && S > 1; --S) {
     const int cq = static_cast<int>(p->n_chunks / S), cr = static_cast<int>(p->n_chunks % S);
     const int stages = cq + (cr > 0 ? 1 : 0) >= 2 ? 2 : 1;

@@ -56,6 +56,15 @@ def test_host_side_argument_checks_need_no_gpu():
     # instead of 2) plus the per-token copy and the scales
     bf, f8 = L.stq1_moe_workspace(4096, 8, 256, 4096, 7168, 0), L.stq1_moe_workspace(4096, 8, 256, 4096, 7168, 2)
     assert f8 == bf - 32768 * 7168 + 4096 * 7168 + 4096 * 4 + 32768 * 4
+    # empty inputs are shape errors, never launches
+    assert L.stq1_gemv(1 << 20, 1 << 20, 1 << 20, 0, 256, 1, None, 0, None) == -1
+    assert L.stq1_moe_gateup(1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 0, 2, 4, 64, 256, 0, None, 0, None) == -1
+    assert L.stq1_swiglu(1 << 20, 1 << 20, 0, 64, None) == -1
+    assert L.stq1_swiglu(1 << 20, 1 << 20, 4, 63, None) == -1
+    assert L.stq1_moe_combine(1 << 20, None, 1 << 20, 0, 8, 64, None) == -1
+    assert L.stq1_moe_ffn(1 << 20, 1 << 20, 1 << 20, 1 << 20, None, 1 << 20, 0, 8, 4, 512, 256, 0, None, 0,
+                          None) == -1
+    assert L.stq1_quantize(1 << 20, None, 0, 256, 0, 3, 1 << 20, None) == -1
     assert L.stq1_quantize(None, None, 4, 256, 0, 3, 1 << 20, None) == -2
     assert L.stq1_quantize(1 << 20, None, 4, 300, 0, 3, 1 << 20, None) == -1
     assert L.stq1_quantize(1 << 20, None, 4, 256, 7, 3, 1 << 20, None) == -8

@@ -225,3 +225,57 @@ def test_bad_arguments_enqueue_nothing():
     with pytest.raises(stq1.Stq1Error, match="ALIGN"):
         stq1.gemv(w[1:], x, 3, 256)
     assert stq1.status() == 0
+
+
+# ---------------------------------------------------------------------------
+# Largest sizes and degenerate cases
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("b", [1, 5])
+def test_gemv_long_rows(b):
+    # K = 65,536: 256 blocks per row (10,752 bytes, a multiple of 16: super-rows of one row)
+    n, k = 64, 65536
+    w = workloads.gaussian_matrix(n, k, 0.01, seed=4242)
+    packed = stq1.quantize_ref(w)
+    x = workloads.activations_bf16(b, k, seed=4243)
+    y = stq1.gemv(_dev(packed), _bf16(x), n, k).cpu().numpy()
+    _assert_close(y, oracle.gemv(packed, x, n, k), oracle.gemv_abs(packed, x, n, k), f"long rows b={b}")
+
+
+def test_gemv_largest_batch():
+    # batch 65,535 (the API's limit) on the tile path
+    n, k, b = 128, 256, 65535
+    packed = stq1.quantize_ref(workloads.gaussian_matrix(n, k, 0.05, seed=11))
+    x = workloads.activations_bf16(b, k, seed=12)
+    y = stq1.gemv(_dev(packed), _bf16(x), n, k).cpu().numpy()
+    _assert_close(y, oracle.gemv(packed, x, n, k), oracle.gemv_abs(packed, x, n, k), "batch 65535")
+
+
+def test_gemv_zero_weights_and_zero_activations():
+    n, k = 130, 1024
+    packed = stq1.quantize_ref(np.zeros((n, k), np.float32))          # every d = 0
+    x = workloads.activations_bf16(3, k, seed=5)
+    assert np.all(stq1.gemv(_dev(packed), _bf16(x), n, k).cpu().numpy() == 0)
+    packed = stq1.quantize_ref(workloads.gaussian_matrix(n, k, 0.02, seed=6))
+    z = np.zeros((2, k), np.uint16)
+    assert np.all(stq1.gemv(_dev(packed), _bf16(z), n, k).cpu().numpy() == 0)
+
+
+def test_moe_most_experts_the_library_takes():
+    # E = 4096 experts (the routing kernel's limit), a few tokens, top-8
+    n, k, E, T, topk = 128, 256, 4096, 3, 8
+    bank = workloads.random_packed_blocks(E * oracle.packed_size(n, k) // 42, seed=77)
+    x = workloads.activations_bf16(T, k, seed=78)
+    ids = workloads.zipf_topk_ids(T, E, topk, seed=79)
+    wts = workloads.softmax_route_weights(T, topk, seed=80)
+    _moe_check(bank, x, ids, wts, n, k, E, flags=1)
+
+
+def test_moe_one_token_every_expert():
+    n, k, E = 256, 512, 4
+    experts = [stq1.quantize_ref(workloads.gaussian_matrix(n, k, 0.02, seed=90 + e)) for e in range(E)]
+    x = workloads.activations_bf16(1, k, seed=91)
+    ids = np.arange(E, dtype=np.int32).reshape(1, E)
+    wts = np.full((1, E), 0.25, np.float32)
+    _moe_check(experts, x, ids, wts, n, k, E, flags=0)
