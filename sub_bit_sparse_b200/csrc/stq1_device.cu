@@ -68,7 +68,7 @@ bool make_b_map(CUtensorMap* map, const void* base, long long rows, long long K,
   const int esize = fp8 ? 1 : 2;
   cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * esize};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcStageBytesK / esize), static_cast<cuuint32_t>(kTcN)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcAtomBytes / esize), static_cast<cuuint32_t>(kTcN)};
   cuuint32_t estride[2] = {1, 1};
   return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
             const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,

@@ -8,9 +8,10 @@
 // accumulator, and CUDA cores add d_{j,b} * slab into an fp32 register
 // accumulator (a5 of the hot path, done once per row, slab and token).
 //
-// Tile: M = 128 weight rows x N = 128 tokens, K in 64-column stages.
-//   warp 0      TMA producer: x tiles (bf16, 128-byte swizzle) into a 4-stage
-//               shared ring (one 2-D tensor copy per stage, no multicast).
+// Tile: M = 128 weight rows x N = 128 tokens, K in stages of two 128-byte
+// swizzle atoms (128 bf16 or 256 E4M3 columns), eight MMAs per stage.
+//   warp 0      TMA producer: x tiles (128-byte swizzle) into a 4-stage shared
+//               ring (two 2-D tensor copies per stage, no multicast).
 //   warp 1      TMEM allocator and the single MMA-issuing thread:
 //               tcgen05.mma.cta_group::1.kind::f16, A from TMEM, B from shared.
 //   warp 18     TMA producer of the packed weights: per 128-row tile, chunks
@@ -28,7 +29,7 @@
 //               release of the TMEM buffer; at the end of the tile, coalesced
 //               stores of y.
 // TMEM (512 columns allocated, one CTA per SM): slab accumulators 2 x 128
-// columns, A stages 8 x 32 columns.  Shared memory: 8 x-tile stages of 16 KB
+// columns, A stages 4 x 64 columns.  Shared memory: 4 x-tile stages of 32 KB
 // and 4 packed-weight stages of up to 15 KB.
 // All waits are bounded; a timeout sets the device error word and makes every
 // role stop at its next wait, so the CTA always reaches the final barrier and
@@ -36,9 +37,9 @@
 //
 // fp8 variant (FP8 = true): x rows arrive as E4M3 codes with one fp32 scale
 // per row, the pattern is expanded to E4M3 +/-1 and 0 (one byte per weight,
-// a 32-bit word per group), the MMA is kind::f8f6f4, and a stage covers 128
-// columns (128 bytes, the same 32 TMEM columns and 16 KB x tile as a bf16
-// stage of 64 columns), so a scale block takes two stages instead of four.
+// a 32-bit word per group), the MMA is kind::f8f6f4, and a stage covers 256
+// columns (256 bytes, the same 64 TMEM columns and 32 KB x tile as a bf16
+// stage of 128 columns), so a scale block is one stage instead of two.
 // The row's scale multiplies the finished sum.
 #pragma once
 
@@ -52,22 +53,25 @@ namespace stq1 {
 
 constexpr int kTcM = 128;
 constexpr int kTcN = 128;
-constexpr int kTcStageBytesK = 128;           // bytes of x per row and stage
-constexpr int kTcKC = 64;                     // K per stage, bf16 (128 bytes)
-constexpr int kTcKC8 = 128;                   // K per stage, fp8 (128 bytes)
-constexpr int kTcStages = 8;
+constexpr int kTcAtomBytes = 128;             // one 128-byte swizzle atom of x per row
+constexpr int kTcAtoms = 2;                   // atoms per stage
+constexpr int kTcStageBytesK = kTcAtoms * kTcAtomBytes;   // 256 bytes of x per row and stage
+constexpr int kTcKC = 128;                    // K per stage, bf16
+constexpr int kTcKC8 = 256;                   // K per stage, fp8
+constexpr int kTcStages = 4;
+constexpr int kTcAStageCols = 64;             // TMEM columns of A per stage (256 bytes per lane)
 template <bool FP8>
 constexpr int tc_kc() { return FP8 ? kTcKC8 : kTcKC; }
 template <bool FP8>
-constexpr int tc_slab_chunks() { return kBlockWeights / tc_kc<FP8>(); }   // 4 (bf16) or 2 (fp8)
+constexpr int tc_slab_chunks() { return kBlockWeights / tc_kc<FP8>(); }   // 2 (bf16) or 1 (fp8)
 constexpr int kTcThreads = 608;
 constexpr int kTcAStages = 4;                    // packed-weight chunks in flight
 constexpr int kTcDecoders = 256;                 // threads: 8 warps
 constexpr int kTcEpilogue = 256;                 // threads: 8 warps
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcColD = 0;               // 2 x 128
-constexpr uint32_t kTcColA = 256;             // kTcStages x 32
-constexpr int kTcBStageBytes = kTcN * kTcStageBytesK;   // 16 KB
+constexpr uint32_t kTcColA = 256;             // kTcStages x 64
+constexpr int kTcBStageBytes = kTcN * kTcStageBytesK;   // 32 KB (two 16 KB atoms)
 // shared layout (offsets from a 1024-aligned base)
 constexpr int kTcOffB = 0;
 constexpr int kTcOffA = kTcStages * kTcBStageBytes;                // 131072: packed-weight ring
@@ -253,11 +257,12 @@ __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t 
                                                uint32_t bar_empty, uint32_t& it) {
 #pragma unroll
   for (int q = 0; q < tc_slab_chunks<FP8>(); ++q) {
-    uint32_t v[16];
+    uint32_t v[32];
+    // this half's qs words of the stage: bf16 2 words (16 groups, 2 columns each),
+    // fp8 4 words (32 groups, 1 column each)
 #pragma unroll
-    for (int w = 0; w < (FP8 ? 2 : 1); ++w) {
-      // qs word i: groups 8i .. 8i+7
-      const int i = FP8 ? 4 * q + 2 * HALF + w : 2 * q + HALF;
+    for (int w = 0; w < (FP8 ? 4 : 2); ++w) {
+      const int i = FP8 ? 4 * HALF + w : 4 * q + 2 * HALF + w;   // qs word i: groups 8i .. 8i+7
       const uint32_t hb = (i < 4 ? H0 : H1) >> (8 * (i & 3));
       const uint32_t ce = ((Q[i] << 2) & 0x3C3C3C3Cu) | (((hb & 0x55u) * 0x01041040u) & 0x40404040u);
       const uint32_t co = ((Q[i] >> 2) & 0x3C3C3C3Cu) | (((hb & 0xAAu) * 0x00820820u) & 0x40404040u);
@@ -278,10 +283,10 @@ __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t 
           asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(x1) : "r"(ae));
           asm volatile("ld.shared.u32 %0, [%1];" : "=r"(y0) : "r"(ao));
           asm volatile("ld.shared.u32 %0, [%1+128];" : "=r"(y1) : "r"(ao));
-          v[4 * m] = x0;
-          v[4 * m + 1] = x1;
-          v[4 * m + 2] = y0;
-          v[4 * m + 3] = y1;
+          v[16 * w + 4 * m] = x0;
+          v[16 * w + 4 * m + 1] = x1;
+          v[16 * w + 4 * m + 2] = y0;
+          v[16 * w + 4 * m + 3] = y1;
         }
       }
     }
@@ -289,7 +294,7 @@ __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t 
     const uint32_t use = it / kTcStages;
     if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) return false;
     tc_fence_after();
-    STQ1_TMEM_ST16(tmem_a_lane + kTcColA + 32 * s + 16 * HALF, v);
+    STQ1_TMEM_ST32(tmem_a_lane + kTcColA + kTcAStageCols * s + 32 * HALF, v);
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(bar_full_a + 8 * s);
@@ -372,7 +377,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
           const uint32_t s = it % kTcStages, use = it / kTcStages;
           if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) { *abort = 1; break; }
           mbar_arrive_expect_tx(bar_full_b + 8 * s, kTcBStageBytes);
-          tma_load_2d(sB + s * kTcBStageBytes, &tmap_b, kc * KC, b_row, bar_full_b + 8 * s);
+#pragma unroll
+          for (int at = 0; at < kTcAtoms; ++at)
+            tma_load_2d(sB + s * kTcBStageBytes + at * (kTcN * kTcAtomBytes), &tmap_b, kc * KC + at * (KC / kTcAtoms),
+                        b_row, bar_full_b + 8 * s);
         }
       }
       if (*abort) {
@@ -396,10 +404,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
             if (!mbar_wait_bounded(bar_full_b + 8 * s, use & 1) ||
                 !mbar_wait_bounded(bar_full_a + 8 * s, use & 1)) { *abort = 1; break; }
             tc_fence_after();
-            const uint64_t bdesc = smem_desc_sw128(sB + s * kTcBStageBytes);
 #pragma unroll
             for (int kk = 0; kk < kTcStageBytesK / 32; ++kk) {   // 32 bytes of K per MMA
-              tc_mma_ts<FP8>(d_tmem, tmem + kTcColA + 32 * s + 8 * kk, bdesc + 2 * kk, tc_idesc<FP8>(),
+              const uint64_t bdesc =
+                  smem_desc_sw128(sB + s * kTcBStageBytes + (kk >> 2) * (kTcN * kTcAtomBytes)) + 2 * (kk & 3);
+              tc_mma_ts<FP8>(d_tmem, tmem + kTcColA + kTcAStageCols * s + 8 * kk, bdesc, tc_idesc<FP8>(),
                              (q > 0 || kk > 0) ? 1u : 0u);
             }
             tc_commit(bar_empty + 8 * s);
