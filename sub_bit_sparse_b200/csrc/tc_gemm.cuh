@@ -54,27 +54,31 @@ namespace stq1 {
 constexpr int kTcM = 128;
 constexpr int kTcN = 128;
 constexpr int kTcAtomBytes = 128;             // one 128-byte swizzle atom of x per row
-constexpr int kTcAtoms = 2;                   // atoms per stage
-constexpr int kTcStageBytesK = kTcAtoms * kTcAtomBytes;   // 256 bytes of x per row and stage
-constexpr int kTcKC = 128;                    // K per stage, bf16
-constexpr int kTcKC8 = 256;                   // K per stage, fp8
-constexpr int kTcStages = 4;
-constexpr int kTcAStageCols = 64;             // TMEM columns of A per stage (256 bytes per lane)
+constexpr int kTcMaxStages = 4;
+// Pipeline geometry: a stage is one 256-column scale block of K, i.e. four
+// 128-byte atoms of bf16 x (two of E4M3), so 128 KB of x tiles and 256 TMEM
+// columns of A give 2 (bf16) or 4 (fp8) stages.
 template <bool FP8>
-constexpr int tc_kc() { return FP8 ? kTcKC8 : kTcKC; }
-template <bool FP8>
-constexpr int tc_slab_chunks() { return kBlockWeights / tc_kc<FP8>(); }   // 2 (bf16) or 1 (fp8)
+struct TcGeom {
+  static constexpr int atoms = FP8 ? 2 : 4;                  // swizzle atoms per stage
+  static constexpr int stages = 8 / atoms;
+  static constexpr int kc = kBlockWeights;                   // K per stage
+  static constexpr int a_cols = 32 * atoms;                  // TMEM columns of A per stage
+  static constexpr int b_stage_bytes = kTcN * kTcAtomBytes * atoms;
+  static constexpr int mmas = 4 * atoms;                     // 32 bytes of K per MMA
+};
+
 constexpr int kTcThreads = 608;
 constexpr int kTcAStages = 4;                    // packed-weight chunks in flight
 constexpr int kTcDecoders = 256;                 // threads: 8 warps
 constexpr int kTcEpilogue = 256;                 // threads: 8 warps
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcColD = 0;               // 2 x 128
-constexpr uint32_t kTcColA = 256;             // kTcStages x 64
-constexpr int kTcBStageBytes = kTcN * kTcStageBytesK;   // 32 KB (two 16 KB atoms)
+constexpr uint32_t kTcColA = 256;             // stages x a_cols = 256
+constexpr int kTcBRingBytes = 8 * kTcN * kTcAtomBytes;   // 128 KB of x tiles
 // shared layout (offsets from a 1024-aligned base)
 constexpr int kTcOffB = 0;
-constexpr int kTcOffA = kTcStages * kTcBStageBytes;                // 131072: packed-weight ring
+constexpr int kTcOffA = kTcBRingBytes;                             // 131072: packed-weight ring
 constexpr int kTcOffTable = kTcOffA + kTcAStages * kPackedStageMax; // 2 x 128 B decode tables
 static_assert(kTcOffTable % 256 == 0, "decode tables must be 256-aligned");
 constexpr int kTcOffBar = kTcOffTable + 256;
@@ -255,14 +259,18 @@ template <bool FP8, int HALF>
 __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t H0, uint32_t H1,
                                                uint32_t tables, uint32_t tmem_a_lane, uint32_t bar_full_a,
                                                uint32_t bar_empty, uint32_t& it) {
+  using G = TcGeom<FP8>;
+  const uint32_t s = it % G::stages;
+  const uint32_t use = it / G::stages;
+  bool waited = false;
+  // this half's 32 groups (qs words 4 * HALF .. 4 * HALF + 3) in pieces of 32 TMEM
+  // columns: bf16 two pieces of 16 groups (2 columns each), fp8 one of 32 groups
 #pragma unroll
-  for (int q = 0; q < tc_slab_chunks<FP8>(); ++q) {
+  for (int piece = 0; piece < (FP8 ? 1 : 2); ++piece) {
     uint32_t v[32];
-    // this half's qs words of the stage: bf16 2 words (16 groups, 2 columns each),
-    // fp8 4 words (32 groups, 1 column each)
 #pragma unroll
     for (int w = 0; w < (FP8 ? 4 : 2); ++w) {
-      const int i = FP8 ? 4 * HALF + w : 4 * q + 2 * HALF + w;   // qs word i: groups 8i .. 8i+7
+      const int i = 4 * HALF + (FP8 ? w : 2 * piece + w);      // qs word i: groups 8i .. 8i+7
       const uint32_t hb = (i < 4 ? H0 : H1) >> (8 * (i & 3));
       const uint32_t ce = ((Q[i] << 2) & 0x3C3C3C3Cu) | (((hb & 0x55u) * 0x01041040u) & 0x40404040u);
       const uint32_t co = ((Q[i] >> 2) & 0x3C3C3C3Cu) | (((hb & 0xAAu) * 0x00820820u) & 0x40404040u);
@@ -290,16 +298,17 @@ __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t 
         }
       }
     }
-    const uint32_t s = it % kTcStages;
-    const uint32_t use = it / kTcStages;
-    if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) return false;
-    tc_fence_after();
-    STQ1_TMEM_ST32(tmem_a_lane + kTcColA + kTcAStageCols * s + 32 * HALF, v);
-    tmem_wait_st();
-    tc_fence_before();
-    mbar_arrive(bar_full_a + 8 * s);
-    ++it;
+    if (!waited) {
+      if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) return false;
+      tc_fence_after();
+      waited = true;
+    }
+    STQ1_TMEM_ST32(tmem_a_lane + kTcColA + G::a_cols * s + (G::a_cols / 2) * HALF + 32 * piece, v);
   }
+  tmem_wait_st();
+  tc_fence_before();
+  mbar_arrive(bar_full_a + 8 * s);
+  ++it;
   return true;
 }
 
@@ -307,8 +316,8 @@ template <bool FP8>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap wmap,
                const __grid_constant__ CUtensorMap tmap_w, const TcArgs a) {
-  constexpr int KC = tc_kc<FP8>();
-  constexpr int kSlabChunks = tc_slab_chunks<FP8>();
+  using G = TcGeom<FP8>;
+  constexpr int KC = G::kc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
@@ -329,7 +338,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kTcStages; ++i) {
+    for (int i = 0; i < kTcMaxStages; ++i) {
       mbar_init(bar_full_b + 8 * i, 1);
       mbar_init(bar_full_a + 8 * i, kTcDecoders);
       mbar_init(bar_empty + 8 * i, 1);
@@ -374,19 +383,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
         const int tile = static_cast<int>(item / a.n_mtiles);
         const int b_row = a.tile_info ? a.tile_info[4 * tile + 1] : tile * kTcN;
         for (int kc = 0; kc < n_chunks; ++kc, ++it) {
-          const uint32_t s = it % kTcStages, use = it / kTcStages;
+          const uint32_t s = it % G::stages, use = it / G::stages;
           if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) { *abort = 1; break; }
-          mbar_arrive_expect_tx(bar_full_b + 8 * s, kTcBStageBytes);
+          mbar_arrive_expect_tx(bar_full_b + 8 * s, G::b_stage_bytes);
 #pragma unroll
-          for (int at = 0; at < kTcAtoms; ++at)
-            tma_load_2d(sB + s * kTcBStageBytes + at * (kTcN * kTcAtomBytes), &tmap_b, kc * KC + at * (KC / kTcAtoms),
+          for (int at = 0; at < G::atoms; ++at)
+            tma_load_2d(sB + s * G::b_stage_bytes + at * (kTcN * kTcAtomBytes), &tmap_b, kc * KC + at * (KC / G::atoms),
                         b_row, bar_full_b + 8 * s);
         }
       }
       if (*abort) {
         // let the last tensor copies land before the CTA can exit (bounded)
-        for (uint32_t j = it > kTcStages ? it - kTcStages : 0; j < it; ++j)
-          mbar_wait_bounded(bar_full_b + 8 * (j % kTcStages), (j / kTcStages) & 1);
+        for (uint32_t j = it > G::stages ? it - G::stages : 0; j < it; ++j)
+          mbar_wait_bounded(bar_full_b + 8 * (j % G::stages), (j / G::stages) & 1);
       }
     }
   } else if (warp == 1) {
@@ -399,19 +408,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
           if (!mbar_wait_bounded(bar_d_empty + 8 * p, (puse & 1) ^ 1)) { *abort = 1; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem + kTcColD + p * kTcN;
-          for (int q = 0; q < kSlabChunks; ++q, ++it) {
-            const uint32_t s = it % kTcStages, use = it / kTcStages;
+          {
+            const uint32_t s = it % G::stages, use = it / G::stages;
             if (!mbar_wait_bounded(bar_full_b + 8 * s, use & 1) ||
                 !mbar_wait_bounded(bar_full_a + 8 * s, use & 1)) { *abort = 1; break; }
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < kTcStageBytesK / 32; ++kk) {   // 32 bytes of K per MMA
+            for (int kk = 0; kk < G::mmas; ++kk) {
               const uint64_t bdesc =
-                  smem_desc_sw128(sB + s * kTcBStageBytes + (kk >> 2) * (kTcN * kTcAtomBytes)) + 2 * (kk & 3);
-              tc_mma_ts<FP8>(d_tmem, tmem + kTcColA + kTcAStageCols * s + 8 * kk, bdesc, tc_idesc<FP8>(),
-                             (q > 0 || kk > 0) ? 1u : 0u);
+                  smem_desc_sw128(sB + s * G::b_stage_bytes + (kk >> 2) * (kTcN * kTcAtomBytes)) + 2 * (kk & 3);
+              tc_mma_ts<FP8>(d_tmem, tmem + kTcColA + G::a_cols * s + 8 * kk, bdesc, tc_idesc<FP8>(),
+                             kk > 0 ? 1u : 0u);
             }
             tc_commit(bar_empty + 8 * s);
+            ++it;
           }
           if (*abort) break;
           tc_commit(bar_d_full + 8 * p);
