@@ -70,6 +70,7 @@ extern "C" {
 /* stq1_moe_gateup flags. */
 #define STQ1_MOE_WEIGHT_UP 1      /* multiply rows N/2..N-1 (the up half) by the routing weight */
 #define STQ1_MOE_FP8 2            /* tile path: E4M3 activations (per-token fp32 scale), fp8 MMAs */
+#define STQ1_MOE_SKIP_FOREIGN 4   /* ids outside [0, E) give y = 0 without an error (expert parallelism) */
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 int stq1_version(void);
@@ -182,10 +183,10 @@ size_t stq1_moe_workspace(int T, int topk, int E, int64_t N, int64_t K, int flag
  *                  (may be NULL otherwise).
  *   y              device, [T, topk, N] fp32 (fully overwritten; a slot whose
  *                  id is out of range is set to 0 and flagged in the error word).
- *   flags          STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8.
+ *   flags          STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8 | STQ1_MOE_SKIP_FOREIGN.
  *   ws, ws_bytes   device workspace, at least stq1_moe_workspace(...) bytes
  *                  (computed with the same flags).
- * Requires N even, K % 256 == 0, 1 <= topk <= E.
+ * Requires N even, K % 256 == 0, 1 <= topk <= E (any topk with STQ1_MOE_SKIP_FOREIGN).
  * Paths: with few token-slot pairs per routed expert (decode) the lookup-table
  * kernel runs; with many (prefill) the tensor-core tile kernel.
  * STQ1_MOE_FP8 applies to the tile kernel only: each token row of x is
@@ -251,6 +252,23 @@ size_t stq1_moe_ffn_workspace(int T, int topk, int E, int64_t N, int64_t H, int 
 int stq1_moe_ffn(const void* gateup_blocks, const void* down_blocks, const uint16_t* x,
                  const int32_t* topk_ids, const float* topk_weights, float* out, int T, int topk, int E,
                  int64_t N, int64_t H, int flags, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * stq1_moe_ffn_local_workspace / stq1_moe_ffn_local -- one rank's share of an
+ * expert-parallel MoE feed-forward layer: the experts [expert_begin,
+ * expert_begin + E_local) of E, held in gateup_local / down_local (E_local
+ * matrices each, as stq1_moe_ffn), applied to every (token, slot) pair routed
+ * to them; pairs routed to other ranks' experts contribute 0.  `out` [T, H]
+ * is this rank's partial sum; the layer's output is the sum of all ranks'
+ * partials (an all-reduce).  topk_ids hold global expert ids.  Other
+ * arguments as stq1_moe_ffn; ws at least stq1_moe_ffn_local_workspace(...).
+ * Errors: as stq1_moe_ffn.
+ */
+size_t stq1_moe_ffn_local_workspace(int T, int topk, int E_local, int64_t N, int64_t H, int flags);
+int stq1_moe_ffn_local(const void* gateup_local, const void* down_local, const uint16_t* x,
+                       const int32_t* topk_ids, const float* topk_weights, float* out, int T, int topk,
+                       int E_local, int expert_begin, int64_t N, int64_t H, int flags, void* ws,
+                       size_t ws_bytes, void* stream);
 
 /*
  * stq1_quantize_x_e4m3 -- the activation quantization of the fp8 tile variant

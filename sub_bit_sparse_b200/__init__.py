@@ -33,6 +33,7 @@ ENC_PLAIN = 0
 ENC_SHERRY = 1
 MOE_WEIGHT_UP = 1
 MOE_FP8 = 2
+MOE_SKIP_FOREIGN = 4
 BLOCK_BYTES = 42
 BLOCK_WEIGHTS = 256
 
@@ -61,6 +62,11 @@ SIGNATURES = {
     "stq1_moe_ffn": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                 _c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
                                 _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "stq1_moe_ffn_local_workspace": (_c.c_size_t, [_c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64,
+                                                    _c.c_int]),
+    "stq1_moe_ffn_local": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                      _c.c_void_p, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64,
+                                      _c.c_int, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "stq1_quantize": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int, _c.c_int,
                                  _c.c_void_p, _c.c_void_p]),
     "stq1_quantize_x_e4m3": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p, _c.c_void_p,
@@ -324,6 +330,32 @@ def moe_ffn(gateup_blocks, down_blocks, x, topk_ids, topk_weights, n: int, hidde
                               n_experts, n, hidden, flags, None if ws is None else ws.data_ptr(),
                               0 if ws is None else ws.numel(), _stream(x))
     _check("stq1_moe_ffn", rc)
+    return out
+
+
+def moe_ffn_local(gateup_local, down_local, x, topk_ids, topk_weights, n: int, hidden: int, n_local: int,
+                  expert_begin: int, flags: int = 0, out=None, ws=None):
+    """This rank's partial MoE feed-forward output [T, hidden] for experts
+    [expert_begin, expert_begin + n_local); pairs routed elsewhere contribute 0."""
+    torch = _torch()
+    _require(gateup_local, torch.uint8, "gateup_local")
+    _require(down_local, torch.uint8, "down_local")
+    _require(x, torch.bfloat16, "x")
+    _require(topk_ids, torch.int32, "topk_ids")
+    if topk_weights is not None:
+        _require(topk_weights, torch.float32, "topk_weights")
+    t, topk = topk_ids.shape
+    if out is None:
+        out = torch.empty((t, hidden), dtype=torch.float32, device=x.device)
+    _require(out, torch.float32, "out")
+    lib = _load()
+    if ws is None:
+        ws = workspace(lib.stq1_moe_ffn_local_workspace(t, topk, n_local, n, hidden, flags), x.device, kind="ffn")
+    rc = lib.stq1_moe_ffn_local(gateup_local.data_ptr(), down_local.data_ptr(), x.data_ptr(), topk_ids.data_ptr(),
+                                None if topk_weights is None else topk_weights.data_ptr(), out.data_ptr(), t, topk,
+                                n_local, expert_begin, n, hidden, flags, None if ws is None else ws.data_ptr(),
+                                0 if ws is None else ws.numel(), _stream(x))
+    _check("stq1_moe_ffn_local", rc)
     return out
 
 

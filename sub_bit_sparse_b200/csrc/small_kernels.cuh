@@ -11,7 +11,8 @@ namespace stq1 {
 // One CTA: histogram of ids, exclusive scans of pair counts and of tile
 // counts, tile table, then a scatter of pair ids into per-expert segments.
 // A pair p = t * topk + s.  Pairs with an id outside [0, E) get y = 0 and set
-// STQ1_DEV_BAD_EXPERT.  Order inside a segment is unspecified (it does not
+// STQ1_DEV_BAD_EXPERT, unless skip_foreign (expert parallelism: ids of
+// experts another rank holds) makes them a silent zero.  Order inside a segment is unspecified (it does not
 // change any result: every output row is computed on its own).
 // tile_info[4 * i] = expert, first pair offset, pair count (<= tile_tokens), 0.
 // n_tiles[0] = number of tiles, n_tiles[1] = number of pairs with a valid id.
@@ -21,7 +22,7 @@ constexpr int kRouteThreads = 1024;
 __global__ void __launch_bounds__(kRouteThreads)
 route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_tokens,
              int* __restrict__ pairs_out, int* __restrict__ tile_info, int* __restrict__ n_tiles,
-             float* __restrict__ y, int N) {
+             float* __restrict__ y, int N, int skip_foreign) {
   extern __shared__ int sm[];
   griddep_wait();           // ids may come from the previous kernel in the stream
   griddep_launch_dependents();
@@ -33,7 +34,7 @@ route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_token
   for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
     const int e = ids[p];
     if (e < 0 || e >= E) {
-      flag_error(STQ1_DEV_BAD_EXPERT);
+      if (!skip_foreign) flag_error(STQ1_DEV_BAD_EXPERT);
       float* yr = y + static_cast<long long>(p) * N;
       for (int j = 0; j < N; ++j) yr[j] = 0.f;
     } else {
@@ -129,6 +130,7 @@ direct_gemv_kernel(const uint8_t* __restrict__ W, long long expert_bytes, int E,
                    const uint16_t* __restrict__ x, const int32_t* __restrict__ ids, int topk,
                    const float* __restrict__ route_w, int flags, float* __restrict__ y, int N,
                    int K, int rows_out) {
+  const bool skip_foreign = (flags & STQ1_MOE_SKIP_FOREIGN) != 0;
   const int nb = K / kBlockWeights;
   const long long gw = blockIdx.x * 8LL + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -141,7 +143,7 @@ direct_gemv_kernel(const uint8_t* __restrict__ W, long long expert_bytes, int E,
     if (e < 0 || e >= E) {
       if (lane == 0) {
         y[static_cast<long long>(p) * N + j] = 0.f;
-        flag_error(STQ1_DEV_BAD_EXPERT);
+        if (!skip_foreign) flag_error(STQ1_DEV_BAD_EXPERT);
       }
       return;
     }
@@ -218,6 +220,14 @@ swiglu_kernel(const float* __restrict__ y, uint16_t* __restrict__ act, long long
     const double s = g / (1.0 + exp(-g));
     act[i] = bf16_bits_from_f64(s * u);
   }
+}
+
+// ids[i] - begin: the routing ids of one rank's expert range (expert parallelism).
+__global__ void __launch_bounds__(256)
+shift_ids_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ out, long long n, int begin) {
+  griddep_wait();
+  griddep_launch_dependents();
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n; i += 256LL * gridDim.x) out[i] = ids[i] - begin;
 }
 
 // out[t, h] = sum_s w[t, s] * y[t, s, h] (plain sum without w), fp32 in slot order.

@@ -502,8 +502,10 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
                                int64_t K, int flags, void* ws, size_t ws_bytes, void* stream) {
   if (!expert_blocks || !x || !topk_ids || !y) return STQ1_ERR_NULL;
   if ((flags & STQ1_MOE_WEIGHT_UP) && !topk_weights) return STQ1_ERR_NULL;
-  if (flags & ~(STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8)) return STQ1_ERR_ARG;
-  if (T <= 0 || topk <= 0 || E <= 0 || topk > E || E > kMaxExperts || N <= 0 || (N & 1) || K <= 0 ||
+  if (flags & ~(STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8 | STQ1_MOE_SKIP_FOREIGN)) return STQ1_ERR_ARG;
+  // with STQ1_MOE_SKIP_FOREIGN a rank may hold fewer experts than a token picks
+  const bool foreign = (flags & STQ1_MOE_SKIP_FOREIGN) != 0;
+  if (T <= 0 || topk <= 0 || E <= 0 || (!foreign && topk > E) || E > kMaxExperts || N <= 0 || (N & 1) || K <= 0 ||
       K % kBlockWeights || N > (1LL << 30) || K > (1LL << 30) ||
       static_cast<long long>(T) * topk > (1LL << 30))
     return STQ1_ERR_SHAPE;
@@ -531,7 +533,7 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   }
 
   rc = launch_pdl(route_kernel, 1, kRouteThreads, 3 * E * sizeof(int), s, topk_ids, n_pairs, E, m.tile_tokens,
-                  pairs, tiles, ntiles, y, static_cast<int>(N));
+                  pairs, tiles, ntiles, y, static_cast<int>(N), (flags & STQ1_MOE_SKIP_FOREIGN) ? 1 : 0);
   if (rc != STQ1_OK) return rc;
   if (m.tiles) {
     void* xperm = wsb + m.xperm_off;
@@ -688,7 +690,7 @@ extern "C" int stq1_moe_ffn(const void* gateup_blocks, const void* down_blocks, 
                             const int32_t* topk_ids, const float* topk_weights, float* out, int T, int topk, int E,
                             int64_t N, int64_t H, int flags, void* ws, size_t ws_bytes, void* stream) {
   if (!gateup_blocks || !down_blocks || !x || !topk_ids || !out) return STQ1_ERR_NULL;
-  if (flags & ~(STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8)) return STQ1_ERR_ARG;
+  if (flags & ~(STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8 | STQ1_MOE_SKIP_FOREIGN)) return STQ1_ERR_ARG;
   if (T <= 0 || topk <= 0 || E <= 0 || N <= 0 || (N & 1) || H <= 0 || H % kBlockWeights || (N / 2) % kBlockWeights ||
       (H & 1) || static_cast<long long>(T) * topk > (1LL << 30))
     return STQ1_ERR_SHAPE;
@@ -707,10 +709,36 @@ extern "C" int stq1_moe_ffn(const void* gateup_blocks, const void* down_blocks, 
   rc = stq1_swiglu(ygu, act, P, N, stream);
   if (rc != STQ1_OK) return rc;
   // down projection: each pair is its own token (ids [T, topk] read as [P, 1])
-  rc = stq1_moe_gateup(down_blocks, act, topk_ids, nullptr, yd, P, 1, E, H, N / 2, flags & STQ1_MOE_FP8,
-                       wsb + f.moe_off, f.moe_bytes, stream);
+  rc = stq1_moe_gateup(down_blocks, act, topk_ids, nullptr, yd, P, 1, E, H, N / 2,
+                       flags & (STQ1_MOE_FP8 | STQ1_MOE_SKIP_FOREIGN), wsb + f.moe_off, f.moe_bytes, stream);
   if (rc != STQ1_OK) return rc;
   return stq1_moe_combine(yd, (flags & STQ1_MOE_WEIGHT_UP) ? nullptr : topk_weights, out, T, topk, H, stream);
+}
+
+extern "C" size_t stq1_moe_ffn_local_workspace(int T, int topk, int E_local, int64_t N, int64_t H, int flags) {
+  const size_t w = stq1_moe_ffn_workspace(T, topk, E_local, N, H, flags);
+  return w ? w + round16(static_cast<size_t>(T) * topk * sizeof(int32_t)) : 0;
+}
+
+extern "C" int stq1_moe_ffn_local(const void* gateup_local, const void* down_local, const uint16_t* x,
+                                  const int32_t* topk_ids, const float* topk_weights, float* out, int T, int topk,
+                                  int E_local, int expert_begin, int64_t N, int64_t H, int flags, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  if (!topk_ids || !ws) return !topk_ids ? STQ1_ERR_NULL : STQ1_ERR_WORKSPACE;
+  if (T <= 0 || topk <= 0 || E_local <= 0 || expert_begin < 0) return STQ1_ERR_SHAPE;
+  const size_t need = stq1_moe_ffn_local_workspace(T, topk, E_local, N, H, flags);
+  if (need == 0) return STQ1_ERR_SHAPE;
+  if (ws_bytes < need) return STQ1_ERR_WORKSPACE;
+  if (!aligned16(ws)) return STQ1_ERR_ALIGN;
+  // this rank's view of the routing: ids of its range start at 0, others fall outside [0, E_local)
+  int32_t* ids_local = static_cast<int32_t*>(ws);
+  const size_t ids_bytes = round16(static_cast<size_t>(T) * topk * sizeof(int32_t));
+  const long long n = static_cast<long long>(T) * topk;
+  int rc = launch_pdl(shift_ids_kernel, static_cast<unsigned>(std::min<long long>((n + 255) / 256, 1024)), 256, 0,
+                      static_cast<cudaStream_t>(stream), topk_ids, ids_local, n, expert_begin);
+  if (rc != STQ1_OK) return rc;
+  return stq1_moe_ffn(gateup_local, down_local, x, ids_local, topk_weights, out, T, topk, E_local, N, H,
+                      flags | STQ1_MOE_SKIP_FOREIGN, static_cast<uint8_t*>(ws) + ids_bytes, ws_bytes - ids_bytes, stream);
 }
 
 extern "C" int stq1_set_path(int path) {
