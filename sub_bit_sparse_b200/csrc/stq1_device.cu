@@ -284,6 +284,21 @@ bool want_tiles(long long nb, long long units) {
   return units >= kTcMinBatch;
 }
 
+// Plain GEMV from kTcMinBatch tokens on: the tile kernel when it is expected to
+// be faster.  Calibrated on [4096, 7168] and [18432, 7168] (CUDA graphs of
+// distinct matrices): the table kernel costs about 5.7e-8 us per token and
+// weight (its shared-memory lookups grow with the tokens); a tile-kernel wave
+// of (128-token, 128-row) items costs about 1.36 us per 256-column block of K.
+bool want_tiles_gemv(long long N, long long nb, long long batch) {
+  if (!want_tiles(nb, batch)) return false;
+  if (g_path == 2) return true;
+  const double table_us = 5.7e-8 * static_cast<double>(batch) * static_cast<double>(N) * nb * kBlockWeights;
+  const long long items = ((batch + kTcN - 1) / kTcN) * ((N + kTcM - 1) / kTcM);
+  const long long waves = (items + sm_count() - 1) / sm_count();
+  const double tiles_us = 1.36 * static_cast<double>(waves) * nb;
+  return tiles_us < table_us;
+}
+
 int smem_per_sm() {
   static int cache[kMaxDevices] = {};
   const int dev = current_device();
@@ -331,7 +346,7 @@ void plan_table(GemvPlan* p, long long N, long long K, int batch, bool one_wave)
 GemvPlan plan_gemv(long long N, long long K, int batch) {
   GemvPlan p{};
   const long long nb = K / kBlockWeights;
-  p.tile_path = want_tiles(nb, batch);
+  p.tile_path = want_tiles_gemv(N, nb, batch);
   if (p.tile_path) return p;
   p.table_path = (nb % 2 == 0);
   plan_table(&p, N, K, batch, true);
