@@ -75,6 +75,18 @@ design notes):
    of the down projection; the down projection is the same STQ1_0 matmul per
    routed (token, slot) pair; the combine is sum_s w[t, s] * y_down[t, s]
    (or the plain sum when the weights were applied to the up half).
+9. Mixed-precision allocation (the pages: per-layer bit widths picked by
+   full-Hessian sensitivity, greedily by error reduction per added byte,
+   between STQ1_0 and a 2.06-bpw partner format that is third-party): the
+   partner here is STQ2, a format of this library at the same rate: per 256
+   weights an fp16 scale d = fp16(amax) and 64 bytes of 2-bit codes (weight k
+   at bits 2 (k mod 4) of byte k / 4), code q meaning (2q - 3) d / 3, chosen
+   as the nearest level (ties: the lower code).  A layer's error under a
+   format is tr(D H D^T) with D = W - W^ and H = X^T X over its calibration
+   rows x; the diagonal (imatrix) score keeps only H's diagonal.  Greedy:
+   start from STQ1_0 everywhere, upgrade layers in order of error reduction
+   per added byte (ties: lower layer index) while the total stays within the
+   byte budget.
 """
 
 from __future__ import annotations
@@ -589,6 +601,71 @@ def moe_ffn(gateup_packed, down_packed, x_bits, ids, weights, n: int, hidden: in
         return out
     wa = np.ones((T, topk)) if w is None else np.abs(np.asarray(w, dtype=np.float32).astype(np.float64))
     return out, np.einsum("ts,tsh->th", wa, ya)
+
+
+# ---------------------------------------------------------------------------
+# Mixed-precision allocation (reading 9)
+# ---------------------------------------------------------------------------
+
+STQ2_BLOCK_BYTES = 66
+
+
+def encode_stq2(w: np.ndarray) -> np.ndarray:
+    """[N, K] fp32 -> STQ2 bytes: per block fp16(amax), then 2-bit nearest-level codes."""
+    blocks = np.asarray(w, dtype=np.float32).reshape(-1, BLOCK_WEIGHTS).astype(np.float64)
+    amax = np.max(np.abs(blocks), axis=1)
+    d_bits = fp16_bits(amax)
+    d = fp16_value(d_bits)
+    levels = d[:, None] * (2.0 * np.arange(4) - 3.0)[None, :] / 3.0            # [B, 4]
+    dist = np.abs(blocks[:, :, None] - levels[:, None, :])                       # [B, 256, 4]
+    q = np.argmin(dist, axis=2).astype(np.uint8)                                 # first minimum = lower code
+    out = np.zeros((blocks.shape[0], STQ2_BLOCK_BYTES), dtype=np.uint8)
+    out[:, 0] = d_bits & 0xFF
+    out[:, 1] = d_bits >> 8
+    qq = q.reshape(-1, 64, 4).astype(np.uint32)
+    out[:, 2:] = (qq[:, :, 0] | (qq[:, :, 1] << 2) | (qq[:, :, 2] << 4) | (qq[:, :, 3] << 6)).astype(np.uint8)
+    return out.reshape(-1)
+
+
+def decode_stq2(packed: np.ndarray, n: int, k: int) -> np.ndarray:
+    """STQ2 bytes -> [n, k] fp64."""
+    b = np.asarray(packed, dtype=np.uint8).reshape(-1, STQ2_BLOCK_BYTES)
+    d = fp16_value(b[:, 0].astype(np.uint16) | (b[:, 1].astype(np.uint16) << 8))
+    codes = np.stack([(b[:, 2:] >> (2 * i)) & 3 for i in range(4)], axis=2).reshape(-1, BLOCK_WEIGHTS)
+    return (d[:, None] * (2.0 * codes - 3.0) / 3.0).reshape(n, k)
+
+
+def hessian_error(w: np.ndarray, w_hat: np.ndarray, x: np.ndarray) -> float:
+    """tr(D H D^T) with D = w - w_hat [N, K] and H = x^T x, x [n_cal, K] (fp64)."""
+    d = np.asarray(w, dtype=np.float64) - np.asarray(w_hat, dtype=np.float64)
+    h = np.asarray(x, dtype=np.float64).T @ np.asarray(x, dtype=np.float64)
+    return float(np.sum((d @ h) * d))
+
+
+def diagonal_error(w: np.ndarray, w_hat: np.ndarray, x: np.ndarray) -> float:
+    """The imatrix score: sum_k H_kk D_jk^2 over rows j."""
+    d = np.asarray(w, dtype=np.float64) - np.asarray(w_hat, dtype=np.float64)
+    hd = np.sum(np.asarray(x, dtype=np.float64) ** 2, axis=0)
+    return float(np.sum(d * d * hd[None, :]))
+
+
+def greedy_allocate(err_low, err_high, bytes_low, bytes_high, budget) -> np.ndarray:
+    """Per layer: True = the higher-bit format.  Start all low; upgrade in order of
+    (err_low - err_high) / (bytes_high - bytes_low), descending (ties: lower index),
+    while the total bytes stay within the budget (a layer that does not fit is skipped)."""
+    el, eh = np.asarray(err_low, float), np.asarray(err_high, float)
+    bl, bh = np.asarray(bytes_low, float), np.asarray(bytes_high, float)
+    gain = (el - eh) / (bh - bl)
+    order = sorted(range(len(el)), key=lambda i: (-gain[i], i))
+    pick = np.zeros(len(el), dtype=bool)
+    total = float(np.sum(bl))
+    for i in order:
+        if gain[i] <= 0:
+            break
+        if total + bh[i] - bl[i] <= budget:
+            pick[i] = True
+            total += bh[i] - bl[i]
+    return pick
 
 
 def half_from_struct(x: float) -> int:
