@@ -253,6 +253,12 @@ def run_gpu(args):
     except Exception as exc:  # reported, never hidden
         encoder = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
+    # --- mixed-precision allocation: layer scoring on the tensor cores ---
+    try:
+        mix = run_mix(torch, stq1, device, stream, args, world, timed, bf16_peak, hbm_peak)
+    except Exception as exc:  # reported, never hidden
+        mix = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     # --- end to end through the public API with host buffers ---
     e2e = run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier)
 
@@ -277,6 +283,7 @@ def run_gpu(args):
         "moe_prefill": prefill,
         "moe_ffn_decode": ffn,
         "encoder": encoder,
+        "mix_allocation": mix,
         "e2e": e2e,
         "gpu_launches": args.steps * STACK,
         "clocks": clk.summary(),
@@ -438,6 +445,109 @@ def run_encoder(torch, stq1, device, stream):
     res["host_threads"] = os.cpu_count()
     res["gpu_equals_host"] = bool(np.array_equal(host, outs["sherry"]))
     res["config"] = "decode matrix [4096, 7168], Sherry 3 rounds with calibration importance; plain = amax"
+    return res
+
+
+MIX_LAYERS, MIX_N, MIX_K, MIX_CAL = 77, 4096, 7168, 512
+
+
+def _mix_inputs(torch, device, n_layers, seed=2025):
+    import workloads
+    w = torch.empty((n_layers, MIX_N, MIX_K), dtype=torch.float32, device=device)
+    x = torch.empty((n_layers, MIX_CAL, MIX_K), dtype=torch.bfloat16, device=device)
+    for l in range(n_layers):
+        wl, xl = workloads.mix_layer_torch(MIX_N, MIX_K, MIX_CAL, l, seed, device)
+        w[l].copy_(wl)
+        x[l].copy_(xl)
+        del wl, xl
+    return w, x
+
+
+def _ranks(v):
+    r = np.empty(len(v))
+    r[np.argsort(v, kind="stable")] = np.arange(len(v))
+    return r
+
+
+def run_mix(torch, stq1, device, stream, args, world, timed, bf16_peak, hbm_peak):
+    """Mixed-precision allocation study: 77 layers of one [4096, 7168] matrix
+    each with 512 calibration rows; STQ1_0 (Sherry, 3 rounds) versus STQ2
+    (importance-fitted, 3 rounds) for every layer, both scored under the full and the diagonal Hessian on the
+    tensor cores, then the greedy per-byte allocation at the pages' split
+    (29 layers low, 48 high)."""
+    L, n, k, nc = MIX_LAYERS, MIX_N, MIX_K, MIX_CAL
+    w, x = _mix_inputs(torch, device, L)
+    with torch.cuda.stream(stream):
+        h = stq1.hessian_diag(x)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        p_low = torch.cat([stq1.quantize_gpu(w[l], h[l], mode="sherry", rounds=3) for l in range(L)])
+        e1.record(stream)
+        p_high = torch.cat([stq1.stq2_quantize(w[l], h[l], rounds=3) for l in range(L)])
+        e2 = torch.cuda.Event(enable_timing=True)
+        e2.record(stream)
+    torch.cuda.synchronize()
+    enc_ms = e0.elapsed_time(e1)
+    enc2_ms = e1.elapsed_time(e2)
+    out_low = torch.empty((L, 2), dtype=torch.float64, device=device)
+    out_high = torch.empty((L, 2), dtype=torch.float64, device=device)
+    flops = 2.0 * L * n * k * nc
+    res = {}
+    for name, fmt, pk, o, bb in (("stq1_0", stq1.FMT_STQ1_0, p_low, out_low, 42),
+                                 ("stq2", stq1.FMT_STQ2, p_high, out_high, 66)):
+        def step():
+            stq1.hessian_error(fmt, pk, w, x, h, out=o)
+        steps = 5
+        g = time_graph(torch, step, steps, 3, stream)
+        ms = timed(g, steps) / steps
+        del g
+        nbytes = L * (n * k * 4 + n * k // 256 * bb + nc * k * 2 + k * 4)
+        t_hbm, t_tc = nbytes / (hbm_peak * 1e9), flops / (bf16_peak * 1e12)
+        res[name] = {"ms_per_call": round(ms, 4), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                     "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+                     "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / hbm_peak, 4),
+                     "tensor_frac": round(flops / (ms * 1e-3) / 1e12 / bf16_peak, 4),
+                     "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                     "roofline_frac": round(max(t_hbm, t_tc) / (ms * 1e-3), 4),
+                     "algorithmic_bytes": nbytes, "flops": flops}
+    torch.cuda.synchronize()
+    assert stq1.status() == 0
+    el, eh = out_low.cpu().numpy(), out_high.cpu().numpy()
+    b_low, b_high = float(n * k // 256 * 42), float(n * k // 256 * 66)
+    bl, bh = np.full(L, b_low), np.full(L, b_high)
+    budget = 29 * b_low + 48 * b_high
+    import time
+    t0 = time.perf_counter()
+    pick_full = stq1.mix_allocate(el[:, 0], eh[:, 0], bl, bh, budget)
+    alloc_ms = (time.perf_counter() - t0) * 1e3
+    pick_diag = stq1.mix_allocate(el[:, 1], eh[:, 1], bl, bh, budget)
+    gain_full = (el[:, 0] - eh[:, 0]) / (bh - bl)
+    gain_diag = (el[:, 1] - eh[:, 1]) / (bh - bl)
+    rf, rd = _ranks(gain_full), _ranks(gain_diag)
+    spearman = float(np.corrcoef(rf, rd)[0, 1])
+    sens_rank = float(np.corrcoef(_ranks(el[:, 0]), _ranks(el[:, 1]))[0, 1])
+
+    def total(pick):
+        return float(np.sum(np.where(pick, eh[:, 0], el[:, 0])))
+
+    res.update({
+        "layers": L, "layer_shape": [n, k], "calibration_rows": nc,
+        "picked_high_full": int(pick_full.sum()), "picked_high_diag": int(pick_diag.sum()),
+        "picks_differ": int(np.sum(pick_full != pick_diag)),
+        "full_error_of_full_allocation": total(pick_full),
+        "full_error_of_diag_allocation": total(pick_diag),
+        "full_error_all_stq1_0": float(el[:, 0].sum()), "full_error_all_stq2": float(eh[:, 0].sum()),
+        "spearman_gain_full_vs_diag": round(spearman, 4),
+        "spearman_stq1_error_full_vs_diag": round(sens_rank, 4),
+        "avg_bpw": round((29 * 1.3125 + 48 * 2.0625) / 77, 4),
+        "sherry_encode_ms_all_layers": round(enc_ms, 2), "stq2_encode_ms_all_layers": round(enc2_ms, 2),
+        "allocate_ms": round(alloc_ms, 3),
+        "kernel": "hess_score_kernel", "peak_hbm_gbs": hbm_peak, "peak_bf16_tflops": bf16_peak,
+        "config": "77 layers x [4096, 7168] fp32 weights, 512 bf16 calibration rows each (synthetic: "
+                  "correlated channels, weights partly along the shared directions), all layers per call",
+    })
+    del w, x, p_low, p_high
+    torch.cuda.empty_cache()
     return res
 
 
@@ -639,6 +749,16 @@ def profile_case(args):
     import sub_bit_sparse_b200 as stq1
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
+    if args.profile_case == "mix":
+        # four layers (about 500 MB of weights, larger than L2), one scoring call each format
+        w, x = _mix_inputs(torch, device, 4)
+        h = stq1.hessian_diag(x)
+        pk = torch.cat([stq1.quantize_gpu(w[l], h[l], mode="sherry", rounds=3) for l in range(4)])
+        for _ in range(3):
+            o = stq1.hessian_error(stq1.FMT_STQ1_0, pk, w, x, h)
+        torch.cuda.synchronize()
+        print("profile case done", o.cpu().numpy().tolist())
+        return
     if args.profile_case in ("moe", "prefill"):
         stream = torch.cuda.Stream(device)
         fn = run_moe if args.profile_case == "moe" else run_prefill
@@ -664,7 +784,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", default=None, choices=["gemv", "moe", "prefill"])
+    ap.add_argument("--profile-case", default=None, choices=["gemv", "moe", "prefill", "mix"])
     ap.add_argument("--sweep", action="store_true", help="crossover sweep (18432 x 7168, batch 1..1024)")
     args = ap.parse_args()
     if args.sweep:

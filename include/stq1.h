@@ -72,6 +72,10 @@ extern "C" {
 #define STQ1_MOE_FP8 2            /* tile path: E4M3 activations (per-token fp32 scale), fp8 MMAs */
 #define STQ1_MOE_SKIP_FOREIGN 4   /* ids outside [0, E) give y = 0 without an error (expert parallelism) */
 
+/* Weight formats for stq1_hessian_error. */
+#define STQ1_FMT_STQ1_0 0         /* 42 bytes per 256 weights (1.3125 bpw) */
+#define STQ1_FMT_STQ2 1           /* 66 bytes per 256 weights (2.0625 bpw), see stq1_quantize_stq2 */
+
 /* Library version (major * 10000 + minor * 100 + patch). */
 int stq1_version(void);
 
@@ -330,6 +334,96 @@ int stq1_set_path(int path);
  * synchronisation itself fails.
  */
 int stq1_status(void* stream, int* device_err);
+
+/*
+ * ---- Mixed-precision allocation ----
+ * The pages let calibration data choose each layer's bit width: sensitivity is
+ * the layer's error under the full Hessian H = X^T X of its calibration
+ * inputs, and layers move from STQ1_0 to a 2.06-bpw format greedily by error
+ * reduction per added byte ("AngelSlim Shrinks ..." bullet list;
+ * lemmy.durstig.online post 66506, "Full-Hessian scoring").  The pages'
+ * partner format is third-party; the partner here is STQ2, defined below.
+ */
+
+/*
+ * stq1_quantize_stq2 -- STQ2 encoder (GPU).  Per 256 weights (66 bytes): bytes
+ * 0-1 the fp16 scale d, then 64 code bytes: weight k of the block at bits
+ * 2 (k mod 4) of code byte k / 4; code q means the level (d (2q - 3)) / 3.
+ * rounds = 0: d = fp16(max |w|) (round to nearest even, saturating at 65504)
+ * and each weight takes the nearest level, ties to the lower code.
+ * rounds > 0: the pages fit the partner format with the importance matrix
+ * (lemmy.durstig.online post 66506, "Full-Hessian scoring"), and STQ2 is fit
+ * the way the Sherry scale is: starting from those codes, `rounds` times
+ * d = 3 sum h w m / sum h m^2 (m = 2q - 3, k ascending; the weighted
+ * least-squares scale for fixed codes), then the nearest levels at that d;
+ * the stored scale is fp16 of one more fit.  All in fp64 with a fixed order,
+ * so the bytes are those of the oracle's encoder.
+ *   W       device, [N, K] fp32 row-major, 16-byte aligned.
+ *   h       device, [K] fp32 importance per column, 4-byte aligned, or NULL
+ *           (h = 1).  A block whose h is all zero uses h = 1.
+ *   rounds  0..1000.
+ *   out     device, N*K/256*66 bytes, 2-byte aligned (fully overwritten).
+ * Asynchronous on `stream`.  A NaN/Inf weight, or a negative or non-finite
+ * importance, sets STQ1_DEV_BAD_VALUE in the device error word and the block
+ * is written as zeros.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE (K % 256, non-positive sizes),
+ * STQ1_ERR_ARG (rounds), STQ1_ERR_ALIGN, STQ1_ERR_CUDA.
+ */
+int stq1_quantize_stq2(const float* W, const float* h, int64_t N, int64_t K, int rounds, uint8_t* out,
+                       void* stream);
+
+/*
+ * stq1_hessian_diag -- diagonal of each layer's calibration Hessian (GPU):
+ * h[l][k] = sum over r of x[l][r][k]^2, summed in fp64 and rounded once to
+ * fp32.  This is the per-column importance (imatrix) the Sherry encoder and
+ * the diagonal score use.
+ *   x  device, [L][rows][K] bf16 bits, 2-byte aligned.
+ *   h  device, [L][K] fp32, 4-byte aligned (fully overwritten).
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE (non-positive sizes, L > 65535),
+ * STQ1_ERR_ALIGN, STQ1_ERR_CUDA.
+ */
+int stq1_hessian_diag(const uint16_t* x, int64_t L, int64_t rows, int64_t K, float* h, void* stream);
+
+/*
+ * stq1_hessian_error -- per-layer quantisation error under the full and the
+ * diagonal Hessian (GPU, tensor cores).  For each layer l, with
+ * D = W[l] - decode(packed[l]) [N, K] and X = x[l] [n_cal, K]:
+ *   out[2l]     = tr(D X^T X D^T) = sum over calibration rows c and output
+ *                 rows j of (sum_k D[j,k] X[c,k])^2   (the full score)
+ *   out[2l + 1] = sum over j, k of h[l][k] D[j,k]^2   (the diagonal score;
+ *                 with h from stq1_hessian_diag it is the imatrix score)
+ * D is formed in fp32 and rounded to bf16 for the contraction (fp32
+ * accumulation), so the full score carries a relative error of the order of
+ * 2^-9 per element of D; the diagonal score is formed from the fp32 D.
+ *   format  STQ1_FMT_STQ1_0 or STQ1_FMT_STQ2.
+ *   packed  device, [L][N][K/256 * bytes per block], 2-byte aligned.
+ *   W       device, [L][N][K] fp32, 16-byte aligned (the unquantised weights).
+ *   x       device, [L][n_cal][K] bf16 bits, 16-byte aligned.
+ *   h       device, [L][K] fp32, 16-byte aligned.
+ *   out     device, [L][2] fp64, 8-byte aligned (zeroed on `stream`, then
+ *           accumulated by the kernel; the order of the additions is not fixed).
+ * Asynchronous on `stream`.  A wait that runs out sets STQ1_DEV_WAIT_LIMIT.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_ARG (format), STQ1_ERR_SHAPE (K % 256,
+ * non-positive sizes), STQ1_ERR_ALIGN, STQ1_ERR_CUDA.
+ */
+int stq1_hessian_error(int format, const void* packed, const float* W, const uint16_t* x, const float* h,
+                       int64_t L, int64_t N, int64_t K, int64_t n_cal, double* out, void* stream);
+
+/*
+ * stq1_mix_allocate -- greedy layer allocation (host, deterministic).  Start
+ * with every layer in the lower format; visit layers in decreasing order of
+ * gain = (err_low - err_high) / (bytes_high - bytes_low) (ties: lower index);
+ * stop at the first gain <= 0; upgrade a layer when total + cost <= budget,
+ * where total starts as the sum of bytes_low in layer order and grows by each
+ * upgrade's cost = bytes_high - bytes_low (a layer that does not fit is
+ * skipped and later ones are still tried).  All arithmetic is IEEE fp64.
+ *   err_low, err_high, bytes_low, bytes_high  host, [n_layers] fp64.
+ *   pick  host, [n_layers]: 1 = the higher format, 0 = the lower.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE (n_layers <= 0), STQ1_ERR_VALUE
+ * (a non-finite input, or bytes_high <= bytes_low).
+ */
+int stq1_mix_allocate(const double* err_low, const double* err_high, const double* bytes_low,
+                      const double* bytes_high, int64_t n_layers, double budget, uint8_t* pick);
 
 #ifdef __cplusplus
 }

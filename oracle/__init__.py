@@ -14,5 +14,6 @@ from .stq1 import (  # noqa: F401
     decode, dequant_bf16, gemv, gemv_abs, tolerance, route_pairs, moe_gateup,
     half_from_struct, E4M3_MAX, e4m3_value, e4m3_round, quantize_x_e4m3, moe_gateup_fp8,
     bf16_bits_from_f64, silu, swiglu_bf16, moe_combine, moe_ffn,
-    STQ2_BLOCK_BYTES, encode_stq2, decode_stq2, hessian_error, diagonal_error, greedy_allocate,
+    STQ2_BLOCK_BYTES, encode_stq2, decode_stq2, stq2_codes, stq2_wls_scale, stq2_weighted_error,
+    hessian_error, diagonal_error, greedy_allocate,
 )

@@ -79,14 +79,18 @@ design notes):
    full-Hessian sensitivity, greedily by error reduction per added byte,
    between STQ1_0 and a 2.06-bpw partner format that is third-party): the
    partner here is STQ2, a format of this library at the same rate: per 256
-   weights an fp16 scale d = fp16(amax) and 64 bytes of 2-bit codes (weight k
-   at bits 2 (k mod 4) of byte k / 4), code q meaning (2q - 3) d / 3, chosen
-   as the nearest level (ties: the lower code).  A layer's error under a
+   weights an fp16 scale d and 64 bytes of 2-bit codes (weight k at bits
+   2 (k mod 4) of byte k / 4), code q meaning (2q - 3) d / 3, chosen as the
+   nearest level (ties: the lower code).  The pages' partner is fitted with
+   the importance matrix, so STQ2 is too: d starts at fp16(amax) and is then
+   fit like the Sherry scale, by weighted least squares alternating with the
+   code choice.  A layer's error under a
    format is tr(D H D^T) with D = W - W^ and H = X^T X over its calibration
    rows x; the diagonal (imatrix) score keeps only H's diagonal.  Greedy:
    start from STQ1_0 everywhere, upgrade layers in order of error reduction
    per added byte (ties: lower layer index) while the total stays within the
-   byte budget.
+   byte budget; byte totals are summed in layer order, then grown one upgrade
+   at a time.
 """
 
 from __future__ import annotations
@@ -610,21 +614,77 @@ def moe_ffn(gateup_packed, down_packed, x_bits, ids, weights, n: int, hidden: in
 STQ2_BLOCK_BYTES = 66
 
 
-def encode_stq2(w: np.ndarray) -> np.ndarray:
-    """[N, K] fp32 -> STQ2 bytes: per block fp16(amax), then 2-bit nearest-level codes."""
-    blocks = np.asarray(w, dtype=np.float32).reshape(-1, BLOCK_WEIGHTS).astype(np.float64)
-    amax = np.max(np.abs(blocks), axis=1)
-    d_bits = fp16_bits(amax)
+def _stq2_levels(d: np.ndarray) -> np.ndarray:
+    """[B] fp64 scales -> [B, 4] levels (d * (2q - 3)) / 3."""
+    return d[:, None] * (2.0 * np.arange(4) - 3.0)[None, :] / 3.0
+
+
+def stq2_codes(wb: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """Nearest level per weight (ties: the lower code).  wb fp64 [B, 256], d fp64 [B]."""
+    dist = np.abs(wb[:, :, None] - _stq2_levels(d)[:, None, :])
+    return np.argmin(dist, axis=2)                                           # first minimum
+
+
+def stq2_wls_scale(wb: np.ndarray, hb: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """Weighted least-squares scale for fixed codes: with m_k = 2 q_k - 3 the level
+    of weight k is d m_k / 3, and the minimiser of sum_k h_k (w_k - d m_k / 3)^2 is
+    d = 3 sum h_k w_k m_k / sum h_k m_k^2, summed over k ascending (sequential fp64)."""
+    m = 2.0 * q - 3.0
+    num = np.zeros(wb.shape[0])
+    den = np.zeros(wb.shape[0])
+    for k in range(BLOCK_WEIGHTS):
+        num = num + (hb[:, k] * wb[:, k]) * m[:, k]
+        den = den + hb[:, k] * (m[:, k] * m[:, k])
+    return (3.0 * num) / den
+
+
+def stq2_weighted_error(wb: np.ndarray, hb: np.ndarray, d: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """sum_k h_k (w_k - d m_k / 3)^2 per block (fp64)."""
+    lev = np.take_along_axis(_stq2_levels(d), q, axis=1)
+    return np.sum(hb * (wb - lev) ** 2, axis=1)
+
+
+def encode_stq2(w: np.ndarray, h: np.ndarray | None = None, rounds: int = 0, trace: bool = False):
+    """[N, K] fp32 -> STQ2 bytes.
+
+    rounds = 0: d = fp16(amax), codes nearest at that d.  rounds > 0: starting
+    from those codes, ``rounds`` times fit d by weighted least squares (h per
+    column; None means h = 1; a block whose h is all zero uses h = 1) and
+    re-pick the nearest levels at that d; then store fp16 of one more fit.
+    """
+    w = np.asarray(w, dtype=np.float32)
+    if not np.all(np.isfinite(w)):
+        raise OracleValueError("non-finite weight")
+    n, k = w.shape
+    wb = w.reshape(-1, BLOCK_WEIGHTS).astype(np.float64)
+    B = wb.shape[0]
+    if h is None:
+        hcol = np.ones(k)
+    else:
+        hcol = np.asarray(h, dtype=np.float32).astype(np.float64)
+        if hcol.shape != (k,) or not np.all(np.isfinite(hcol)) or np.any(hcol < 0):
+            raise OracleValueError("importance must be finite, >= 0, one value per column")
+    hb = np.broadcast_to(hcol.reshape(1, k), (n, k)).reshape(B, BLOCK_WEIGHTS).copy()
+    hb[~np.any(hb != 0.0, axis=1)] = 1.0
+    d_bits = fp16_bits(np.max(np.abs(wb), axis=1))
     d = fp16_value(d_bits)
-    levels = d[:, None] * (2.0 * np.arange(4) - 3.0)[None, :] / 3.0            # [B, 4]
-    dist = np.abs(blocks[:, :, None] - levels[:, None, :])                       # [B, 256, 4]
-    q = np.argmin(dist, axis=2).astype(np.uint8)                                 # first minimum = lower code
-    out = np.zeros((blocks.shape[0], STQ2_BLOCK_BYTES), dtype=np.uint8)
+    q = stq2_codes(wb, d)
+    hist = [(d.copy(), q.copy())]
+    if rounds > 0:
+        for _ in range(rounds):
+            d = stq2_wls_scale(wb, hb, q)
+            q = stq2_codes(wb, d)
+            hist.append((d.copy(), q.copy()))
+        d_bits = fp16_bits(stq2_wls_scale(wb, hb, q))
+    out = np.zeros((B, STQ2_BLOCK_BYTES), dtype=np.uint8)
     out[:, 0] = d_bits & 0xFF
     out[:, 1] = d_bits >> 8
-    qq = q.reshape(-1, 64, 4).astype(np.uint32)
+    qq = q.astype(np.uint32).reshape(B, 64, 4)
     out[:, 2:] = (qq[:, :, 0] | (qq[:, :, 1] << 2) | (qq[:, :, 2] << 4) | (qq[:, :, 3] << 6)).astype(np.uint8)
-    return out.reshape(-1)
+    out = out.reshape(-1)
+    if trace:
+        return out, {"rounds": hist, "h_blocks": hb}
+    return out
 
 
 def decode_stq2(packed: np.ndarray, n: int, k: int) -> np.ndarray:
@@ -636,10 +696,14 @@ def decode_stq2(packed: np.ndarray, n: int, k: int) -> np.ndarray:
 
 
 def hessian_error(w: np.ndarray, w_hat: np.ndarray, x: np.ndarray) -> float:
-    """tr(D H D^T) with D = w - w_hat [N, K] and H = x^T x, x [n_cal, K] (fp64)."""
+    """tr(D H D^T) with D = w - w_hat [N, K] and H = x^T x, x [n_cal, K] (fp64).
+
+    Evaluated as the sum over calibration rows of the squared outputs of D,
+    sum_c ||D x_c||^2, which is the same number (tr(D X^T X D^T) = ||X D^T||_F^2)
+    without forming the K x K matrix H."""
     d = np.asarray(w, dtype=np.float64) - np.asarray(w_hat, dtype=np.float64)
-    h = np.asarray(x, dtype=np.float64).T @ np.asarray(x, dtype=np.float64)
-    return float(np.sum((d @ h) * d))
+    y = np.asarray(x, dtype=np.float64) @ d.T
+    return float(np.sum(y * y))
 
 
 def diagonal_error(w: np.ndarray, w_hat: np.ndarray, x: np.ndarray) -> float:
@@ -658,13 +722,16 @@ def greedy_allocate(err_low, err_high, bytes_low, bytes_high, budget) -> np.ndar
     gain = (el - eh) / (bh - bl)
     order = sorted(range(len(el)), key=lambda i: (-gain[i], i))
     pick = np.zeros(len(el), dtype=bool)
-    total = float(np.sum(bl))
+    total = 0.0
+    for v in bl:                         # left to right, one rounding per addition
+        total += float(v)
     for i in order:
         if gain[i] <= 0:
             break
-        if total + bh[i] - bl[i] <= budget:
+        cost = float(bh[i] - bl[i])
+        if total + cost <= budget:
             pick[i] = True
-            total += bh[i] - bl[i]
+            total += cost
     return pick
 
 

@@ -36,6 +36,9 @@ MOE_FP8 = 2
 MOE_SKIP_FOREIGN = 4
 BLOCK_BYTES = 42
 BLOCK_WEIGHTS = 256
+FMT_STQ1_0 = 0
+FMT_STQ2 = 1
+STQ2_BLOCK_BYTES = 66
 
 # Every symbol include/stq1.h declares: name -> (restype, argtypes)
 _c = ctypes
@@ -71,6 +74,15 @@ SIGNATURES = {
                                  _c.c_void_p, _c.c_void_p]),
     "stq1_quantize_x_e4m3": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p, _c.c_void_p,
                                         _c.c_void_p]),
+    "stq1_quantize_stq2": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int, _c.c_void_p,
+                                      _c.c_void_p]),
+    "stq1_hessian_diag": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int64, _c.c_void_p,
+                                     _c.c_void_p]),
+    "stq1_hessian_error": (_c.c_int, [_c.c_int, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                      _c.c_int64, _c.c_int64, _c.c_int64, _c.c_int64, _c.c_void_p,
+                                      _c.c_void_p]),
+    "stq1_mix_allocate": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64,
+                                     _c.c_double, _c.c_void_p]),
 }
 
 
@@ -374,6 +386,72 @@ def quantize_gpu(w, h=None, mode: str = "plain", rounds: int = 3, out=None):
                                _stream(w))
     _check("stq1_quantize", rc)
     return out
+
+
+def stq2_quantize(w, h=None, rounds: int = 0, out=None):
+    """fp32 [N, K] CUDA tensor -> packed STQ2 bytes (uint8 CUDA tensor, N*K/256*66).
+
+    rounds = 0 is the amax encoding; rounds > 0 fits the scale to the
+    per-column importance h (fp32 [K], or None for h = 1)."""
+    torch = _torch()
+    _require(w, torch.float32, "w")
+    n, k = w.shape
+    if h is not None:
+        _require(h, torch.float32, "h")
+    if out is None:
+        out = torch.empty((n * (k // BLOCK_WEIGHTS) * STQ2_BLOCK_BYTES,), dtype=torch.uint8, device=w.device)
+    _require(out, torch.uint8, "out")
+    rc = _load().stq1_quantize_stq2(w.data_ptr(), None if h is None else h.data_ptr(), n, k, rounds,
+                                    out.data_ptr(), _stream(w))
+    _check("stq1_quantize_stq2", rc)
+    return out
+
+
+def hessian_diag(x, out=None):
+    """bf16 calibration rows [L, rows, K] (or [rows, K]) -> fp32 [L, K]: sum over rows of x^2."""
+    torch = _torch()
+    _require(x, torch.bfloat16, "x")
+    x3 = x if x.dim() == 3 else x.unsqueeze(0)
+    nl, rows, k = x3.shape
+    if out is None:
+        out = torch.empty((nl, k), dtype=torch.float32, device=x.device)
+    _require(out, torch.float32, "out")
+    _check("stq1_hessian_diag", _load().stq1_hessian_diag(x3.data_ptr(), nl, rows, k, out.data_ptr(), _stream(x)))
+    return out
+
+
+def hessian_error(fmt: int, packed, w, x, h, out=None):
+    """Per-layer (full, diagonal) Hessian error of a quantised weight set.
+
+    packed: uint8 [L * N * K/256 * block bytes]; w: fp32 [L, N, K]; x: bf16
+    [L, n_cal, K]; h: fp32 [L, K].  Returns fp64 [L, 2] on the device.
+    """
+    torch = _torch()
+    _require(packed, torch.uint8, "packed")
+    _require(w, torch.float32, "w")
+    _require(x, torch.bfloat16, "x")
+    _require(h, torch.float32, "h")
+    nl, n, k = w.shape
+    n_cal = x.shape[1]
+    if out is None:
+        out = torch.empty((nl, 2), dtype=torch.float64, device=w.device)
+    _require(out, torch.float64, "out")
+    rc = _load().stq1_hessian_error(fmt, packed.data_ptr(), w.data_ptr(), x.data_ptr(), h.data_ptr(), nl, n, k,
+                                    n_cal, out.data_ptr(), _stream(w))
+    _check("stq1_hessian_error", rc)
+    return out
+
+
+def mix_allocate(err_low, err_high, bytes_low, bytes_high, budget: float) -> np.ndarray:
+    """Greedy per-byte layer allocation (host): bool [L], True = the higher-bit format."""
+    arrs = [np.ascontiguousarray(v, dtype=np.float64) for v in (err_low, err_high, bytes_low, bytes_high)]
+    n = arrs[0].shape[0]
+    if any(a.shape != (n,) for a in arrs):
+        raise ValueError("all four inputs must be 1-D of the same length")
+    pick = np.zeros(max(n, 1), dtype=np.uint8)
+    rc = _load().stq1_mix_allocate(*(a.ctypes.data for a in arrs), n, float(budget), pick.ctypes.data)
+    _check("stq1_mix_allocate", rc)
+    return pick[:n].astype(bool)
 
 
 def quantize_x_e4m3(x, out=None, scales=None):

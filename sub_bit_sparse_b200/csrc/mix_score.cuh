@@ -1,0 +1,443 @@
+// Mixed-precision allocation kernels: the STQ2 partner-format encoder, the
+// diagonal of the calibration Hessian, and the per-layer error under the full
+// and the diagonal Hessian.
+//
+// The pages let calibration data pick each layer's format: sensitivity is the
+// error under the full Hessian H = X^T X (the off-diagonal terms are what the
+// diagonal imatrix score misses), and layers move to the higher-bit format
+// greedily by error reduction per added byte ("AngelSlim Shrinks ..."
+// bullet list; lemmy.durstig.online post 66506, "Full-Hessian scoring").  The
+// pages' partner format is third-party; STQ2 is this library's format at the
+// same 2.0625 bits per weight: per 256 weights an fp16 scale d and 64 bytes of
+// 2-bit codes, weight k at bits 2 (k mod 4) of code byte k / 4, code q meaning
+// (2q - 3) d / 3; d is fit to the importance matrix like the Sherry scale.
+//
+// Layer error: E = tr(D H D^T) = ||D X^T||_F^2 with D = W - W^ [N, K] and
+// X [n_cal, K].  It is a dense contraction, so the scoring kernel is a
+// tcgen05 GEMM: decode warps write D (bf16, 128-byte swizzled, K-major) into
+// shared memory, TMA brings 256 calibration rows, one thread issues
+// 128 x 256 x 16 MMAs into a TMEM accumulator, and the epilogue sums the
+// squares of the 128 x 256 tile.  The sum over calibration rows is additive,
+// so calibration chunks of 256 rows are separate CTAs (no split-K reduction
+// before the square).
+
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "device_common.cuh"
+#include "encode_device.cuh"
+#include "tc_gemm.cuh"
+
+namespace stq1 {
+
+constexpr int kStq2BlockBytes = 66;
+constexpr int kStq2OffCodes = 2;
+
+// ---------------------------------------------------------------------------
+// STQ2 encoder: one thread per 256-weight block (staged in shared memory like
+// the STQ1_0 encoder).  d starts at fp16(amax) with each weight at its nearest
+// level (d m_q) / 3, m_q = 2q - 3 (ties: the lower code); then `rounds` times
+// d is refit by weighted least squares, d = 3 sum h w m / sum h m^2 (k
+// ascending), and the levels re-picked; the stored scale is fp16 of one more
+// fit.  Every real-valued step is fp64 with the round-to-nearest intrinsics,
+// so the bytes do not depend on contraction or scheduling.
+// ---------------------------------------------------------------------------
+constexpr int kStq2EncBlocks = 64;              // blocks (threads) per CTA
+
+__device__ __forceinline__ void stq2_pick(const float* w, double d, uint32_t (&qw)[16]) {
+  double lev[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) lev[q] = __ddiv_rn(__dmul_rn(d, static_cast<double>(2 * q - 3)), 3.0);
+#pragma unroll 1
+  for (int j = 0; j < 16; ++j) {
+    uint32_t word = 0;
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+      const double wk = static_cast<double>(w[16 * j + i]);
+      int best = 0;
+      double bd = fabs(__dsub_rn(wk, lev[0]));
+#pragma unroll
+      for (int q = 1; q < 4; ++q) {
+        const double dq = fabs(__dsub_rn(wk, lev[q]));
+        if (dq < bd) { bd = dq; best = q; }
+      }
+      word |= static_cast<uint32_t>(best) << (2 * i);
+    }
+    qw[j] = word;
+  }
+}
+
+__device__ __forceinline__ double stq2_wls(const float* w, const float* h, const uint32_t (&qw)[16]) {
+  double num = 0.0, den = 0.0;
+#pragma unroll 1
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t word = qw[j];
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+      const int k = 16 * j + i;
+      const double m = static_cast<double>(2 * static_cast<int>((word >> (2 * i)) & 3u) - 3);
+      const double hk = h ? static_cast<double>(h[k]) : 1.0;
+      num = __dadd_rn(num, __dmul_rn(__dmul_rn(hk, static_cast<double>(w[k])), m));
+      den = __dadd_rn(den, __dmul_rn(hk, __dmul_rn(m, m)));
+    }
+  }
+  return __ddiv_rn(__dmul_rn(3.0, num), den);
+}
+
+__global__ void __launch_bounds__(kStq2EncBlocks)
+stq2_encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long long n_blocks, int nb,
+                   int rounds, uint8_t* __restrict__ out) {
+  extern __shared__ float sw[];                   // [kStq2EncBlocks][kEncPitch]
+  const long long b0 = static_cast<long long>(blockIdx.x) * kStq2EncBlocks;
+  const int nblk = static_cast<int>(min(static_cast<long long>(kStq2EncBlocks), n_blocks - b0));
+  griddep_wait();                                 // W may come from the previous kernel
+  const float4* src = reinterpret_cast<const float4*>(W + b0 * kBlockWeights);
+  for (int f = threadIdx.x; f < nblk * (kBlockWeights / 4); f += kStq2EncBlocks) {
+    const float4 v = __ldg(src + f);
+    float* d = sw + (f >> 6) * kEncPitch + 4 * (f & 63);
+    d[0] = v.x;
+    d[1] = v.y;
+    d[2] = v.z;
+    d[3] = v.w;
+  }
+  __syncthreads();
+  if (threadIdx.x >= nblk) return;
+  const long long b = b0 + threadIdx.x;
+  const float* w = sw + threadIdx.x * kEncPitch;
+  const float* h = hcol ? hcol + (b % nb) * kBlockWeights : nullptr;
+  bool finite = true;
+  float amax = 0.f;
+  for (int k = 0; k < kBlockWeights; ++k) {
+    finite = finite && isfinite(w[k]);
+    amax = fmaxf(amax, fabsf(w[k]));
+  }
+  if (h) {
+    bool hany = false;
+    for (int k = 0; k < kBlockWeights; ++k) {
+      const float hk = h[k];
+      finite = finite && isfinite(hk) && hk >= 0.f;
+      hany = hany || hk != 0.f;
+    }
+    if (!hany) h = nullptr;                       // an all-zero importance block uses h = 1
+  }
+  uint16_t* o16 = reinterpret_cast<uint16_t*>(out + b * kStq2BlockBytes);   // 2-byte aligned
+  if (!finite) {
+    flag_error(STQ1_DEV_BAD_VALUE);
+    for (int i = 0; i < kStq2BlockBytes / 2; ++i) o16[i] = 0;
+    return;
+  }
+  uint16_t d_bits = enc_half_bits(static_cast<double>(amax));
+  uint32_t qw[16];
+  stq2_pick(w, static_cast<double>(__half2float(__ushort_as_half(d_bits))), qw);
+  if (rounds > 0) {
+    for (int r = 0; r < rounds; ++r) stq2_pick(w, stq2_wls(w, h, qw), qw);
+    d_bits = enc_half_bits(stq2_wls(w, h, qw));
+  }
+  o16[0] = d_bits;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) o16[1 + i] = static_cast<uint16_t>(qw[i >> 1] >> (16 * (i & 1)));
+}
+
+// ---------------------------------------------------------------------------
+// Diagonal of the calibration Hessian: h[l][k] = sum_r x[l][r][k]^2 (bf16
+// inputs; squares exact in fp64, summed in fp64, one rounding to fp32).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+hess_diag_kernel(const uint16_t* __restrict__ x, long long rows, long long K, float* __restrict__ h) {
+  const long long k = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  const long long l = blockIdx.y;
+  griddep_wait();
+  if (k >= K) return;
+  const uint16_t* xs = x + l * rows * K + k;
+  double s = 0.0;
+  for (long long r = 0; r < rows; ++r) {
+    const double v = static_cast<double>(bf16_bits_to_f32(__ldg(xs + r * K)));
+    s = __dadd_rn(s, __dmul_rn(v, v));
+  }
+  h[l * K + k] = __double2float_rn(s);
+}
+
+// ---------------------------------------------------------------------------
+// Layer error kernel.
+// ---------------------------------------------------------------------------
+constexpr int kHsM = 128;                       // weight rows per CTA (MMA M)
+constexpr int kHsKC = 64;                       // K per stage: one 128-byte atom of bf16
+constexpr int kHsMaxCal = 256;                  // calibration rows per CTA (MMA N)
+constexpr int kHsStages = 2;
+constexpr int kHsDecWarps = 8;
+constexpr int kHsThreads = 64 + 32 * kHsDecWarps;   // producer, MMA, decoders
+constexpr int kHsAStage = kHsM * 128;               // 16 KB
+constexpr int kHsBStage = kHsMaxCal * 128;          // 32 KB
+constexpr int kHsOffB = kHsStages * kHsAStage;
+constexpr int kHsOffBar = kHsOffB + kHsStages * kHsBStage;
+constexpr int kHsOffMisc = kHsOffBar + 128;
+constexpr int kHsSmemBytes = 1024 + kHsOffMisc + 16;   // two CTAs per SM
+
+struct HsArgs {
+  const float* W;           // [L][N][K] fp32
+  const uint8_t* packed;    // [L][N][K/256 * bb]
+  const float* h;           // [L][K] fp32 (diagonal of H)
+  double* out;              // [L][2]: full, diagonal (accumulated)
+  long long N, K;
+  int bb;                   // bytes per block: 42 (STQ1_0) or 66 (STQ2)
+  int n_mtiles, n_cchunks;
+  int box_rows;             // calibration rows per TMA box / MMA N (multiple of 16)
+  uint32_t tmem_cols;
+  uint32_t idesc;
+};
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], bf16 x bf16 -> fp32
+__device__ __forceinline__ void tc_mma_ss_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__host__ __device__ constexpr uint32_t hs_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(kHsM >> 4) << 24);
+}
+
+// Raw code bits of 8 consecutive columns (two groups) of one row, packed in
+// one word: the fp16 scale in bits 0-15, then (STQ1_0) the qs byte of the two
+// groups in bits 16-23 and their two select bits in bits 24-25, or (STQ2) the
+// 16 code bits in bits 16-31.
+template <int FMT>
+__device__ __forceinline__ uint32_t hs_load_raw(const uint8_t* blk, int k_in_block) {
+  const uint32_t d = __ldg(reinterpret_cast<const uint16_t*>(blk));
+  if constexpr (FMT == 0) {
+    const int g0 = k_in_block >> 2;                               // even group
+    const uint32_t qs = __ldg(blk + kOffQs + (g0 >> 1));
+    const uint32_t qh = (static_cast<uint32_t>(__ldg(blk + kOffQh + (g0 >> 3))) >> (g0 & 7)) & 3u;
+    return d | (qs << 16) | (qh << 24);
+  } else {
+    const uint32_t q = __ldg(reinterpret_cast<const uint16_t*>(blk + kStq2OffCodes + (k_in_block >> 2)));
+    return d | (q << 16);
+  }
+}
+
+// Decoded weights of those 8 columns (fp32).
+template <int FMT>
+__device__ __forceinline__ void hs_decode_raw(uint32_t raw, float wh[8]) {
+  const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(raw & 0xFFFFu)));
+  if constexpr (FMT == 0) {
+    const uint32_t qs = (raw >> 16) & 0xFFu, qh = raw >> 24;
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      // code = t << 4 | n: zero lane z = n >> 2; the non-zero lanes in order carry
+      // +1, -(bit 1 of n), -(bit 0 of n); t negates all three
+      const uint32_t n = (qs >> (4 * g)) & 15u, t = (qh >> g) & 1u;
+      const uint32_t z = n >> 2;
+      const float s = t ? -d : d;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t p = static_cast<uint32_t>(i) - (static_cast<uint32_t>(i) > z ? 1u : 0u);
+        const uint32_t neg = p == 1 ? ((n >> 1) & 1u) : (p == 2 ? (n & 1u) : 0u);
+        wh[4 * g + i] = (static_cast<uint32_t>(i) == z) ? 0.f : (neg ? -s : s);
+      }
+    }
+  } else {
+    const uint32_t q = raw >> 16;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      wh[i] = __fdiv_rn(d * static_cast<float>(2 * static_cast<int>((q >> (2 * i)) & 3u) - 3), 3.0f);
+  }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kHsThreads, 2)
+hess_score_kernel(const __grid_constant__ CUtensorMap xmap, const HsArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sbase = (sraw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - sraw);
+  const uint32_t sA = sbase, sB = sbase + kHsOffB;
+  const uint32_t bar = sbase + kHsOffBar;
+  // full_b[2] @0, full_a[2] @16, empty[2] @32, d_full @48, drain @56
+  const uint32_t bar_full_b = bar, bar_full_a = bar + 16, bar_empty = bar + 32;
+  const uint32_t bar_d_full = bar + 48, bar_drain = bar + 56;
+  volatile int* s_misc = reinterpret_cast<volatile int*>(sgen + kHsOffMisc);   // [0] tmem, [1] abort
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int item = blockIdx.x;
+  const int cc = item % a.n_cchunks;
+  const int mt = (item / a.n_cchunks) % a.n_mtiles;
+  const int l = item / (a.n_cchunks * a.n_mtiles);
+  const int n_steps = static_cast<int>(a.K / kHsKC);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kHsStages; ++i) {
+      mbar_init(bar_full_b + 8 * i, 1);
+      mbar_init(bar_full_a + 8 * i, kHsDecWarps);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    mbar_init(bar_d_full, 1);
+    mbar_init(bar_drain, 1);
+    s_misc[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + kHsOffMisc, a.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(s_misc[0]);
+  volatile int* abort = s_misc + 1;
+  griddep_wait();                                    // inputs may come from the previous kernel
+
+  if (warp == 0) {
+    // ---------------- TMA producer: calibration rows ----------------
+    if (lane == 0) {
+      int ks = 0;
+      for (; ks < n_steps && !*abort; ++ks) {
+        const uint32_t s = ks % kHsStages, use = ks / kHsStages;
+        if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) { *abort = 1; break; }
+        mbar_arrive_expect_tx(bar_full_b + 8 * s, static_cast<uint32_t>(a.box_rows) * 128u);
+        tma_load_3d(sB + s * kHsBStage, &xmap, ks * kHsKC, cc * kHsMaxCal, l, bar_full_b + 8 * s);
+      }
+      // let the copies in flight land before the CTA can exit (bounded)
+      for (int j = ks > kHsStages ? ks - kHsStages : 0; j < ks; ++j)
+        mbar_wait_bounded(bar_full_b + 8 * (j % kHsStages), (j / kHsStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      for (int ks = 0; ks < n_steps && !*abort; ++ks) {
+        const uint32_t s = ks % kHsStages, use = ks / kHsStages;
+        if (!mbar_wait_bounded(bar_full_b + 8 * s, use & 1) ||
+            !mbar_wait_bounded(bar_full_a + 8 * s, use & 1)) { *abort = 1; break; }
+        tc_fence_after();
+        const uint64_t adesc = smem_desc_sw128(sA + s * kHsAStage);
+        const uint64_t bdesc = smem_desc_sw128(sB + s * kHsBStage);
+#pragma unroll
+        for (int kk = 0; kk < kHsKC / 16; ++kk)
+          tc_mma_ss_bf16(tmem, adesc + 2 * kk, bdesc + 2 * kk, a.idesc, (ks | kk) != 0 ? 1u : 0u);
+        tc_commit(bar_empty + 8 * s);
+      }
+      if (!*abort) tc_commit(bar_d_full);
+      // every MMA issued so far has completed once this arrives
+      tc_commit(bar_drain);
+      mbar_wait_bounded(bar_drain, 0);
+    }
+  } else {
+    // ---------------- decoders, then the epilogue ----------------
+    const int t = threadIdx.x - 64;
+    const int c = t & 7;                       // 8-column chunk within the 64-column step
+    const int r0 = t >> 3;                     // rows r0 + 32 i
+    const long long nb = a.K / kBlockWeights;
+    const bool want_diag = (cc == 0);
+    double diag = 0.0;
+    for (int ks = 0; ks < n_steps && !*abort; ++ks) {
+      const uint32_t s = ks % kHsStages, use = ks / kHsStages;
+      const long long k0 = static_cast<long long>(ks) * kHsKC + c * 8;
+      const long long blkk = k0 / kBlockWeights;
+      const int kin = static_cast<int>(k0 % kBlockWeights);
+      float hk[8];
+      if (want_diag) {
+        const float4* hp = reinterpret_cast<const float4*>(a.h + l * a.K + k0);
+        const float4 h0 = __ldg(hp), h1 = __ldg(hp + 1);
+        hk[0] = h0.x; hk[1] = h0.y; hk[2] = h0.z; hk[3] = h0.w;
+        hk[4] = h1.x; hk[5] = h1.y; hk[6] = h1.z; hk[7] = h1.w;
+      }
+      // loads first: they do not need the shared-memory slot
+      float4 wv[4][2];
+      uint32_t raw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const long long row = static_cast<long long>(mt) * kHsM + r0 + 32 * i;
+        if (row < a.N) {
+          const float4* wp = reinterpret_cast<const float4*>(a.W + (l * a.N + row) * a.K + k0);
+          wv[i][0] = __ldcs(wp);
+          wv[i][1] = __ldcs(wp + 1);
+          raw[i] = hs_load_raw<FMT>(a.packed + ((l * a.N + row) * nb + blkk) * a.bb, kin);
+        } else {
+          wv[i][0] = wv[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+          raw[i] = 0;                            // d = 0: decodes to zeros
+        }
+      }
+      if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) { *abort = 1; break; }
+      float part = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = r0 + 32 * i;
+        const float w8[8] = {wv[i][0].x, wv[i][0].y, wv[i][0].z, wv[i][0].w,
+                             wv[i][1].x, wv[i][1].y, wv[i][1].z, wv[i][1].w};
+        float wh[8], dv[8];
+        hs_decode_raw<FMT>(raw[i], wh);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dv[e] = w8[e] - wh[e];
+        if (want_diag) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) part = fmaf(hk[e] * dv[e], dv[e], part);
+        }
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 p2 = __floats2bfloat162_rn(dv[2 * e], dv[2 * e + 1]);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&p2);
+        }
+        const uint32_t dst = sA + s * kHsAStage + r * 128 + ((c ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
+                     "r"(pk[2]), "r"(pk[3])
+                     : "memory");
+      }
+      diag += static_cast<double>(part);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_full_a + 8 * s);
+    }
+    // diagonal score: once per (layer, row tile)
+    if (want_diag) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) diag += __shfl_xor_sync(0xffffffffu, diag, o);
+      if (lane == 0 && !*abort) atomicAdd(a.out + 2 * l + 1, diag);
+    }
+    // full score: sum of squares of the accumulator tile
+    double full = 0.0;
+    if (!*abort && mbar_wait_bounded(bar_d_full, 0)) {
+      tc_fence_after();
+      const int q = warp & 3;                       // TMEM lane quarter this warp may access
+      const int half = (warp - 2) >> 2;
+      for (int j = half; j < a.box_rows / 16; j += 2) {
+        uint32_t v[16];
+        STQ1_TMEM_LD16(tmem + (static_cast<uint32_t>(32 * q) << 16) + 16 * j, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const double y = static_cast<double>(__uint_as_float(v[e]));
+          full += y * y;
+        }
+      }
+    } else {
+      *abort = 1;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) full += __shfl_xor_sync(0xffffffffu, full, o);
+    if (lane == 0 && !*abort) atomicAdd(a.out + 2 * l, full);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, a.tmem_cols);
+  }
+}
+
+}  // namespace stq1

@@ -11,6 +11,7 @@
 #include "device_common.cuh"
 #include "encode_device.cuh"
 #include "gemv_lut.cuh"
+#include "mix_score.cuh"
 #include "small_kernels.cuh"
 #include "tc_gemm.cuh"
 
@@ -101,7 +102,13 @@ int ensure_configured() {
       cudaFuncSetAttribute(tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kTcSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(encode_smem_bytes())) != cudaSuccess)
+                           static_cast<int>(encode_smem_bytes())) != cudaSuccess ||
+      cudaFuncSetAttribute(stq2_encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kStq2EncBlocks * kEncPitch * sizeof(float))) != cudaSuccess ||
+      cudaFuncSetAttribute(hess_score_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kHsSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(hess_score_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kHsSmemBytes) != cudaSuccess)
     return STQ1_ERR_CUDA;
   // split-K clusters of up to 16 CTAs (above the portable 8); a refusal only
   // disables the cluster path
@@ -876,4 +883,95 @@ extern "C" int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float*
   else
     lut_gemv_kernel<4><<<grid, kLutThreads, smem, s>>>(maps.w, maps.t, a);
   return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Mixed-precision allocation: STQ2 encoder, Hessian diagonal, layer error.
+// ---------------------------------------------------------------------------
+
+extern "C" int stq1_quantize_stq2(const float* W, const float* h, int64_t N, int64_t K, int rounds, uint8_t* out,
+                                  void* stream) {
+  if (!W || !out) return STQ1_ERR_NULL;
+  if (N <= 0 || K <= 0 || K % kBlockWeights || N > (1LL << 40) / K) return STQ1_ERR_SHAPE;
+  if (rounds < 0 || rounds > 1000) return STQ1_ERR_ARG;
+  if (!aligned16(W) || (reinterpret_cast<uintptr_t>(out) & 1) || (reinterpret_cast<uintptr_t>(h) & 3))
+    return STQ1_ERR_ALIGN;
+  const long long n_blocks = N * (K / kBlockWeights);
+  const long long grid = (n_blocks + kStq2EncBlocks - 1) / kStq2EncBlocks;
+  if (grid >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  int rc = ensure_configured();
+  if (rc != STQ1_OK) return rc;
+  return launch_pdl(stq2_encode_kernel, static_cast<unsigned>(grid), kStq2EncBlocks,
+                    static_cast<size_t>(kStq2EncBlocks) * kEncPitch * sizeof(float), static_cast<cudaStream_t>(stream),
+                    W, h, n_blocks, static_cast<int>(K / kBlockWeights), rounds, out);
+}
+
+extern "C" int stq1_hessian_diag(const uint16_t* x, int64_t L, int64_t rows, int64_t K, float* h, void* stream) {
+  if (!x || !h) return STQ1_ERR_NULL;
+  if (L <= 0 || rows <= 0 || K <= 0 || L > 65535 || rows > (1LL << 40) / K || L > (1LL << 40) / (rows * K))
+    return STQ1_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(x) & 1) || (reinterpret_cast<uintptr_t>(h) & 3)) return STQ1_ERR_ALIGN;
+  const long long gx = (K + 255) / 256;
+  if (gx >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  return launch_pdl_cluster(hess_diag_kernel, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(L)), 256, 0,
+                            static_cast<cudaStream_t>(stream), 1u, x, static_cast<long long>(rows),
+                            static_cast<long long>(K), h);
+}
+
+namespace {
+
+// 3-D map over calibration rows [L][n_cal][K] of bf16: box = 64 columns (one
+// 128-byte swizzle atom) x box_rows rows x 1 layer; rows past n_cal read as zero.
+bool make_cal_map(CUtensorMap* map, const void* base, long long L, long long n_cal, long long K, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(n_cal), static_cast<cuuint64_t>(L)};
+  cuuint64_t gstride[2] = {static_cast<cuuint64_t>(K) * 2, static_cast<cuuint64_t>(n_cal * K) * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kHsKC), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" int stq1_hessian_error(int format, const void* packed, const float* W, const uint16_t* x,
+                                  const float* h, int64_t L, int64_t N, int64_t K, int64_t n_cal, double* out,
+                                  void* stream) {
+  if (!packed || !W || !x || !h || !out) return STQ1_ERR_NULL;
+  if (format != STQ1_FMT_STQ1_0 && format != STQ1_FMT_STQ2) return STQ1_ERR_ARG;
+  if (L <= 0 || N <= 0 || n_cal <= 0 || K < kBlockWeights || K % kBlockWeights) return STQ1_ERR_SHAPE;
+  if (K > (1LL << 31) - 1 || n_cal > (1LL << 31) - 1 || L > (1LL << 31) - 1) return STQ1_ERR_SHAPE;
+  if (N > (1LL << 40) / K || L > (1LL << 40) / (N * K) || L > (1LL << 40) / (n_cal * K)) return STQ1_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(x) || !aligned16(h) || (reinterpret_cast<uintptr_t>(packed) & 1) ||
+      (reinterpret_cast<uintptr_t>(out) & 7))
+    return STQ1_ERR_ALIGN;
+  const long long n_mtiles = (N + kHsM - 1) / kHsM;
+  const long long n_cchunks = (n_cal + kHsMaxCal - 1) / kHsMaxCal;
+  const long long items = L * n_mtiles * n_cchunks;
+  if (items >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  int rc = ensure_configured();
+  if (rc != STQ1_OK) return rc;
+  const int box_rows = static_cast<int>(std::min<long long>(kHsMaxCal, (n_cal + 15) / 16 * 16));
+  CUtensorMap map;
+  if (!make_cal_map(&map, x, L, n_cal, K, box_rows)) return STQ1_ERR_CUDA;
+  HsArgs a{};
+  a.W = W;
+  a.packed = static_cast<const uint8_t*>(packed);
+  a.h = h;
+  a.out = out;
+  a.N = N;
+  a.K = K;
+  a.bb = format == STQ1_FMT_STQ1_0 ? kBlockBytes : kStq2BlockBytes;
+  a.n_mtiles = static_cast<int>(n_mtiles);
+  a.n_cchunks = static_cast<int>(n_cchunks);
+  a.box_rows = box_rows;
+  a.tmem_cols = box_rows <= 32 ? 32u : (box_rows <= 64 ? 64u : (box_rows <= 128 ? 128u : 256u));
+  a.idesc = hs_idesc(box_rows);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(out, 0, static_cast<size_t>(L) * 2 * sizeof(double), s) != cudaSuccess) return STQ1_ERR_CUDA;
+  if (format == STQ1_FMT_STQ1_0)
+    return launch_pdl(hess_score_kernel<0>, static_cast<unsigned>(items), kHsThreads, kHsSmemBytes, s, map, a);
+  return launch_pdl(hess_score_kernel<1>, static_cast<unsigned>(items), kHsThreads, kHsSmemBytes, s, map, a);
 }

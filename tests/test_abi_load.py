@@ -75,3 +75,24 @@ def test_host_side_argument_checks_need_no_gpu():
     assert L.stq1_quantize_x_e4m3(1 << 20, 4, 250, 1 << 20, 1 << 20, None) == -1
     assert L.stq1_quantize_x_e4m3(1 << 20, 0, 256, 1 << 20, 1 << 20, None) == -1
     assert L.stq1_quantize_x_e4m3((1 << 20) + 2, 4, 256, 1 << 20, 1 << 20, None) == -6
+    # mixed-precision allocation entries
+    assert L.stq1_quantize_stq2(None, None, 4, 256, 0, 1 << 20, None) == -2
+    assert L.stq1_quantize_stq2(1 << 20, None, 0, 256, 0, 1 << 20, None) == -1
+    assert L.stq1_quantize_stq2(1 << 20, None, 4, 300, 0, 1 << 20, None) == -1
+    assert L.stq1_quantize_stq2(1 << 20, None, 4, 256, -1, 1 << 20, None) == -8
+    assert L.stq1_quantize_stq2((1 << 20) + 4, None, 4, 256, 0, 1 << 20, None) == -6
+    assert L.stq1_quantize_stq2(1 << 20, (1 << 20) + 2, 4, 256, 3, 1 << 20, None) == -6
+    assert L.stq1_hessian_diag(None, 1, 4, 256, 1 << 20, None) == -2
+    assert L.stq1_hessian_diag(1 << 20, 0, 4, 256, 1 << 20, None) == -1
+    assert L.stq1_hessian_diag(1 << 20, 1, 0, 256, 1 << 20, None) == -1
+    assert L.stq1_hessian_diag(1 << 20, 70000, 4, 256, 1 << 20, None) == -1
+    P = 1 << 20
+    assert L.stq1_hessian_error(0, None, P, P, P, 1, 4, 256, 4, P, None) == -2
+    assert L.stq1_hessian_error(2, P, P, P, P, 1, 4, 256, 4, P, None) == -8
+    assert L.stq1_hessian_error(0, P, P, P, P, 1, 4, 300, 4, P, None) == -1
+    assert L.stq1_hessian_error(0, P, P, P, P, 0, 4, 256, 4, P, None) == -1
+    assert L.stq1_hessian_error(0, P, P, P, P, 1, 0, 256, 4, P, None) == -1
+    assert L.stq1_hessian_error(0, P, P, P, P, 1, 4, 256, 0, P, None) == -1
+    assert L.stq1_hessian_error(1, P + 1, P, P, P, 1, 4, 256, 4, P, None) == -6
+    assert L.stq1_hessian_error(1, P, P, P + 8, P, 1, 4, 256, 4, P, None) == -6
+    assert L.stq1_hessian_error(1, P, P, P, P, 1, 4, 256, 4, P + 4, None) == -6

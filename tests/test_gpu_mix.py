@@ -1,0 +1,231 @@
+"""Mixed-precision allocation kernels against the oracle (needs a B200).
+
+- stq1_quantize_stq2: byte-identical to the oracle's encode_stq2, plain and
+  importance-fitted (the scale fits and level choices are fp64 on both sides,
+  in the same evaluation order).
+- stq1_hessian_diag: within one fp32 rounding of the oracle's fp64 sum.
+- stq1_hessian_error: the full score tr(D H D^T) forms D in fp32 and rounds it to
+  bf16 for the tensor cores (fp32 accumulation).  Rounding to nearest is
+  zero-mean, so over many (calibration row, output row) pairs the relative
+  effect on the score stays of order 2^-8 / sqrt(pairs) plus a bias of order
+  2^-16; a CPU replay of that rounding on the shapes below gave at most 4.1e-5,
+  and the test allows 1e-3 where there are at least 1024 pairs.  Below that the
+  test uses the worst-case bound: each output y_cj may move by
+  (2^-8 + (K + 2) 2^-24) sum_k |D_jk x_ck|.  The diagonal score is formed from
+  the fp32 D in fp32 partial sums: relative 1e-5.
+- stq1_mix_allocate on the GPU scores picks exactly what the oracle's greedy
+  picks on the same numbers.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import sub_bit_sparse_b200 as stq1
+
+U_BF16 = 2.0 ** -8
+REL_FULL = 1e-3
+REL_DIAG = 1e-5
+
+
+def _dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return t if dtype is None else t.view(dtype)
+
+
+# ---------------------------------------------------------------------------
+# STQ2 encoder
+# ---------------------------------------------------------------------------
+
+
+def _stq2_gpu(w, h=None, rounds=0):
+    hd = None if h is None else _dev(np.asarray(h, np.float32))
+    out = stq1.stq2_quantize(_dev(w.astype(np.float32)), hd, rounds=rounds).cpu().numpy()
+    assert stq1.status() == 0
+    return out
+
+
+def _stq2_edge_matrix():
+    rng = np.random.default_rng(2718)
+    w = (rng.standard_normal((6, 1024)) * 0.02).astype(np.float32)
+    w[0, 0:256] = 0.0                                       # d = 0: every weight takes code 0
+    w[1, 0:256] = np.tile([3.0, 0.0, 2.0, -2.0], 64)        # midway values: ties to the lower code
+    w[1, 256:512] = -0.0
+    w[2, 0:256] *= 1e7                                      # d saturates at 65504
+    w[2, 256:512] = 70000.0                                 # amax past the fp16 range
+    w[3, 0:256] *= 1e-6                                     # subnormal fp16 scales
+    w[4, 512:768] = rng.choice([-3.0, -1.0, 1.0, 3.0], 256)  # exactly on the levels
+    return w
+
+
+@pytest.mark.parametrize("rounds", [0, 1, 3])
+@pytest.mark.parametrize("shape", [(1, 256), (7, 1024), (129, 2048)])
+def test_stq2_encoder_matches_oracle(shape, rounds):
+    n, k = shape
+    w = workloads.expert_like_matrix(n, k, seeds=(n, k, 9))
+    h = workloads.calibration_importance(k, seed=k)
+    assert np.array_equal(_stq2_gpu(w, h, rounds), oracle.encode_stq2(w, h, rounds=rounds))
+    if rounds:
+        assert np.array_equal(_stq2_gpu(w, None, rounds), oracle.encode_stq2(w, None, rounds=rounds))
+
+
+@pytest.mark.parametrize("rounds", [0, 3])
+def test_stq2_encoder_edge_blocks(rounds):
+    w = _stq2_edge_matrix()
+    h = workloads.calibration_importance(1024, seed=3)
+    h[256:512] = 0.0                                     # a block column with zero importance
+    h[700] = 0.0
+    for hh in (h, None):
+        assert np.array_equal(_stq2_gpu(w, hh, rounds), oracle.encode_stq2(w, hh, rounds=rounds))
+
+
+def test_stq2_encoder_full_layer_sampled():
+    # one [4096, 7168] layer, fitted to its calibration importance: 64 sampled rows
+    w, x = workloads.mix_layer(4096, 7168, 64, layer=0, seed=31)
+    h = _h_oracle(x)
+    g = _stq2_gpu(w, h, 3).reshape(4096, -1)
+    rows = np.random.default_rng(1).choice(4096, 64, replace=False)
+    assert np.array_equal(g[rows], oracle.encode_stq2(w[rows], h, rounds=3).reshape(64, -1))
+
+
+def test_stq2_encoder_flags_non_finite():
+    w = np.zeros((2, 512), np.float32)
+    w[0, 3] = np.nan
+    w[1, 300] = np.inf
+    out = stq1.stq2_quantize(_dev(w), rounds=2).cpu().numpy()
+    assert stq1.status() & stq1.DEV_BAD_VALUE
+    assert not out.reshape(4, 66)[[0, 3]].any()
+
+
+# ---------------------------------------------------------------------------
+# Hessian diagonal and layer error
+# ---------------------------------------------------------------------------
+
+
+def _layers(n_layers, n, k, n_cal, seed):
+    ws, xs = zip(*(workloads.mix_layer(n, k, n_cal, layer=l, seed=seed) for l in range(n_layers)))
+    return np.stack(ws), np.stack(xs)
+
+
+def _h_oracle(x_bits):
+    x = workloads.f32_from_bf16_bits(x_bits).astype(np.float64)
+    return np.sum(x * x, axis=-2).astype(np.float32)
+
+
+def test_hessian_diag_matches_oracle():
+    _, x = _layers(3, 8, 768, 37, seed=5)
+    h = stq1.hessian_diag(_dev(x, torch.bfloat16)).cpu().numpy()
+    want = _h_oracle(x)
+    assert np.all(np.abs(h.astype(np.float64) - want) <= np.spacing(want).astype(np.float64))
+
+
+def _check_scores(got, w, packed, x_bits, h, fmt, n, k):
+    x = workloads.f32_from_bf16_bits(x_bits).astype(np.float64)
+    wh = oracle.decode(packed, n, k) if fmt == stq1.FMT_STQ1_0 else oracle.decode_stq2(packed, n, k)
+    full = oracle.hessian_error(w, wh, x)
+    diag = oracle.diagonal_error(w, wh, x)
+    pairs = n * x.shape[0]
+    if pairs >= 1024:
+        assert abs(got[0] - full) <= REL_FULL * full, (got[0], full)
+    else:
+        d = w.astype(np.float64) - wh
+        y = d @ x.T
+        e = (U_BF16 + (k + 2) * 2.0 ** -24) * (np.abs(d) @ np.abs(x).T)
+        assert abs(got[0] - full) <= float(np.sum(e * (2 * np.abs(y) + e))) + 1e-300, (got[0], full)
+    # the device takes h rounded to fp32; the oracle's diagonal uses the exact sum
+    assert abs(got[1] - diag) <= REL_DIAG * diag + 1e-300, (got[1], diag)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("n,k,n_cal", [(300, 768, 40), (300, 768, 300), (128, 512, 256), (1, 256, 1),
+                                       (5, 256, 17)])
+def test_hessian_error_matches_oracle(fmt, n, k, n_cal):
+    n_layers = 3 if n * k * n_cal < 1e8 else 1
+    w, x = _layers(n_layers, n, k, n_cal, seed=n + k + n_cal)
+    h = _h_oracle(x)
+    if fmt == stq1.FMT_STQ1_0:
+        packed = [oracle.encode_sherry(w[l], h[l], rounds=3) for l in range(n_layers)]
+    else:
+        packed = [oracle.encode_stq2(w[l], h[l], rounds=3) for l in range(n_layers)]
+    got = stq1.hessian_error(fmt, _dev(np.concatenate(packed)), _dev(w), _dev(x, torch.bfloat16),
+                             _dev(h)).cpu().numpy()
+    assert stq1.status() == 0
+    for l in range(n_layers):
+        _check_scores(got[l], w[l], packed[l], x[l], h[l], fmt, n, k)
+
+
+def test_hessian_error_zero_difference_is_zero():
+    # weights that STQ2 represents exactly: both scores are exactly zero
+    rng = np.random.default_rng(4)
+    w = (rng.choice([-3.0, -1.0, 1.0, 3.0], size=(1, 130, 512)) * 0.25).astype(np.float32)
+    w[:, :, ::256] = 0.75                                   # amax 0.75 in every block
+    _, x = _layers(1, 8, 512, 64, seed=3)
+    packed = oracle.encode_stq2(w[0])
+    assert np.array_equal(oracle.decode_stq2(packed, 130, 512), w[0].astype(np.float64))
+    got = stq1.hessian_error(stq1.FMT_STQ2, _dev(packed), _dev(w), _dev(x, torch.bfloat16),
+                             _dev(_h_oracle(x))).cpu().numpy()
+    assert np.array_equal(got, np.zeros((1, 2)))
+
+
+def _oracle_packed(fmt, w, h):
+    return (oracle.encode_sherry(w, h, rounds=3) if fmt == stq1.FMT_STQ1_0
+            else oracle.encode_stq2(w, h, rounds=3))
+
+
+def test_hessian_error_full_layer_shape():
+    # the study's layer shape ([4096, 7168], 512 calibration rows), two layers,
+    # in the launch configuration the study uses (all layers in one call);
+    # the oracle encodes and scores both layers in full
+    n, k, n_cal = 4096, 7168, 512
+    w, x = _layers(2, n, k, n_cal, seed=77)
+    h = _h_oracle(x)
+    wd, xd, hd = _dev(w), _dev(x, torch.bfloat16), _dev(h)
+    for fmt in (stq1.FMT_STQ1_0, stq1.FMT_STQ2):
+        packed = [_oracle_packed(fmt, w[l], h[l]) for l in range(2)]
+        got = stq1.hessian_error(fmt, _dev(np.concatenate(packed)), wd, xd, hd).cpu().numpy()
+        assert stq1.status() == 0
+        for l in range(2):
+            _check_scores(got[l], w[l], packed[l], x[l], h[l], fmt, n, k)
+
+
+def test_allocation_from_gpu_scores_agrees_with_the_oracle():
+    # same encoded layers on both sides; only the scoring precision differs, so
+    # the picks agree wherever the gains at the budget's edge are not near-ties
+    n_layers, n, k, n_cal = 12, 256, 1024, 128
+    w, x = _layers(n_layers, n, k, n_cal, seed=12)
+    h = _h_oracle(x)
+    p1 = [_oracle_packed(stq1.FMT_STQ1_0, w[l], h[l]) for l in range(n_layers)]
+    p2 = [_oracle_packed(stq1.FMT_STQ2, w[l], h[l]) for l in range(n_layers)]
+    wd, xd, hd = _dev(w), _dev(x, torch.bfloat16), _dev(h)
+    g1 = stq1.hessian_error(stq1.FMT_STQ1_0, _dev(np.concatenate(p1)), wd, xd, hd).cpu().numpy()
+    g2 = stq1.hessian_error(stq1.FMT_STQ2, _dev(np.concatenate(p2)), wd, xd, hd).cpu().numpy()
+    xf = workloads.f32_from_bf16_bits(x).astype(np.float64)
+    o1 = np.array([oracle.hessian_error(w[l], oracle.decode(p1[l], n, k), xf[l]) for l in range(n_layers)])
+    o2 = np.array([oracle.hessian_error(w[l], oracle.decode_stq2(p2[l], n, k), xf[l]) for l in range(n_layers)])
+    bl = np.full(n_layers, n * k // 256 * 42.0)
+    bh = np.full(n_layers, n * k // 256 * 66.0)
+    budget = float(np.sum(bl) + 5 * (bh[0] - bl[0]))
+    gains = np.sort((o1 - o2) / (bh - bl))[::-1]
+    margin = (gains[4] - gains[5]) / abs(gains[4])
+    got = stq1.mix_allocate(g1[:, 0], g2[:, 0], bl, bh, budget)
+    want = oracle.greedy_allocate(o1, o2, bl, bh, budget)
+    assert got.sum() == want.sum() == 5
+    if margin > 4 * REL_FULL:
+        assert np.array_equal(got, want)
+
+
+def test_hessian_error_rejects_bad_arguments():
+    w = torch.zeros((1, 4, 256), dtype=torch.float32, device="cuda")
+    x = torch.zeros((1, 4, 256), dtype=torch.bfloat16, device="cuda")
+    h = torch.zeros((1, 256), dtype=torch.float32, device="cuda")
+    pk = torch.zeros(4 * 66, dtype=torch.uint8, device="cuda")
+    with pytest.raises(stq1.Stq1Error):
+        stq1.hessian_error(7, pk, w, x, h)
+    with pytest.raises(stq1.Stq1Error):
+        stq1.hessian_error(1, pk, w[:, :, :128].contiguous(), x[:, :, :128].contiguous(), h[:, :128].contiguous())

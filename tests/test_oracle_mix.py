@@ -5,8 +5,8 @@ error reduction per added byte, between STQ1_0 and a 2.06-bpw partner format
 ("AngelSlim Shrinks ..." bullet list; lemmy.durstig.online post 66506,
 "Full-Hessian scoring").  The partner here is STQ2, this library's 2-bit
 format at the same rate.  Each check ties the oracle to something outside it:
-hand-built blocks with known codes and ties, the per-row sum of squares that
-tr(D H D^T) equals, the diagonal form when calibration columns are orthogonal,
+hand-built blocks with known codes and ties, tr(D H D^T) written out with H
+formed explicitly, the diagonal form when calibration columns are orthogonal,
 and brute force over all layer subsets where greedy is optimal.
 """
 
@@ -80,25 +80,75 @@ def test_stq2_beats_stq1_on_gaussian_weights():
     assert e2 < 0.6 * e1
 
 
+def test_stq2_wls_scale_is_the_weighted_least_squares_minimiser():
+    # against a library least-squares solve of the sqrt(h)-weighted system
+    rng = np.random.default_rng(21)
+    wb = rng.standard_normal((5, 256)) * 0.02
+    hb = rng.uniform(0.0, 4.0, (5, 256))
+    q = rng.integers(0, 4, (5, 256))
+    got = oracle.stq2_wls_scale(wb, hb, q)
+    for b in range(5):
+        a = (np.sqrt(hb[b]) * (2.0 * q[b] - 3.0) / 3.0)[:, None]
+        want = np.linalg.lstsq(a, np.sqrt(hb[b]) * wb[b], rcond=None)[0][0]
+        assert got[b] == pytest.approx(want, rel=1e-12)
+
+
+def test_stq2_fit_never_increases_the_weighted_error():
+    w = workloads.expert_like_matrix(8, 1024, seeds=(31, 32, 33))
+    h = workloads.calibration_importance(1024, seed=34)
+    _, tr = oracle.encode_stq2(w, h, rounds=5, trace=True)
+    wb = w.reshape(-1, 256).astype(np.float64)
+    hb = tr["h_blocks"]
+    errs = [oracle.stq2_weighted_error(wb, hb, d, q) for d, q in tr["rounds"]]
+    for a, b in zip(errs, errs[1:]):
+        assert np.all(b <= a * (1 + 1e-12) + 1e-300)
+    assert np.sum(errs[-1]) < 0.95 * np.sum(errs[0])
+
+
+def test_stq2_fit_follows_the_important_columns():
+    # one large weight on an unimportant column sets amax; the fit shrinks d
+    # towards the small weights that carry the importance
+    w = np.full((1, 256), 0.01, np.float32)
+    w[0, 0] = 1.0
+    h = np.ones(256, np.float32)
+    h[0] = 1e-6
+    plain = oracle.encode_stq2(w)
+    fitted = oracle.encode_stq2(w, h, rounds=3)
+    d_plain = oracle.fp16_value(plain[0] | (np.uint16(plain[1]) << 8))
+    d_fit = oracle.fp16_value(fitted[0] | (np.uint16(fitted[1]) << 8))
+    assert d_plain == oracle.fp16_value(oracle.fp16_bits(1.0))
+    assert d_fit < 0.1
+    err = lambda p: float(np.sum(h * (w[0] - oracle.decode_stq2(p, 1, 256)[0]) ** 2))
+    assert err(fitted) < 0.01 * err(plain)
+
+
+def test_stq2_zero_importance_block_uses_unit_weights():
+    w = workloads.gaussian_matrix(2, 512, 0.02, seed=8)
+    h = np.ones(512, np.float32)
+    h[:256] = 0.0
+    a = oracle.encode_stq2(w, h, rounds=2)
+    b = oracle.encode_stq2(w, np.ones(512, np.float32), rounds=2)
+    assert np.array_equal(a.reshape(2, 2, 66)[:, 0], b.reshape(2, 2, 66)[:, 0])
+
+
 # ---------------------------------------------------------------------------
 # Layer error under the full and the diagonal Hessian
 # ---------------------------------------------------------------------------
 
 
 def _brute_force_error(w, wh, x):
-    """sum over calibration rows c and output rows j of (sum_k D_jk x_ck)^2, as loops."""
+    """The definition, as loops: H_kl = sum_c x_ck x_cl, then sum_j sum_k sum_l D_jk H_kl D_jl."""
     n, k = w.shape
+    h = [[sum(float(x[c, a]) * float(x[c, b]) for c in range(x.shape[0])) for b in range(k)] for a in range(k)]
     total = 0.0
-    for c in range(x.shape[0]):
-        for j in range(n):
-            s = 0.0
-            for i in range(k):
-                s += (float(w[j, i]) - float(wh[j, i])) * float(x[c, i])
-            total += s * s
+    for j in range(n):
+        for a in range(k):
+            for b in range(k):
+                total += (float(w[j, a]) - float(wh[j, a])) * h[a][b] * (float(w[j, b]) - float(wh[j, b]))
     return total
 
 
-def test_hessian_error_equals_the_sum_of_squared_outputs():
+def test_hessian_error_equals_the_trace_definition():
     rng = np.random.default_rng(3)
     w = rng.standard_normal((3, 8))
     wh = rng.standard_normal((3, 8))
@@ -217,16 +267,18 @@ def test_greedy_budget_extremes():
     assert oracle.greedy_allocate(el, eh, bl, bh, budget=48.0).all()
 
 
-@pytest.mark.parametrize("mistake", ["diagonal_for_full", "gain_without_bytes", "stq2_levels_by_half"])
+@pytest.mark.parametrize("mistake", ["diagonal_for_full", "gain_without_bytes", "stq2_levels_by_half",
+                                     "stq2_fit_unweighted"])
 def test_planted_mix_mistakes_are_caught(monkeypatch, mistake):
     import oracle.stq1 as o
 
     def passes():
         try:
             test_stq2_hand_built_block()
-            test_hessian_error_equals_the_sum_of_squared_outputs()
+            test_hessian_error_equals_the_trace_definition()
             test_diagonal_misses_correlation()
             test_greedy_orders_by_reduction_per_byte_not_by_reduction()
+            test_stq2_wls_scale_is_the_weighted_least_squares_minimiser()
         except AssertionError:
             return False
         return True
@@ -248,6 +300,9 @@ def test_planted_mix_mistakes_are_caught(monkeypatch, mistake):
                     pick[i], total = True, total + bh[i] - bl[i]
             return pick
         plant("greedy_allocate", by_reduction)
+    elif mistake == "stq2_fit_unweighted":
+        orig_wls = o.stq2_wls_scale
+        plant("stq2_wls_scale", lambda wb, hb, q: orig_wls(wb, np.ones_like(hb), q))
     elif mistake == "stq2_levels_by_half":
         orig_dec = o.decode_stq2
         plant("decode_stq2", lambda p, n, k: orig_dec(p, n, k) * 1.5)

@@ -212,3 +212,63 @@ def gateup_outputs(p: int, n: int, seed: int) -> np.ndarray:
     flat[idx] = rng.choice([-1e3, 1e3, 0.0], size=idx.size)
     return y.astype(np.float32)
 
+
+
+# ---------------------------------------------------------------------------
+# Mixed-precision allocation study: one [n, k] matrix and n_cal calibration
+# rows per layer, with layer-to-layer differences in how strongly the
+# calibration channels are correlated and how much of the weights lie along
+# the correlated directions (the pages score 77 MoE layers; lemmy.durstig.online
+# post 66506, "Full-Hessian scoring").
+# ---------------------------------------------------------------------------
+
+MIX_RANK = 16
+
+
+def mix_layer_params(layer: int, seed: int):
+    """(rho, beta) of a layer: correlation strength of the calibration channels
+    in [0, 0.9] and weight alignment with the shared directions in [0, 1]."""
+    rng = np.random.default_rng([seed, layer, 0])
+    return float(rng.uniform(0.0, 0.9)), float(rng.uniform(0.0, 1.0))
+
+
+def mix_layer(n: int, k: int, n_cal: int, layer: int, seed: int):
+    """(w fp32 [n, k], x bf16 bits [n_cal, k]) of one layer (NumPy).
+
+    x = tau * (sqrt(1 - rho^2) z + rho g V): z [n_cal, k] and g [n_cal, 16]
+    standard normal, V [16, k] normal with variance 1/16, per-channel tau
+    log-uniform in [0.25, 4].  w = s_r * (N(0, 1) + beta A V): per-row s_r
+    log-uniform in [0.005, 0.05], A [n, 16] standard normal.
+    """
+    rho, beta = mix_layer_params(layer, seed)
+    rng = np.random.default_rng([seed, layer, 1])
+    v = rng.standard_normal((MIX_RANK, k)) / np.sqrt(MIX_RANK)
+    tau = np.exp(rng.uniform(np.log(0.25), np.log(4.0), size=k))
+    z = rng.standard_normal((n_cal, k))
+    g = rng.standard_normal((n_cal, MIX_RANK))
+    x = tau[None, :] * (np.sqrt(1.0 - rho * rho) * z + rho * (g @ v))
+    s = np.exp(rng.uniform(np.log(0.005), np.log(0.05), size=n))
+    a = rng.standard_normal((n, MIX_RANK))
+    w = s[:, None] * (rng.standard_normal((n, k)) + beta * (a @ v))
+    return w.astype(np.float32), bf16_bits_from_f32(x.astype(np.float32))
+
+
+def mix_layer_torch(n: int, k: int, n_cal: int, layer: int, seed: int, device):
+    """The same recipe drawn on a torch device (torch's generator: other
+    numbers than mix_layer, same distributions), for study sizes that NumPy
+    would take minutes to draw.  Returns (w fp32 [n, k], x bf16 [n_cal, k])."""
+    import torch
+    rho, beta = mix_layer_params(layer, seed)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed * 1000003 + layer)
+    f32 = torch.float32
+    v = torch.randn((MIX_RANK, k), generator=gen, device=device, dtype=f32) / MIX_RANK ** 0.5
+    tau = torch.exp(torch.empty(k, device=device, dtype=f32).uniform_(np.log(0.25), np.log(4.0), generator=gen))
+    z = torch.randn((n_cal, k), generator=gen, device=device, dtype=f32)
+    g = torch.randn((n_cal, MIX_RANK), generator=gen, device=device, dtype=f32)
+    x = tau[None, :] * ((1.0 - rho * rho) ** 0.5 * z + rho * (g @ v))
+    s = torch.exp(torch.empty(n, device=device, dtype=f32).uniform_(np.log(0.005), np.log(0.05), generator=gen))
+    a = torch.randn((n, MIX_RANK), generator=gen, device=device, dtype=f32)
+    w = torch.randn((n, k), generator=gen, device=device, dtype=f32)
+    w.add_(beta * (a @ v)).mul_(s[:, None])
+    return w, x.to(torch.bfloat16)
