@@ -172,7 +172,8 @@ constexpr int kHsAStage = kHsM * 128;               // 16 KB
 constexpr int kHsBStage = kHsMaxCal * 128;          // 32 KB
 constexpr int kHsOffB = kHsStages * kHsAStage;
 constexpr int kHsOffBar = kHsOffB + kHsStages * kHsBStage;
-constexpr int kHsOffMisc = kHsOffBar + 128;
+constexpr int kHsOffTab = kHsOffBar + 128;          // code -> lane values: 32 (STQ1_0) or 256 (STQ2) x 16 B
+constexpr int kHsOffMisc = kHsOffTab + 256 * 16;
 constexpr int kHsSmemBytes = 1024 + kHsOffMisc + 16;   // two CTAs per SM
 
 struct HsArgs {
@@ -231,32 +232,32 @@ __device__ __forceinline__ uint32_t hs_load_raw(const uint8_t* blk, int k_in_blo
   }
 }
 
-// Decoded weights of those 8 columns (fp32).
+// Lane values of a code word, as four floats: STQ1_0 codes (32 entries, the
+// pattern's -1 / 0 / +1; d multiplies them) or STQ2 code bytes (256 entries,
+// m = 2q - 3 of the byte's four weights; d / 3 multiplies them).
 template <int FMT>
-__device__ __forceinline__ void hs_decode_raw(uint32_t raw, float wh[8]) {
-  const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(raw & 0xFFFFu)));
+__device__ __forceinline__ void hs_fill_table(float4* tab) {
   if constexpr (FMT == 0) {
-    const uint32_t qs = (raw >> 16) & 0xFFu, qh = raw >> 24;
-#pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      // code = t << 4 | n: zero lane z = n >> 2; the non-zero lanes in order carry
-      // +1, -(bit 1 of n), -(bit 0 of n); t negates all three
-      const uint32_t n = (qs >> (4 * g)) & 15u, t = (qh >> g) & 1u;
-      const uint32_t z = n >> 2;
-      const float s = t ? -d : d;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t p = static_cast<uint32_t>(i) - (static_cast<uint32_t>(i) > z ? 1u : 0u);
-        const uint32_t neg = p == 1 ? ((n >> 1) & 1u) : (p == 2 ? (n & 1u) : 0u);
-        wh[4 * g + i] = (static_cast<uint32_t>(i) == z) ? 0.f : (neg ? -s : s);
-      }
+    if (threadIdx.x < 32) {
+      int v[4];
+      code_pattern(threadIdx.x, v);
+      tab[threadIdx.x] = make_float4(static_cast<float>(v[0]), static_cast<float>(v[1]), static_cast<float>(v[2]),
+                                     static_cast<float>(v[3]));
     }
   } else {
-    const uint32_t q = raw >> 16;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      wh[i] = __fdiv_rn(d * static_cast<float>(2 * static_cast<int>((q >> (2 * i)) & 3u) - 3), 3.0f);
+    for (int b = threadIdx.x; b < 256; b += blockDim.x)
+      tab[b] = make_float4(static_cast<float>(2 * (b & 3) - 3), static_cast<float>(2 * ((b >> 2) & 3) - 3),
+                           static_cast<float>(2 * ((b >> 4) & 3) - 3), static_cast<float>(2 * ((b >> 6) & 3) - 3));
   }
+}
+
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 
 template <int FMT>
@@ -266,7 +267,7 @@ hess_score_kernel(const __grid_constant__ CUtensorMap xmap, const HsArgs a) {
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - sraw);
-  const uint32_t sA = sbase, sB = sbase + kHsOffB;
+  const uint32_t sA = sbase, sB = sbase + kHsOffB, sTab = sbase + kHsOffTab;
   const uint32_t bar = sbase + kHsOffBar;
   // full_b[2] @0, full_a[2] @16, empty[2] @32, d_full @48, drain @56
   const uint32_t bar_full_b = bar, bar_full_a = bar + 16, bar_empty = bar + 32;
@@ -291,6 +292,7 @@ hess_score_kernel(const __grid_constant__ CUtensorMap xmap, const HsArgs a) {
     s_misc[1] = 0;
     fence_mbar_init();
   }
+  hs_fill_table<FMT>(reinterpret_cast<float4*>(sgen + kHsOffTab));
   if (warp == 1) {
     tmem_alloc(sbase + kHsOffMisc, a.tmem_cols);
     tmem_relinquish();
@@ -379,10 +381,24 @@ hess_score_kernel(const __grid_constant__ CUtensorMap xmap, const HsArgs a) {
         const int r = r0 + 32 * i;
         const float w8[8] = {wv[i][0].x, wv[i][0].y, wv[i][0].z, wv[i][0].w,
                              wv[i][1].x, wv[i][1].y, wv[i][1].z, wv[i][1].w};
-        float wh[8], dv[8];
-        hs_decode_raw<FMT>(raw[i], wh);
+        // D = w - d v: one fused multiply-add per weight, v from the lane table
+        const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(raw[i] & 0xFFFFu)));
+        float4 v0, v1;
+        float sc;
+        if constexpr (FMT == 0) {
+          const uint32_t qs = (raw[i] >> 16) & 0xFFu, qh = raw[i] >> 24;
+          v0 = lds_f4(sTab + 16u * ((qs & 15u) | ((qh & 1u) << 4)));
+          v1 = lds_f4(sTab + 16u * ((qs >> 4) | ((qh >> 1) << 4)));
+          sc = d;
+        } else {
+          v0 = lds_f4(sTab + 16u * ((raw[i] >> 16) & 0xFFu));
+          v1 = lds_f4(sTab + 16u * (raw[i] >> 24));
+          sc = __fdiv_rn(d, 3.0f);
+        }
+        const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float dv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dv[e] = w8[e] - wh[e];
+        for (int e = 0; e < 8; ++e) dv[e] = fmaf(-sc, vv[e], w8[e]);
         if (want_diag) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) part = fmaf(hk[e] * dv[e], dv[e], part);
