@@ -328,6 +328,19 @@ int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float* y, int64_t
 int stq1_set_path(int path);
 
 /*
+ * stq1_selftest_wait -- exercises the failure-detection path without a fault:
+ * one thread waits, through the bounded wait every kernel of this library
+ * uses, on a barrier phase that is completed first (arrive = 1) or that
+ * nothing completes (arrive = 0).  With arrive = 0 the wait gives up after
+ * its bound (2^14 suspended tries of at most 100 us each, so under two
+ * seconds), records STQ1_DEV_WAIT_LIMIT in the device error word and the
+ * kernel returns; the context stays usable.  Read the outcome with
+ * stq1_status.  Asynchronous on `stream`.
+ * Errors: STQ1_ERR_ARG (arrive not 0 or 1), STQ1_ERR_CUDA.
+ */
+int stq1_selftest_wait(int arrive, void* stream);
+
+/*
  * stq1_status -- synchronise `stream`, return STQ1_OK if no device error was
  * recorded since the last call, else STQ1_ERR_DEVICE with the bits in
  * *device_err (may be NULL).  Clears the word.  STQ1_ERR_CUDA if the

@@ -81,6 +81,7 @@ SIGNATURES = {
     "stq1_hessian_error": (_c.c_int, [_c.c_int, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                       _c.c_int64, _c.c_int64, _c.c_int64, _c.c_int64, _c.c_void_p,
                                       _c.c_void_p]),
+    "stq1_selftest_wait": (_c.c_int, [_c.c_int, _c.c_void_p]),
     "stq1_mix_allocate": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64,
                                      _c.c_double, _c.c_void_p]),
 }
@@ -476,6 +477,14 @@ PATH_AUTO, PATH_TABLE, PATH_TILES = 0, 1, 2
 def set_path(path: int) -> None:
     """Selects the matmul kernel process-wide (0 by size, 1 table kernel, 2 tile kernel)."""
     _check("stq1_set_path", _load().stq1_set_path(path))
+
+
+def selftest_wait(arrive: bool, stream=None) -> int:
+    """Runs the bounded-wait self-test (see include/stq1.h) and returns the device error bits."""
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    _check("stq1_selftest_wait", _load().stq1_selftest_wait(1 if arrive else 0, ctypes.c_void_p(s.cuda_stream)))
+    return status(s)
 
 
 def status(stream=None) -> int:

@@ -248,4 +248,20 @@ combine_kernel(const float* __restrict__ y, const float* __restrict__ w, float* 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Self-test of the failure path: one thread waits, through the same bounded
+// wait every kernel uses, on an mbarrier phase that `arrive` completes or
+// (arrive = 0) nothing completes.  In the second case the wait gives up after
+// its bound and records STQ1_DEV_WAIT_LIMIT; the kernel then returns normally.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) wait_selftest_kernel(int arrive) {
+  __shared__ __align__(8) uint64_t bar_storage;
+  if (threadIdx.x != 0) return;
+  const uint32_t bar = smem_u32(&bar_storage);
+  mbar_init(bar, 1);
+  fence_mbar_init();
+  if (arrive) mbar_arrive(bar);
+  mbar_wait_bounded(bar, 0);
+}
+
 }  // namespace stq1

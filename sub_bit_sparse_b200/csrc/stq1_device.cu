@@ -769,6 +769,12 @@ extern "C" int stq1_set_path(int path) {
   return STQ1_OK;
 }
 
+extern "C" int stq1_selftest_wait(int arrive, void* stream) {
+  if (arrive != 0 && arrive != 1) return STQ1_ERR_ARG;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(arrive);
+  return launch_status();
+}
+
 extern "C" int stq1_status(void* stream, int* device_err) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return STQ1_ERR_CUDA;
   int v = 0;
