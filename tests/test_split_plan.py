@@ -1,0 +1,40 @@
+"""The table GEMV's K-split plan, read through the workspace query (no GPU).
+
+stq1_gemv_workspace returns 2048 counter bytes plus S * batch * N * 4 bytes of
+partial sums when the plan splits K into S > 1 pieces, and 0 otherwise, so the
+plan's S can be checked on the host.  Without a device the planner assumes a
+148-SM part with 228 KB of shared memory per SM, the B200's figures.
+"""
+
+import pytest
+
+import sub_bit_sparse_b200 as stq1
+
+
+def _split(n, k, b):
+    ws = stq1.LIB.stq1_gemv_workspace(n, k, b)
+    if ws == 0:
+        return 1
+    assert (ws - 2048) % (b * n * 4) == 0
+    return (ws - 2048) // (b * n * 4)
+
+
+@pytest.mark.parametrize("n,k,b,want", [
+    (4096, 7168, 1, 14),    # 32 slabs x 14 one-chunk pieces = 448 CTAs (about 3 per SM)
+    (4096, 7168, 2, 4),     # two-token units aim at a quarter of the CTAs: 32 x 4, pieces of <= 4 chunks
+    (18432, 7168, 2, 1),    # 144 two-token units already exceed that target: no split
+    (18432, 7168, 1, 4),    # 144 slabs x 4 pieces (the longest piece of 4 chunks, 14 = 4+4+3+3)
+])
+def test_split_of_the_benchmark_shapes(n, k, b, want):
+    assert _split(n, k, b) == want
+
+
+@pytest.mark.parametrize("b", [1, 2, 4, 8])
+@pytest.mark.parametrize("n,k", [(4096, 7168), (18432, 7168), (512, 2048), (1000, 4096)])
+def test_pieces_are_as_few_as_the_longest_piece_allows(n, k, b):
+    # the plan never uses more pieces than its longest piece needs
+    chunks = k // 512
+    s = _split(n, k, b)
+    assert 1 <= s <= min(chunks, 16)
+    longest = -(-chunks // s)
+    assert s == -(-chunks // longest)
