@@ -292,6 +292,22 @@ int stq1_quantize_x_e4m3(const uint16_t* x, int64_t T, int64_t K, uint8_t* q, fl
                          void* stream);
 
 /*
+ * stq1_gemv_prefetch -- stq1_gemv, and while it runs its CTAs ask the GPU to
+ * bring the next_bytes bytes at W_next into L2 (cp.async.bulk.prefetch; no
+ * completion is awaited and nothing waits for it), so that a following call
+ * whose weights are W_next finds them in L2 instead of waiting for HBM.  For
+ * a chain of matmuls over known matrices (the layers of a decode step).
+ * Results are those of stq1_gemv.  Only the lookup-table path (batch below
+ * the tile path's threshold) issues the prefetch.
+ *   W_next      device pointer, 16-byte aligned, only read; NULL: no prefetch.
+ *   next_bytes  bytes to prefetch (rounded down to a multiple of 16); >= 0.
+ * Errors: those of stq1_gemv; STQ1_ERR_SHAPE (next_bytes < 0), STQ1_ERR_ALIGN
+ * (W_next not 16-byte aligned).
+ */
+int stq1_gemv_prefetch(const void* W_packed, const uint16_t* x, float* y, int64_t N, int64_t K, int batch,
+                       void* workspace, size_t ws_bytes, const void* W_next, int64_t next_bytes, void* stream);
+
+/*
  * stq1_gemv_noalloc -- stq1_gemv without a caller workspace and without any
  * allocation.  The source pages have no counterpart; this entry point exists
  * for callers that cannot allocate device memory or keep a workspace: hosts

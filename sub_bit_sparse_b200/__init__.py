@@ -50,6 +50,8 @@ SIGNATURES = {
     "stq1_gemv_workspace": (_c.c_size_t, [_c.c_int64, _c.c_int64, _c.c_int]),
     "stq1_gemv": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int,
                              _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "stq1_gemv_prefetch": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int,
+                                      _c.c_void_p, _c.c_size_t, _c.c_void_p, _c.c_int64, _c.c_void_p]),
     "stq1_moe_workspace": (_c.c_size_t, [_c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int]),
     "stq1_moe_gateup": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                    _c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
@@ -233,8 +235,11 @@ def dequant(w_packed, n: int, k: int, out=None):
     return out
 
 
-def gemv(w_packed, x, n: int, k: int, out=None, ws=None):
-    """y [b, n] fp32 = W^ x for x [b, k] bf16."""
+def gemv(w_packed, x, n: int, k: int, out=None, ws=None, prefetch=None):
+    """y [b, n] fp32 = W^ x for x [b, k] bf16.
+
+    prefetch: the packed weights (uint8 CUDA tensor) of a following call, to be
+    brought into L2 while this one runs (stq1_gemv_prefetch)."""
     torch = _torch()
     _require(w_packed, torch.uint8, "w_packed")
     _require(x, torch.bfloat16, "x")
@@ -245,10 +250,17 @@ def gemv(w_packed, x, n: int, k: int, out=None, ws=None):
     lib = _load()
     if ws is None:
         ws = workspace(lib.stq1_gemv_workspace(n, k, b), x.device)
-    rc = lib.stq1_gemv(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b,
-                       None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
-                       _stream(x))
-    _check("stq1_gemv", rc)
+    if prefetch is None:
+        rc = lib.stq1_gemv(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b,
+                           None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
+                           _stream(x))
+        _check("stq1_gemv", rc)
+        return out
+    _require(prefetch, torch.uint8, "prefetch")
+    rc = lib.stq1_gemv_prefetch(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b,
+                                None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
+                                prefetch.data_ptr(), prefetch.numel(), _stream(x))
+    _check("stq1_gemv_prefetch", rc)
     return out
 
 

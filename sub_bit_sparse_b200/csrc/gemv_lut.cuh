@@ -64,6 +64,8 @@ struct LutArgs {
   int S, cq, cr;             // K splits; split s has cq chunks, plus one if s < cr
   int flags;
   int cluster;               // 1: the S splits of a (tile, slab) form one thread-block cluster
+  const uint8_t* next;       // bytes to bring into L2 for a following call, or nullptr
+  long long next_bytes;      // multiple of 16
 };
 
 // Spread bits 0, 2, 4, 6 of x to bit 6 of bytes 0..3 (other bits cleared).
@@ -206,6 +208,19 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
   if (threadIdx.x == 0) {
     issue(c0, 0);
     if (NS == 2) issue(c0 + 1, 1);
+  }
+  // The next call's weights: each CTA asks for its share to be brought into
+  // L2 (no completion is tracked; nothing here reads them).
+  if (a.next != nullptr && threadIdx.x == 32) {
+    const long long n_cta = static_cast<long long>(gridDim.x) * gridDim.y;
+    const long long cta = static_cast<long long>(blockIdx.y) * gridDim.x + blockIdx.x;
+    const long long share = ((a.next_bytes + n_cta - 1) / n_cta + 15) & ~15LL;
+    const long long off = cta * share;
+    if (off < a.next_bytes) {
+      const long long len = min(share, a.next_bytes - off);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.next + off), "r"(static_cast<uint32_t>(len))
+                   : "memory");
+    }
   }
   if (a.tile_info == nullptr) griddep_wait();
   griddep_launch_dependents();

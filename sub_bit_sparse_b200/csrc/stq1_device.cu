@@ -397,8 +397,9 @@ extern "C" size_t stq1_gemv_workspace(int64_t N, int64_t K, int batch) {
   return p.counter_bytes + round16(p.partial_bytes);
 }
 
-extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int64_t N, int64_t K,
-                         int batch, void* workspace, size_t ws_bytes, void* stream) {
+namespace {
+int gemv_impl(const void* W_packed, const uint16_t* x, float* y, int64_t N, int64_t K, int batch,
+              void* workspace, size_t ws_bytes, const void* W_next, int64_t next_bytes, void* stream) {
   if (!W_packed || !x || !y) return STQ1_ERR_NULL;
   if (N <= 0 || K <= 0 || K % kBlockWeights || batch <= 0 || batch > 65535 ||
       N > (1LL << 31) - 1 || K > (1LL << 31) - 1)
@@ -460,6 +461,9 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
   a.n_slabs = p.n_slabs;
   set_split(&a, p.n_chunks, p.S);
   a.flags = 0;
+  a.next = static_cast<const uint8_t*>(W_next);
+  a.next_bytes = W_next ? (next_bytes & ~static_cast<int64_t>(15)) : 0;
+  if (a.next_bytes <= 0) a.next = nullptr;
   const long long units = static_cast<long long>(p.n_tiles) * p.n_slabs;
   if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
   const dim3 grid(static_cast<unsigned>(units), static_cast<unsigned>(p.S));
@@ -477,6 +481,20 @@ extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int6
   // caller's scratch buffer
   if (p.S > 1 && p.S <= kMaxClusterRanks && go(p.S) == STQ1_OK) return STQ1_OK;
   return go(1);
+}
+}  // namespace
+
+extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int64_t N, int64_t K,
+                         int batch, void* workspace, size_t ws_bytes, void* stream) {
+  return gemv_impl(W_packed, x, y, N, K, batch, workspace, ws_bytes, nullptr, 0, stream);
+}
+
+extern "C" int stq1_gemv_prefetch(const void* W_packed, const uint16_t* x, float* y, int64_t N, int64_t K,
+                                  int batch, void* workspace, size_t ws_bytes, const void* W_next,
+                                  int64_t next_bytes, void* stream) {
+  if (next_bytes < 0) return STQ1_ERR_SHAPE;
+  if (W_next && !aligned16(W_next)) return STQ1_ERR_ALIGN;
+  return gemv_impl(W_packed, x, y, N, K, batch, workspace, ws_bytes, W_next, next_bytes, stream);
 }
 
 namespace stq1 {

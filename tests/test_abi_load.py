@@ -76,6 +76,9 @@ def test_host_side_argument_checks_need_no_gpu():
     assert L.stq1_quantize_x_e4m3(1 << 20, 0, 256, 1 << 20, 1 << 20, None) == -1
     assert L.stq1_quantize_x_e4m3((1 << 20) + 2, 4, 256, 1 << 20, 1 << 20, None) == -6
     assert L.stq1_selftest_wait(2, None) == -8
+    assert L.stq1_gemv_prefetch(1 << 20, 1 << 20, 1 << 20, 16, 256, 1, None, 0, 1 << 20, -16, None) == -1
+    assert L.stq1_gemv_prefetch(1 << 20, 1 << 20, 1 << 20, 16, 256, 1, None, 0, (1 << 20) + 8, 64, None) == -6
+    assert L.stq1_gemv_prefetch(1 << 20, 1 << 20, 1 << 20, 16, 300, 1, None, 0, None, 0, None) == -1
     # mixed-precision allocation entries
     assert L.stq1_quantize_stq2(None, None, 4, 256, 0, 1 << 20, None) == -2
     assert L.stq1_quantize_stq2(1 << 20, None, 0, 256, 0, 1 << 20, None) == -1

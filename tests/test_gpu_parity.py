@@ -106,6 +106,24 @@ def test_gemv_decode_workload_full(decode_workload, b):
     _assert_close(y, oracle.gemv(packed, xb, n, k), oracle.gemv_abs(packed, xb, n, k), f"cfg2 b={b}")
 
 
+@pytest.mark.parametrize("b", [1, 2, 8])
+def test_gemv_prefetch_leaves_results_unchanged(decode_workload, b):
+    # stq1_gemv_prefetch only adds L2 prefetches of another matrix: same bits as
+    # stq1_gemv, and the oracle's tolerance; prefetch lengths that are not a
+    # multiple of 16, empty, or the matrix itself
+    packed, x = decode_workload
+    n, k = 4096, 7168
+    wd, xd = _dev(packed), _bf16(x[:b])
+    other = _dev(np.roll(packed, 4242))
+    y0 = stq1.gemv(wd, xd, n, k).clone()
+    for nxt in (other, other[: other.numel() - 37], other[:0], wd):
+        y = stq1.gemv(wd, xd, n, k, prefetch=nxt)
+        assert torch.equal(y, y0)
+    assert stq1.status() == 0
+    _assert_close(y0.cpu().numpy(), oracle.gemv(packed, x[:b], n, k), oracle.gemv_abs(packed, x[:b], n, k),
+                  f"prefetch b={b}")
+
+
 def test_gemv_repeatable_and_workspace_left_zero(decode_workload):
     packed, x = decode_workload
     wd, xd = _dev(packed), _bf16(x[:1])
