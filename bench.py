@@ -746,8 +746,9 @@ def kernel_traffic(kernel):
 
 def profile_case(args):
     """Small launch sequence for ncu captures: the decode GEMV on 64 distinct
-    [4096, 7168] matrices (308 MB, larger than L2), 32 launches, batch 1
-    (or the MoE decode call with --profile-case moe)."""
+    [4096, 7168] matrices (308 MB, larger than L2), 32 launches, batch 1, each
+    prefetching the next matrix as the bench's chain does (or the MoE decode
+    call with --profile-case moe)."""
     import torch
     import sub_bit_sparse_b200 as stq1
     device = torch.device("cuda", 0)
@@ -773,8 +774,13 @@ def profile_case(args):
     xs = torch.from_numpy(x_bits.view(np.int16)).to(device).view(torch.bfloat16)
     y = torch.empty((1, N_ROWS), dtype=torch.float32, device=device)
     ws = stq1.workspace(stq1.LIB.stq1_gemv_workspace(N_ROWS, K_COLS, 1), device)
+    # read a buffer larger than L2 first: the dirty lines left by building the
+    # stack are written back here, not during the captured launches
+    clean = torch.empty(64 << 20, dtype=torch.float32, device=device)
+    float(clean.sum())
+    del clean
     for i in range(32):
-        stq1.gemv(stack[i % STACK], xs[:1], N_ROWS, K_COLS, out=y, ws=ws)
+        stq1.gemv(stack[i % STACK], xs[:1], N_ROWS, K_COLS, out=y, ws=ws, prefetch=stack[(i + 1) % STACK])
     torch.cuda.synchronize()
     print("profile case done", float(y.abs().sum()))
 
