@@ -45,6 +45,27 @@ FP8_OVER_BF16 = 2.0                        # nominal dense fp8 / bf16 tensor rat
 HBM_NOMINAL_GBS = 8000.0
 
 
+def measure_fp8_peak(torch, device, n=8192, reps=10):
+    """Dense E4M3 tensor throughput on this GPU, TFLOP/s: best of `reps`
+    torch._scaled_mm calls on n^3 (fp32 accumulation, bf16 output)."""
+    a = torch.randn((n, n), device=device).to(torch.float8_e4m3fn)
+    b = torch.randn((n, n), device=device).to(torch.float8_e4m3fn).t()   # column-major operand
+    one = torch.ones((), dtype=torch.float32, device=device)
+    for _ in range(3):
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del a, b
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -261,6 +282,12 @@ def run_gpu(args):
     except Exception as exc:  # reported, never hidden
         mix = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
+    # --- crossover between the kernels on [18432, 7168], batches 1 .. 1024 ---
+    try:
+        xover = crossover(torch, stq1, device, stream, (1, 4, 16, 64, 256, 1024), reps_cap=1024)
+    except Exception as exc:  # reported, never hidden
+        xover = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     # --- end to end through the public API with host buffers ---
     e2e = run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier)
 
@@ -286,6 +313,7 @@ def run_gpu(args):
         "moe_ffn_decode": ffn,
         "encoder": encoder,
         "mix_allocation": mix,
+        "crossover": xover,
         "e2e": e2e,
         "gpu_launches": args.steps * STACK,
         "clocks": clk.summary(),
@@ -383,7 +411,11 @@ def run_prefill(torch, stq1, device, stream, args, world, timed, bf16_peak):
     flops = 2.0 * 4096 * 8 * n * k
     out = {}
     ys = {}
-    for name, flags, peak in (("bf16", 0, bf16_peak), ("fp8", stq1.MOE_FP8, bf16_peak * FP8_OVER_BF16)):
+    try:
+        fp8_peak, fp8_kind = measure_fp8_peak(torch, device), "measured in this run (torch._scaled_mm E4M3 8192^3)"
+    except Exception as exc:  # reported, never hidden
+        fp8_peak, fp8_kind = bf16_peak * FP8_OVER_BF16, f"measured bf16 x 2 (nominal ratio; fp8 probe failed: {exc})"[:200]
+    for name, flags, peak in (("bf16", 0, bf16_peak), ("fp8", stq1.MOE_FP8, fp8_peak)):
         y = torch.empty((4096, 8, n), dtype=torch.float32, device=device)
         ws = stq1.workspace(stq1.LIB.stq1_moe_workspace(4096, 8, E, n, k, flags), device, kind="moe")
 
@@ -411,9 +443,10 @@ def run_prefill(torch, stq1, device, stream, args, world, timed, bf16_peak):
     res = out["bf16"]
     res["bf16_peak_tflops"] = bf16_peak
     res["fp8"] = out["fp8"]
+    res["fp8"]["peak_kind"] = fp8_kind
     res["config"] = ("256 experts x [4096, 7168] STQ1_0, 4096 tokens, Zipf(1.1) top-8 (32,768 pairs), "
                      "tcgen05 tiles, A = decoded +/-1 in TMEM (bf16, kind::f16; fp8: E4M3, kind::f8f6f4 with "
-                     "per-token E4M3 activations), fp32 per-block scale; fp8 peak = measured bf16 x 2 (nominal ratio)")
+                     "per-token E4M3 activations), fp32 per-block scale")
     return res
 
 
@@ -553,14 +586,12 @@ def run_mix(torch, stq1, device, stream, args, world, timed, bf16_peak, hbm_peak
     return res
 
 
-def run_sweep(args):
-    """Crossover sweep: one [18432, 7168] matrix, batch 1..1024 (the stated
-    1, 4, 16, 64, 256, 1024 plus 2, 8 and 32 around the crossover), both kernels."""
-    import torch
+def crossover(torch, stq1, device, stream, batches, reps_cap=4096):
+    """Crossover between the kernels on one [18432, 7168] matrix with the decode
+    matrix's statistics: per batch, each forced path and the library's own
+    choice, timed in a CUDA graph of launches over rotating copies larger than
+    L2 (GB/s of packed weights and dense-equivalent TFLOP/s)."""
     import workloads
-    import sub_bit_sparse_b200 as stq1
-    device = torch.device("cuda", 0)
-    torch.cuda.set_device(device)
     w, h, x = workloads.crossover_inputs()
     n, k = w.shape
     packed = stq1.quantize_ref(w, h, mode="sherry")
@@ -568,38 +599,59 @@ def run_sweep(args):
     copies = max(2, (300 * 1024 * 1024) // pb + 1)          # rotate > 2 x L2
     wd = torch.from_numpy(packed).to(device)
     stack = torch.stack([torch.roll(wd.view(-1, 42), shifts=i * 7919, dims=0).reshape(-1) for i in range(copies)])
+    del wd
     xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
-    y = torch.empty((1024, n), dtype=torch.float32, device=device)
-    batches = (1, 2, 4, 8, 16, 32, 64, 256, 1024)
+    y = torch.empty((max(batches), n), dtype=torch.float32, device=device)
     ws = stq1.workspace(max(stq1.LIB.stq1_gemv_workspace(n, k, b) for b in batches), device)
-    out = []
-    stream = torch.cuda.Stream(device)
-    for b in batches:
-        row = {"batch": b}
-        for name, path in (("table", stq1.PATH_TABLE), ("tiles", stq1.PATH_TILES)):
-            stq1.set_path(path)
+    paths = (("table", stq1.PATH_TABLE), ("tiles", stq1.PATH_TILES), ("auto", stq1.PATH_AUTO))
+    rows = []
+    try:
+        for b in batches:
+            row = {"batch": b}
             xb = xd[:b].contiguous()
-            reps = max(2, min(copies, 4096 // b))
+            for name, path in paths:
+                stq1.set_path(path)
+                reps = max(2, min(copies, reps_cap // b))
 
-            def step():
-                for i in range(reps):
-                    stq1.gemv(stack[i % copies], xb, n, k, out=y[:b], ws=ws)
+                def step():
+                    for i in range(reps):
+                        stq1.gemv(stack[i % copies], xb, n, k, out=y[:b], ws=ws)
 
-            g = time_graph(torch, step, 1, 3, stream)
-            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            with torch.cuda.stream(stream):
-                s0.record(stream)
-                g.replay()
-                s1.record(stream)
-            torch.cuda.synchronize()
-            ms = s0.elapsed_time(s1) / reps
-            del g
-            row[name] = {"ms": round(ms, 4), "gbs": round(pb / (ms * 1e-3) / 1e9, 1),
-                         "tflops": round(2.0 * b * n * k / (ms * 1e-3) / 1e12, 2)}
+                g = time_graph(torch, step, 1, 3, stream)
+                s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    s0.record(stream)
+                    g.replay()
+                    s1.record(stream)
+                torch.cuda.synchronize()
+                ms = s0.elapsed_time(s1) / reps
+                del g
+                row[name] = {"us": round(ms * 1e3, 2), "gbs": round(pb / (ms * 1e-3) / 1e9, 1),
+                             "tflops": round(2.0 * b * n * k / (ms * 1e-3) / 1e12, 2)}
+            rows.append(row)
+    finally:
         stq1.set_path(stq1.PATH_AUTO)
-        out.append(row)
+    faster = [r["batch"] for r in rows if r["tiles"]["us"] < r["table"]["us"]]
+    del stack, y
+    return {"matrix": [n, k], "packed_bytes": int(pb), "rows": rows,
+            "tiles_faster_from_batch": min(faster) if faster else None,
+            "config": "one [18432, 7168] STQ1_0 matrix (decode-matrix statistics, Sherry 3 rounds), bf16 batch "
+                      "prefix of x [1024, 7168]; CUDA graph over rotating copies (> 2 x L2); table = lookup-table "
+                      "kernel, tiles = tcgen05 tile kernel, auto = the library's own choice"}
+
+
+def run_sweep(args):
+    """Crossover sweep: the stated batches 1, 4, 16, 64, 256, 1024 plus 2, 8 and
+    32 around the crossover."""
+    import torch
+    import sub_bit_sparse_b200 as stq1
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device)
+    res = crossover(torch, stq1, device, stream, (1, 2, 4, 8, 16, 32, 64, 256, 1024))
+    for row in res["rows"]:
         print(json.dumps(row), flush=True)
-    print(json.dumps({"sweep": "crossover", "matrix": [n, k], "packed_bytes": int(pb), "rows": out}))
+    print(json.dumps({"sweep": "crossover", **res}))
 
 
 def run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier):
@@ -610,7 +662,7 @@ def run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier):
     yh = torch.empty((STACK, 1, N_ROWS), dtype=torch.float32).pin_memory()
     xd = torch.empty((1, K_COLS), dtype=torch.bfloat16, device=device)
     yd = torch.empty((STACK, 1, N_ROWS), dtype=torch.float32, device=device)
-    steps = max(1, args.steps // 10)
+    steps = max(20, args.steps // 2)
 
     def one():
         xd.copy_(xh, non_blocking=True)
@@ -642,6 +694,7 @@ def run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier):
 
 
 def _blas_threads():
+    """Threads the oracle's fp64 matmul runs on (the BLAS pool; the decode is one thread)."""
     try:
         from threadpoolctl import threadpool_info
         info = threadpool_info()
@@ -668,7 +721,7 @@ def cpu_baseline(packed, x_bits, seconds=10.0):
     dt = time.perf_counter() - t0
     rb = (K_COLS // 256) * 42
     return {"value": round(n * rows * rb / dt / 1e9, 6), "unit": "GB/s", "cores": _blas_threads(),
-            "kind": "oracle",
+            "host_cores": os.cpu_count(), "kind": "oracle",
             "sample": f"{n} oracle GEMVs of {rows} x {K_COLS} rows of the WLS-encoded decode matrix, "
                       f"batch 1, {dt:.1f} s"}
 
@@ -710,7 +763,7 @@ def run_reference(args):
         "data": "synthetic",
         "config": bench_config(int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": _blas_threads(),
-                         "kind": "oracle",
+                         "host_cores": os.cpu_count(), "kind": "oracle",
                          "sample": f"each step: decode + fp64 GEMV of {rows} of the 4096 rows x {K_COLS} of the "
                                    "decode matrix, batch 1 (a bounded sample of the workload)"},
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -78,7 +78,7 @@ def build(verbose: bool = False, force: bool = False, ptxas_verbose: bool = Fals
         _run(cmd, verbose)
         objs.append(obj)
     tmp = LIB + ".tmp"
-    _run([nvcc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-lpthread"], verbose)
+    _run([nvcc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-lpthread", "-ldl"], verbose)
     os.replace(tmp, LIB)
     return LIB
 

@@ -217,7 +217,9 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
     const long long share = ((a.next_bytes + n_cta - 1) / n_cta + 15) & ~15LL;
     const long long off = cta * share;
     if (off < a.next_bytes) {
-      const long long len = min(share, a.next_bytes - off);
+      // the prefetch length is a 32-bit count: a share above 1 GiB is cut
+      // there (the rest of it is simply not prefetched)
+      const long long len = min(min(share, a.next_bytes - off), 1LL << 30);
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.next + off), "r"(static_cast<uint32_t>(len))
                    : "memory");
     }

@@ -1,12 +1,14 @@
 // C-ABI entry points of libstq1.so (device side).  Argument checks happen on the
 // host before anything is enqueued; every entry point returns an STQ1_* code.
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
 #include <utility>
 
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "device_common.cuh"
 #include "encode_device.cuh"
@@ -33,34 +35,51 @@ static_assert(kTargetUnits * sizeof(int) <= kCounterBytes, "counter region too s
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// An NVTX range around each entry point, so that a profiler's timeline shows
+// which library call enqueued which kernels (nearly free without a profiler).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Path selection: 0 = by size, 1 = table kernel, 2 = tensor-core tile kernel.
-int g_path = 0;
+// Atomic so that a call on another host thread reads either value, never a torn one.
+std::atomic<int> g_path{0};
 constexpr int kTcMinBatch = 16;       // stq1_gemv: batches from here use the tile kernel
 constexpr int kTcMinPairsPerExpert = 16;
 constexpr int kMoeTableTokens = 2;    // MoE decode tiles: pairs per table-kernel unit
 
-int sm_count() {
-  static int cache[kMaxDevices] = {};
+// Per-device attribute caches.  Several host threads may make their first
+// call at once: a cache slot is an atomic written with the same value by
+// whichever thread gets there, so a reader sees 0 (and asks the runtime) or
+// the final value.
+int device_attr_cached(std::atomic<int>* cache, cudaDeviceAttr attr, int fallback) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  if (!cache[dev]) {
-    int v = 0;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = v > 0 ? v : 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return fallback;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, attr, dev) != cudaSuccess || v <= 0) v = fallback;
+    cache[dev].store(v, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return v;
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+std::atomic<int> g_sm_count[kMaxDevices];
+int sm_count() { return device_attr_cached(g_sm_count, cudaDevAttrMultiProcessorCount, 148); }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda
+// link); a function-local static is initialised once, thread-safely.
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -88,11 +107,16 @@ int current_device() {
 }
 
 // Per-device one-time kernel attribute setup (dynamic shared memory limits).
+// The first call on a device holds a lock while it sets the attributes, so a
+// call on another host thread never launches before they are in place.
+std::atomic<bool> g_configured[kMaxDevices];
+std::mutex g_config_mutex;
 int ensure_configured() {
-  static bool done[kMaxDevices] = {};
   const int dev = current_device();
   if (dev < 0) return STQ1_ERR_CUDA;
-  if (done[dev]) return STQ1_OK;
+  if (g_configured[dev].load(std::memory_order_acquire)) return STQ1_OK;
+  std::lock_guard<std::mutex> lock(g_config_mutex);
+  if (g_configured[dev].load(std::memory_order_relaxed)) return STQ1_OK;
   if (cudaFuncSetAttribute(lut_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(lut_smem_bytes_max(1))) != cudaSuccess ||
       cudaFuncSetAttribute(lut_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -120,7 +144,7 @@ int ensure_configured() {
   cudaFuncSetAttribute(lut_gemv_kernel<2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaFuncSetAttribute(lut_gemv_kernel<4>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaGetLastError();
-  done[dev] = true;
+  g_configured[dev].store(true, std::memory_order_release);
   return STQ1_OK;
 }
 
@@ -310,16 +334,9 @@ bool want_tiles_gemv(long long N, long long nb, long long batch) {
   return tiles_us < table_us;
 }
 
+std::atomic<int> g_smem_per_sm[kMaxDevices];
 int smem_per_sm() {
-  static int cache[kMaxDevices] = {};
-  const int dev = current_device();
-  if (dev < 0) return 228 * 1024;
-  if (!cache[dev]) {
-    int v = 0;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-    cache[dev] = v > 0 ? v : 228 * 1024;
-  }
-  return cache[dev];
+  return device_attr_cached(g_smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, 228 * 1024);
 }
 
 // Work split of the table kernel: (token tile, 128-row slab) units, each cut
@@ -380,6 +397,7 @@ using namespace stq1;
 
 extern "C" int stq1_dequant(const void* W_packed, uint16_t* W_bf16, int64_t N, int64_t K,
                             void* stream) {
+  NvtxRange nvtx_range("stq1_dequant");
   if (!W_packed || !W_bf16) return STQ1_ERR_NULL;
   if (N <= 0 || K <= 0 || K % kBlockWeights) return STQ1_ERR_SHAPE;
   if (!aligned16(W_packed) || !aligned16(W_bf16)) return STQ1_ERR_ALIGN;
@@ -486,12 +504,14 @@ int gemv_impl(const void* W_packed, const uint16_t* x, float* y, int64_t N, int6
 
 extern "C" int stq1_gemv(const void* W_packed, const uint16_t* x, float* y, int64_t N, int64_t K,
                          int batch, void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("stq1_gemv");
   return gemv_impl(W_packed, x, y, N, K, batch, workspace, ws_bytes, nullptr, 0, stream);
 }
 
 extern "C" int stq1_gemv_prefetch(const void* W_packed, const uint16_t* x, float* y, int64_t N, int64_t K,
                                   int batch, void* workspace, size_t ws_bytes, const void* W_next,
                                   int64_t next_bytes, void* stream) {
+  NvtxRange nvtx_range("stq1_gemv_prefetch");
   if (next_bytes < 0) return STQ1_ERR_SHAPE;
   if (W_next && !aligned16(W_next)) return STQ1_ERR_ALIGN;
   return gemv_impl(W_packed, x, y, N, K, batch, workspace, ws_bytes, W_next, next_bytes, stream);
@@ -546,6 +566,7 @@ extern "C" size_t stq1_moe_workspace(int T, int topk, int E, int64_t N, int64_t 
 extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, const int32_t* topk_ids,
                                const float* topk_weights, float* y, int T, int topk, int E, int64_t N,
                                int64_t K, int flags, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("stq1_moe_gateup");
   if (!expert_blocks || !x || !topk_ids || !y) return STQ1_ERR_NULL;
   if ((flags & STQ1_MOE_WEIGHT_UP) && !topk_weights) return STQ1_ERR_NULL;
   if (flags & ~(STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8 | STQ1_MOE_SKIP_FOREIGN)) return STQ1_ERR_ARG;
@@ -657,6 +678,7 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
 
 extern "C" int stq1_quantize(const float* W, const float* h, int64_t N, int64_t K, int mode, int rounds,
                              uint8_t* out, void* stream) {
+  NvtxRange nvtx_range("stq1_quantize");
   if (!W || !out) return STQ1_ERR_NULL;
   if (N <= 0 || K <= 0 || K % kBlockWeights) return STQ1_ERR_SHAPE;
   if (mode != STQ1_ENC_PLAIN && mode != STQ1_ENC_SHERRY) return STQ1_ERR_ARG;
@@ -675,6 +697,7 @@ extern "C" int stq1_quantize(const float* W, const float* h, int64_t N, int64_t 
 
 extern "C" int stq1_quantize_x_e4m3(const uint16_t* x, int64_t T, int64_t K, uint8_t* q, float* scales,
                                     void* stream) {
+  NvtxRange nvtx_range("stq1_quantize_x_e4m3");
   if (!x || !q || !scales) return STQ1_ERR_NULL;
   if (T <= 0 || K <= 0 || K % 16 || T > (1LL << 31) - 1) return STQ1_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(q)) return STQ1_ERR_ALIGN;
@@ -685,6 +708,7 @@ extern "C" int stq1_quantize_x_e4m3(const uint16_t* x, int64_t T, int64_t K, uin
 }
 
 extern "C" int stq1_swiglu(const float* y, uint16_t* act, int64_t P, int64_t N, void* stream) {
+  NvtxRange nvtx_range("stq1_swiglu");
   if (!y || !act) return STQ1_ERR_NULL;
   if (P <= 0 || N <= 0 || (N & 1) || N > (1LL << 31) - 1 || P > (1LL << 40) / N) return STQ1_ERR_SHAPE;
   const long long total = P * (N / 2);
@@ -695,6 +719,7 @@ extern "C" int stq1_swiglu(const float* y, uint16_t* act, int64_t P, int64_t N, 
 
 extern "C" int stq1_moe_combine(const float* y, const float* w, float* out, int64_t T, int topk, int64_t H,
                                 void* stream) {
+  NvtxRange nvtx_range("stq1_moe_combine");
   if (!y || !out) return STQ1_ERR_NULL;
   if (T <= 0 || topk <= 0 || H <= 0 || H > (1LL << 31) - 1 || T > (1LL << 40) / (H * topk)) return STQ1_ERR_SHAPE;
   const long long total = T * H;
@@ -735,6 +760,7 @@ extern "C" size_t stq1_moe_ffn_workspace(int T, int topk, int E, int64_t N, int6
 extern "C" int stq1_moe_ffn(const void* gateup_blocks, const void* down_blocks, const uint16_t* x,
                             const int32_t* topk_ids, const float* topk_weights, float* out, int T, int topk, int E,
                             int64_t N, int64_t H, int flags, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("stq1_moe_ffn");
   if (!gateup_blocks || !down_blocks || !x || !topk_ids || !out) return STQ1_ERR_NULL;
   if (flags & ~(STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8 | STQ1_MOE_SKIP_FOREIGN)) return STQ1_ERR_ARG;
   if (T <= 0 || topk <= 0 || E <= 0 || N <= 0 || (N & 1) || H <= 0 || H % kBlockWeights || (N / 2) % kBlockWeights ||
@@ -770,6 +796,7 @@ extern "C" int stq1_moe_ffn_local(const void* gateup_local, const void* down_loc
                                   const int32_t* topk_ids, const float* topk_weights, float* out, int T, int topk,
                                   int E_local, int expert_begin, int64_t N, int64_t H, int flags, void* ws,
                                   size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("stq1_moe_ffn_local");
   if (!topk_ids || !ws) return !topk_ids ? STQ1_ERR_NULL : STQ1_ERR_WORKSPACE;
   if (T <= 0 || topk <= 0 || E_local <= 0 || expert_begin < 0) return STQ1_ERR_SHAPE;
   const size_t need = stq1_moe_ffn_local_workspace(T, topk, E_local, N, H, flags);
@@ -789,17 +816,19 @@ extern "C" int stq1_moe_ffn_local(const void* gateup_local, const void* down_loc
 
 extern "C" int stq1_set_path(int path) {
   if (path < 0 || path > 2) return STQ1_ERR_ARG;
-  g_path = path;
+  g_path.store(path);
   return STQ1_OK;
 }
 
 extern "C" int stq1_selftest_wait(int arrive, void* stream) {
+  NvtxRange nvtx_range("stq1_selftest_wait");
   if (arrive != 0 && arrive != 1) return STQ1_ERR_ARG;
   wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(arrive);
   return launch_status();
 }
 
 extern "C" int stq1_status(void* stream, int* device_err) {
+  NvtxRange nvtx_range("stq1_status");
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return STQ1_ERR_CUDA;
   int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_dev_err, sizeof(int)) != cudaSuccess) return STQ1_ERR_CUDA;
@@ -833,11 +862,14 @@ constexpr size_t kStaticScratchBytes = static_cast<size_t>(1) << 20;   // 1 MiB
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 uint8_t* g_static_scratch_ptr[kMaxDevices] = {};
+std::mutex g_static_scratch_mutex;
 
-// One-time set-up per device, with that device current.
+// One-time set-up per device, with that device current (under a lock: two
+// host threads making their first call at once look the address up once).
 int static_scratch(uint8_t** out) {
   const int dev = current_device();
   if (dev < 0) return STQ1_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
   if (!g_static_scratch_ptr[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || ptr == nullptr)
@@ -853,6 +885,7 @@ int static_scratch(uint8_t** out) {
 
 extern "C" int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float* y, int64_t N,
                                  int64_t K, int batch, void* stream) {
+  NvtxRange nvtx_range("stq1_gemv_noalloc");
   if (!W_packed || !x || !y) return STQ1_ERR_NULL;
   if (N <= 0 || K <= 0 || K % kBlockWeights || batch <= 0 || batch > 65535 ||
       N > (1LL << 31) - 1 || K > (1LL << 31) - 1)
@@ -921,6 +954,7 @@ extern "C" int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float*
 
 extern "C" int stq1_quantize_stq2(const float* W, const float* h, int64_t N, int64_t K, int rounds, uint8_t* out,
                                   void* stream) {
+  NvtxRange nvtx_range("stq1_quantize_stq2");
   if (!W || !out) return STQ1_ERR_NULL;
   if (N <= 0 || K <= 0 || K % kBlockWeights || N > (1LL << 40) / K) return STQ1_ERR_SHAPE;
   if (rounds < 0 || rounds > 1000) return STQ1_ERR_ARG;
@@ -937,6 +971,7 @@ extern "C" int stq1_quantize_stq2(const float* W, const float* h, int64_t N, int
 }
 
 extern "C" int stq1_hessian_diag(const uint16_t* x, int64_t L, int64_t rows, int64_t K, float* h, void* stream) {
+  NvtxRange nvtx_range("stq1_hessian_diag");
   if (!x || !h) return STQ1_ERR_NULL;
   if (L <= 0 || rows <= 0 || K <= 0 || L > 65535 || rows > (1LL << 40) / K || L > (1LL << 40) / (rows * K))
     return STQ1_ERR_SHAPE;
@@ -969,6 +1004,7 @@ bool make_cal_map(CUtensorMap* map, const void* base, long long L, long long n_c
 extern "C" int stq1_hessian_error(int format, const void* packed, const float* W, const uint16_t* x,
                                   const float* h, int64_t L, int64_t N, int64_t K, int64_t n_cal, double* out,
                                   void* stream) {
+  NvtxRange nvtx_range("stq1_hessian_error");
   if (!packed || !W || !x || !h || !out) return STQ1_ERR_NULL;
   if (format != STQ1_FMT_STQ1_0 && format != STQ1_FMT_STQ2) return STQ1_ERR_ARG;
   if (L <= 0 || N <= 0 || n_cal <= 0 || K < kBlockWeights || K % kBlockWeights) return STQ1_ERR_SHAPE;
