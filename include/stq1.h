@@ -148,11 +148,14 @@ size_t stq1_gemv_workspace(int64_t N, int64_t K, int batch);
 
 /*
  * stq1_gemv -- y[t, j] = sum_k W^[j, k] x[t, k], fp32 accumulation.
- * The decoded weight is never materialised: codes are expanded through a
- * per-group lookup table of the activation sums, so the weight side has no
- * multiplies ("Runtime" section of the lemmy post: STQ1_0 CUDA kernels).
- * Small batches use the lookup-table kernel; larger batches the tensor-core
- * tile kernel.
+ * The decoded weight is never materialised in memory ("Runtime" section of
+ * the lemmy post: STQ1_0 CUDA kernels).  One token uses the lookup-table
+ * kernel: codes index per-group tables of the activation sums, so the weight
+ * side has no multiplies.  2 to 15 tokens use the tensor-core decode kernel:
+ * each group's code is expanded once in registers to bf16 +/-1 and 0 and
+ * contracted against up to 8 tokens per MMA (fp32 accumulation, d applied
+ * per 256-weight block in fp32).  Larger batches use the tensor-core tile
+ * kernel when it is expected to be faster (see stq1_set_path).
  *   W_packed   device, [N, K] STQ1_0 blocks, 16-byte aligned.
  *   x          device, [batch, K] bf16 bits, row-major, 16-byte aligned.
  *   y          device, [batch, N] fp32, row-major (fully overwritten).
@@ -191,15 +194,16 @@ size_t stq1_moe_workspace(int T, int topk, int E, int64_t N, int64_t K, int flag
  *   ws, ws_bytes   device workspace, at least stq1_moe_workspace(...) bytes
  *                  (computed with the same flags).
  * Requires N even, K % 256 == 0, 1 <= topk <= E (any topk with STQ1_MOE_SKIP_FOREIGN).
- * Paths: with few token-slot pairs per routed expert (decode) the lookup-table
- * kernel runs; with many (prefill) the tensor-core tile kernel.
+ * Paths: with few token-slot pairs per routed expert (decode) the tensor-core
+ * decode kernel runs (units of up to 8 pairs of one expert); with many
+ * (prefill) the tensor-core tile kernel.
  * STQ1_MOE_FP8 applies to the tile kernel only: each token row of x is
  * quantized to E4M3 as by stq1_quantize_x_e4m3, the +/-1 weight patterns are
  * E4M3 too, the MMAs run in fp8 with fp32 accumulation and y is multiplied by
  * the row's scale.  The weights stay exact; the activations carry E4M3's
  * relative error (up to 2^-4), so this variant is outside the accuracy bound
- * below and its error is measured, not bounded.  The table kernel ignores the
- * flag.
+ * below and its error is measured, not bounded.  The decode kernels (table
+ * and tensor-core decode) ignore the flag.
  * Accuracy (without STQ1_MOE_FP8): as stq1_gemv, per output.
  * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_ALIGN, STQ1_ERR_WORKSPACE,
  * STQ1_ERR_ARG, STQ1_ERR_CUDA.
@@ -334,12 +338,18 @@ int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float* y, int64_t
                       int batch, void* stream);
 
 /*
- * stq1_set_path -- process-wide choice between the two matmul kernels, for
- * testing and crossover measurements: 0 = by size (default: batches of 16 or
- * more tokens, and MoE calls averaging 16 or more pairs per routed expert, use
- * the tensor-core tile kernel), 1 = always the lookup-table kernel, 2 = the tile
- * kernel whenever the shape allows it (K / 256 even).  Not thread-safe with
- * concurrent calls.  Errors: STQ1_ERR_ARG.
+ * stq1_set_path -- process-wide choice between the matmul kernels, for testing
+ * and crossover measurements: 0 = by size (default: one token uses the
+ * lookup-table kernel; 2 to 15 tokens, and MoE calls averaging fewer than 16
+ * pairs per routed expert, the tensor-core decode kernel; 16 or more tokens,
+ * and MoE calls averaging 16 or more pairs per routed expert, the tensor-core
+ * tile kernel when it is expected to be faster), 1 = always the lookup-table
+ * kernel, 2 = the tile kernel whenever the shape allows it, 3 = the
+ * tensor-core decode kernel (up to 8 tokens per unit) whenever the shape
+ * allows it.  "Allows" means K / 256 even; other shapes use a generic kernel.
+ * The value is read atomically by each call: a call that overlaps a change
+ * on another host thread uses either the old or the new choice.
+ * Errors: STQ1_ERR_ARG.
  */
 int stq1_set_path(int path);
 

@@ -483,11 +483,12 @@ def quantize_x_e4m3(x, out=None, scales=None):
     return out, scales
 
 
-PATH_AUTO, PATH_TABLE, PATH_TILES = 0, 1, 2
+PATH_AUTO, PATH_TABLE, PATH_TILES, PATH_MMA = 0, 1, 2, 3
 
 
 def set_path(path: int) -> None:
-    """Selects the matmul kernel process-wide (0 by size, 1 table kernel, 2 tile kernel)."""
+    """Selects the matmul kernel process-wide (0 by size, 1 table kernel, 2 tile kernel,
+    3 tensor-core decode kernel)."""
     _check("stq1_set_path", _load().stq1_set_path(path))
 
 

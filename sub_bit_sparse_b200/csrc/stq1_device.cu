@@ -13,6 +13,7 @@
 #include "device_common.cuh"
 #include "encode_device.cuh"
 #include "gemv_lut.cuh"
+#include "gemv_mma.cuh"
 #include "mix_score.cuh"
 #include "small_kernels.cuh"
 #include "tc_gemm.cuh"
@@ -44,7 +45,8 @@ struct NvtxRange {
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
-// Path selection: 0 = by size, 1 = table kernel, 2 = tensor-core tile kernel.
+// Path selection: 0 = by size, 1 = table kernel, 2 = tensor-core tile kernel,
+// 3 = tensor-core decode kernel (mma.sync, few tokens).
 // Atomic so that a call on another host thread reads either value, never a torn one.
 std::atomic<int> g_path{0};
 constexpr int kTcMinBatch = 16;       // stq1_gemv: batches from here use the tile kernel
@@ -136,7 +138,9 @@ int ensure_configured() {
       cudaFuncSetAttribute(hess_score_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kHsSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(hess_score_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kHsSmemBytes) != cudaSuccess)
+                           kHsSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(mma_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(mma_smem_bytes_max())) != cudaSuccess)
     return STQ1_ERR_CUDA;
   // split-K clusters of up to 16 CTAs (above the portable 8); a refusal only
   // disables the cluster path
@@ -309,12 +313,12 @@ int lut_stages(const LutArgs& a) { return a.cq + (a.cr > 0 ? 1 : 0) >= 2 ? 2 : 1
 struct GemvPlan {
   int n_tiles, n_slabs, S, n_chunks, tt;
   size_t partial_bytes, counter_bytes;
-  bool table_path, tile_path;
+  bool table_path, tile_path, mma_path;
 };
 
 bool want_tiles(long long nb, long long units) {
   if (nb % 2 != 0) return false;          // the tile kernel needs 4-byte-aligned rows
-  if (g_path == 1) return false;
+  if (g_path == 1 || g_path == 3) return false;
   if (g_path == 2) return true;
   return units >= kTcMinBatch;
 }
@@ -373,15 +377,52 @@ void plan_table(GemvPlan* p, long long N, long long K, int batch, bool one_wave)
   p->S = static_cast<int>(std::max<long long>(1, S));
 }
 
+// Tensor-core decode kernel for few tokens: 2 .. 15 tokens by default (one
+// token keeps the table kernel, whose per-group cost is lower), any batch
+// when forced.  Rows need an even number of blocks (chunks of two).
+bool want_mma(long long nb, int batch) {
+  if (nb % 2 != 0) return false;
+  const int path = g_path;
+  if (path == 3) return true;
+  if (path != 0) return false;
+  return batch >= 2;
+}
+
+// Work split of the tensor-core decode kernel: (8-token tile, 128-row slab)
+// units, each cut into S pieces of K (whole steps of four blocks) so that
+// there are about two CTAs per SM, then reduced to the fewest pieces with
+// the same longest piece.
+void plan_mma(GemvPlan* p, long long N, long long K, int batch) {
+  const long long nb = K / kBlockWeights;
+  p->n_tiles = (batch + kMmaTokens - 1) / kMmaTokens;
+  p->n_slabs = static_cast<int>((N + kMmaRows - 1) / kMmaRows);
+  p->n_chunks = static_cast<int>(nb / 2);
+  const long long steps = (p->n_chunks + 1) / 2;
+  const long long units0 = static_cast<long long>(p->n_tiles) * p->n_slabs;
+  const long long target = 2LL * sm_count();
+  long long S = units0 < target ? (target + units0 - 1) / units0 : 1;
+  // split K only while the arrival counters of the units fit their region
+  if (units0 * static_cast<long long>(sizeof(int)) > static_cast<long long>(kCounterBytes)) S = 1;
+  S = std::max<long long>(1, std::min<long long>(S, steps));
+  const long long longest = (steps + S - 1) / S;
+  if (longest > 0) S = (steps + longest - 1) / longest;
+  p->S = static_cast<int>(S);
+}
+
 GemvPlan plan_gemv(long long N, long long K, int batch) {
   GemvPlan p{};
   const long long nb = K / kBlockWeights;
   p.tile_path = want_tiles_gemv(N, nb, batch);
   if (p.tile_path) return p;
-  p.table_path = (nb % 2 == 0);
-  plan_table(&p, N, K, batch, true);
-  if (!p.table_path) p.S = 1;
-  if (p.table_path && p.S > 1) {
+  if (want_mma(nb, batch)) {
+    p.mma_path = true;
+    plan_mma(&p, N, K, batch);
+  } else {
+    p.table_path = (nb % 2 == 0);
+    plan_table(&p, N, K, batch, true);
+    if (!p.table_path) p.S = 1;
+  }
+  if ((p.table_path || p.mma_path) && p.S > 1) {
     p.partial_bytes = static_cast<size_t>(p.S) * batch * N * sizeof(float);
     p.counter_bytes = kCounterBytes;
   }
@@ -456,6 +497,32 @@ int gemv_impl(const void* W_packed, const uint16_t* x, float* y, int64_t N, int6
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
     return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
   }
+  if (p.mma_path) {
+    MmaArgs m{};
+    PackedMaps maps;
+    rc = packed_maps_cached(&maps, &m.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
+    if (rc != STQ1_OK) return rc;
+    m.x = x;
+    m.y = y;
+    m.counters = p.S > 1 ? static_cast<int*>(workspace) : nullptr;
+    m.partial = p.S > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes) : nullptr;
+    m.N = static_cast<int>(N);
+    m.K = static_cast<int>(K);
+    m.topk = 1;
+    m.batch = batch;
+    m.rows_out = batch;
+    m.n_slabs = p.n_slabs;
+    m.n_chunks = p.n_chunks;
+    const int steps = (p.n_chunks + 1) / 2;
+    m.S = p.S;
+    m.sq = steps / p.S;
+    m.sr = steps % p.S;
+    m.flags = 0;
+    const long long units = static_cast<long long>(p.n_tiles) * p.n_slabs;
+    if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
+    return launch_pdl_cluster(mma_gemv_kernel, dim3(static_cast<unsigned>(units), static_cast<unsigned>(p.S)),
+                              kMmaThreads, mma_smem_bytes(m.g.stage_bytes), s, 1u, maps.w, maps.t, m);
+  }
   if (!p.table_path) {
     const long long warps = static_cast<long long>(batch) * N;
     direct_gemv_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(
@@ -522,7 +589,7 @@ namespace {
 struct MoePlan {
   size_t pairs_off, tiles_off, ntiles_off, xperm_off, xq_off, sq_off, sperm_off, total;
   int max_tiles, tile_tokens;
-  bool tiles, fp8;
+  bool tiles, fp8, mma;
 };
 MoePlan plan_moe(int T, int topk, int E, long long K, int flags) {
   MoePlan m{};
@@ -530,7 +597,8 @@ MoePlan plan_moe(int T, int topk, int E, long long K, int flags) {
   const long long nb = K / kBlockWeights;
   const long long active = std::min<long long>(E, n_pairs);
   m.tiles = want_tiles(nb, n_pairs >= kTcMinPairsPerExpert * active ? kTcMinBatch : 0);
-  m.tile_tokens = m.tiles ? kTcN : kMoeTableTokens;
+  m.mma = !m.tiles && nb % 2 == 0 && g_path != 1;
+  m.tile_tokens = m.tiles ? kTcN : (m.mma ? kMmaTokens : kMoeTableTokens);
   m.max_tiles = static_cast<int>(std::min<long long>(n_pairs, n_pairs / m.tile_tokens + active));
   size_t off = 0;
   m.pairs_off = off;
@@ -645,6 +713,33 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
     if (m.fp8) return launch_pdl(tc_gemm_kernel<true>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
     return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
+  }
+  if (m.mma) {
+    MmaArgs a{};
+    PackedMaps maps;
+    rc = packed_maps_cached(&maps, &a.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
+                            rowbytes, N % residue_period(rowbytes) != 0);
+    if (rc != STQ1_OK) return rc;
+    a.x = x;
+    a.y = y;
+    a.tile_info = tiles;
+    a.n_tiles_dev = ntiles;
+    a.pairs = pairs;
+    a.route_w = topk_weights;
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.topk = topk;
+    a.rows_out = n_pairs;
+    a.n_slabs = static_cast<int>((N + kMmaRows - 1) / kMmaRows);
+    a.n_chunks = static_cast<int>(nb / 2);
+    a.S = 1;
+    a.sq = (a.n_chunks + 1) / 2;
+    a.sr = 0;
+    a.flags = flags;
+    const long long units = static_cast<long long>(m.max_tiles) * a.n_slabs;
+    if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
+    return launch_pdl_cluster(mma_gemv_kernel, dim3(static_cast<unsigned>(units)), kMmaThreads,
+                              mma_smem_bytes(a.g.stage_bytes), s, 1u, maps.w, maps.t, a);
   }
   LutArgs a{};
   PackedMaps maps;
@@ -815,7 +910,7 @@ extern "C" int stq1_moe_ffn_local(const void* gateup_local, const void* down_loc
 }
 
 extern "C" int stq1_set_path(int path) {
-  if (path < 0 || path > 2) return STQ1_ERR_ARG;
+  if (path < 0 || path > 3) return STQ1_ERR_ARG;
   g_path.store(path);
   return STQ1_OK;
 }
