@@ -257,8 +257,11 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const PackedRow pr = packed_row(a.g, R0, 64 * rh + 16 * rt + gq + 8 * u);
-      slot[2 * rt + u] = pr.slot;
       ok[2 * rt + u] = slab * kMmaRows + pr.rho < a.N;
+      // A row outside the matrix has no slot in the stage (its computed slot
+      // can lie past the stage's tail slots): read slot 0 instead, whose
+      // bytes are in bounds, and give the row scale 0.
+      slot[2 * rt + u] = ok[2 * rt + u] ? pr.slot : 0u;
       if (u == 0) res_of_tile[rt] = pr.res;
     }
   }
@@ -335,7 +338,7 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
           cA = load_quarter<0>(st + slot[2 * rt] + o, q);
           cB = load_quarter<0>(st + slot[2 * rt + 1] + o, q);
         }
-        // rows outside the matrix: scale 0 (their codes are whatever the copy brought)
+        // rows outside the matrix: scale 0 (their codes are slot 0's bytes)
         if (!ok[2 * rt]) cA.d = 0.f;
         if (!ok[2 * rt + 1]) cB.d = 0.f;
         mma_tile_block(cA, cB, xb, table, acc[rt]);
