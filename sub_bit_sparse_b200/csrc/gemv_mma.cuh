@@ -4,9 +4,10 @@
 // four weights is one of 32 patterns in {-d, 0, +d} with one zero lane
 // (lemmy.durstig.online post 66506, "Four weights, five bits"), so the
 // pattern is exact in bf16 and only d is not.  Each group's 5-bit code is
-// expanded once into bf16 values +/-2 and 0 -- one 4-byte load from a
-// 32-entry shared table (the four lanes' high bytes) and two byte permutes
-// that place them into the two A-operand registers -- and the tensor core
+// expanded once into bf16 values +/-2 and 0 -- two 4-byte loads from two
+// 32-entry shared tables that hold, per code, lanes 0-1 and lanes 2-3 as
+// ready bf16 pairs (each table is 128 bytes, so a warp's 32 lookups hit 32
+// distinct banks), i.e. the two A-operand registers -- and the tensor core
 // contracts the pattern against the bf16 activations of all tokens of the
 // unit with fp32 accumulation.  The decode cost per weight does not depend
 // on the number of tokens, unlike the lookup-table kernel, whose table loads
@@ -48,7 +49,7 @@ constexpr int kMmaRows = kSlabRows;              // 128 rows per unit
 constexpr int kMmaStepBlocks = 4;                // blocks consumed per step (two chunks)
 constexpr int kMmaStages = 4;                    // packed-weight chunks in flight
 constexpr int kMmaXStepBytes = kMmaStepBlocks * kMmaTokens * kBlockWeights * 2;   // 16 KB
-constexpr int kMmaOffTable = 0;                  // 32 x 4 bytes (256-aligned base)
+constexpr int kMmaOffTable = 0;                  // 2 x 32 x 4 bytes (256-aligned base)
 constexpr int kMmaOffBar = 256;                  // kMmaStages mbarriers
 constexpr int kMmaOffX = 512;                    // 2 x 16 KB of staged activations
 constexpr int kMmaOffStage = kMmaOffX + 2 * kMmaXStepBytes;
@@ -145,12 +146,20 @@ __device__ __forceinline__ void code_offsets(uint32_t Q, uint32_t hb, uint32_t& 
   co = ((Q >> 2) & 0x3C3C3C3Cu) | (((hb & 0xAAu) * 0x00820820u) & 0x40404040u);
 }
 
+template <int OFF>
+__device__ __forceinline__ uint32_t lds_u32_off(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
+  return v;
+}
+
 // The two A registers (lanes 0, 1 and lanes 2, 3 as bf16 pairs) of the group
-// whose table offset is byte m of `c`.
+// whose table offset is byte m of `c`: the offset is spliced into the
+// 256-aligned table base, the second table sits 128 bytes above the first.
 __device__ __forceinline__ void decode_group(uint32_t c, int m, uint32_t table, uint32_t& lo, uint32_t& hi) {
-  const uint32_t r = lds_u32(__byte_perm(c, table, 0x7650u | static_cast<uint32_t>(m)));
-  lo = __byte_perm(r, 0u, 0x1404u);
-  hi = __byte_perm(r, 0u, 0x3424u);
+  const uint32_t addr = __byte_perm(c, table, 0x7650u | static_cast<uint32_t>(m));
+  lo = lds_u32_off<0>(addr);
+  hi = lds_u32_off<128>(addr);
 }
 
 // One 16-row tile of one block: 16 MMAs into a fresh accumulator, then added
@@ -162,7 +171,8 @@ __device__ __forceinline__ void mma_tile_block(const QuarterCodes& cA, const Qua
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const uint32_t QA = half ? cA.Q1 : cA.Q0, QB = half ? cB.Q1 : cB.Q0;
-    const uint32_t hA = (cA.S >> (8 * half)) & 0xFFu, hB = (cB.S >> (8 * half)) & 0xFFu;
+    // code_offsets looks at bits 0..7 only
+    const uint32_t hA = half ? (cA.S >> 8) : cA.S, hB = half ? (cB.S >> 8) : cB.S;
     uint32_t eA, oA, eB, oB;
     code_offsets(QA, hA, eA, oA);
     code_offsets(QB, hB, eB, oB);
@@ -227,12 +237,15 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
 
   // ---- set-up: decode table, barriers, first copies ----
   if (threadIdx.x < 32) {
+    // bf16 +2 = 0x4000, -2 = 0xC000, 0 = 0x0000; lanes 0, 1 then lanes 2, 3
     int v[4];
     code_pattern(threadIdx.x, v);
-    uint32_t r = 0;
+    uint32_t h[4];
 #pragma unroll
-    for (int l = 0; l < 4; ++l) r |= (v[l] == 0 ? 0u : (v[l] > 0 ? 0x40u : 0xC0u)) << (8 * l);
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 4u * threadIdx.x), "r"(r) : "memory");
+    for (int l = 0; l < 4; ++l) h[l] = v[l] == 0 ? 0u : (v[l] > 0 ? 0x4000u : 0xC000u);
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 4u * threadIdx.x), "r"(h[0] | (h[1] << 16)) : "memory");
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 128u + 4u * threadIdx.x), "r"(h[2] | (h[3] << 16))
+                 : "memory");
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMmaStages; ++i) mbar_init(bar0 + 8u * i, 1);

@@ -16,19 +16,23 @@ namespace stq1 {
 // change any result: every output row is computed on its own).
 // tile_info[4 * i] = expert, first pair offset, pair count (<= tile_tokens), 0.
 // n_tiles[0] = number of tiles, n_tiles[1] = number of pairs with a valid id.
+// With small_max > 0, an expert with at most small_max pairs gets one tile in
+// a second table, tile_small (same format), counted in n_tiles[2]; the other
+// experts' tiles go to tile_info as before.  Decode sends the two tables to
+// different kernels.
 // ---------------------------------------------------------------------------
 constexpr int kRouteThreads = 1024;
 
 __global__ void __launch_bounds__(kRouteThreads)
-route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_tokens,
-             int* __restrict__ pairs_out, int* __restrict__ tile_info, int* __restrict__ n_tiles,
-             float* __restrict__ y, int N, int skip_foreign) {
+route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_tokens, int small_max,
+             int* __restrict__ pairs_out, int* __restrict__ tile_info, int* __restrict__ tile_small,
+             int* __restrict__ n_tiles, float* __restrict__ y, int N, int skip_foreign) {
   extern __shared__ int sm[];
   griddep_wait();           // ids may come from the previous kernel in the stream
   griddep_launch_dependents();
   int* cnt = sm;            // [E]
   int* off = sm + E;        // [E]
-  int* tst = sm + 2 * E;    // [E]
+  int* tst = sm + 2 * E;    // [E] first tile of the expert in its table
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
@@ -42,38 +46,54 @@ route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_token
     }
   }
   __syncthreads();
+  // tiles of an expert with c pairs: in the small table one (c <= small_max),
+  // else ceil(c / tile_tokens) in the main table
+  auto big_tiles = [&](int c) { return c > small_max ? (c + tile_tokens - 1) / tile_tokens : 0; };
+  auto small_tiles = [&](int c) { return (c > 0 && c <= small_max) ? 1 : 0; };
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     const int per = (E + 31) / 32;
     const int lo = min(E, lane * per), hi = min(E, lo + per);
-    int s1 = 0, s2 = 0;
+    int s1 = 0, s2 = 0, s3 = 0;
     for (int e = lo; e < hi; ++e) {
       s1 += cnt[e];
-      s2 += (cnt[e] + tile_tokens - 1) / tile_tokens;
+      s2 += big_tiles(cnt[e]);
+      s3 += small_tiles(cnt[e]);
     }
-    int i1 = s1, i2 = s2;
+    int i1 = s1, i2 = s2, i3 = s3;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
       const int v1 = __shfl_up_sync(0xffffffffu, i1, d);
       const int v2 = __shfl_up_sync(0xffffffffu, i2, d);
-      if (lane >= d) { i1 += v1; i2 += v2; }
+      const int v3 = __shfl_up_sync(0xffffffffu, i3, d);
+      if (lane >= d) { i1 += v1; i2 += v2; i3 += v3; }
     }
-    int r1 = i1 - s1, r2 = i2 - s2;
+    int r1 = i1 - s1, r2 = i2 - s2, r3 = i3 - s3;
     for (int e = lo; e < hi; ++e) {
       off[e] = r1;
-      tst[e] = r2;
+      tst[e] = small_tiles(cnt[e]) ? r3 : r2;
       r1 += cnt[e];
-      r2 += (cnt[e] + tile_tokens - 1) / tile_tokens;
+      r2 += big_tiles(cnt[e]);
+      r3 += small_tiles(cnt[e]);
     }
     if (lane == 31) {
-      n_tiles[0] = i2;       // tiles
+      n_tiles[0] = i2;       // tiles in the main table
       n_tiles[1] = i1;       // pairs with a valid expert id
+      n_tiles[2] = i3;       // tiles in the small table
     }
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int c = cnt[e];
-    const int nt = (c + tile_tokens - 1) / tile_tokens;
+    if (small_tiles(c)) {
+      int* ti = tile_small + 4 * tst[e];
+      ti[0] = e;
+      ti[1] = off[e];
+      ti[2] = c;
+      ti[3] = 0;
+      continue;
+    }
+    const int nt = big_tiles(c);
     for (int k = 0; k < nt; ++k) {
       int* ti = tile_info + 4 * (tst[e] + k);
       ti[0] = e;

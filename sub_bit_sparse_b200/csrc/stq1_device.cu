@@ -587,10 +587,15 @@ extern "C" int stq1_gemv_prefetch(const void* W_packed, const uint16_t* x, float
 namespace stq1 {
 namespace {
 struct MoePlan {
-  size_t pairs_off, tiles_off, ntiles_off, xperm_off, xq_off, sq_off, sperm_off, total;
-  int max_tiles, tile_tokens;
+  size_t pairs_off, tiles_off, small_off, ntiles_off, xperm_off, xq_off, sq_off, sperm_off, total;
+  int max_tiles, tile_tokens, small_max, max_small;
   bool tiles, fp8, mma;
 };
+// Decode with the tensor-core kernel: experts with at most this many routed
+// pairs go to the lookup-table kernel instead, whose cost per weight is lower
+// for one or two tokens (one table load per token and group against a fixed
+// decode of about a dozen instructions per group on the tensor-core path).
+constexpr int kMoeSmallMax = 2;
 MoePlan plan_moe(int T, int topk, int E, long long K, int flags) {
   MoePlan m{};
   const long long n_pairs = static_cast<long long>(T) * topk;
@@ -600,11 +605,15 @@ MoePlan plan_moe(int T, int topk, int E, long long K, int flags) {
   m.mma = !m.tiles && nb % 2 == 0 && g_path != 1;
   m.tile_tokens = m.tiles ? kTcN : (m.mma ? kMmaTokens : kMoeTableTokens);
   m.max_tiles = static_cast<int>(std::min<long long>(n_pairs, n_pairs / m.tile_tokens + active));
+  m.small_max = m.mma ? kMoeSmallMax : 0;
+  m.max_small = m.mma ? static_cast<int>(active) : 0;
   size_t off = 0;
   m.pairs_off = off;
   off += round16(n_pairs * sizeof(int));
   m.tiles_off = off;
   off += round16(static_cast<size_t>(m.max_tiles) * 4 * sizeof(int));
+  m.small_off = off;
+  off += round16(static_cast<size_t>(m.max_small) * 4 * sizeof(int));
   m.ntiles_off = off;
   off += 16;
   m.fp8 = m.tiles && (flags & STQ1_MOE_FP8);
@@ -657,6 +666,7 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   int* pairs = reinterpret_cast<int*>(wsb + m.pairs_off);
   int* tiles = reinterpret_cast<int*>(wsb + m.tiles_off);
+  int* tiles_small = reinterpret_cast<int*>(wsb + m.small_off);
   int* ntiles = reinterpret_cast<int*>(wsb + m.ntiles_off);
 
   if (nb % 2 != 0) {
@@ -668,7 +678,8 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   }
 
   rc = launch_pdl(route_kernel, 1, kRouteThreads, 3 * E * sizeof(int), s, topk_ids, n_pairs, E, m.tile_tokens,
-                  pairs, tiles, ntiles, y, static_cast<int>(N), (flags & STQ1_MOE_SKIP_FOREIGN) ? 1 : 0);
+                  m.small_max, pairs, tiles, tiles_small, ntiles, y, static_cast<int>(N),
+                  (flags & STQ1_MOE_SKIP_FOREIGN) ? 1 : 0);
   if (rc != STQ1_OK) return rc;
   if (m.tiles) {
     void* xperm = wsb + m.xperm_off;
@@ -720,6 +731,31 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
     rc = packed_maps_cached(&maps, &a.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
                             rowbytes, N % residue_period(rowbytes) != 0);
     if (rc != STQ1_OK) return rc;
+    // experts with one or two pairs: the lookup-table kernel (small tile table)
+    {
+      LutArgs l{};
+      l.g = a.g;
+      l.x = x;
+      l.y = y;
+      l.tile_info = tiles_small;
+      l.n_tiles_dev = ntiles + 2;
+      l.pairs = pairs;
+      l.route_w = topk_weights;
+      l.N = static_cast<int>(N);
+      l.K = static_cast<int>(K);
+      l.topk = topk;
+      l.rows_out = n_pairs;
+      l.n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
+      set_split(&l, static_cast<int>(nb / kLutKC), 1);
+      l.flags = flags;
+      l.cluster = 0;
+      const long long lunits = static_cast<long long>(m.max_small) * l.n_slabs;
+      if (lunits >= (1LL << 31)) return STQ1_ERR_SHAPE;
+      rc = launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(lunits)), kLutThreads,
+                              lut_smem_bytes(kMoeTableTokens, lut_stages(l), l.g.stage_bytes, 1), s, 1u, maps.w,
+                              maps.t, l);
+      if (rc != STQ1_OK) return rc;
+    }
     a.x = x;
     a.y = y;
     a.tile_info = tiles;

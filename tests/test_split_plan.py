@@ -1,4 +1,4 @@
-"""The table GEMV's K-split plan, read through the workspace query (no GPU).
+"""The GEMV kernels' K-split plans, read through the workspace query (no GPU).
 
 stq1_gemv_workspace returns 2048 counter bytes plus S * batch * N * 4 bytes of
 partial sums when the plan splits K into S > 1 pieces, and 0 otherwise, so the
@@ -9,6 +9,20 @@ plan's S can be checked on the host.  Without a device the planner assumes a
 import pytest
 
 import sub_bit_sparse_b200 as stq1
+
+
+@pytest.fixture
+def table_path():
+    stq1.set_path(stq1.PATH_TABLE)
+    yield
+    stq1.set_path(stq1.PATH_AUTO)
+
+
+@pytest.fixture
+def mma_path():
+    stq1.set_path(stq1.PATH_MMA)
+    yield
+    stq1.set_path(stq1.PATH_AUTO)
 
 
 def _split(n, k, b):
@@ -25,16 +39,33 @@ def _split(n, k, b):
     (18432, 7168, 2, 1),    # 144 two-token units already exceed that target: no split
     (18432, 7168, 1, 4),    # 144 slabs x 4 pieces (the longest piece of 4 chunks, 14 = 4+4+3+3)
 ])
-def test_split_of_the_benchmark_shapes(n, k, b, want):
+def test_split_of_the_benchmark_shapes(table_path, n, k, b, want):
     assert _split(n, k, b) == want
 
 
 @pytest.mark.parametrize("b", [1, 2, 4, 8])
 @pytest.mark.parametrize("n,k", [(4096, 7168), (18432, 7168), (512, 2048), (1000, 4096)])
-def test_pieces_are_as_few_as_the_longest_piece_allows(n, k, b):
+def test_pieces_are_as_few_as_the_longest_piece_allows(table_path, n, k, b):
     # the plan never uses more pieces than its longest piece needs
     chunks = k // 512
     s = _split(n, k, b)
     assert 1 <= s <= min(chunks, 16)
     longest = -(-chunks // s)
     assert s == -(-chunks // longest)
+
+
+# Tensor-core decode kernel: (8-token tile, 128-row slab) units, K split in
+# whole steps of four blocks (two chunks) to about two CTAs per SM.
+@pytest.mark.parametrize("n,k,b,want", [
+    (4096, 7168, 8, 7),     # 32 units want 10 pieces; 7 steps allow 7
+    (4096, 7168, 12, 4),    # 64 units (two token tiles) want 5 pieces of 7 steps: longest 2 -> 4 pieces
+    (18432, 7168, 8, 3),    # 144 units want 3 pieces; longest 3 steps -> 3 (3 + 2 + 2)
+    (512, 2048, 4, 2),      # 4 units, 2 steps
+    (37888, 7168, 4, 1),    # 296 units: already two per SM
+])
+def test_mma_split(mma_path, n, k, b, want):
+    s = _split(n, k, b)
+    steps = -(-(k // 512) // 2)
+    longest = -(-steps // s)
+    assert s == -(-steps // longest)      # as few pieces as the longest piece allows
+    assert s == want
