@@ -590,7 +590,9 @@ def crossover(torch, stq1, device, stream, batches, reps_cap=4096):
     """Crossover between the kernels on one [18432, 7168] matrix with the decode
     matrix's statistics: per batch, each forced path and the library's own
     choice, timed in a CUDA graph of launches over rotating copies larger than
-    L2 (GB/s of packed weights and dense-equivalent TFLOP/s)."""
+    L2 (GB/s of packed weights and dense-equivalent TFLOP/s): the lookup-table
+    kernel, the tensor-core decode kernel (mma.sync), the tcgen05 tile kernel
+    and the library's own choice."""
     import workloads
     w, h, x = workloads.crossover_inputs()
     n, k = w.shape
@@ -602,8 +604,15 @@ def crossover(torch, stq1, device, stream, batches, reps_cap=4096):
     del wd
     xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
     y = torch.empty((max(batches), n), dtype=torch.float32, device=device)
-    ws = stq1.workspace(max(stq1.LIB.stq1_gemv_workspace(n, k, b) for b in batches), device)
-    paths = (("table", stq1.PATH_TABLE), ("tiles", stq1.PATH_TILES), ("auto", stq1.PATH_AUTO))
+    paths = (("table", stq1.PATH_TABLE), ("mma", stq1.PATH_MMA), ("tiles", stq1.PATH_TILES), ("auto", stq1.PATH_AUTO))
+    need = 0
+    try:
+        for _, path in paths:                                 # each kernel's plan has its own split
+            stq1.set_path(path)
+            need = max([need] + [stq1.LIB.stq1_gemv_workspace(n, k, b) for b in batches])
+    finally:
+        stq1.set_path(stq1.PATH_AUTO)
+    ws = stq1.workspace(need, device)
     rows = []
     try:
         for b in batches:
@@ -631,13 +640,14 @@ def crossover(torch, stq1, device, stream, batches, reps_cap=4096):
             rows.append(row)
     finally:
         stq1.set_path(stq1.PATH_AUTO)
-    faster = [r["batch"] for r in rows if r["tiles"]["us"] < r["table"]["us"]]
+    faster = [r["batch"] for r in rows if r["tiles"]["us"] < min(r["table"]["us"], r["mma"]["us"])]
     del stack, y
     return {"matrix": [n, k], "packed_bytes": int(pb), "rows": rows,
             "tiles_faster_from_batch": min(faster) if faster else None,
             "config": "one [18432, 7168] STQ1_0 matrix (decode-matrix statistics, Sherry 3 rounds), bf16 batch "
                       "prefix of x [1024, 7168]; CUDA graph over rotating copies (> 2 x L2); table = lookup-table "
-                      "kernel, tiles = tcgen05 tile kernel, auto = the library's own choice"}
+                      "kernel, mma = tensor-core decode kernel, tiles = tcgen05 tile kernel, auto = the library's "
+                      "own choice"}
 
 
 def run_sweep(args):

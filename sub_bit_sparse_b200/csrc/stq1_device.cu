@@ -377,15 +377,20 @@ void plan_table(GemvPlan* p, long long N, long long K, int batch, bool one_wave)
   p->S = static_cast<int>(std::max<long long>(1, S));
 }
 
-// Tensor-core decode kernel for few tokens: 2 .. 15 tokens by default (one
-// token keeps the table kernel, whose per-group cost is lower), any batch
-// when forced.  Rows need an even number of blocks (chunks of two).
+// Tensor-core decode kernel for few tokens: 5 .. 15 tokens by default, any
+// batch when forced.  Its cost per weight does not depend on the token count;
+// the table kernel's grows with it.  Measured (CUDA graphs of distinct
+// matrices): on [4096, 7168] 12.6-13.0 us at 1-8 tokens against the table
+// kernel's 5.0 / 7.2 / 10.3 / 16.5 us at 1 / 2 / 4 / 8; on [18432, 7168]
+// 26.0-26.9 us against 15.5 / 19.1 / 27.5 / 49.9 us.  Rows need an even
+// number of blocks (chunks of two).
+constexpr int kMmaMinBatch = 5;
 bool want_mma(long long nb, int batch) {
   if (nb % 2 != 0) return false;
   const int path = g_path;
   if (path == 3) return true;
   if (path != 0) return false;
-  return batch >= 2;
+  return batch >= kMmaMinBatch;
 }
 
 // Work split of the tensor-core decode kernel: (8-token tile, 128-row slab)
