@@ -271,6 +271,13 @@ int stq1_moe_ffn(const void* gateup_blocks, const void* down_blocks, const uint1
  * is this rank's partial sum; the layer's output is the sum of all ranks'
  * partials (an all-reduce).  topk_ids hold global expert ids.  Other
  * arguments as stq1_moe_ffn; ws at least stq1_moe_ffn_local_workspace(...).
+ * Only this rank's pairs are computed and stored: they are grouped by expert
+ * on the device, gate/up writes one row per local pair, SwiGLU and the down
+ * projection run over those rows only (the down projection reuses the
+ * grouping), and the combine gathers each token's local rows; nothing is
+ * written for pairs of other ranks.  (Shapes whose H / 256 or N / 512 is odd
+ * run the whole-layer chain with foreign pairs zeroed instead.)
+ * All pointers 16-byte aligned.
  * Errors: as stq1_moe_ffn.
  */
 size_t stq1_moe_ffn_local_workspace(int T, int topk, int E_local, int64_t N, int64_t H, int flags);

@@ -66,6 +66,9 @@ struct LutArgs {
   int cluster;               // 1: the S splits of a (tile, slab) form one thread-block cluster
   const uint8_t* next;       // bytes to bring into L2 for a following call, or nullptr
   long long next_bytes;      // multiple of 16
+  int compact;               // MoE: bit 0 = output row of a pair is its position in `pairs`
+                             // (else the pair id); bit 1 = its activation row is that position
+                             // (else pair id / topk).  Routing weights are always by pair id.
 };
 
 // Spread bits 0, 2, 4, 6 of x to bit 6 of bytes 0..3 (other bits cleared).
@@ -160,7 +163,7 @@ __device__ __forceinline__ void lut_build(const uint2 (&xv)[kLutMaxTT], uint32_t
 template <int TT>
 __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wmap, const CUtensorMap* tmap, long long R0,
                          int slab, int split, int unit, const uint16_t* const (&xr)[kLutMaxTT],
-                         const int (&orow)[kLutMaxTT], uint8_t* smem) {
+                         const int (&orow)[kLutMaxTT], const int (&wrow)[kLutMaxTT], uint8_t* smem) {
   const int c0 = split * a.cq + min(split, a.cr);
   const int c1 = c0 + a.cq + (split < a.cr ? 1 : 0);
   const int half = threadIdx.x >> 7;               // block of the chunk this thread decodes
@@ -275,7 +278,7 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
       for (int t = 0; t < TT; ++t) {
         float v = 0.f;
         for (int i = 0; i < 2 * a.S; ++i) v += lds_f32_addr(red + 4u * ((t * 2 * a.S + i) * per + local));
-        if (up) v *= a.route_w[orow[t]];
+        if (up) v *= a.route_w[wrow[t]];
         a.y[static_cast<long long>(orow[t]) * a.N + row] = v;
       }
     }
@@ -300,7 +303,7 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
         float v = acc[t];
-        if (up) v *= a.route_w[orow[t]];
+        if (up) v *= a.route_w[wrow[t]];
         a.y[static_cast<long long>(orow[t]) * a.N + row] = v;
       }
     }
@@ -332,7 +335,7 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
       float v = 0.f;
       for (int sp = 0; sp < a.S; ++sp)
         v += __ldcg(&a.partial[(static_cast<long long>(sp) * a.rows_out + orow[t]) * a.N + row]);
-      if (up) v *= a.route_w[orow[t]];
+      if (up) v *= a.route_w[wrow[t]];
       a.y[static_cast<long long>(orow[t]) * a.N + row] = v;
     }
   }
@@ -352,7 +355,7 @@ lut_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
   const int tile = unit / a.n_slabs;
   const int slab = unit - tile * a.n_slabs;
   const uint16_t* xr[kLutMaxTT];
-  int orow[kLutMaxTT];
+  int orow[kLutMaxTT], wrow[kLutMaxTT];
   int cnt, expert = 0;
   if (a.tile_info) {
     griddep_wait();                                  // the tile table comes from the routing kernel
@@ -362,9 +365,11 @@ lut_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
     cnt = a.tile_info[4 * tile + 2];
 #pragma unroll
     for (int t = 0; t < kLutMaxTT; ++t) {
-      const int p = a.pairs[off + (t < cnt ? t : 0)];
-      orow[t] = p;
-      xr[t] = a.x + static_cast<long long>(p / a.topk) * a.K;
+      const int pos = off + (t < cnt ? t : 0);
+      const int p = a.pairs[pos];
+      orow[t] = (a.compact & 1) ? pos : p;
+      wrow[t] = p;
+      xr[t] = a.x + static_cast<long long>((a.compact & 2) ? pos : p / a.topk) * a.K;
     }
   } else {
     const int t0 = tile * kLutMaxTT;
@@ -372,29 +377,30 @@ lut_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
 #pragma unroll
     for (int t = 0; t < kLutMaxTT; ++t) {
       orow[t] = t0 + (t < cnt ? t : 0);
+      wrow[t] = orow[t];
       xr[t] = a.x + static_cast<long long>(orow[t]) * a.K;
     }
   }
   const long long R0 = static_cast<long long>(expert) * a.N + static_cast<long long>(slab) * kLutRows;
   if constexpr (TTMAX >= 4) {
     if (cnt >= 4) {
-      lut_unit<4>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, smem);
+      lut_unit<4>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, wrow, smem);
       return;
     }
   }
   if constexpr (TTMAX >= 3) {
     if (cnt == 3) {
-      lut_unit<3>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, smem);
+      lut_unit<3>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, wrow, smem);
       return;
     }
   }
   if constexpr (TTMAX >= 2) {
     if (cnt == 2) {
-      lut_unit<2>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, smem);
+      lut_unit<2>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, wrow, smem);
       return;
     }
   }
-  lut_unit<1>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, smem);
+  lut_unit<1>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, wrow, smem);
 }
 
 // Dynamic shared memory: tables, barriers, stages and (cluster split K) the

@@ -73,6 +73,9 @@ struct MmaArgs {
   int n_chunks;              // chunks (two blocks each) of K
   int S, sq, sr;             // K splits over steps: split s has sq steps, plus one if s < sr
   int flags;
+  int compact;               // MoE: bit 0 = output row of a pair is its position in `pairs`
+                             // (else the pair id); bit 1 = its activation row is that position
+                             // (else pair id / topk).  Routing weights are always by pair id.
 };
 
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
@@ -222,11 +225,13 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
     cnt = min(kMmaTokens, a.batch - tile * kMmaTokens);
   }
   auto out_row = [&](int t) -> int {               // output row of token t (< cnt)
-    return a.tile_info ? a.pairs[off + t] : tile * kMmaTokens + t;
+    if (!a.tile_info) return tile * kMmaTokens + t;
+    return (a.compact & 1) ? off + t : a.pairs[off + t];
   };
   auto x_row = [&](int t) -> const uint16_t* {     // activation row of token t (clamped)
     const int tt = t < cnt ? t : 0;
-    const int r = a.tile_info ? a.pairs[off + tt] / a.topk : tile * kMmaTokens + tt;
+    int r = tile * kMmaTokens + tt;
+    if (a.tile_info) r = (a.compact & 2) ? off + tt : a.pairs[off + tt] / a.topk;
     return a.x + static_cast<long long>(r) * a.K;
   };
 
@@ -394,7 +399,7 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
   __syncthreads();
   const bool up_flag = (a.flags & STQ1_MOE_WEIGHT_UP) != 0;
   float vals[4];
-  int orows[4], rows[4];
+  int orows[4], rows[4], wrows[4];
   bool good[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -408,6 +413,7 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
     good[k] = t < cnt && row < a.N;
     rows[k] = row;
     orows[k] = good[k] ? out_row(t) : 0;
+    wrows[k] = (good[k] && a.tile_info) ? a.pairs[off + t] : 0;
     vals[k] = v;
   }
   if (a.S == 1) {
@@ -415,7 +421,7 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
     for (int k = 0; k < 4; ++k) {
       if (!good[k]) continue;
       float v = vals[k];
-      if (up_flag && rows[k] >= a.N / 2) v *= a.route_w[orows[k]];
+      if (up_flag && rows[k] >= a.N / 2) v *= a.route_w[wrows[k]];
       a.y[static_cast<long long>(orows[k]) * a.N + rows[k]] = v;
     }
     return;
@@ -440,7 +446,7 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
     float v = 0.f;
     for (int sp = 0; sp < a.S; ++sp)
       v += __ldcg(&a.partial[(static_cast<long long>(sp) * a.rows_out + orows[k]) * a.N + rows[k]]);
-    if (up_flag && rows[k] >= a.N / 2) v *= a.route_w[orows[k]];
+    if (up_flag && rows[k] >= a.N / 2) v *= a.route_w[wrows[k]];
     a.y[static_cast<long long>(orows[k]) * a.N + rows[k]] = v;
   }
   if (threadIdx.x == 0) a.counters[unit] = 0;

@@ -20,14 +20,20 @@ namespace stq1 {
 // a second table, tile_small (same format), counted in n_tiles[2]; the other
 // experts' tiles go to tile_info as before.  Decode sends the two tables to
 // different kernels.
+// inv (optional): inv[p] = the position of pair p in pairs_out, or -1 for a
+// pair whose id is out of range -- the row of p in outputs that are stored
+// compactly, in pairs_out order.  y (optional): the rows of out-of-range
+// pairs are zeroed in y [n_pairs, N] (a compact caller passes nullptr).
 // ---------------------------------------------------------------------------
 constexpr int kRouteThreads = 1024;
 
 __global__ void __launch_bounds__(kRouteThreads)
 route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_tokens, int small_max,
              int* __restrict__ pairs_out, int* __restrict__ tile_info, int* __restrict__ tile_small,
-             int* __restrict__ n_tiles, float* __restrict__ y, int N, int skip_foreign) {
+             int* __restrict__ n_tiles, int* __restrict__ inv, float* __restrict__ y, int N, int skip_foreign) {
   extern __shared__ int sm[];
+  __shared__ int s_bad[kRouteThreads];      // out-of-range pairs to zero, this round
+  __shared__ int s_nbad;
   griddep_wait();           // ids may come from the previous kernel in the stream
   griddep_launch_dependents();
   int* cnt = sm;            // [E]
@@ -35,17 +41,33 @@ route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_token
   int* tst = sm + 2 * E;    // [E] first tile of the expert in its table
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
-  for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
-    const int e = ids[p];
-    if (e < 0 || e >= E) {
-      if (!skip_foreign) flag_error(STQ1_DEV_BAD_EXPERT);
-      float* yr = y + static_cast<long long>(p) * N;
-      for (int j = 0; j < N; ++j) yr[j] = 0.f;
-    } else {
-      atomicAdd(&cnt[e], 1);
+  // Rounds of blockDim pairs: count valid ids; the rows of invalid ones are
+  // zeroed by the whole block (float4 stores along each row).
+  for (int p0 = 0; p0 < n_pairs; p0 += blockDim.x) {
+    if (threadIdx.x == 0) s_nbad = 0;
+    __syncthreads();
+    const int p = p0 + static_cast<int>(threadIdx.x);
+    if (p < n_pairs) {
+      const int e = ids[p];
+      if (e < 0 || e >= E) {
+        if (!skip_foreign) flag_error(STQ1_DEV_BAD_EXPERT);
+        if (inv) inv[p] = -1;
+        if (y) s_bad[atomicAdd(&s_nbad, 1)] = p;
+      } else {
+        atomicAdd(&cnt[e], 1);
+      }
     }
+    __syncthreads();
+    const int nbad = s_nbad;
+    if (nbad > 0) {
+      for (long long i = threadIdx.x; i < static_cast<long long>(nbad) * N; i += blockDim.x) {
+        const int r = static_cast<int>(i / N);
+        const int j = static_cast<int>(i - static_cast<long long>(r) * N);
+        y[static_cast<long long>(s_bad[r]) * N + j] = 0.f;
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
   // tiles of an expert with c pairs: in the small table one (c <= small_max),
   // else ceil(c / tile_tokens) in the main table
   auto big_tiles = [&](int c) { return c > small_max ? (c + tile_tokens - 1) / tile_tokens : 0; };
@@ -108,6 +130,7 @@ route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_token
     if (e < 0 || e >= E) continue;
     const int pos = atomicSub(&cnt[e], 1) - 1;
     pairs_out[off[e] + pos] = p;
+    if (inv) inv[p] = off[e] + pos;
   }
 }
 
@@ -228,10 +251,13 @@ __device__ __forceinline__ uint16_t bf16_bits_from_f64(double x) {
 // act[p, j] = bf16(SiLU(g) * u), g = y[p, j], u = y[p, half + j], SiLU(v) =
 // v / (1 + e^-v), in fp64 (the down projection's bf16 input, rounded once).
 __global__ void __launch_bounds__(256)
-swiglu_kernel(const float* __restrict__ y, uint16_t* __restrict__ act, long long P, int half) {
+swiglu_kernel(const float* __restrict__ y, uint16_t* __restrict__ act, long long P, int half,
+              const int* __restrict__ n_rows) {
   griddep_wait();
   griddep_launch_dependents();
-  const long long total = P * half;
+  // n_rows (optional, device): only the first *n_rows rows are in use
+  const long long rows = n_rows ? min(P, static_cast<long long>(*n_rows)) : P;
+  const long long total = rows * half;
   for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += 256LL * gridDim.x) {
     const long long p = i / half;
     const int j = static_cast<int>(i - p * half);
@@ -264,6 +290,29 @@ combine_kernel(const float* __restrict__ y, const float* __restrict__ w, float* 
     float acc = 0.f;
     for (int s = 0; s < topk; ++s) acc = w ? fmaf(w[t * topk + s], yt[static_cast<long long>(s) * H], acc)
                                            : acc + yt[static_cast<long long>(s) * H];
+    out[i] = acc;
+  }
+}
+
+// Combine of one rank's compact outputs: out[t, h] = sum over slots s whose
+// pair is local (inv[t * topk + s] >= 0) of w[t, s] * y[inv[...], h] (plain
+// sum without w), fp32 in slot order; 0 where no slot is local.
+__global__ void __launch_bounds__(256)
+combine_compact_kernel(const float* __restrict__ y, const float* __restrict__ w, const int* __restrict__ inv,
+                       float* __restrict__ out, long long T, int topk, int H) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const long long total = T * H;
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += 256LL * gridDim.x) {
+    const long long t = i / H;
+    const int h = static_cast<int>(i - t * H);
+    float acc = 0.f;
+    for (int s = 0; s < topk; ++s) {
+      const int r = inv[t * topk + s];
+      if (r < 0) continue;
+      const float v = y[static_cast<long long>(r) * H + h];
+      acc = w ? fmaf(w[t * topk + s], v, acc) : acc + v;
+    }
     out[i] = acc;
   }
 }

@@ -645,6 +645,148 @@ extern "C" size_t stq1_moe_workspace(int T, int topk, int E, int64_t N, int64_t 
   return plan_moe(T, topk, E, K, flags).total;
 }
 
+namespace stq1 {
+namespace {
+
+// Routing tables one MoE call computes once (route_kernel) and its matmuls read.
+struct MoeTables {
+  int* pairs;         // pair ids grouped by expert
+  int* tiles;         // main tile table
+  int* tiles_small;   // tiles of experts with few pairs (tensor-core decode path)
+  int* ntiles;        // [0] main tiles, [1] pairs with a valid id, [2] small tiles
+};
+
+// Device scratch of one matmul over routed pairs on the tile path.
+struct MoeScratch {
+  void* xperm;        // activation rows in pair order (bf16, or E4M3 bytes)
+  uint8_t* xq;        // E4M3 codes of the activation rows (fp8)
+  float* sq;          // their per-row scales (fp8)
+  float* sperm;       // scales in pair order (fp8)
+};
+
+// The matmul over routed pairs, on tables the route kernel already fills.
+// `compact` bit 0: pair i of the grouped list writes output row i (else row
+// pairs[i]); bit 1: its activation row is row i of x (else pairs[i] / topk).
+// x_rows = rows of x (tokens, or the compact rows).  Routing weights are
+// always indexed by pair id.
+int moe_compute(const MoePlan& m, const MoeTables& tb, const MoeScratch& sc, const void* expert_blocks,
+                const uint16_t* x, int x_rows, const float* topk_weights, float* y, int topk, int n_pairs, int E,
+                long long N, long long K, int flags, int compact, cudaStream_t s) {
+  const long long nb = K / kBlockWeights;
+  const long long rowbytes = nb * kBlockBytes;
+  int rc;
+  if (m.tiles) {
+    const void* B = x;
+    float* xscale = nullptr;
+    if (m.fp8) {
+      rc = launch_pdl(quant_e4m3_kernel, static_cast<unsigned>(x_rows), kQuantThreads, 0, s, x, static_cast<int>(K),
+                      sc.xq, sc.sq);
+      if (rc != STQ1_OK) return rc;
+      if (compact & 2) {
+        B = sc.xq;                                   // compact rows are already in pair order
+        xscale = sc.sq;
+      } else {
+        rc = launch_pdl(gather_rows8_kernel, static_cast<unsigned>(n_pairs), 256, 0, s,
+                        static_cast<const uint8_t*>(sc.xq), static_cast<const float*>(sc.sq),
+                        static_cast<const int*>(tb.pairs), static_cast<const int*>(tb.ntiles + 1), n_pairs, topk,
+                        static_cast<int>(K), static_cast<uint8_t*>(sc.xperm), sc.sperm);
+        if (rc != STQ1_OK) return rc;
+        B = sc.xperm;
+        xscale = sc.sperm;
+      }
+    } else if (!(compact & 2)) {
+      rc = launch_pdl(gather_rows_kernel, static_cast<unsigned>(n_pairs), 256, 0, s, x,
+                      static_cast<const int*>(tb.pairs), static_cast<const int*>(tb.ntiles + 1), n_pairs, topk,
+                      static_cast<int>(K), static_cast<uint16_t*>(sc.xperm));
+      if (rc != STQ1_OK) return rc;
+      B = sc.xperm;
+    }
+    CUtensorMap map;
+    if (!make_b_map(&map, B, n_pairs, K, m.fp8)) return STQ1_ERR_CUDA;
+    TcArgs t{};
+    PackedMaps pm;
+    rc = packed_maps_cached(&pm, &t.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
+                            rowbytes, N % residue_period(rowbytes) != 0);
+    if (rc != STQ1_OK) return rc;
+    t.y = y;
+    t.tile_info = tb.tiles;
+    t.n_tiles_dev = tb.ntiles;
+    t.pairs = (compact & 1) ? nullptr : tb.pairs;
+    t.wpairs = tb.pairs;
+    t.route_w = topk_weights;
+    t.xscale = xscale;
+    t.n_tiles = m.max_tiles;
+    t.N = static_cast<int>(N);
+    t.K = static_cast<int>(K);
+    t.nb = static_cast<int>(nb);
+    t.n_mtiles = static_cast<int>((N + kTcM - 1) / kTcM);
+    t.batch = 0;
+    t.flags = flags;
+    const long long items = static_cast<long long>(m.max_tiles) * t.n_mtiles;
+    const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
+    if (m.fp8) return launch_pdl(tc_gemm_kernel<true>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
+    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
+  }
+  PackedMaps maps;
+  PackedGeom geom;
+  rc = packed_maps_cached(&maps, &geom, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
+                          rowbytes, N % residue_period(rowbytes) != 0);
+  if (rc != STQ1_OK) return rc;
+  // lookup-table kernel: every tile (table path) or the experts with few pairs
+  if (!m.mma || m.max_small > 0) {
+    LutArgs l{};
+    l.g = geom;
+    l.x = x;
+    l.y = y;
+    l.tile_info = m.mma ? tb.tiles_small : tb.tiles;
+    l.n_tiles_dev = m.mma ? tb.ntiles + 2 : tb.ntiles;
+    l.pairs = tb.pairs;
+    l.route_w = topk_weights;
+    l.N = static_cast<int>(N);
+    l.K = static_cast<int>(K);
+    l.topk = topk;
+    l.rows_out = n_pairs;
+    l.n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
+    set_split(&l, static_cast<int>(nb / kLutKC), 1);
+    l.flags = flags;
+    l.cluster = 0;
+    l.compact = compact;
+    const long long lunits = static_cast<long long>(m.mma ? m.max_small : m.max_tiles) * l.n_slabs;
+    if (lunits >= (1LL << 31)) return STQ1_ERR_SHAPE;
+    rc = launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(lunits)), kLutThreads,
+                            lut_smem_bytes(kMoeTableTokens, lut_stages(l), l.g.stage_bytes, 1), s, 1u, maps.w, maps.t,
+                            l);
+    if (rc != STQ1_OK || !m.mma) return rc;
+  }
+  // tensor-core decode kernel: the other experts, in tiles of up to 8 pairs
+  MmaArgs a{};
+  a.g = geom;
+  a.x = x;
+  a.y = y;
+  a.tile_info = tb.tiles;
+  a.n_tiles_dev = tb.ntiles;
+  a.pairs = tb.pairs;
+  a.route_w = topk_weights;
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.topk = topk;
+  a.rows_out = n_pairs;
+  a.n_slabs = static_cast<int>((N + kMmaRows - 1) / kMmaRows);
+  a.n_chunks = static_cast<int>(nb / 2);
+  a.S = 1;
+  a.sq = (a.n_chunks + 1) / 2;
+  a.sr = 0;
+  a.flags = flags;
+  a.compact = compact;
+  const long long units = static_cast<long long>(m.max_tiles) * a.n_slabs;
+  if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  return launch_pdl_cluster(mma_gemv_kernel, dim3(static_cast<unsigned>(units)), kMmaThreads,
+                            mma_smem_bytes(a.g.stage_bytes), s, 1u, maps.w, maps.t, a);
+}
+
+}  // namespace
+}  // namespace stq1
+
 extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, const int32_t* topk_ids,
                                const float* topk_weights, float* y, int T, int topk, int E, int64_t N,
                                int64_t K, int flags, void* ws, size_t ws_bytes, void* stream) {
@@ -669,10 +811,16 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   const long long rowbytes = nb * kBlockBytes;
   const int n_pairs = T * topk;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  int* pairs = reinterpret_cast<int*>(wsb + m.pairs_off);
-  int* tiles = reinterpret_cast<int*>(wsb + m.tiles_off);
-  int* tiles_small = reinterpret_cast<int*>(wsb + m.small_off);
-  int* ntiles = reinterpret_cast<int*>(wsb + m.ntiles_off);
+  MoeTables tb;
+  tb.pairs = reinterpret_cast<int*>(wsb + m.pairs_off);
+  tb.tiles = reinterpret_cast<int*>(wsb + m.tiles_off);
+  tb.tiles_small = reinterpret_cast<int*>(wsb + m.small_off);
+  tb.ntiles = reinterpret_cast<int*>(wsb + m.ntiles_off);
+  MoeScratch sc;
+  sc.xperm = wsb + m.xperm_off;
+  sc.xq = wsb + m.xq_off;
+  sc.sq = reinterpret_cast<float*>(wsb + m.sq_off);
+  sc.sperm = reinterpret_cast<float*>(wsb + m.sperm_off);
 
   if (nb % 2 != 0) {
     const long long warps = static_cast<long long>(n_pairs) * N;
@@ -683,133 +831,10 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
   }
 
   rc = launch_pdl(route_kernel, 1, kRouteThreads, 3 * E * sizeof(int), s, topk_ids, n_pairs, E, m.tile_tokens,
-                  m.small_max, pairs, tiles, tiles_small, ntiles, y, static_cast<int>(N),
-                  (flags & STQ1_MOE_SKIP_FOREIGN) ? 1 : 0);
+                  m.small_max, tb.pairs, tb.tiles, tb.tiles_small, tb.ntiles, static_cast<int*>(nullptr), y,
+                  static_cast<int>(N), (flags & STQ1_MOE_SKIP_FOREIGN) ? 1 : 0);
   if (rc != STQ1_OK) return rc;
-  if (m.tiles) {
-    void* xperm = wsb + m.xperm_off;
-    float* sperm = reinterpret_cast<float*>(wsb + m.sperm_off);
-    if (m.fp8) {
-      uint8_t* xq = wsb + m.xq_off;
-      float* sq = reinterpret_cast<float*>(wsb + m.sq_off);
-      rc = launch_pdl(quant_e4m3_kernel, static_cast<unsigned>(T), kQuantThreads, 0, s, x, static_cast<int>(K), xq,
-                      sq);
-      if (rc != STQ1_OK) return rc;
-      rc = launch_pdl(gather_rows8_kernel, static_cast<unsigned>(n_pairs), 256, 0, s,
-                      static_cast<const uint8_t*>(xq), static_cast<const float*>(sq), static_cast<const int*>(pairs),
-                      static_cast<const int*>(ntiles + 1), n_pairs, topk, static_cast<int>(K),
-                      static_cast<uint8_t*>(xperm), sperm);
-    } else {
-      rc = launch_pdl(gather_rows_kernel, static_cast<unsigned>(n_pairs), 256, 0, s, x,
-                      static_cast<const int*>(pairs), static_cast<const int*>(ntiles + 1), n_pairs, topk,
-                      static_cast<int>(K), static_cast<uint16_t*>(xperm));
-    }
-    if (rc != STQ1_OK) return rc;
-    CUtensorMap map;
-    if (!make_b_map(&map, xperm, n_pairs, K, m.fp8)) return STQ1_ERR_CUDA;
-    TcArgs t{};
-    PackedMaps pm;
-    rc = packed_maps_cached(&pm, &t.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
-                          rowbytes, N % residue_period(rowbytes) != 0);
-    if (rc != STQ1_OK) return rc;
-    t.y = y;
-    t.tile_info = tiles;
-    t.n_tiles_dev = ntiles;
-    t.pairs = pairs;
-    t.route_w = topk_weights;
-    t.xscale = m.fp8 ? sperm : nullptr;
-    t.n_tiles = m.max_tiles;
-    t.N = static_cast<int>(N);
-    t.K = static_cast<int>(K);
-    t.nb = static_cast<int>(nb);
-    t.n_mtiles = static_cast<int>((N + kTcM - 1) / kTcM);
-    t.batch = 0;
-    t.flags = flags;
-    const long long items = static_cast<long long>(m.max_tiles) * t.n_mtiles;
-    const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
-    if (m.fp8) return launch_pdl(tc_gemm_kernel<true>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
-    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
-  }
-  if (m.mma) {
-    MmaArgs a{};
-    PackedMaps maps;
-    rc = packed_maps_cached(&maps, &a.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
-                            rowbytes, N % residue_period(rowbytes) != 0);
-    if (rc != STQ1_OK) return rc;
-    // experts with one or two pairs: the lookup-table kernel (small tile table)
-    {
-      LutArgs l{};
-      l.g = a.g;
-      l.x = x;
-      l.y = y;
-      l.tile_info = tiles_small;
-      l.n_tiles_dev = ntiles + 2;
-      l.pairs = pairs;
-      l.route_w = topk_weights;
-      l.N = static_cast<int>(N);
-      l.K = static_cast<int>(K);
-      l.topk = topk;
-      l.rows_out = n_pairs;
-      l.n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
-      set_split(&l, static_cast<int>(nb / kLutKC), 1);
-      l.flags = flags;
-      l.cluster = 0;
-      const long long lunits = static_cast<long long>(m.max_small) * l.n_slabs;
-      if (lunits >= (1LL << 31)) return STQ1_ERR_SHAPE;
-      rc = launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(lunits)), kLutThreads,
-                              lut_smem_bytes(kMoeTableTokens, lut_stages(l), l.g.stage_bytes, 1), s, 1u, maps.w,
-                              maps.t, l);
-      if (rc != STQ1_OK) return rc;
-    }
-    a.x = x;
-    a.y = y;
-    a.tile_info = tiles;
-    a.n_tiles_dev = ntiles;
-    a.pairs = pairs;
-    a.route_w = topk_weights;
-    a.N = static_cast<int>(N);
-    a.K = static_cast<int>(K);
-    a.topk = topk;
-    a.rows_out = n_pairs;
-    a.n_slabs = static_cast<int>((N + kMmaRows - 1) / kMmaRows);
-    a.n_chunks = static_cast<int>(nb / 2);
-    a.S = 1;
-    a.sq = (a.n_chunks + 1) / 2;
-    a.sr = 0;
-    a.flags = flags;
-    const long long units = static_cast<long long>(m.max_tiles) * a.n_slabs;
-    if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
-    return launch_pdl_cluster(mma_gemv_kernel, dim3(static_cast<unsigned>(units)), kMmaThreads,
-                              mma_smem_bytes(a.g.stage_bytes), s, 1u, maps.w, maps.t, a);
-  }
-  LutArgs a{};
-  PackedMaps maps;
-  const int P = residue_period(rowbytes);
-  rc = packed_maps_cached(&maps, &a.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
-                     rowbytes, N % P != 0);
-  if (rc != STQ1_OK) return rc;
-  a.x = x;
-  a.y = y;
-  a.partial = nullptr;
-  a.counters = nullptr;
-  a.tile_info = tiles;
-  a.n_tiles_dev = ntiles;
-  a.pairs = pairs;
-  a.route_w = topk_weights;
-  a.N = static_cast<int>(N);
-  a.K = static_cast<int>(K);
-  a.topk = topk;
-  a.batch = 0;
-  a.rows_out = n_pairs;
-  a.n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
-  set_split(&a, static_cast<int>(nb / kLutKC), 1);
-  a.flags = flags;
-  a.cluster = 0;
-  const long long units = static_cast<long long>(m.max_tiles) * a.n_slabs;
-  if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
-  return launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(units)), kLutThreads,
-                            lut_smem_bytes(kMoeTableTokens, lut_stages(a), a.g.stage_bytes, 1), s, 1u, maps.w, maps.t,
-                            a);
+  return moe_compute(m, tb, sc, expert_blocks, x, T, topk_weights, y, topk, n_pairs, E, N, K, flags, 0, s);
 }
 
 extern "C" int stq1_quantize(const float* W, const float* h, int64_t N, int64_t K, int mode, int rounds,
@@ -850,7 +875,7 @@ extern "C" int stq1_swiglu(const float* y, uint16_t* act, int64_t P, int64_t N, 
   const long long total = P * (N / 2);
   const long long grid = std::min<long long>((total + 255) / 256, 148LL * 16);
   return launch_pdl(swiglu_kernel, static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream), y, act, P,
-                    static_cast<int>(N / 2));
+                    static_cast<int>(N / 2), static_cast<const int*>(nullptr));
 }
 
 extern "C" int stq1_moe_combine(const float* y, const float* w, float* out, int64_t T, int topk, int64_t H,
@@ -923,7 +948,57 @@ extern "C" int stq1_moe_ffn(const void* gateup_blocks, const void* down_blocks, 
   return stq1_moe_combine(yd, (flags & STQ1_MOE_WEIGHT_UP) ? nullptr : topk_weights, out, T, topk, H, stream);
 }
 
+namespace stq1 {
+namespace {
+// One rank's share of an expert-parallel layer, stored compactly: only the
+// pairs routed to this rank's experts are computed and stored, in the order
+// of the grouped pair list; inv maps each (token, slot) pair to its row or -1.
+struct FfnLocalPlan {
+  MoePlan m;                       // routing and matmul plan (gate/up shape; the down shares the tables)
+  size_t ids_off, pairs_off, tiles_off, small_off, ntiles_off, inv_off;
+  size_t xperm_off, xq_off, sq_off, sperm_off;   // tile-path scratch, sized for both projections
+  size_t ygu_off, act_off, yd_off, total;
+  bool compact;                    // false: rows with an odd number of blocks (generic kernels)
+};
+FfnLocalPlan plan_ffn_local(int T, int topk, int E_local, long long N, long long H, int flags) {
+  FfnLocalPlan f{};
+  const long long P = static_cast<long long>(T) * topk;
+  f.compact = (H / kBlockWeights) % 2 == 0 && (N / 2 / kBlockWeights) % 2 == 0;
+  f.m = plan_moe(T, topk, E_local, H, flags);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off += round16(bytes); return o; };
+  f.ids_off = take(P * sizeof(int32_t));
+  f.pairs_off = take(P * sizeof(int));
+  f.tiles_off = take(static_cast<size_t>(f.m.max_tiles) * 4 * sizeof(int));
+  f.small_off = take(static_cast<size_t>(f.m.max_small) * 4 * sizeof(int));
+  f.ntiles_off = take(16);
+  f.inv_off = take(P * sizeof(int));
+  const long long kmax = std::max(H, N / 2);
+  f.xperm_off = f.xq_off = f.sq_off = f.sperm_off = off;
+  if (f.m.tiles) {
+    f.xperm_off = take(static_cast<size_t>(P) * H * (f.m.fp8 ? 1 : 2));   // gate/up gather
+    if (f.m.fp8) {
+      f.xq_off = take(static_cast<size_t>(std::max<long long>(T, P)) * kmax);
+      f.sq_off = take(static_cast<size_t>(std::max<long long>(T, P)) * sizeof(float));
+      f.sperm_off = take(static_cast<size_t>(P) * sizeof(float));
+    }
+  }
+  f.ygu_off = take(static_cast<size_t>(P) * N * sizeof(float));
+  f.act_off = take(static_cast<size_t>(P) * (N / 2) * sizeof(uint16_t));
+  f.yd_off = take(static_cast<size_t>(P) * H * sizeof(float));
+  f.total = off;
+  return f;
+}
+}  // namespace
+}  // namespace stq1
+
 extern "C" size_t stq1_moe_ffn_local_workspace(int T, int topk, int E_local, int64_t N, int64_t H, int flags) {
+  if (T <= 0 || topk <= 0 || E_local <= 0 || N <= 0 || (N & 1) || H <= 0 || H % kBlockWeights ||
+      (N / 2) % kBlockWeights)
+    return 0;
+  const FfnLocalPlan f = plan_ffn_local(T, topk, E_local, N, H, flags);
+  if (f.compact) return f.total;
+  // generic shapes: shifted ids, then the whole-layer chain with foreign pairs skipped
   const size_t w = stq1_moe_ffn_workspace(T, topk, E_local, N, H, flags);
   return w ? w + round16(static_cast<size_t>(T) * topk * sizeof(int32_t)) : 0;
 }
@@ -933,21 +1008,69 @@ extern "C" int stq1_moe_ffn_local(const void* gateup_local, const void* down_loc
                                   int E_local, int expert_begin, int64_t N, int64_t H, int flags, void* ws,
                                   size_t ws_bytes, void* stream) {
   NvtxRange nvtx_range("stq1_moe_ffn_local");
-  if (!topk_ids || !ws) return !topk_ids ? STQ1_ERR_NULL : STQ1_ERR_WORKSPACE;
-  if (T <= 0 || topk <= 0 || E_local <= 0 || expert_begin < 0) return STQ1_ERR_SHAPE;
+  if (!gateup_local || !down_local || !x || !topk_ids || !out) return STQ1_ERR_NULL;
+  if (!ws) return STQ1_ERR_WORKSPACE;
+  if (flags & ~(STQ1_MOE_WEIGHT_UP | STQ1_MOE_FP8 | STQ1_MOE_SKIP_FOREIGN)) return STQ1_ERR_ARG;
+  if (T <= 0 || topk <= 0 || E_local <= 0 || expert_begin < 0 || E_local > kMaxExperts) return STQ1_ERR_SHAPE;
   const size_t need = stq1_moe_ffn_local_workspace(T, topk, E_local, N, H, flags);
-  if (need == 0) return STQ1_ERR_SHAPE;
+  if (need == 0 || static_cast<long long>(T) * topk > (1LL << 30)) return STQ1_ERR_SHAPE;
   if (ws_bytes < need) return STQ1_ERR_WORKSPACE;
-  if (!aligned16(ws)) return STQ1_ERR_ALIGN;
-  // this rank's view of the routing: ids of its range start at 0, others fall outside [0, E_local)
-  int32_t* ids_local = static_cast<int32_t*>(ws);
-  const size_t ids_bytes = round16(static_cast<size_t>(T) * topk * sizeof(int32_t));
-  const long long n = static_cast<long long>(T) * topk;
-  int rc = launch_pdl(shift_ids_kernel, static_cast<unsigned>(std::min<long long>((n + 255) / 256, 1024)), 256, 0,
-                      static_cast<cudaStream_t>(stream), topk_ids, ids_local, n, expert_begin);
+  if (!aligned16(ws) || !aligned16(gateup_local) || !aligned16(down_local) || !aligned16(x)) return STQ1_ERR_ALIGN;
+  int rc = ensure_configured();
   if (rc != STQ1_OK) return rc;
-  return stq1_moe_ffn(gateup_local, down_local, x, ids_local, topk_weights, out, T, topk, E_local, N, H,
-                      flags | STQ1_MOE_SKIP_FOREIGN, static_cast<uint8_t*>(ws) + ids_bytes, ws_bytes - ids_bytes, stream);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long n = static_cast<long long>(T) * topk;
+  const FfnLocalPlan f = plan_ffn_local(T, topk, E_local, N, H, flags);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  // this rank's view of the routing: ids of its range start at 0, others fall outside [0, E_local)
+  int32_t* ids_local = reinterpret_cast<int32_t*>(wsb + (f.compact ? f.ids_off : 0));
+  rc = launch_pdl(shift_ids_kernel, static_cast<unsigned>(std::min<long long>((n + 255) / 256, 1024)), 256, 0, s,
+                  topk_ids, ids_local, n, expert_begin);
+  if (rc != STQ1_OK) return rc;
+  if (!f.compact) {
+    const size_t ids_bytes = round16(static_cast<size_t>(n) * sizeof(int32_t));
+    return stq1_moe_ffn(gateup_local, down_local, x, ids_local, topk_weights, out, T, topk, E_local, N, H,
+                        flags | STQ1_MOE_SKIP_FOREIGN, wsb + ids_bytes, ws_bytes - ids_bytes, stream);
+  }
+  const int P = static_cast<int>(n);
+  MoeTables tb;
+  tb.pairs = reinterpret_cast<int*>(wsb + f.pairs_off);
+  tb.tiles = reinterpret_cast<int*>(wsb + f.tiles_off);
+  tb.tiles_small = reinterpret_cast<int*>(wsb + f.small_off);
+  tb.ntiles = reinterpret_cast<int*>(wsb + f.ntiles_off);
+  int* inv = reinterpret_cast<int*>(wsb + f.inv_off);
+  MoeScratch sc;
+  sc.xperm = wsb + f.xperm_off;
+  sc.xq = wsb + f.xq_off;
+  sc.sq = reinterpret_cast<float*>(wsb + f.sq_off);
+  sc.sperm = reinterpret_cast<float*>(wsb + f.sperm_off);
+  float* ygu = reinterpret_cast<float*>(wsb + f.ygu_off);
+  uint16_t* act = reinterpret_cast<uint16_t*>(wsb + f.act_off);
+  float* yd = reinterpret_cast<float*>(wsb + f.yd_off);
+  // group the local pairs by expert; foreign pairs get no row (inv = -1) and nothing is written for them
+  rc = launch_pdl(route_kernel, 1, kRouteThreads, 3 * E_local * sizeof(int), s, static_cast<const int32_t*>(ids_local),
+                  P, E_local, f.m.tile_tokens, f.m.small_max, tb.pairs, tb.tiles, tb.tiles_small, tb.ntiles, inv,
+                  static_cast<float*>(nullptr), static_cast<int>(N), 1);
+  if (rc != STQ1_OK) return rc;
+  // gate/up of the local pairs into compact rows (routing weight on the up half with STQ1_MOE_WEIGHT_UP)
+  rc = moe_compute(f.m, tb, sc, gateup_local, x, T, topk_weights, ygu, topk, P, E_local, N, H, flags, 1, s);
+  if (rc != STQ1_OK) return rc;
+  // SwiGLU over the rows in use (their count is on the device)
+  const long long half = N / 2;
+  const long long grid = std::min<long long>((n * half + 255) / 256, 148LL * 16);
+  rc = launch_pdl(swiglu_kernel, static_cast<unsigned>(grid), 256, 0, s, static_cast<const float*>(ygu), act, n,
+                  static_cast<int>(half), static_cast<const int*>(tb.ntiles + 1));
+  if (rc != STQ1_OK) return rc;
+  // down projection on the same tables: compact rows in, compact rows out
+  rc = moe_compute(f.m, tb, sc, down_local, act, P, nullptr, yd, 1, P, E_local, H, N / 2,
+                   flags & STQ1_MOE_FP8, 3, s);
+  if (rc != STQ1_OK) return rc;
+  // combine through the pair -> row map (plain sum when the weight went on the up half)
+  const long long total = static_cast<long long>(T) * H;
+  const long long cgrid = std::min<long long>((total + 255) / 256, 148LL * 16);
+  return launch_pdl(combine_compact_kernel, static_cast<unsigned>(cgrid), 256, 0, s, static_cast<const float*>(yd),
+                    (flags & STQ1_MOE_WEIGHT_UP) ? static_cast<const float*>(nullptr) : topk_weights,
+                    static_cast<const int*>(inv), out, static_cast<long long>(T), topk, static_cast<int>(H));
 }
 
 extern "C" int stq1_set_path(int path) {

@@ -84,7 +84,8 @@ static_assert(kTcOffTable % 256 == 0, "decode tables must be 256-aligned");
 constexpr int kTcOffBar = kTcOffTable + 256;
 constexpr int kTcOffPairs = kTcOffBar + 512;                       // kTcN ints
 constexpr int kTcOffScale = kTcOffPairs + kTcN * 4;                // kTcN floats (fp8)
-constexpr int kTcOffMisc = kTcOffScale + kTcN * 4;
+constexpr int kTcOffWrow = kTcOffScale + kTcN * 4;                 // kTcN ints: routing-weight index
+constexpr int kTcOffMisc = kTcOffWrow + kTcN * 4;
 constexpr int kTcSmemBytes = 1024 + kTcOffMisc + 64;   // > 114 KB: one CTA per SM
 
 struct TcArgs {
@@ -93,6 +94,7 @@ struct TcArgs {
   const int* tile_info;      // [tiles, 4] expert, first B row, count, pad (nullptr: plain)
   const int* n_tiles_dev;    // device tile count (MoE) or nullptr
   const int* pairs;          // output row of each B row (MoE) or nullptr (identity)
+  const int* wpairs;         // routing-weight index of each B row, or nullptr (the output row)
   const float* route_w;
   const float* xscale;       // fp8: scale of each B row, nullptr otherwise
   int n_tiles;               // plain: token tiles
@@ -334,6 +336,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
   const uint32_t bar_pk_full = bar + 256, bar_pk_empty = bar + 288;
   int* s_pairs = reinterpret_cast<int*>(sgen + kTcOffPairs);
   float* s_scale = reinterpret_cast<float*>(sgen + kTcOffScale);
+  int* s_wrow = reinterpret_cast<int*>(sgen + kTcOffWrow);
   volatile int* s_misc = reinterpret_cast<volatile int*>(sgen + kTcOffMisc);   // [0] tmem base, [1] abort
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -488,6 +491,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
       named_bar(1, kTcEpilogue);                     // previous tile's stores are done
       if (et < kTcN) {
         s_pairs[et] = et < cnt ? (a.pairs ? a.pairs[b_row + et] : b_row + et) : -1;
+        s_wrow[et] = et < cnt ? (a.wpairs ? a.wpairs[b_row + et] : s_pairs[et]) : 0;
         if constexpr (FP8) s_scale[et] = et < cnt ? a.xscale[b_row + et] : 0.f;
       }
       named_bar(1, kTcEpilogue);
@@ -541,7 +545,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
           if (pair >= 0) {
             float v = acc[j];
             if constexpr (FP8) v *= s_scale[kCols * chalf + j];
-            if (up) v *= a.route_w[pair];
+            if (up) v *= a.route_w[s_wrow[kCols * chalf + j]];
             a.y[static_cast<long long>(pair) * a.N + row] = v;
           }
         }

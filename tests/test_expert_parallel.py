@@ -84,12 +84,18 @@ def test_partial_outputs_sum_to_the_whole_layer(world):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("world", [1, 4])
-def test_rank_shares_on_one_gpu_sum_to_the_oracle(world):
+@pytest.mark.parametrize("n,hidden,T,flags", [
+    (512, 512, 24, 0),      # down rows of one block (odd count): the generic whole-layer chain per rank
+    (1024, 512, 24, 0),     # compact rank rows: few pairs per expert (table and tensor-core decode kernels)
+    (1024, 512, 24, 1),     # the same with the routing weight on the up half
+    (1024, 512, 600, 0),    # compact rank rows, many pairs per expert: the tcgen05 tile kernel
+])
+def test_rank_shares_on_one_gpu_sum_to_the_oracle(world, n, hidden, T, flags):
     # The per-rank kernels of a G-way expert-parallel layer, run one after the
     # other on one GPU (no collective: the sum is taken here), against the
     # oracle's whole layer.
     import sub_bit_sparse_b200 as stq1
-    n, hidden, E, T, topk = 512, 512, 8, 24, 3
+    E, topk = 8, 3
     gu = [stq1.quantize_ref(workloads.gaussian_matrix(n, hidden, 0.05, seed=1100 + e)) for e in range(E)]
     dn = [stq1.quantize_ref(workloads.gaussian_matrix(hidden, n // 2, 0.05, seed=1200 + e)) for e in range(E)]
     x = workloads.activations_bf16(T, hidden, seed=13)
@@ -101,10 +107,10 @@ def test_rank_shares_on_one_gpu_sum_to_the_oracle(world):
     for r in range(world):
         b, c = expert_range(E, world, r)
         part = stq1.moe_ffn_local(dev(np.concatenate(gu[b:b + c])), dev(np.concatenate(dn[b:b + c])), xd,
-                                  dev(ids.astype(np.int32)), dev(wts), n, hidden, c, b)
+                                  dev(ids.astype(np.int32)), dev(wts), n, hidden, c, b, flags=flags)
         total += part
     assert stq1.status() == 0                          # foreign ids are not errors
-    ref, scale = oracle.moe_ffn(gu, dn, x, ids, wts, n, hidden, abs_sum=True)
+    ref, scale = oracle.moe_ffn(gu, dn, x, ids, wts, n, hidden, flags=flags, abs_sum=True)
     err = np.abs(total.cpu().numpy().astype(np.float64) - ref)
     # Bound for a sum of `world` partials: rank r's partial covers its own slots,
     # so it is within 1e-3 * S_r + 1e-6 of the oracle's partial (S_r = its share
