@@ -287,6 +287,49 @@ int stq1_moe_ffn_local(const void* gateup_local, const void* down_local, const u
                        size_t ws_bytes, void* stream);
 
 /*
+ * stq1_ep_dispatch / stq1_ep_combine -- the token exchange of an
+ * expert-parallel MoE layer whose tokens are spread over the ranks as well
+ * (prefill).  The pages ran the model on eight GPUs without describing the
+ * split ("Tencent's 200GB Hy4-preview ...", "The catch: not a drop-in GGUF");
+ * this is the plain expert-parallel reading: each rank sends every (token,
+ * slot) pair to the rank that holds its expert, that rank runs the pair
+ * through its experts (stq1_moe_ffn_local with the received rows as tokens,
+ * topk = 1), and the results come back to be summed per token.  The exchange
+ * itself (an all-to-all over NCCL) is the caller's.
+ * Ownership: the E experts are split into `world` contiguous ranges, the first
+ * E % world ranks holding one expert more.
+ *
+ * stq1_ep_dispatch groups this rank's pairs p = t * topk + s by owner rank:
+ *   topk_ids  device, [T, topk] int32 global expert ids.
+ *   x         device, [T, K] bf16 bits, 16-byte aligned, K % 8 == 0.
+ *   topk_weights  device, [T, topk] fp32, read only when w_send is not NULL.
+ *   order     device, [T * topk] int32: order[i] = the pair sent i-th.
+ *   inv       device, [T * topk] int32: inv[p] = i (or -1 for an id outside
+ *             [0, E), which is sent nowhere and sets STQ1_DEV_BAD_EXPERT).
+ *   counts    device, [world + 1] int32: pairs sent to each rank, in rank
+ *             order (rank r's rows are the counts[r] rows after those of
+ *             ranks < r), then the total.
+ *   local_ids device, [T * topk] int32: local_ids[i] = the expert of pair
+ *             order[i] within its owner's range.
+ *   x_send    device, [T * topk, K] bf16: x_send[i] = x[order[i] / topk]
+ *             (rows past counts[world] are left untouched), 16-byte aligned.
+ *   w_send    device, [T * topk] fp32: w_send[i] = topk_weights[order[i]], or
+ *             NULL.
+ * Rows of one rank are in no particular order (the order changes no result).
+ *
+ * stq1_ep_combine: out[t, h] = sum over slots s with inv[t * topk + s] >= 0
+ * of rows[inv[t * topk + s], h], fp32 in slot order (0 without such a slot);
+ * rows = [T * topk, H] fp32, the results returned in send order.
+ * Both are asynchronous on `stream`.
+ * Errors: STQ1_ERR_NULL, STQ1_ERR_SHAPE, STQ1_ERR_ALIGN, STQ1_ERR_CUDA.
+ */
+int stq1_ep_dispatch(const int32_t* topk_ids, const uint16_t* x, const float* topk_weights, int T, int topk, int E,
+                     int world, int64_t K, int32_t* order, int32_t* inv, int32_t* counts, int32_t* local_ids,
+                     uint16_t* x_send, float* w_send, void* stream);
+int stq1_ep_combine(const float* rows, const int32_t* inv, float* out, int64_t T, int topk, int64_t H,
+                    void* stream);
+
+/*
  * stq1_quantize_x_e4m3 -- the activation quantization of the fp8 tile variant
  * (the pages have no fp8 step; this is the library's choice).  Per row t of
  * x: amax = max |x[t, k]|, inv = 448 / amax and scales[t] = amax / 448 (IEEE

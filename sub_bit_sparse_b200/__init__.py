@@ -84,6 +84,11 @@ SIGNATURES = {
                                       _c.c_int64, _c.c_int64, _c.c_int64, _c.c_int64, _c.c_void_p,
                                       _c.c_void_p]),
     "stq1_selftest_wait": (_c.c_int, [_c.c_int, _c.c_void_p]),
+    "stq1_ep_dispatch": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int, _c.c_int, _c.c_int,
+                                    _c.c_int64, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                    _c.c_void_p, _c.c_void_p]),
+    "stq1_ep_combine": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int, _c.c_int64,
+                                   _c.c_void_p]),
     "stq1_mix_allocate": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64,
                                      _c.c_double, _c.c_void_p]),
 }
@@ -481,6 +486,48 @@ def quantize_x_e4m3(x, out=None, scales=None):
     rc = _load().stq1_quantize_x_e4m3(x.data_ptr(), t, k, out.data_ptr(), scales.data_ptr(), _stream(x))
     _check("stq1_quantize_x_e4m3", rc)
     return out, scales
+
+
+def ep_dispatch(topk_ids, x, topk_weights, n_experts: int, world: int):
+    """Groups this rank's (token, slot) pairs by the rank owning their expert
+    (stq1_ep_dispatch).  Returns (order, inv, counts [world + 1], local_ids,
+    x_send [T*topk, K], w_send or None), all CUDA tensors."""
+    torch = _torch()
+    _require(topk_ids, torch.int32, "topk_ids")
+    _require(x, torch.bfloat16, "x")
+    t, topk = topk_ids.shape
+    k = x.shape[1]
+    n = t * topk
+    dev = x.device
+    order = torch.empty(n, dtype=torch.int32, device=dev)
+    inv = torch.empty(n, dtype=torch.int32, device=dev)
+    counts = torch.empty(world + 1, dtype=torch.int32, device=dev)
+    local_ids = torch.empty(n, dtype=torch.int32, device=dev)
+    x_send = torch.empty((n, k), dtype=torch.bfloat16, device=dev)
+    w_send = None
+    if topk_weights is not None:
+        _require(topk_weights, torch.float32, "topk_weights")
+        w_send = torch.empty(n, dtype=torch.float32, device=dev)
+    rc = _load().stq1_ep_dispatch(topk_ids.data_ptr(), x.data_ptr(),
+                                  None if topk_weights is None else topk_weights.data_ptr(), t, topk, n_experts,
+                                  world, k, order.data_ptr(), inv.data_ptr(), counts.data_ptr(), local_ids.data_ptr(),
+                                  x_send.data_ptr(), None if w_send is None else w_send.data_ptr(), _stream(x))
+    _check("stq1_ep_dispatch", rc)
+    return order, inv, counts, local_ids, x_send, w_send
+
+
+def ep_combine(rows, inv, t: int, topk: int, out=None):
+    """out [t, H] = per-token sum of the returned rows through inv (stq1_ep_combine)."""
+    torch = _torch()
+    _require(rows, torch.float32, "rows")
+    _require(inv, torch.int32, "inv")
+    h = rows.shape[1]
+    if out is None:
+        out = torch.empty((t, h), dtype=torch.float32, device=rows.device)
+    _require(out, torch.float32, "out")
+    rc = _load().stq1_ep_combine(rows.data_ptr(), inv.data_ptr(), out.data_ptr(), t, topk, h, _stream(rows))
+    _check("stq1_ep_combine", rc)
+    return out
 
 
 PATH_AUTO, PATH_TABLE, PATH_TILES, PATH_MMA = 0, 1, 2, 3

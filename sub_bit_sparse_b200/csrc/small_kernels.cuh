@@ -318,6 +318,86 @@ combine_compact_kernel(const float* __restrict__ y, const float* __restrict__ w,
 }
 
 // ---------------------------------------------------------------------------
+// Expert parallelism with token dispatch.  The E experts are split into world
+// contiguous ranges, the first E % world ranks holding one more (the split of
+// sub_bit_sparse_b200.ep.expert_range).  Pairs p = t * topk + s are grouped by
+// the rank that owns expert ids[p], in rank order.  Inside a rank's segment
+// the order is that of the atomic slot counters; it changes no result, since
+// every row is computed on its own and the combine adds a token's rows in
+// slot order through inv.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int expert_owner(int e, int E, int world) {
+  const int base = E / world, extra = E % world;
+  const int split = extra * (base + 1);
+  return e < split ? e / (base + 1) : extra + (e - split) / base;
+}
+__device__ __forceinline__ int expert_begin(int r, int E, int world) {
+  const int base = E / world, extra = E % world;
+  return r * base + min(r, extra);
+}
+
+// order[i] = pair sent i-th; inv[p] = i; counts[r] = pairs sent to rank r,
+// counts[world] = all pairs sent; local[i] = the expert id of pair order[i]
+// within its owner's range.  Invalid ids (outside [0, E)) are sent nowhere
+// (inv = -1) and flagged in the device error word.
+constexpr int kDispatchThreads = 1024;
+__global__ void __launch_bounds__(kDispatchThreads)
+ep_dispatch_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int world, int* __restrict__ order,
+                   int* __restrict__ inv, int* __restrict__ counts, int32_t* __restrict__ local) {
+  extern __shared__ int sm[];
+  int* cnt = sm;                  // [world]
+  int* cur = sm + world;          // [world] next slot of each rank
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int r = threadIdx.x; r < world; r += blockDim.x) cnt[r] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
+    const int e = ids[p];
+    if (e >= 0 && e < E) atomicAdd(&cnt[expert_owner(e, E, world)], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int r = 0; r < world; ++r) {
+      cur[r] = run;
+      counts[r] = cnt[r];
+      run += cnt[r];
+    }
+    counts[world] = run;
+  }
+  __syncthreads();
+  for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
+    const int e = ids[p];
+    if (e < 0 || e >= E) {
+      inv[p] = -1;
+      flag_error(STQ1_DEV_BAD_EXPERT);
+      continue;
+    }
+    const int r = expert_owner(e, E, world);
+    const int i = atomicAdd(&cur[r], 1);
+    order[i] = p;
+    inv[p] = i;
+    local[i] = e - expert_begin(r, E, world);
+  }
+}
+
+// Rows of one dispatch: xs[i] = x[order[i] / topk] (bf16 rows of K), ws[i] =
+// w[order[i]] (w optional).  One CTA per sent pair, 16-byte copies (K % 8 == 0).
+__global__ void __launch_bounds__(256)
+ep_gather_kernel(const uint16_t* __restrict__ x, const float* __restrict__ w, const int* __restrict__ order,
+                 const int* __restrict__ n_sent, int topk, int K, uint16_t* __restrict__ xs, float* __restrict__ ws) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int i = blockIdx.x;
+  if (i >= *n_sent) return;
+  const int p = order[i];
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<long long>(p / topk) * K);
+  uint4* dst = reinterpret_cast<uint4*>(xs + static_cast<long long>(i) * K);
+  for (int c = threadIdx.x; c < K / 8; c += blockDim.x) dst[c] = src[c];
+  if (w && threadIdx.x == 0) ws[i] = w[p];
+}
+
+// ---------------------------------------------------------------------------
 // Self-test of the failure path: one thread waits, through the same bounded
 // wait every kernel uses, on an mbarrier phase that `arrive` completes or
 // (arrive = 0) nothing completes.  In the second case the wait gives up after

@@ -1073,6 +1073,40 @@ extern "C" int stq1_moe_ffn_local(const void* gateup_local, const void* down_loc
                     static_cast<const int*>(inv), out, static_cast<long long>(T), topk, static_cast<int>(H));
 }
 
+extern "C" int stq1_ep_dispatch(const int32_t* topk_ids, const uint16_t* x, const float* topk_weights, int T,
+                                int topk, int E, int world, int64_t K, int32_t* order, int32_t* inv, int32_t* counts,
+                                int32_t* local_ids, uint16_t* x_send, float* w_send, void* stream) {
+  NvtxRange nvtx_range("stq1_ep_dispatch");
+  if (!topk_ids || !x || !order || !inv || !counts || !local_ids || !x_send) return STQ1_ERR_NULL;
+  if (w_send && !topk_weights) return STQ1_ERR_NULL;
+  if (T <= 0 || topk <= 0 || E <= 0 || world <= 0 || world > E || world > 4096 || K <= 0 || K % 8 ||
+      static_cast<long long>(T) * topk > (1LL << 30) || K > (1LL << 30))
+    return STQ1_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(x_send)) return STQ1_ERR_ALIGN;
+  int rc = ensure_configured();
+  if (rc != STQ1_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = T * topk;
+  rc = launch_pdl(ep_dispatch_kernel, 1, kDispatchThreads, 2 * world * sizeof(int), s, topk_ids, n, E, world, order,
+                  inv, counts, local_ids);
+  if (rc != STQ1_OK) return rc;
+  return launch_pdl(ep_gather_kernel, static_cast<unsigned>(n), 256, 0, s, x, w_send ? topk_weights : nullptr,
+                    static_cast<const int*>(order), static_cast<const int*>(counts + world), topk,
+                    static_cast<int>(K), x_send, w_send);
+}
+
+extern "C" int stq1_ep_combine(const float* rows, const int32_t* inv, float* out, int64_t T, int topk, int64_t H,
+                               void* stream) {
+  NvtxRange nvtx_range("stq1_ep_combine");
+  if (!rows || !inv || !out) return STQ1_ERR_NULL;
+  if (T <= 0 || topk <= 0 || H <= 0 || H > (1LL << 31) - 1 || T > (1LL << 40) / (H * topk)) return STQ1_ERR_SHAPE;
+  const long long total = T * H;
+  const long long grid = std::min<long long>((total + 255) / 256, 148LL * 16);
+  return launch_pdl(combine_compact_kernel, static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream),
+                    rows, static_cast<const float*>(nullptr), static_cast<const int*>(inv), out,
+                    static_cast<long long>(T), topk, static_cast<int>(H));
+}
+
 extern "C" int stq1_set_path(int path) {
   if (path < 0 || path > 3) return STQ1_ERR_ARG;
   g_path.store(path);
