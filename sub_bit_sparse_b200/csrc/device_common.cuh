@@ -43,6 +43,20 @@ __device__ __forceinline__ void code_pattern(unsigned code, int v[4]) {
   v[lc] = (n & 1u) ? -s : s;
 }
 
+// Compile-time loop helper: f(IntC<0>{}) ... f(IntC<N-1>{}).
+template <int I>
+struct IntC {
+  static constexpr int value = I;
+};
+template <typename F, int... Is>
+__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, Is...>) {
+  (f(IntC<Is>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
 // ---- PTX wrappers ----
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

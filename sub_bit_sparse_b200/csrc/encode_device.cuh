@@ -15,8 +15,8 @@
 
 namespace stq1 {
 
-constexpr int kEncThreads = 64;                  // blocks per CTA
-constexpr int kEncPitch = kBlockWeights + 1;     // floats per staged block (odd: conflict-free reads)
+constexpr int kEncThreads = 128;                 // blocks per CTA (one thread each)
+constexpr int kEncPitch = kBlockWeights + 1;     // floats per block staged by the STQ2 encoder (odd: conflict-free)
 
 // fp64 -> IEEE binary16 bits, round to nearest even, saturating at +/-65504:
 // 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits, subnormal quantum
@@ -68,116 +68,198 @@ __device__ __forceinline__ void enc_group_lane(const float* w, int& z, uint32_t&
   }
 }
 
-// Weighted least-squares scale over the non-zero lanes, k ascending; with a zero
-// denominator the unweighted mean of |w| over the 192 non-zero lanes.
-__device__ __forceinline__ double enc_wls(const float* w, const float* h, const uint8_t* z) {
+// Per-block state in registers, processed eight groups at a time by a
+// runtime loop of eight iterations: the zero lanes (two bits per group, 128
+// bits) and the sign masks (four bits per group, 256 bits) rotate by one
+// chunk per iteration, so the chunk in use is always the low 16 bits of z[0]
+// and all of neg[0] -- no indexing with a loop variable, hence no
+// local-memory arrays.
+struct EncState {
+  uint32_t z[4];      // zero lanes: chunk c (groups 8c .. 8c+7) in bits 16 (c mod 2) of word c / 2, rotated
+  uint32_t neg[8];    // sign masks: chunk c in word c (rotated)
+  __device__ __forceinline__ void rotate(uint32_t z16) {   // z16 = the current chunk's (new) zero lanes
+    z[0] = (z[0] >> 16) | (z[1] << 16);
+    z[1] = (z[1] >> 16) | (z[2] << 16);
+    z[2] = (z[2] >> 16) | (z[3] << 16);
+    z[3] = (z[3] >> 16) | (z16 << 16);
+    const uint32_t n0 = neg[0];
+#pragma unroll
+    for (int i = 0; i < 7; ++i) neg[i] = neg[i + 1];
+    neg[7] = n0;
+  }
+};
+
+// Sums of the weighted least-squares scale over the non-zero lanes, added in
+// ascending k: num = sum h|w|, den = sum h, num1 = sum |w| (for a zero den).
+struct WlsSums {
   double num = 0.0, den = 0.0, num1 = 0.0;
-  for (int k = 0; k < kBlockWeights; ++k) {
-    if ((k & 3) == z[k >> 2]) continue;
-    const double aw = fabs(static_cast<double>(w[k]));
-    const double hk = h ? static_cast<double>(h[k]) : 1.0;
+  __device__ __forceinline__ void add(double aw, double hk) {
     num = __dadd_rn(num, __dmul_rn(hk, aw));
     den = __dadd_rn(den, hk);
     num1 = __dadd_rn(num1, aw);
   }
-  if (den == 0.0) return __ddiv_rn(num1, static_cast<double>(kBlockWeights - kGroupsPerBlock));
-  return __ddiv_rn(num, den);
-}
+  // d = num / den; with a zero denominator the mean |w| over the 192 non-zero lanes
+  __device__ __forceinline__ double scale() const {
+    if (den == 0.0) return __ddiv_rn(num1, static_cast<double>(kBlockWeights - kGroupsPerBlock));
+    return __ddiv_rn(num, den);
+  }
+};
 
-__global__ void __launch_bounds__(kEncThreads)
+// One thread encodes one block, reading it from global memory (L1/L2) once
+// per pass: no shared staging, so the number of blocks in flight per SM is set
+// by registers, which is what hides the latency of the sequential fp64 sums.
+// Passes: lanes and checks; the scale of the initial lanes; then per Sherry
+// round one pass that picks every group's zero lane with that round's d and,
+// group by group in the same ascending order, adds the group's new non-zero
+// lanes to the sums of the next d.  The additions happen in exactly the order
+// of a separate fit over k = 0..255, so the bytes do not change.
+__global__ void __launch_bounds__(kEncThreads, 4)
 encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long long n_blocks, int nb, int mode,
               int rounds, uint8_t* __restrict__ out) {
-  extern __shared__ float sw[];                   // [kEncThreads][kEncPitch]
-  const long long b0 = static_cast<long long>(blockIdx.x) * kEncThreads;
-  const int nblk = static_cast<int>(min(static_cast<long long>(kEncThreads), n_blocks - b0));
   griddep_wait();
   griddep_launch_dependents();
-  // the CTA's blocks are one contiguous span of W (row-major [N, K], blocks in storage order)
-  const float4* src = reinterpret_cast<const float4*>(W + b0 * kBlockWeights);
-  for (int f = threadIdx.x; f < nblk * (kBlockWeights / 4); f += kEncThreads) {
-    const float4 v = __ldg(src + f);
-    float* d = sw + (f >> 6) * kEncPitch + 4 * (f & 63);
-    d[0] = v.x;
-    d[1] = v.y;
-    d[2] = v.z;
-    d[3] = v.w;
-  }
-  __syncthreads();
-  if (threadIdx.x >= nblk) return;
-  const long long b = b0 + threadIdx.x;
-  const float* w = sw + threadIdx.x * kEncPitch;
-  const float* h = (mode == STQ1_ENC_SHERRY && hcol) ? hcol + (b % nb) * kBlockWeights : nullptr;
+  const long long b = static_cast<long long>(blockIdx.x) * kEncThreads + threadIdx.x;
+  if (b >= n_blocks) return;
+  const float4* w4 = reinterpret_cast<const float4*>(W + b * kBlockWeights);   // one group per float4
+  const float4* h4 = (mode == STQ1_ENC_SHERRY && hcol)
+                         ? reinterpret_cast<const float4*>(hcol + (b % nb) * kBlockWeights)
+                         : nullptr;
 
-  bool finite = true;
-  for (int k = 0; k < kBlockWeights; ++k) finite = finite && isfinite(w[k]);
-  bool hany = false;
-  if (h) {
-    for (int k = 0; k < kBlockWeights; ++k) {
-      const float hk = h[k];
-      finite = finite && isfinite(hk) && hk >= 0.f;
-      hany = hany || hk != 0.f;
-    }
-    if (!hany) h = nullptr;                      // an all-zero importance block uses h = 1
-  }
-  uint8_t* ob = out + b * kBlockBytes;
-  if (!finite) {
-    flag_error(STQ1_DEV_BAD_VALUE);
-    for (int i = 0; i < kBlockBytes; ++i) ob[i] = 0;
-    return;
-  }
-
-  uint8_t z[kGroupsPerBlock];
-  uint32_t negs[kGroupsPerBlock / 8];             // 4 bits per group
-  for (int i = 0; i < kGroupsPerBlock / 8; ++i) negs[i] = 0u;
-  for (int g = 0; g < kGroupsPerBlock; ++g) {
-    int zl;
-    uint32_t neg;
-    enc_group_lane(w + 4 * g, zl, neg);
-    z[g] = static_cast<uint8_t>(zl);
-    negs[g >> 3] |= neg << (4 * (g & 7));
-  }
-  uint16_t d_bits;
-  if (mode == STQ1_ENC_PLAIN) {
-    float amax = 0.f;
-    for (int k = 0; k < kBlockWeights; ++k) amax = fmaxf(amax, fabsf(w[k]));
-    d_bits = enc_half_bits(static_cast<double>(amax));
-  } else {
-    for (int r = 0; r < rounds; ++r) {
-      const double d = enc_wls(w, h, z);
-      for (int g = 0; g < kGroupsPerBlock; ++g) {
-        int best_l = 0;
-        double best = 0.0;
+  // pass 1: zero lanes (least |w|), sign masks, amax, checks
+  EncState st;
+  bool finite = true, hany = false;
+  float amax = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < 8; ++c) {
+    uint32_t z16 = 0u, n32 = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 v = __ldg(w4 + 8 * c + i);
+      const float wg[4] = {v.x, v.y, v.z, v.w};
+      int zl;
+      uint32_t neg;
+      enc_group_lane(wg, zl, neg);
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        finite = finite && isfinite(wg[l]);
+        amax = fmaxf(amax, fabsf(wg[l]));
+      }
+      if (h4) {
+        const float4 hv = __ldg(h4 + 8 * c + i);
+        const float hg[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
         for (int l = 0; l < 4; ++l) {
-          const int k = 4 * g + l;
-          const double aw = fabs(static_cast<double>(w[k]));
-          const double hd = __dmul_rn(h ? static_cast<double>(h[k]) : 1.0, d);
-          const double delta = __dmul_rn(hd, __dsub_rn(__dmul_rn(2.0, aw), d));
-          if (l == 0 || delta < best) {
-            best = delta;
-            best_l = l;
-          }
+          finite = finite && isfinite(hg[l]) && hg[l] >= 0.f;
+          hany = hany || hg[l] != 0.f;
         }
-        z[g] = static_cast<uint8_t>(best_l);
       }
+      z16 |= static_cast<uint32_t>(zl) << (2 * i);
+      n32 |= neg << (4 * i);
     }
-    d_bits = enc_half_bits(enc_wls(w, h, z));
+    // fill the rotating state in chunk order: after 8 iterations chunk c sits in its place
+    st.neg[0] = n32;
+    st.rotate(z16);
   }
-  // pack: d, qs (even group in the low nibble), qh (group g at bit g & 7 of byte g >> 3)
-  uint8_t blk[kBlockBytes];
-  blk[0] = static_cast<uint8_t>(d_bits & 0xFF);
-  blk[1] = static_cast<uint8_t>(d_bits >> 8);
-  for (int i = 2; i < kBlockBytes; ++i) blk[i] = 0;
-  for (int g = 0; g < kGroupsPerBlock; ++g) {
-    const uint32_t c = enc_group_code(z[g], (negs[g >> 3] >> (4 * (g & 7))) & 15u);
-    blk[kOffQs + (g >> 1)] |= static_cast<uint8_t>((c & 15u) << (4 * (g & 1)));
-    blk[kOffQh + (g >> 3)] |= static_cast<uint8_t>(((c >> 4) & 1u) << (g & 7));
+  uint16_t* o16 = reinterpret_cast<uint16_t*>(out + b * kBlockBytes);   // 2-byte aligned
+  if (!finite) {
+    flag_error(STQ1_DEV_BAD_VALUE);
+    for (int i = 0; i < kBlockBytes / 2; ++i) o16[i] = 0;
+    return;
   }
-  // the block starts on a 2-byte boundary: 21 halfword stores
-  uint16_t* o16 = reinterpret_cast<uint16_t*>(ob);
-  for (int i = 0; i < kBlockBytes / 2; ++i) o16[i] = static_cast<uint16_t>(blk[2 * i] | (blk[2 * i + 1] << 8));
+  if (!hany) h4 = nullptr;                       // an all-zero importance block uses h = 1
+
+  uint16_t d_bits;
+  if (mode == STQ1_ENC_PLAIN) {
+    d_bits = enc_half_bits(static_cast<double>(amax));
+  } else {
+    // pass 2: the scale of the initial lanes
+    WlsSums sums;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t z16 = st.z[0] & 0xFFFFu;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 v = __ldg(w4 + 8 * c + i);
+        const float wg[4] = {v.x, v.y, v.z, v.w};
+        float hg[4] = {1.f, 1.f, 1.f, 1.f};
+        if (h4) {
+          const float4 hv = __ldg(h4 + 8 * c + i);
+          hg[0] = hv.x; hg[1] = hv.y; hg[2] = hv.z; hg[3] = hv.w;
+        }
+        const int zg = static_cast<int>((z16 >> (2 * i)) & 3u);
+#pragma unroll
+        for (int l = 0; l < 4; ++l)
+          if (l != zg) sums.add(fabs(static_cast<double>(wg[l])), static_cast<double>(hg[l]));
+      }
+      st.rotate(z16);
+    }
+    double d = sums.scale();
+    // one pass per round: zero lanes at d, and the sums of the next d
+#pragma unroll 1
+    for (int r = 0; r < rounds; ++r) {
+      WlsSums next;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t z16 = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 v = __ldg(w4 + 8 * c + i);
+          const float wg[4] = {v.x, v.y, v.z, v.w};
+          float hg[4] = {1.f, 1.f, 1.f, 1.f};
+          if (h4) {
+            const float4 hv = __ldg(h4 + 8 * c + i);
+            hg[0] = hv.x; hg[1] = hv.y; hg[2] = hv.z; hg[3] = hv.w;
+          }
+          double aw[4];
+          int best_l = 0;
+          double best = 0.0;
+#pragma unroll
+          for (int l = 0; l < 4; ++l) {
+            aw[l] = fabs(static_cast<double>(wg[l]));
+            const double hd = __dmul_rn(static_cast<double>(hg[l]), d);
+            const double delta = __dmul_rn(hd, __dsub_rn(__dmul_rn(2.0, aw[l]), d));
+            if (l == 0 || delta < best) {
+              best = delta;
+              best_l = l;
+            }
+          }
+          z16 |= static_cast<uint32_t>(best_l) << (2 * i);
+#pragma unroll
+          for (int l = 0; l < 4; ++l)
+            if (l != best_l) next.add(aw[l], static_cast<double>(hg[l]));
+        }
+        st.rotate(z16);
+      }
+      d = next.scale();
+    }
+    d_bits = enc_half_bits(d);
+  }
+  // pack: d, qs (even group in the low nibble), qh (group g at bit g & 7 of byte g >> 3);
+  // chunk c gives qs bytes 4c .. 4c+3 and qh byte c (the block starts on a 2-byte boundary)
+  o16[0] = d_bits;
+  uint32_t qh2 = 0u;
+#pragma unroll 1
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t z16 = st.z[0] & 0xFFFFu;
+    const uint32_t n32 = st.neg[0];
+    uint32_t qs = 0u, qh = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t code = enc_group_code(static_cast<int>((z16 >> (2 * i)) & 3u), (n32 >> (4 * i)) & 15u);
+      qs |= (code & 15u) << (4 * i);
+      qh |= ((code >> 4) & 1u) << i;
+    }
+    o16[1 + 2 * c] = static_cast<uint16_t>(qs & 0xFFFFu);
+    o16[2 + 2 * c] = static_cast<uint16_t>(qs >> 16);
+    qh2 |= qh << (8 * (c & 1));
+    if (c & 1) {
+      o16[17 + (c >> 1)] = static_cast<uint16_t>(qh2);
+      qh2 = 0u;
+    }
+    st.rotate(z16);
+  }
 }
 
-inline size_t encode_smem_bytes() { return static_cast<size_t>(kEncThreads) * kEncPitch * sizeof(float); }
+inline size_t encode_smem_bytes() { return 0; }   // blocks are read from global memory
 
 }  // namespace stq1

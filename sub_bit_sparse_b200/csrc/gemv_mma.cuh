@@ -170,7 +170,9 @@ __device__ __forceinline__ void decode_group(uint32_t c, int m, uint32_t table, 
 // patterns for rows outside the matrix); xb = B fragments of the block.
 __device__ __forceinline__ void mma_tile_block(const QuarterCodes& cA, const QuarterCodes& cB,
                                                const uint32_t (&xb)[32], uint32_t table, float (&acc)[4]) {
-  float blk[4] = {0.f, 0.f, 0.f, 0.f};
+  // two accumulators (even and odd groups) so that consecutive MMAs do not
+  // wait on each other
+  float blk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const uint32_t QA = half ? cA.Q1 : cA.Q0, QB = half ? cB.Q1 : cB.Q0;
@@ -185,13 +187,13 @@ __device__ __forceinline__ void mma_tile_block(const QuarterCodes& cA, const Qua
       uint32_t a0, a2, a1, a3;
       decode_group((i & 1) ? oA : eA, i >> 1, table, a0, a2);
       decode_group((i & 1) ? oB : eB, i >> 1, table, a1, a3);
-      mma_bf16_16816(blk, a0, a1, a2, a3, xb[2 * m], xb[2 * m + 1]);
+      mma_bf16_16816(blk[i & 1], a0, a1, a2, a3, xb[2 * m], xb[2 * m + 1]);
     }
   }
-  acc[0] = fmaf(cA.d, blk[0], acc[0]);
-  acc[1] = fmaf(cA.d, blk[1], acc[1]);
-  acc[2] = fmaf(cB.d, blk[2], acc[2]);
-  acc[3] = fmaf(cB.d, blk[3], acc[3]);
+  acc[0] = fmaf(cA.d, blk[0][0] + blk[1][0], acc[0]);
+  acc[1] = fmaf(cA.d, blk[0][1] + blk[1][1], acc[1]);
+  acc[2] = fmaf(cB.d, blk[0][2] + blk[1][2], acc[2]);
+  acc[3] = fmaf(cB.d, blk[0][3] + blk[1][3], acc[3]);
 }
 
 // Grid: x = unit = tile * n_slabs + slab, y = K split.

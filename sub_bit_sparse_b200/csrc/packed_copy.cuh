@@ -116,20 +116,6 @@ __device__ __forceinline__ void packed_issue_chunk(const PackedGeom& g, const CU
   }
 }
 
-// Compile-time loop helper.
-template <int I>
-struct IntC {
-  static constexpr int value = I;
-};
-template <typename F, int... Is>
-__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, Is...>) {
-  (f(IntC<Is>{}), ...);
-}
-template <int N, typename F>
-__device__ __forceinline__ void static_for(F&& f) {
-  static_for_impl(f, std::make_integer_sequence<int, N>{});
-}
-
 __device__ __forceinline__ uint32_t win_word(const uint32_t* w, int p) {
   // p is a compile-time constant after unrolling
   return (p & 3) ? __funnelshift_r(w[p >> 2], w[(p >> 2) + 1], 8 * (p & 3)) : w[p >> 2];
