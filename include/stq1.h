@@ -36,6 +36,15 @@
  *     device error word, skips the bad item and finishes; stq1_status()
  *     reads and clears that word.
  *   - bf16 and fp16 values are passed as uint16_t bit patterns.
+ *   - Host threads: every call may be made from any thread.  The library's
+ *     process-wide state (per-device configuration, cached device
+ *     attributes and tensor maps, the path setting) is set up under locks or
+ *     atomics.  What a caller passes in is not: two calls that share a
+ *     workspace must not overlap.  The device error word is one per device
+ *     and process, so a stq1_status() read reports errors of every thread's
+ *     calls on that device.
+ *   - Each entry point opens an NVTX range named after it, so a profiler's
+ *     timeline shows which call enqueued which kernels.
  */
 #ifndef STQ1_H
 #define STQ1_H
