@@ -71,6 +71,7 @@ extern "C" {
 #define STQ1_DEV_BAD_EXPERT 1     /* a topk id was outside [0, E); its slot was skipped */
 #define STQ1_DEV_WAIT_LIMIT 2     /* a bounded wait inside a kernel gave up */
 #define STQ1_DEV_BAD_VALUE 4      /* (stq1_quantize) NaN/Inf weight or negative/non-finite importance */
+#define STQ1_DEV_BOUNDS 8         /* (debug build) an index failed a bounds check; its access was skipped */
 
 /* Encoder modes for stq1_quantize_ref and stq1_quantize. */
 #define STQ1_ENC_PLAIN 0          /* amax scale, smallest-|w| lane zeroed */
@@ -427,6 +428,40 @@ int stq1_set_path(int path);
  * Errors: STQ1_ERR_ARG (arrive not 0 or 1), STQ1_ERR_CUDA.
  */
 int stq1_selftest_wait(int arrive, void* stream);
+
+/*
+ * Debug build.  The library also builds as libstq1_debug.so, compiled with
+ * STQ1_DEBUG.  That build bounds-checks the indices its kernels take from
+ * device memory and from the call's geometry before using them:
+ *   - the routing tables: tile counts against the table's size; each tile's
+ *     expert, pair range and token count; each pair id and activation row;
+ *   - the shared-memory windows a row is read from;
+ *   - the shared-memory destinations of every tensor copy;
+ *   - the output and routing-weight rows of the tile kernel;
+ *   - the rows the gathers, the dispatch and the combines touch.
+ * A failed check records STQ1_DEV_BOUNDS in the device error word and skips
+ * the access (a unit leaves, a row is zeroed or not stored, a copy is not
+ * issued), so results are wrong but nothing reads or writes out of bounds.
+ * It is the stand-in for a memory checker; the release build has no checks
+ * and the same results.
+ *
+ * stq1_build_flags -- STQ1_BUILD_DEBUG if this library is the debug build,
+ * else 0.
+ */
+#define STQ1_BUILD_DEBUG 1
+int stq1_build_flags(void);
+
+/*
+ * stq1_selftest_bounds -- exercises the debug build's bounds check without an
+ * out-of-bounds access: one thread stores into a 32-entry shared array at
+ * `index` if 0 <= index < bound passes the check.  The address is masked
+ * into the array, so any arguments are safe.  In the debug build an index
+ * outside [0, bound) records STQ1_DEV_BOUNDS and skips the store; the release
+ * build does not check.  Read the outcome with stq1_status.  Asynchronous on
+ * `stream`.
+ * Errors: STQ1_ERR_CUDA.
+ */
+int stq1_selftest_bounds(int index, int bound, void* stream);
 
 /*
  * stq1_status -- synchronise `stream`, return STQ1_OK if no device error was

@@ -18,7 +18,9 @@ import threading
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libstq1.so")
+# STQ1_DEBUG=1 in the environment at import selects the bounds-checking build
+DEBUG_BUILD = os.environ.get("STQ1_DEBUG", "") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "libstq1_debug.so" if DEBUG_BUILD else "libstq1.so")
 
 OK = 0
 ERRORS = {
@@ -29,6 +31,8 @@ ERRORS = {
 DEV_BAD_EXPERT = 1
 DEV_WAIT_LIMIT = 2
 DEV_BAD_VALUE = 4
+DEV_BOUNDS = 8
+BUILD_DEBUG = 1
 ENC_PLAIN = 0
 ENC_SHERRY = 1
 MOE_WEIGHT_UP = 1
@@ -84,6 +88,8 @@ SIGNATURES = {
                                       _c.c_int64, _c.c_int64, _c.c_int64, _c.c_int64, _c.c_void_p,
                                       _c.c_void_p]),
     "stq1_selftest_wait": (_c.c_int, [_c.c_int, _c.c_void_p]),
+    "stq1_selftest_bounds": (_c.c_int, [_c.c_int, _c.c_int, _c.c_void_p]),
+    "stq1_build_flags": (_c.c_int, []),
     "stq1_ep_dispatch": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int, _c.c_int, _c.c_int, _c.c_int,
                                     _c.c_int64, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                     _c.c_void_p, _c.c_void_p]),
@@ -115,8 +121,9 @@ def _load():
         if _lib is None:
             if not os.path.exists(LIB_PATH):
                 raise ImportError(
-                    f"libstq1.so not found at {LIB_PATH}; build it with "
-                    "`python -m sub_bit_sparse_b200.build` (needs the CUDA toolkit)")
+                    f"{os.path.basename(LIB_PATH)} not found at {LIB_PATH}; build it with "
+                    "`python -m sub_bit_sparse_b200.build`" + (" --debug" if DEBUG_BUILD else "")
+                    + " (needs the CUDA toolkit)")
             lib = ctypes.CDLL(LIB_PATH)
             for name, (res, args) in SIGNATURES.items():
                 fn = getattr(lib, name)
@@ -545,6 +552,19 @@ def selftest_wait(arrive: bool, stream=None) -> int:
     s = torch.cuda.current_stream() if stream is None else stream
     _check("stq1_selftest_wait", _load().stq1_selftest_wait(1 if arrive else 0, ctypes.c_void_p(s.cuda_stream)))
     return status(s)
+
+
+def selftest_bounds(index: int, bound: int, stream=None) -> int:
+    """Runs the bounds-check self-test (see include/stq1.h) and returns the device error bits."""
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    _check("stq1_selftest_bounds", _load().stq1_selftest_bounds(int(index), int(bound), ctypes.c_void_p(s.cuda_stream)))
+    return status(s)
+
+
+def build_flags() -> int:
+    """BUILD_DEBUG if the loaded library is the bounds-checking build, else 0."""
+    return int(_load().stq1_build_flags())
 
 
 def status(stream=None) -> int:

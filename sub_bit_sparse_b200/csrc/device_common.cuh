@@ -26,6 +26,29 @@ __device__ int g_dev_err;
 
 __device__ __forceinline__ void flag_error(int bits) { atomicOr(&g_dev_err, bits); }
 
+// Bounds checks of the debug build (compiled with -DSTQ1_DEBUG): a failed
+// check records STQ1_DEV_BOUNDS in the device error word and the caller skips
+// the access it guards.  The release build compiles every check to `true`.
+#ifdef STQ1_DEBUG
+constexpr bool kDebugBuild = true;
+__device__ __forceinline__ bool dbg_check(bool ok) {
+  if (!ok) flag_error(STQ1_DEV_BOUNDS);
+  return ok;
+}
+// [addr, addr + bytes) lies inside this CTA's dynamic shared memory.
+__device__ __forceinline__ bool dbg_smem_range(uint32_t addr, uint32_t bytes) {
+  extern __shared__ __align__(16) uint8_t stq1_dyn_smem[];
+  const uint32_t lo = static_cast<uint32_t>(__cvta_generic_to_shared(stq1_dyn_smem));
+  uint32_t size;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(size));
+  return dbg_check(addr >= lo && addr + bytes <= lo + size);
+}
+#else
+constexpr bool kDebugBuild = false;
+__device__ __forceinline__ bool dbg_check(bool) { return true; }
+__device__ __forceinline__ bool dbg_smem_range(uint32_t, uint32_t) { return true; }
+#endif
+
 // Codebook: code = t << 4 | n; zero lane z = n >> 2; non-zero lanes a < b < c
 // carry +1, -(bit1 of n), -(bit0 of n); t = 1 negates them.  Returns the
 // lane values in {-1, 0, +1} (lemmy.durstig.online post 66506, "Four weights,

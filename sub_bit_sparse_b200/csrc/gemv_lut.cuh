@@ -69,6 +69,8 @@ struct LutArgs {
   int compact;               // MoE: bit 0 = output row of a pair is its position in `pairs`
                              // (else the pair id); bit 1 = its activation row is that position
                              // (else pair id / topk).  Routing weights are always by pair id.
+  int tiles_cap;             // MoE: entries the tile table holds (debug-build checks)
+  int x_rows;                // rows of x (debug-build checks)
 };
 
 // Spread bits 0, 2, 4, 6 of x to bit 6 of bytes 0..3 (other bits cleared).
@@ -174,7 +176,8 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
   const int res = pr.res;                          // residue, uniform over a warp
   const int rho = pr.rho;                          // row within the slab, 0..127
   const int row = slab * kLutRows + rho;           // output row
-  const bool row_ok = row < a.N;
+  // (debug build: the window of a row that is read lies inside the stage)
+  const bool row_ok = row < a.N && dbg_check(pr.slot + kWindowBytes <= static_cast<uint32_t>(a.g.stage_bytes));
   const uint32_t my_slot = pr.slot;
 
   const uint32_t sbase = smem_u32(smem);
@@ -359,14 +362,22 @@ lut_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
   int cnt, expert = 0;
   if (a.tile_info) {
     griddep_wait();                                  // the tile table comes from the routing kernel
-    if (tile >= *a.n_tiles_dev) return;              // whole clusters leave together (same tile)
+    const int n_tiles = *a.n_tiles_dev;
+    if (kDebugBuild && unit == 0 && split == 0 && threadIdx.x == 0) dbg_check(n_tiles <= a.tiles_cap);
+    if (tile >= n_tiles) return;                     // whole clusters leave together (same tile)
     expert = a.tile_info[4 * tile + 0];
     const int off = a.tile_info[4 * tile + 1];
     cnt = a.tile_info[4 * tile + 2];
+    // (debug build: the tile names an expert of the buffer and pairs of the list;
+    // every check depends on the tile only, so a cluster leaves whole)
+    if (!dbg_check(expert >= 0 && (expert + 1LL) * a.N <= a.g.rows_total && cnt >= 1 && cnt <= TTMAX &&
+                   off >= 0 && off + cnt <= a.rows_out))
+      return;
 #pragma unroll
     for (int t = 0; t < kLutMaxTT; ++t) {
       const int pos = off + (t < cnt ? t : 0);
       const int p = a.pairs[pos];
+      if (!dbg_check(p >= 0 && p < a.rows_out && ((a.compact & 2) ? pos : p / a.topk) < a.x_rows)) return;
       orow[t] = (a.compact & 1) ? pos : p;
       wrow[t] = p;
       xr[t] = a.x + static_cast<long long>((a.compact & 2) ? pos : p / a.topk) * a.K;

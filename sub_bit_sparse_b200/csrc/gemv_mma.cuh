@@ -76,6 +76,8 @@ struct MmaArgs {
   int compact;               // MoE: bit 0 = output row of a pair is its position in `pairs`
                              // (else the pair id); bit 1 = its activation row is that position
                              // (else pair id / topk).  Routing weights are always by pair id.
+  int tiles_cap;             // MoE: entries the tile table holds (debug-build checks)
+  int x_rows;                // rows of x (debug-build checks)
 };
 
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
@@ -219,10 +221,23 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
   int cnt, expert = 0, off = 0;
   if (a.tile_info) {
     griddep_wait();                                // the tile table comes from the routing kernel
-    if (tile >= *a.n_tiles_dev) return;
+    const int n_tiles = *a.n_tiles_dev;
+    if (kDebugBuild && unit == 0 && split == 0 && threadIdx.x == 0) dbg_check(n_tiles <= a.tiles_cap);
+    if (tile >= n_tiles) return;
     expert = a.tile_info[4 * tile + 0];
     off = a.tile_info[4 * tile + 1];
     cnt = a.tile_info[4 * tile + 2];
+    if constexpr (kDebugBuild) {
+      // the tile names an expert of the buffer and pairs of the list, and each
+      // pair's activation row exists (uniform over the CTA: it leaves whole)
+      bool ok = expert >= 0 && (expert + 1LL) * a.N <= a.g.rows_total && cnt >= 1 && cnt <= kMmaTokens &&
+                off >= 0 && off + cnt <= a.rows_out;
+      for (int t = 0; ok && t < cnt; ++t) {
+        const int p = a.pairs[off + t];
+        ok = p >= 0 && p < a.rows_out && ((a.compact & 2) ? off + t : p / a.topk) < a.x_rows;
+      }
+      if (!dbg_check(ok)) return;
+    }
   } else {
     cnt = min(kMmaTokens, a.batch - tile * kMmaTokens);
   }
@@ -277,7 +292,9 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const PackedRow pr = packed_row(a.g, R0, 64 * rh + 16 * rt + gq + 8 * u);
-      ok[2 * rt + u] = slab * kMmaRows + pr.rho < a.N;
+      // (debug build: the window of a row that is read lies inside the stage)
+      ok[2 * rt + u] = slab * kMmaRows + pr.rho < a.N &&
+                       dbg_check(pr.slot + kWindowBytes <= static_cast<uint32_t>(a.g.stage_bytes));
       // A row outside the matrix has no slot in the stage (its computed slot
       // can lie past the stage's tail slots): read slot 0 instead, whose
       // bytes are in bounds, and give the row scale 0.

@@ -263,7 +263,7 @@ __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
 template <int FMT>
 __global__ void __launch_bounds__(kHsThreads, 2)
 hess_score_kernel(const __grid_constant__ CUtensorMap xmap, const HsArgs a) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];   // realigned to 1024 below
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - sraw);

@@ -104,6 +104,19 @@ __device__ __forceinline__ void packed_issue_chunk(const PackedGeom& g, const CU
   const long long t0 = g.tail_row0 > R0 ? g.tail_row0 : R0;
   const long long t1 = g.rows_total < R0 + kSlabRows ? g.rows_total : R0 + kSlabRows;
   if (t1 > t0) ntail = static_cast<int>(t1 - t0);
+  if constexpr (kDebugBuild) {
+    // every box inside the stage's buffers, every tail row in its slot
+    const int tfirst = static_cast<int>(t0 - g.tail_row0);
+    const bool ok = (!main || dbg_smem_range(dst, static_cast<uint32_t>((P - 1) * g.buf_bytes +
+                                                                       g.box_h * kWindowBytes))) &&
+                    (ntail == 0 || (dbg_check(tfirst >= 0 && tfirst + ntail <= kTailSlots) &&
+                                    dbg_smem_range(dst + P * g.buf_bytes + tfirst * kTailSlotBytes,
+                                                   static_cast<uint32_t>(ntail * kTailSlotBytes))));
+    if (!ok) {
+      mbar_arrive(bar);                            // complete the phase without copies
+      return;
+    }
+  }
   mbar_arrive_expect_tx(bar, (main ? P * g.box_h * kWindowBytes : 0) + ntail * kWindowBytes);
   if (main)
     for (int r = 0; r < P; ++r)

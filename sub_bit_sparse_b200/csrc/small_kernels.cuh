@@ -24,13 +24,16 @@ namespace stq1 {
 // pair whose id is out of range -- the row of p in outputs that are stored
 // compactly, in pairs_out order.  y (optional): the rows of out-of-range
 // pairs are zeroed in y [n_pairs, N] (a compact caller passes nullptr).
+// tiles_cap / small_cap = entries tile_info / tile_small hold (the debug build
+// checks every write against them).
 // ---------------------------------------------------------------------------
 constexpr int kRouteThreads = 1024;
 
 __global__ void __launch_bounds__(kRouteThreads)
 route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_tokens, int small_max,
              int* __restrict__ pairs_out, int* __restrict__ tile_info, int* __restrict__ tile_small,
-             int* __restrict__ n_tiles, int* __restrict__ inv, float* __restrict__ y, int N, int skip_foreign) {
+             int* __restrict__ n_tiles, int* __restrict__ inv, float* __restrict__ y, int N, int skip_foreign,
+             int tiles_cap, int small_cap) {
   extern __shared__ int sm[];
   __shared__ int s_bad[kRouteThreads];      // out-of-range pairs to zero, this round
   __shared__ int s_nbad;
@@ -108,6 +111,7 @@ route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_token
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int c = cnt[e];
     if (small_tiles(c)) {
+      if (!dbg_check(tst[e] >= 0 && tst[e] < small_cap)) continue;
       int* ti = tile_small + 4 * tst[e];
       ti[0] = e;
       ti[1] = off[e];
@@ -117,6 +121,7 @@ route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_token
     }
     const int nt = big_tiles(c);
     for (int k = 0; k < nt; ++k) {
+      if (!dbg_check(tst[e] + k >= 0 && tst[e] + k < tiles_cap)) break;
       int* ti = tile_info + 4 * (tst[e] + k);
       ti[0] = e;
       ti[1] = off[e] + k * tile_tokens;
@@ -129,6 +134,7 @@ route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int tile_token
     const int e = ids[p];
     if (e < 0 || e >= E) continue;
     const int pos = atomicSub(&cnt[e], 1) - 1;
+    if (!dbg_check(pos >= 0 && off[e] + pos < n_pairs)) continue;
     pairs_out[off[e] + pos] = p;
     if (inv) inv[p] = off[e] + pos;
   }
@@ -299,7 +305,7 @@ combine_kernel(const float* __restrict__ y, const float* __restrict__ w, float* 
 // sum without w), fp32 in slot order; 0 where no slot is local.
 __global__ void __launch_bounds__(256)
 combine_compact_kernel(const float* __restrict__ y, const float* __restrict__ w, const int* __restrict__ inv,
-                       float* __restrict__ out, long long T, int topk, int H) {
+                       float* __restrict__ out, long long T, int topk, int H, long long y_rows) {
   griddep_wait();
   griddep_launch_dependents();
   const long long total = T * H;
@@ -309,7 +315,7 @@ combine_compact_kernel(const float* __restrict__ y, const float* __restrict__ w,
     float acc = 0.f;
     for (int s = 0; s < topk; ++s) {
       const int r = inv[t * topk + s];
-      if (r < 0) continue;
+      if (r < 0 || !dbg_check(r < y_rows)) continue;   // (debug build: y_rows = rows y holds)
       const float v = y[static_cast<long long>(r) * H + h];
       acc = w ? fmaf(w[t * topk + s], v, acc) : acc + v;
     }
@@ -375,6 +381,7 @@ ep_dispatch_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int worl
     }
     const int r = expert_owner(e, E, world);
     const int i = atomicAdd(&cur[r], 1);
+    if (!dbg_check(r >= 0 && r < world && i >= 0 && i < n_pairs)) continue;
     order[i] = p;
     inv[p] = i;
     local[i] = e - expert_begin(r, E, world);
@@ -385,12 +392,14 @@ ep_dispatch_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int worl
 // w[order[i]] (w optional).  One CTA per sent pair, 16-byte copies (K % 8 == 0).
 __global__ void __launch_bounds__(256)
 ep_gather_kernel(const uint16_t* __restrict__ x, const float* __restrict__ w, const int* __restrict__ order,
-                 const int* __restrict__ n_sent, int topk, int K, uint16_t* __restrict__ xs, float* __restrict__ ws) {
+                 const int* __restrict__ n_sent, int topk, int K, uint16_t* __restrict__ xs, float* __restrict__ ws,
+                 int n_pairs) {
   griddep_wait();
   griddep_launch_dependents();
   const int i = blockIdx.x;
   if (i >= *n_sent) return;
   const int p = order[i];
+  if (!dbg_check(p >= 0 && p < n_pairs)) return;   // (debug build: n_pairs = pairs of the dispatch)
   const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<long long>(p / topk) * K);
   uint4* dst = reinterpret_cast<uint4*>(xs + static_cast<long long>(i) * K);
   for (int c = threadIdx.x; c < K / 8; c += blockDim.x) dst[c] = src[c];
@@ -411,6 +420,19 @@ __global__ void __launch_bounds__(32) wait_selftest_kernel(int arrive) {
   fence_mbar_init();
   if (arrive) mbar_arrive(bar);
   mbar_wait_bounded(bar, 0);
+}
+
+// The bounds check of the debug build, seen from outside: thread 0 stores
+// into a 32-entry shared array at `index` only if 0 <= index < bound passes
+// the check.  The store's address is masked to the array, so no build and no
+// argument can reach past it: a debug build records STQ1_DEV_BOUNDS for an
+// index outside [0, bound) and skips the store; a release build does not
+// check.
+__global__ void __launch_bounds__(32) bounds_selftest_kernel(int index, int bound) {
+  __shared__ volatile int s_buf[32];
+  s_buf[threadIdx.x] = 0;
+  __syncwarp();
+  if (threadIdx.x == 0 && dbg_check(index >= 0 && index < bound)) s_buf[index & 31] = 1;
 }
 
 }  // namespace stq1

@@ -498,6 +498,8 @@ int gemv_impl(const void* W_packed, const uint16_t* x, float* y, int64_t N, int6
     t.n_mtiles = static_cast<int>((N + kTcM - 1) / kTcM);
     t.batch = batch;
     t.flags = 0;
+    t.b_rows = batch;
+    t.rows_out = batch;
     const long long items = static_cast<long long>(t.n_tiles) * t.n_mtiles;
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
     return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
@@ -516,6 +518,7 @@ int gemv_impl(const void* W_packed, const uint16_t* x, float* y, int64_t N, int6
     m.topk = 1;
     m.batch = batch;
     m.rows_out = batch;
+    m.x_rows = batch;
     m.n_slabs = p.n_slabs;
     m.n_chunks = p.n_chunks;
     const int steps = (p.n_chunks + 1) / 2;
@@ -548,6 +551,7 @@ int gemv_impl(const void* W_packed, const uint16_t* x, float* y, int64_t N, int6
   a.topk = 1;
   a.batch = batch;
   a.rows_out = batch;
+  a.x_rows = batch;
   a.n_slabs = p.n_slabs;
   set_split(&a, p.n_chunks, p.S);
   a.flags = 0;
@@ -722,6 +726,8 @@ int moe_compute(const MoePlan& m, const MoeTables& tb, const MoeScratch& sc, con
     t.n_mtiles = static_cast<int>((N + kTcM - 1) / kTcM);
     t.batch = 0;
     t.flags = flags;
+    t.b_rows = (compact & 2) ? x_rows : n_pairs;
+    t.rows_out = n_pairs;
     const long long items = static_cast<long long>(m.max_tiles) * t.n_mtiles;
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
     if (m.fp8) return launch_pdl(tc_gemm_kernel<true>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
@@ -751,6 +757,8 @@ int moe_compute(const MoePlan& m, const MoeTables& tb, const MoeScratch& sc, con
     l.flags = flags;
     l.cluster = 0;
     l.compact = compact;
+    l.tiles_cap = m.mma ? m.max_small : m.max_tiles;
+    l.x_rows = x_rows;
     const long long lunits = static_cast<long long>(m.mma ? m.max_small : m.max_tiles) * l.n_slabs;
     if (lunits >= (1LL << 31)) return STQ1_ERR_SHAPE;
     rc = launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(lunits)), kLutThreads,
@@ -778,6 +786,8 @@ int moe_compute(const MoePlan& m, const MoeTables& tb, const MoeScratch& sc, con
   a.sr = 0;
   a.flags = flags;
   a.compact = compact;
+  a.tiles_cap = m.max_tiles;
+  a.x_rows = x_rows;
   const long long units = static_cast<long long>(m.max_tiles) * a.n_slabs;
   if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
   return launch_pdl_cluster(mma_gemv_kernel, dim3(static_cast<unsigned>(units)), kMmaThreads,
@@ -832,7 +842,7 @@ extern "C" int stq1_moe_gateup(const void* expert_blocks, const uint16_t* x, con
 
   rc = launch_pdl(route_kernel, 1, kRouteThreads, 3 * E * sizeof(int), s, topk_ids, n_pairs, E, m.tile_tokens,
                   m.small_max, tb.pairs, tb.tiles, tb.tiles_small, tb.ntiles, static_cast<int*>(nullptr), y,
-                  static_cast<int>(N), (flags & STQ1_MOE_SKIP_FOREIGN) ? 1 : 0);
+                  static_cast<int>(N), (flags & STQ1_MOE_SKIP_FOREIGN) ? 1 : 0, m.max_tiles, m.max_small);
   if (rc != STQ1_OK) return rc;
   return moe_compute(m, tb, sc, expert_blocks, x, T, topk_weights, y, topk, n_pairs, E, N, K, flags, 0, s);
 }
@@ -1050,7 +1060,7 @@ extern "C" int stq1_moe_ffn_local(const void* gateup_local, const void* down_loc
   // group the local pairs by expert; foreign pairs get no row (inv = -1) and nothing is written for them
   rc = launch_pdl(route_kernel, 1, kRouteThreads, 3 * E_local * sizeof(int), s, static_cast<const int32_t*>(ids_local),
                   P, E_local, f.m.tile_tokens, f.m.small_max, tb.pairs, tb.tiles, tb.tiles_small, tb.ntiles, inv,
-                  static_cast<float*>(nullptr), static_cast<int>(N), 1);
+                  static_cast<float*>(nullptr), static_cast<int>(N), 1, f.m.max_tiles, f.m.max_small);
   if (rc != STQ1_OK) return rc;
   // gate/up of the local pairs into compact rows (routing weight on the up half with STQ1_MOE_WEIGHT_UP)
   rc = moe_compute(f.m, tb, sc, gateup_local, x, T, topk_weights, ygu, topk, P, E_local, N, H, flags, 1, s);
@@ -1070,7 +1080,7 @@ extern "C" int stq1_moe_ffn_local(const void* gateup_local, const void* down_loc
   const long long cgrid = std::min<long long>((total + 255) / 256, 148LL * 16);
   return launch_pdl(combine_compact_kernel, static_cast<unsigned>(cgrid), 256, 0, s, static_cast<const float*>(yd),
                     (flags & STQ1_MOE_WEIGHT_UP) ? static_cast<const float*>(nullptr) : topk_weights,
-                    static_cast<const int*>(inv), out, static_cast<long long>(T), topk, static_cast<int>(H));
+                    static_cast<const int*>(inv), out, static_cast<long long>(T), topk, static_cast<int>(H), n);
 }
 
 extern "C" int stq1_ep_dispatch(const int32_t* topk_ids, const uint16_t* x, const float* topk_weights, int T,
@@ -1092,7 +1102,7 @@ extern "C" int stq1_ep_dispatch(const int32_t* topk_ids, const uint16_t* x, cons
   if (rc != STQ1_OK) return rc;
   return launch_pdl(ep_gather_kernel, static_cast<unsigned>(n), 256, 0, s, x, w_send ? topk_weights : nullptr,
                     static_cast<const int*>(order), static_cast<const int*>(counts + world), topk,
-                    static_cast<int>(K), x_send, w_send);
+                    static_cast<int>(K), x_send, w_send, n);
 }
 
 extern "C" int stq1_ep_combine(const float* rows, const int32_t* inv, float* out, int64_t T, int topk, int64_t H,
@@ -1104,7 +1114,7 @@ extern "C" int stq1_ep_combine(const float* rows, const int32_t* inv, float* out
   const long long grid = std::min<long long>((total + 255) / 256, 148LL * 16);
   return launch_pdl(combine_compact_kernel, static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream),
                     rows, static_cast<const float*>(nullptr), static_cast<const int*>(inv), out,
-                    static_cast<long long>(T), topk, static_cast<int>(H));
+                    static_cast<long long>(T), topk, static_cast<int>(H), T * topk);
 }
 
 extern "C" int stq1_set_path(int path) {
@@ -1119,6 +1129,14 @@ extern "C" int stq1_selftest_wait(int arrive, void* stream) {
   wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(arrive);
   return launch_status();
 }
+
+extern "C" int stq1_selftest_bounds(int index, int bound, void* stream) {
+  NvtxRange nvtx_range("stq1_selftest_bounds");
+  bounds_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(index, bound);
+  return launch_status();
+}
+
+extern "C" int stq1_build_flags(void) { return kDebugBuild ? STQ1_BUILD_DEBUG : 0; }
 
 extern "C" int stq1_status(void* stream, int* device_err) {
   NvtxRange nvtx_range("stq1_status");
@@ -1225,6 +1243,7 @@ extern "C" int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float*
   a.topk = 1;
   a.batch = batch;
   a.rows_out = batch;
+  a.x_rows = batch;
   a.n_slabs = n_slabs;
   set_split(&a, n_chunks, S);
   a.flags = 0;

@@ -102,6 +102,8 @@ struct TcArgs {
   int n_mtiles;
   int batch;                 // plain: tokens
   int flags;
+  int b_rows;                // rows of B (debug-build checks)
+  int rows_out;              // rows of y (debug-build checks)
 };
 
 // ---- tcgen05 / TMA wrappers ----
@@ -320,7 +322,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
                const __grid_constant__ CUtensorMap tmap_w, const TcArgs a) {
   using G = TcGeom<FP8>;
   constexpr int KC = G::kc;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];   // realigned to 1024 below
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - sraw);
@@ -372,7 +374,22 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
   griddep_wait();                                    // inputs may come from the previous kernel
   griddep_launch_dependents();
 
-  const int n_tiles = a.n_tiles_dev ? *a.n_tiles_dev : a.n_tiles;
+  int n_tiles = a.n_tiles_dev ? *a.n_tiles_dev : a.n_tiles;
+  if constexpr (kDebugBuild) {
+    // every tile of the table names an expert of the buffer and B rows that
+    // exist; otherwise the CTA does no work
+    bool bad = a.n_tiles_dev && n_tiles > a.n_tiles;
+    if (a.tile_info && !bad)
+      for (int t = threadIdx.x; t < n_tiles; t += blockDim.x) {
+        const int e = a.tile_info[4 * t], b = a.tile_info[4 * t + 1], c = a.tile_info[4 * t + 2];
+        if (!(e >= 0 && (e + 1LL) * a.N <= a.g.rows_total && c >= 1 && c <= kTcN && b >= 0 && b + c <= a.b_rows))
+          bad = true;
+      }
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0) dbg_check(false);
+      n_tiles = 0;
+    }
+  }
   const long long n_items = static_cast<long long>(n_tiles) * a.n_mtiles;
   const int n_chunks = a.K / KC;
   const int n_slabs = a.nb;
@@ -492,6 +509,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
       if (et < kTcN) {
         s_pairs[et] = et < cnt ? (a.pairs ? a.pairs[b_row + et] : b_row + et) : -1;
         s_wrow[et] = et < cnt ? (a.wpairs ? a.wpairs[b_row + et] : s_pairs[et]) : 0;
+        // (debug build: a row whose output or routing-weight index is out of range is not stored)
+        if (et < cnt && !dbg_check(s_pairs[et] >= 0 && s_pairs[et] < a.rows_out && s_wrow[et] >= 0 &&
+                                   s_wrow[et] < a.rows_out))
+          s_pairs[et] = -1;
         if constexpr (FP8) s_scale[et] = et < cnt ? a.xscale[b_row + et] : 0.f;
       }
       named_bar(1, kTcEpilogue);
@@ -594,7 +615,8 @@ gather_rows_kernel(const uint16_t* __restrict__ x, const int* __restrict__ pairs
   if (r >= n_rows) return;
   const int nv = n_valid ? *n_valid : n_rows;
   uint4* dst = reinterpret_cast<uint4*>(out + static_cast<long long>(r) * K);
-  if (r >= nv) {
+  // (debug build: a pair id outside the list's range gives a zero row)
+  if (r >= nv || !dbg_check(pairs[r] >= 0 && pairs[r] < n_rows)) {
     for (int i = threadIdx.x; i < K / 8; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
     return;
   }
@@ -657,7 +679,7 @@ gather_rows8_kernel(const uint8_t* __restrict__ q, const float* __restrict__ s, 
   if (r >= n_rows) return;
   const int nv = n_valid ? *n_valid : n_rows;
   uint4* dst = reinterpret_cast<uint4*>(out + static_cast<long long>(r) * K);
-  if (r >= nv) {
+  if (r >= nv || !dbg_check(pairs[r] >= 0 && pairs[r] < n_rows)) {
     for (int i = threadIdx.x; i < K / 16; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) s_out[r] = 0.f;
     return;

@@ -100,3 +100,16 @@ def test_host_side_argument_checks_need_no_gpu():
     assert L.stq1_hessian_error(1, P + 1, P, P, P, 1, 4, 256, 4, P, None) == -6
     assert L.stq1_hessian_error(1, P, P, P + 8, P, 1, 4, 256, 4, P, None) == -6
     assert L.stq1_hessian_error(1, P, P, P, P, 1, 4, 256, 4, P + 4, None) == -6
+
+
+def test_debug_build_exports_the_same_symbols():
+    from sub_bit_sparse_b200 import build as b
+    path = b.build(debug=True)                         # no-op when up to date; nvcc only, no GPU
+    lib = ctypes.CDLL(path)
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    lib.stq1_build_flags.restype = ctypes.c_int
+    assert lib.stq1_build_flags() == 1
+    import sub_bit_sparse_b200 as m
+    if not m.DEBUG_BUILD:
+        assert m.LIB.stq1_build_flags() == 0
