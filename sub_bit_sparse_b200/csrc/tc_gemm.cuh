@@ -8,29 +8,34 @@
 // accumulator, and CUDA cores add d_{j,b} * slab into an fp32 register
 // accumulator (a5 of the hot path, done once per row, slab and token).
 //
-// Tile: M = 128 weight rows x N = 128 tokens, K in stages of two 128-byte
-// swizzle atoms (128 bf16 or 256 E4M3 columns), eight MMAs per stage.
-//   warp 0      TMA producer: x tiles (128-byte swizzle) into a 4-stage shared
-//               ring (two 2-D tensor copies per stage, no multicast).
-//   warp 1      TMEM allocator and the single MMA-issuing thread:
-//               tcgen05.mma.cta_group::1.kind::f16, A from TMEM, B from shared.
+// Tile: M = 128 weight rows x N = 128 tokens, K in stages of one 256-column
+// scale block (bf16: four 128-byte swizzle atoms, 16 MMAs; fp8: two atoms,
+// 8 MMAs).
+//   warp 0      TMA producer: x tiles (128-byte swizzle) into a shared ring
+//               (bf16: 3 stages of 64 KB, fp8: 4 of 32 KB), one 2-D tensor
+//               copy per atom, no multicast.
+//   warps 1, 19 the two MMA-issuing threads (warp 1 also allocates TMEM):
+//               tcgen05.mma.cta_group::1, A from TMEM, B from shared; warp 1
+//               issues the even stages, warp 19 the odd ones, so that one
+//               thread waits for its next stage's operands while the MMAs the
+//               other queued keep the tensor pipe busy.
 //   warp 18     TMA producer of the packed weights: per 128-row tile, chunks
 //               of two blocks (the super-row tensor copies of
-//               packed_copy.cuh) into a 4-stage shared ring.
+//               packed_copy.cuh) into a shared ring (bf16: 2 stages,
+//               fp8: 4).
 //   warps 2-9   decoders, two per TMEM lane quadrant: a thread owns one weight
 //               row (TMEM lane order = the ring's slot order), copies a
 //               chunk's two blocks of codes from shared memory into registers
 //               (releasing the stage), expands each group's 5-bit code to four
 //               bf16 values through a 32-entry table and stores its half of
-//               each stage's 64 columns into TMEM (tcgen05.st), the A operand.
+//               each stage's columns into TMEM (tcgen05.st), the A operand.
 //   warps 10-17 epilogue, two per quadrant (64 token columns each): per slab,
 //               tcgen05.ld of the slab accumulator, fp32 FMA with the row's d
 //               (read from the packed ring),
 //               release of the TMEM buffer; at the end of the tile, coalesced
 //               stores of y.
 // TMEM (512 columns allocated, one CTA per SM): slab accumulators 2 x 128
-// columns, A stages 4 x 64 columns.  Shared memory: 4 x-tile stages of 32 KB
-// and 4 packed-weight stages of up to 15 KB.
+// columns, A stages 256 columns (bf16: 2 x 128, fp8: 4 x 64).
 // All waits are bounded; a timeout sets the device error word and makes every
 // role stop at its next wait, so the CTA always reaches the final barrier and
 // frees its TMEM.
@@ -54,32 +59,43 @@ namespace stq1 {
 constexpr int kTcM = 128;
 constexpr int kTcN = 128;
 constexpr int kTcAtomBytes = 128;             // one 128-byte swizzle atom of x per row
-constexpr int kTcMaxStages = 4;
+constexpr int kTcMaxBStages = 4;
+constexpr int kTcMaxAStages = 4;
+constexpr int kTcMaxPkStages = 4;
 // Pipeline geometry: a stage is one 256-column scale block of K, i.e. four
-// 128-byte atoms of bf16 x (two of E4M3), so 128 KB of x tiles and 256 TMEM
-// columns of A give 2 (bf16) or 4 (fp8) stages.
+// 128-byte atoms of bf16 x (two of E4M3).  bf16: 3 x stages of 64 KB (192
+// KB), so that a stage's copy starts one stage earlier than with two (it
+// takes about as long as a stage's MMAs), and a 2-stage packed-weight ring;
+// fp8: 4 x stages of 32 KB and a 4-stage packed ring (its stages are half
+// as long, so the packed chunks need the deeper ring).  256 TMEM columns of
+// A give 2 (bf16) or 4 (fp8) A stages.
 template <bool FP8>
 struct TcGeom {
   static constexpr int atoms = FP8 ? 2 : 4;                  // swizzle atoms per stage
-  static constexpr int stages = 8 / atoms;
+  static constexpr int b_ring_bytes = (FP8 ? 8 : 12) * kTcN * kTcAtomBytes;
+  static constexpr int b_stages = b_ring_bytes / (kTcN * kTcAtomBytes * atoms);   // x-tile stages
+  static constexpr int a_stages = 8 / atoms;                 // A stages in TMEM
+  static constexpr int pk_stages = FP8 ? 4 : 2;              // packed-weight chunks in flight
   static constexpr int kc = kBlockWeights;                   // K per stage
   static constexpr int a_cols = 32 * atoms;                  // TMEM columns of A per stage
   static constexpr int b_stage_bytes = kTcN * kTcAtomBytes * atoms;
   static constexpr int mmas = 4 * atoms;                     // 32 bytes of K per MMA
 };
 
-constexpr int kTcThreads = 608;
-constexpr int kTcAStages = 4;                    // packed-weight chunks in flight
+constexpr int kTcThreads = 640;
+constexpr int kTcMmaWarp2 = 19;                  // the second MMA issuer (odd stages)
 constexpr int kTcDecoders = 256;                 // threads: 8 warps
 constexpr int kTcEpilogue = 256;                 // threads: 8 warps
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcColD = 0;               // 2 x 128
 constexpr uint32_t kTcColA = 256;             // stages x a_cols = 256
-constexpr int kTcBRingBytes = 8 * kTcN * kTcAtomBytes;   // 128 KB of x tiles
 // shared layout (offsets from a 1024-aligned base)
 constexpr int kTcOffB = 0;
-constexpr int kTcOffA = kTcBRingBytes;                             // 131072: packed-weight ring
-constexpr int kTcOffTable = kTcOffA + kTcAStages * kPackedStageMax; // 2 x 128 B decode tables
+// x ring then packed-weight ring (per geometry), then the rest at fixed offsets
+constexpr int kTcOffTable = (12 * kTcN * kTcAtomBytes + 2 * kPackedStageMax >
+                             8 * kTcN * kTcAtomBytes + 4 * kPackedStageMax)
+                                ? 12 * kTcN * kTcAtomBytes + 2 * kPackedStageMax
+                                : 8 * kTcN * kTcAtomBytes + 4 * kPackedStageMax;   // 2 x 128 B decode tables
 static_assert(kTcOffTable % 256 == 0, "decode tables must be 256-aligned");
 constexpr int kTcOffBar = kTcOffTable + 256;
 constexpr int kTcOffPairs = kTcOffBar + 512;                       // kTcN ints
@@ -87,6 +103,7 @@ constexpr int kTcOffScale = kTcOffPairs + kTcN * 4;                // kTcN float
 constexpr int kTcOffWrow = kTcOffScale + kTcN * 4;                 // kTcN ints: routing-weight index
 constexpr int kTcOffMisc = kTcOffWrow + kTcN * 4;
 constexpr int kTcSmemBytes = 1024 + kTcOffMisc + 64;   // > 114 KB: one CTA per SM
+static_assert(kTcSmemBytes <= 232448, "shared memory per CTA is at most 227 KB");
 
 struct TcArgs {
   PackedGeom g;              // tensor maps' view of the packed weights
@@ -262,10 +279,10 @@ __device__ __forceinline__ void tc_fill_tables(uint32_t* t0, uint32_t* t1) {
 template <bool FP8, int HALF>
 __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t H0, uint32_t H1,
                                                uint32_t tables, uint32_t tmem_a_lane, uint32_t bar_full_a,
-                                               uint32_t bar_empty, uint32_t& it) {
+                                               uint32_t bar_empty_a, uint32_t& it) {
   using G = TcGeom<FP8>;
-  const uint32_t s = it % G::stages;
-  const uint32_t use = it / G::stages;
+  const uint32_t s = it % G::a_stages;
+  const uint32_t use = it / G::a_stages;
   bool waited = false;
   // this half's 32 groups (qs words 4 * HALF .. 4 * HALF + 3) in pieces of 32 TMEM
   // columns: bf16 two pieces of 16 groups (2 columns each), fp8 one of 32 groups
@@ -303,7 +320,7 @@ __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t 
       }
     }
     if (!waited) {
-      if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) return false;
+      if (!mbar_wait_bounded(bar_empty_a + 8 * s, (use & 1) ^ 1)) return false;
       tc_fence_after();
       waited = true;
     }
@@ -327,14 +344,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - sraw);
   const uint32_t sB = sbase + kTcOffB;
-  const uint32_t sA = sbase + kTcOffA;
+  const uint32_t sA = sbase + G::b_ring_bytes;        // packed-weight ring
   const uint32_t sTab = sbase + kTcOffTable;
   const uint32_t bar = sbase + kTcOffBar;
   // barriers: full_b[8] @0, full_a[8] @64, empty[8] @128, d_full[2] @192, d_empty[2] @208, drain @224,
   // packed ring full[4] @256, empty[4] @288
-  const uint32_t bar_full_b = bar, bar_full_a = bar + 64, bar_empty = bar + 128;
-  const uint32_t bar_d_full = bar + 192, bar_d_empty = bar + 208;
-  const uint32_t bar_drain = bar + 224;
+  const uint32_t bar_full_b = bar, bar_empty_b = bar + 48;          // up to 6 each (4 used)
+  const uint32_t bar_full_a = bar + 96, bar_empty_a = bar + 128;     // kTcMaxAStages each
+  const uint32_t bar_d_full = bar + 160, bar_d_empty = bar + 176;
+  const uint32_t bar_drain = bar + 192, bar_drain2 = bar + 200;
   const uint32_t bar_pk_full = bar + 256, bar_pk_empty = bar + 288;
   int* s_pairs = reinterpret_cast<int*>(sgen + kTcOffPairs);
   float* s_scale = reinterpret_cast<float*>(sgen + kTcOffScale);
@@ -343,17 +361,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kTcMaxStages; ++i) {
+    for (int i = 0; i < kTcMaxBStages; ++i) {
       mbar_init(bar_full_b + 8 * i, 1);
+      mbar_init(bar_empty_b + 8 * i, 1);
+    }
+    for (int i = 0; i < kTcMaxAStages; ++i) {
       mbar_init(bar_full_a + 8 * i, kTcDecoders);
-      mbar_init(bar_empty + 8 * i, 1);
+      mbar_init(bar_empty_a + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_d_full + 8 * i, 1);
       mbar_init(bar_d_empty + 8 * i, kTcEpilogue);
     }
-    mbar_init(bar_drain, 1);                         // drain barrier (abort path)
-    for (int i = 0; i < kTcAStages; ++i) {
+    mbar_init(bar_drain, 1);                         // drain barriers (abort path), one per MMA issuer
+    mbar_init(bar_drain2, 1);
+    for (int i = 0; i < kTcMaxPkStages; ++i) {
       mbar_init(bar_pk_full + 8 * i, 1);
       mbar_init(bar_pk_empty + 8 * i, kTcDecoders + kTcEpilogue);
     }
@@ -403,8 +425,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
         const int tile = static_cast<int>(item / a.n_mtiles);
         const int b_row = a.tile_info ? a.tile_info[4 * tile + 1] : tile * kTcN;
         for (int kc = 0; kc < n_chunks; ++kc, ++it) {
-          const uint32_t s = it % G::stages, use = it / G::stages;
-          if (!mbar_wait_bounded(bar_empty + 8 * s, (use & 1) ^ 1)) { *abort = 1; break; }
+          const uint32_t s = it % G::b_stages, use = it / G::b_stages;
+          if (!mbar_wait_bounded(bar_empty_b + 8 * s, (use & 1) ^ 1)) { *abort = 1; break; }
           mbar_arrive_expect_tx(bar_full_b + 8 * s, G::b_stage_bytes);
 #pragma unroll
           for (int at = 0; at < G::atoms; ++at)
@@ -414,43 +436,51 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
       }
       if (*abort) {
         // let the last tensor copies land before the CTA can exit (bounded)
-        for (uint32_t j = it > G::stages ? it - G::stages : 0; j < it; ++j)
-          mbar_wait_bounded(bar_full_b + 8 * (j % G::stages), (j / G::stages) & 1);
+        for (uint32_t j = it > G::b_stages ? it - G::b_stages : 0; j < it; ++j)
+          mbar_wait_bounded(bar_full_b + 8 * (j % G::b_stages), (j / G::b_stages) & 1);
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == 1 || warp == kTcMmaWarp2) {
+    // ---------------- MMA issuers ----------------
+    // Two threads take alternate stages (warp 1 the even ones, the second
+    // issuer warp the odd ones): an issuing thread blocks while the tensor
+    // pipe works through the MMAs it has queued, so one issuer alone leaves
+    // the pipe idle while it waits for the next stage's operands; with two,
+    // one waits while the other's MMAs run.  Each stage has its own
+    // accumulator buffer, A and B stage, and its commits track the MMAs of
+    // the thread that issued them.
     if (lane == 0) {
-      uint32_t it = 0, sc = 0;
+      const uint32_t mine = warp == 1 ? 0u : 1u;
+      const uint32_t drain = warp == 1 ? bar_drain : bar_drain2;
+      uint32_t it = 0;
       for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
-        for (int slab = 0; slab < n_slabs && !*abort; ++slab, ++sc) {
-          const uint32_t p = sc & 1, puse = sc >> 1;
+        for (int slab = 0; slab < n_slabs && !*abort; ++slab, ++it) {
+          if ((it & 1u) != mine) continue;
+          const uint32_t p = it & 1, puse = it >> 1;
           if (!mbar_wait_bounded(bar_d_empty + 8 * p, (puse & 1) ^ 1)) { *abort = 1; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem + kTcColD + p * kTcN;
-          {
-            const uint32_t s = it % G::stages, use = it / G::stages;
-            if (!mbar_wait_bounded(bar_full_b + 8 * s, use & 1) ||
-                !mbar_wait_bounded(bar_full_a + 8 * s, use & 1)) { *abort = 1; break; }
-            tc_fence_after();
+          const uint32_t sb = it % G::b_stages, ub = it / G::b_stages;
+          const uint32_t sa = it % G::a_stages, ua = it / G::a_stages;
+          if (!mbar_wait_bounded(bar_full_b + 8 * sb, ub & 1) ||
+              !mbar_wait_bounded(bar_full_a + 8 * sa, ua & 1)) { *abort = 1; break; }
+          tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < G::mmas; ++kk) {
-              const uint64_t bdesc =
-                  smem_desc_sw128(sB + s * G::b_stage_bytes + (kk >> 2) * (kTcN * kTcAtomBytes)) + 2 * (kk & 3);
-              tc_mma_ts<FP8>(d_tmem, tmem + kTcColA + G::a_cols * s + 8 * kk, bdesc, tc_idesc<FP8>(),
-                             kk > 0 ? 1u : 0u);
-            }
-            tc_commit(bar_empty + 8 * s);
-            ++it;
+          for (int kk = 0; kk < G::mmas; ++kk) {
+            const uint64_t bdesc =
+                smem_desc_sw128(sB + sb * G::b_stage_bytes + (kk >> 2) * (kTcN * kTcAtomBytes)) + 2 * (kk & 3);
+            tc_mma_ts<FP8>(d_tmem, tmem + kTcColA + G::a_cols * sa + 8 * kk, bdesc, tc_idesc<FP8>(),
+                           kk > 0 ? 1u : 0u);
           }
-          if (*abort) break;
+          tc_commit(bar_empty_b + 8 * sb);
+          tc_commit(bar_empty_a + 8 * sa);
           tc_commit(bar_d_full + 8 * p);
         }
       }
       if (*abort) {
         // all MMAs this thread issued must finish before TMEM is freed (bounded)
-        tc_commit(bar_drain);
-        mbar_wait_bounded(bar_drain, 0);
+        tc_commit(drain);
+        mbar_wait_bounded(drain, 0);
       }
     }
   } else if (warp < 10) {
@@ -469,7 +499,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
       const PackedRow pr = packed_row(a.g, R0, 32 * quad + lane);
       const bool row_ok = mt * kTcM + pr.rho < a.N;   // rows past N decode zeros: computed, never stored
       for (int c = 0; c < n_pk; ++c, ++ca) {
-        const uint32_t sa = ca % kTcAStages, ause = ca / kTcAStages;
+        const uint32_t sa = ca % G::pk_stages, ause = ca / G::pk_stages;
         if (!mbar_wait_bounded(bar_pk_full + 8 * sa, ause & 1)) { *abort = 1; ok = false; break; }
         BlockCodes b0 = {}, b1 = {};
         if (row_ok) {
@@ -480,10 +510,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
         }
         mbar_arrive(bar_pk_empty + 8 * sa);          // the codes are in registers now
         const bool okd =
-            (half == 0 ? tc_decode_slab<FP8, 0>(b0.Q, b0.H0, b0.H1, sTab, tmem_lane, bar_full_a, bar_empty, it)
-                       : tc_decode_slab<FP8, 1>(b0.Q, b0.H0, b0.H1, sTab, tmem_lane, bar_full_a, bar_empty, it)) &&
-            (half == 0 ? tc_decode_slab<FP8, 0>(b1.Q, b1.H0, b1.H1, sTab, tmem_lane, bar_full_a, bar_empty, it)
-                       : tc_decode_slab<FP8, 1>(b1.Q, b1.H0, b1.H1, sTab, tmem_lane, bar_full_a, bar_empty, it));
+            (half == 0 ? tc_decode_slab<FP8, 0>(b0.Q, b0.H0, b0.H1, sTab, tmem_lane, bar_full_a, bar_empty_a, it)
+                       : tc_decode_slab<FP8, 1>(b0.Q, b0.H0, b0.H1, sTab, tmem_lane, bar_full_a, bar_empty_a, it)) &&
+            (half == 0 ? tc_decode_slab<FP8, 0>(b1.Q, b1.H0, b1.H1, sTab, tmem_lane, bar_full_a, bar_empty_a, it)
+                       : tc_decode_slab<FP8, 1>(b1.Q, b1.H0, b1.H1, sTab, tmem_lane, bar_full_a, bar_empty_a, it));
         if (!okd) {
           *abort = 1;
           ok = false;
@@ -528,7 +558,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
       for (int slab = 0; slab < n_slabs; ++slab, ++sc) {
         if ((slab & 1) == 0) {
           // the scales of this chunk's two blocks, then release the ring stage
-          const uint32_t sa = ca % kTcAStages, ause = ca / kTcAStages;
+          const uint32_t sa = ca % G::pk_stages, ause = ca / G::pk_stages;
           if (!mbar_wait_bounded(bar_pk_full + 8 * sa, ause & 1)) { *abort = 1; ok = false; break; }
           if (row_ok) {
             const uint32_t w0 = sA + sa * kPackedStageMax + pr.slot +
@@ -582,15 +612,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
         const int e = a.tile_info ? a.tile_info[4 * tile + 0] : 0;
         const long long R0 = static_cast<long long>(e) * a.N + static_cast<long long>(mt) * kTcM;
         for (int c = 0; c < n_pk; ++c, ++ca) {
-          const uint32_t sa = ca % kTcAStages, ause = ca / kTcAStages;
+          const uint32_t sa = ca % G::pk_stages, ause = ca / G::pk_stages;
           if (!mbar_wait_bounded(bar_pk_empty + 8 * sa, (ause & 1) ^ 1)) { *abort = 1; break; }
           packed_issue_chunk(a.g, &wmap, &tmap_w, R0, c, sA + sa * kPackedStageMax, bar_pk_full + 8 * sa);
         }
       }
       if (*abort) {
         // let the last chunk copies land before the CTA can exit (bounded)
-        for (uint32_t j = ca > kTcAStages ? ca - kTcAStages : 0; j < ca; ++j)
-          mbar_wait_bounded(bar_pk_full + 8 * (j % kTcAStages), (j / kTcAStages) & 1);
+        for (uint32_t j = ca > G::pk_stages ? ca - G::pk_stages : 0; j < ca; ++j)
+          mbar_wait_bounded(bar_pk_full + 8 * (j % G::pk_stages), (j / G::pk_stages) & 1);
       }
     }
   }
