@@ -189,14 +189,6 @@ struct HsArgs {
   uint32_t idesc;
 };
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
 
 // D[tmem] (+)= A[smem desc] * B[smem desc], bf16 x bf16 -> fp32
 __device__ __forceinline__ void tc_mma_ss_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,

@@ -88,15 +88,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2-D map over a row-major activation matrix [rows, K] of bf16 (or, fp8, of
 // E4M3 bytes); box = 128 bytes of columns x kTcN rows, 128-byte swizzle,
 // out-of-range rows read as zero.
+// x tiles of the tile kernel as one 3-D copy per stage: dimension 0 = the
+// 128 bytes of one swizzle atom, 1 = rows (row stride K elements), 2 = atoms
+// along K (stride 128 bytes); a box is 128 rows x the stage's atoms, which
+// land atom after atom, 16 KB apart, as the MMA descriptors expect.
 bool make_b_map(CUtensorMap* map, const void* base, long long rows, long long K, bool fp8) {
   auto fn = encode_fn();
   if (!fn) return false;
   const int esize = fp8 ? 1 : 2;
-  cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * esize};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcAtomBytes / esize), static_cast<cuuint32_t>(kTcN)};
-  cuuint32_t estride[2] = {1, 1};
-  return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  const long long atom = kTcAtomBytes / esize;
+  cuuint64_t gdim[3] = {static_cast<cuuint64_t>(atom), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(K / atom)};
+  cuuint64_t gstride[2] = {static_cast<cuuint64_t>(K) * esize, static_cast<cuuint64_t>(kTcAtomBytes)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(atom), static_cast<cuuint32_t>(kTcN),
+                       static_cast<cuuint32_t>(fp8 ? TcGeom<true>::atoms : TcGeom<false>::atoms)};
+  cuuint32_t estride[3] = {1, 1, 1};
+  return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
             const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;

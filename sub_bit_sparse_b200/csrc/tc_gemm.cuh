@@ -176,6 +176,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
 #define STQ1_TMEM_ST32(taddr, v)                                                                  \
   asm volatile(                                                                                   \
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
@@ -428,10 +437,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
           const uint32_t s = it % G::b_stages, use = it / G::b_stages;
           if (!mbar_wait_bounded(bar_empty_b + 8 * s, (use & 1) ^ 1)) { *abort = 1; break; }
           mbar_arrive_expect_tx(bar_full_b + 8 * s, G::b_stage_bytes);
-#pragma unroll
-          for (int at = 0; at < G::atoms; ++at)
-            tma_load_2d(sB + s * G::b_stage_bytes + at * (kTcN * kTcAtomBytes), &tmap_b, kc * KC + at * (KC / G::atoms),
-                        b_row, bar_full_b + 8 * s);
+          // one 3-D copy per stage: (column in atom, row, atom), atoms land 16 KB apart
+          tma_load_3d(sB + s * G::b_stage_bytes, &tmap_b, 0, b_row, kc * G::atoms, bar_full_b + 8 * s);
         }
       }
       if (*abort) {
