@@ -92,7 +92,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 128 bytes of one swizzle atom, 1 = rows (row stride K elements), 2 = atoms
 // along K (stride 128 bytes); a box is 128 rows x the stage's atoms, which
 // land atom after atom, 16 KB apart, as the MMA descriptors expect.
-bool make_b_map(CUtensorMap* map, const void* base, long long rows, long long K, bool fp8) {
+bool make_b_map(CUtensorMap* map, const void* base, long long rows, long long K, bool fp8, int box_rows = kTcN) {
   auto fn = encode_fn();
   if (!fn) return false;
   const int esize = fp8 ? 1 : 2;
@@ -100,7 +100,7 @@ bool make_b_map(CUtensorMap* map, const void* base, long long rows, long long K,
   cuuint64_t gdim[3] = {static_cast<cuuint64_t>(atom), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(K / atom)};
   cuuint64_t gstride[2] = {static_cast<cuuint64_t>(K) * esize, static_cast<cuuint64_t>(kTcAtomBytes)};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(atom), static_cast<cuuint32_t>(kTcN),
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(atom), static_cast<cuuint32_t>(box_rows),
                        static_cast<cuuint32_t>(fp8 ? TcGeom<true>::atoms : TcGeom<false>::atoms)};
   cuuint32_t estride[3] = {1, 1, 1};
   return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
@@ -487,7 +487,9 @@ int gemv_impl(const void* W_packed, const uint16_t* x, float* y, int64_t N, int6
   const long long rowbytes = nb * kBlockBytes;
   if (p.tile_path) {
     CUtensorMap map;
-    if (!make_b_map(&map, x, batch, K, false)) return STQ1_ERR_CUDA;
+    CUtensorMap map_h;                               // half-height boxes for tiles of <= 64 tokens
+    if (!make_b_map(&map, x, batch, K, false) || !make_b_map(&map_h, x, batch, K, false, kTcHalfN))
+      return STQ1_ERR_CUDA;
     TcArgs t{};
     PackedMaps pm;
     rc = packed_maps_cached(&pm, &t.g, static_cast<const uint8_t*>(W_packed), N, rowbytes, false);
@@ -509,7 +511,7 @@ int gemv_impl(const void* W_packed, const uint16_t* x, float* y, int64_t N, int6
     t.rows_out = batch;
     const long long items = static_cast<long long>(t.n_tiles) * t.n_mtiles;
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
-    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
+    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, map_h, pm.w, pm.t, t);
   }
   if (p.mma_path) {
     MmaArgs m{};
@@ -713,7 +715,9 @@ int moe_compute(const MoePlan& m, const MoeTables& tb, const MoeScratch& sc, con
       B = sc.xperm;
     }
     CUtensorMap map;
-    if (!make_b_map(&map, B, n_pairs, K, m.fp8)) return STQ1_ERR_CUDA;
+    CUtensorMap map_h;                               // half-height boxes for tiles of <= 64 pairs
+    if (!make_b_map(&map, B, n_pairs, K, m.fp8) || !make_b_map(&map_h, B, n_pairs, K, m.fp8, kTcHalfN))
+      return STQ1_ERR_CUDA;
     TcArgs t{};
     PackedMaps pm;
     rc = packed_maps_cached(&pm, &t.g, static_cast<const uint8_t*>(expert_blocks), static_cast<long long>(E) * N,
@@ -737,8 +741,9 @@ int moe_compute(const MoePlan& m, const MoeTables& tb, const MoeScratch& sc, con
     t.rows_out = n_pairs;
     const long long items = static_cast<long long>(m.max_tiles) * t.n_mtiles;
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
-    if (m.fp8) return launch_pdl(tc_gemm_kernel<true>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
-    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, pm.w, pm.t, t);
+    if (m.fp8)
+      return launch_pdl(tc_gemm_kernel<true>, grid, kTcThreads, kTcSmemBytes, s, map, map_h, pm.w, pm.t, t);
+    return launch_pdl(tc_gemm_kernel<false>, grid, kTcThreads, kTcSmemBytes, s, map, map_h, pm.w, pm.t, t);
   }
   PackedMaps maps;
   PackedGeom geom;

@@ -252,10 +252,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 // 10-12: bf16 = 1 for kind::f16, E4M3 = 0 for kind::f8f6f4), both K-major,
 // N >> 3 at bit 17, M >> 4 at bit 24.
 template <bool FP8>
-constexpr uint32_t tc_idesc() {
-  return (1u << 4) | (FP8 ? 0u : ((1u << 7) | (1u << 10))) | (static_cast<uint32_t>(kTcN >> 3) << 17) |
+constexpr uint32_t tc_idesc(int n = kTcN) {
+  return (1u << 4) | (FP8 ? 0u : ((1u << 7) | (1u << 10))) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(kTcM >> 4) << 24);
 }
+// Tiles with at most this many pairs (tokens) run half-width: N = 64 MMAs and
+// 64-row x boxes.  Accumulator columns 64..127 then keep stale values, which
+// belong to no pair and are never stored.
+constexpr int kTcHalfN = kTcN / 2;
 
 // bf16 bit patterns of the 32 codes: lanes 0,1 (word 0) and lanes 2,3 (word 1);
 // for fp8 one word per code, lane l in byte l (E4M3 +1 = 0x38, -1 = 0xB8).
@@ -344,7 +348,8 @@ __device__ __forceinline__ bool tc_decode_slab(const uint32_t (&Q)[8], uint32_t 
 
 template <bool FP8>
 __global__ void __launch_bounds__(kTcThreads, 1)
-tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap wmap,
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_bh,
+               const __grid_constant__ CUtensorMap wmap,
                const __grid_constant__ CUtensorMap tmap_w, const TcArgs a) {
   using G = TcGeom<FP8>;
   constexpr int KC = G::kc;
@@ -433,12 +438,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
       for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
         const int tile = static_cast<int>(item / a.n_mtiles);
         const int b_row = a.tile_info ? a.tile_info[4 * tile + 1] : tile * kTcN;
+        const int cnt = a.tile_info ? a.tile_info[4 * tile + 2] : min(kTcN, a.batch - tile * kTcN);
+        const bool half_n = cnt <= kTcHalfN;
         for (int kc = 0; kc < n_chunks; ++kc, ++it) {
           const uint32_t s = it % G::b_stages, use = it / G::b_stages;
           if (!mbar_wait_bounded(bar_empty_b + 8 * s, (use & 1) ^ 1)) { *abort = 1; break; }
-          mbar_arrive_expect_tx(bar_full_b + 8 * s, G::b_stage_bytes);
-          // one 3-D copy per stage: (column in atom, row, atom), atoms land 16 KB apart
-          tma_load_3d(sB + s * G::b_stage_bytes, &tmap_b, 0, b_row, kc * G::atoms, bar_full_b + 8 * s);
+          mbar_arrive_expect_tx(bar_full_b + 8 * s, half_n ? G::b_stage_bytes / 2 : G::b_stage_bytes);
+          // one 3-D copy per stage: (column in atom, row, atom); the atoms land
+          // one after another, 16 KB apart (8 KB for a half-height box)
+          tma_load_3d(sB + s * G::b_stage_bytes, half_n ? &tmap_bh : &tmap_b, 0, b_row, kc * G::atoms,
+                      bar_full_b + 8 * s);
         }
       }
       if (*abort) {
@@ -461,6 +470,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
       const uint32_t drain = warp == 1 ? bar_drain : bar_drain2;
       uint32_t it = 0;
       for (long long item = blockIdx.x; item < n_items && !*abort; item += gridDim.x) {
+        const int tile = static_cast<int>(item / a.n_mtiles);
+        const int cnt = a.tile_info ? a.tile_info[4 * tile + 2] : min(kTcN, a.batch - tile * kTcN);
+        const bool half_n = cnt <= kTcHalfN;
+        const uint32_t idesc = half_n ? tc_idesc<FP8>(kTcHalfN) : tc_idesc<FP8>();
+        // a half-height 3-D copy lands its atoms 8 KB apart instead of 16 KB
+        const uint32_t atom_bytes = (half_n ? kTcHalfN : kTcN) * kTcAtomBytes;
         for (int slab = 0; slab < n_slabs && !*abort; ++slab, ++it) {
           if ((it & 1u) != mine) continue;
           const uint32_t p = it & 1, puse = it >> 1;
@@ -474,10 +489,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < G::mmas; ++kk) {
-            const uint64_t bdesc =
-                smem_desc_sw128(sB + sb * G::b_stage_bytes + (kk >> 2) * (kTcN * kTcAtomBytes)) + 2 * (kk & 3);
-            tc_mma_ts<FP8>(d_tmem, tmem + kTcColA + G::a_cols * sa + 8 * kk, bdesc, tc_idesc<FP8>(),
-                           kk > 0 ? 1u : 0u);
+            const uint64_t bdesc = smem_desc_sw128(sB + sb * G::b_stage_bytes + (kk >> 2) * atom_bytes) + 2 * (kk & 3);
+            tc_mma_ts<FP8>(d_tmem, tmem + kTcColA + G::a_cols * sa + 8 * kk, bdesc, idesc, kk > 0 ? 1u : 0u);
           }
           tc_commit(bar_empty_b + 8 * sb);
           tc_commit(bar_empty_a + 8 * sa);
@@ -583,13 +596,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
         const uint32_t p = sc & 1, puse = sc >> 1;
         if (!mbar_wait_bounded(bar_d_full + 8 * p, puse & 1)) { *abort = 1; ok = false; break; }
         tc_fence_after();
+        if (chalf == 0 || cnt > kTcHalfN) {           // warp-uniform: a half-width tile has no upper columns
 #pragma unroll
-        for (int c = 0; c < kCols / 16; ++c) {
-          uint32_t v[16];
-          STQ1_TMEM_LD16(tmem_lane + kTcColD + p * kTcN + kCols * chalf + 16 * c, v);
-          tmem_wait_ld();
+          for (int c = 0; c < kCols / 16; ++c) {
+            uint32_t v[16];
+            STQ1_TMEM_LD16(tmem_lane + kTcColD + p * kTcN + kCols * chalf + 16 * c, v);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(d, __uint_as_float(v[i]), acc[16 * c + i]);
+            for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(d, __uint_as_float(v[i]), acc[16 * c + i]);
+          }
         }
         tc_fence_before();
         mbar_arrive(bar_d_empty + 8 * p);
