@@ -205,9 +205,18 @@ size_t stq1_moe_workspace(int T, int topk, int E, int64_t N, int64_t K, int flag
  *   ws, ws_bytes   device workspace, at least stq1_moe_workspace(...) bytes
  *                  (computed with the same flags).
  * Requires N even, K % 256 == 0, 1 <= topk <= E (any topk with STQ1_MOE_SKIP_FOREIGN).
- * Paths: with few token-slot pairs per routed expert (decode) the tensor-core
- * decode kernel runs (units of up to 8 pairs of one expert); with many
+ * Paths: with few token-slot pairs per routed expert (decode), experts with
+ * one or two pairs run on the lookup-table kernel and the others on the
+ * tensor-core decode kernel (units of up to 8 pairs of one expert); with many
  * (prefill) the tensor-core tile kernel.
+ * Streams: when a decode call splits its experts this way, the tensor-core
+ * part runs on a second stream that the library keeps per device and host
+ * thread.  It forks from `stream` with an event after the routing kernel and
+ * joins back before the call returns, so work enqueued on `stream` later
+ * waits for both parts.  Under stream capture the fork and the join become
+ * graph edges; the first such call of a thread creates the stream and its two
+ * events, so make it before capturing.  If they cannot be created, both parts
+ * run on `stream`.
  * STQ1_MOE_FP8 applies to the tile kernel only: each token row of x is
  * quantized to E4M3 as by stq1_quantize_x_e4m3, the +/-1 weight patterns are
  * E4M3 too, the MMAs run in fp8 with fp32 accumulation and y is multiplied by

@@ -677,6 +677,34 @@ struct MoeScratch {
   float* sperm;       // scales in pair order (fp8)
 };
 
+// A second stream per device and host thread, with a fork and a join event,
+// for MoE decode calls that split experts between the table and tensor-core
+// kernels: the two launches are independent (disjoint output rows, both read
+// only the routing tables and x), so they run side by side and fill each
+// other's idle issue slots and wave tails.  Created on first use, kept for
+// the thread's lifetime.  Under stream capture the fork and join become graph
+// edges.  If they cannot be created the two kernels run one after the other.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool failed = false;
+};
+SideStream* side_stream() {
+  thread_local SideStream side[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
+  SideStream& ss = side[dev];
+  if (ss.stream == nullptr && !ss.failed) {
+    if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      ss.failed = true;
+    }
+  }
+  return ss.failed ? nullptr : &ss;
+}
+
 // The matmul over routed pairs, on tables the route kernel already fills.
 // `compact` bit 0: pair i of the grouped list writes output row i (else row
 // pairs[i]); bit 1: its activation row is row i of x (else pairs[i] / topk).
@@ -751,33 +779,33 @@ int moe_compute(const MoePlan& m, const MoeTables& tb, const MoeScratch& sc, con
                           rowbytes, N % residue_period(rowbytes) != 0);
   if (rc != STQ1_OK) return rc;
   // lookup-table kernel: every tile (table path) or the experts with few pairs
-  if (!m.mma || m.max_small > 0) {
-    LutArgs l{};
-    l.g = geom;
-    l.x = x;
-    l.y = y;
-    l.tile_info = m.mma ? tb.tiles_small : tb.tiles;
-    l.n_tiles_dev = m.mma ? tb.ntiles + 2 : tb.ntiles;
-    l.pairs = tb.pairs;
-    l.route_w = topk_weights;
-    l.N = static_cast<int>(N);
-    l.K = static_cast<int>(K);
-    l.topk = topk;
-    l.rows_out = n_pairs;
-    l.n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
-    set_split(&l, static_cast<int>(nb / kLutKC), 1);
-    l.flags = flags;
-    l.cluster = 0;
-    l.compact = compact;
-    l.tiles_cap = m.mma ? m.max_small : m.max_tiles;
-    l.x_rows = x_rows;
-    const long long lunits = static_cast<long long>(m.mma ? m.max_small : m.max_tiles) * l.n_slabs;
-    if (lunits >= (1LL << 31)) return STQ1_ERR_SHAPE;
-    rc = launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(lunits)), kLutThreads,
-                            lut_smem_bytes(kMoeTableTokens, lut_stages(l), l.g.stage_bytes, 1), s, 1u, maps.w, maps.t,
-                            l);
-    if (rc != STQ1_OK || !m.mma) return rc;
-  }
+  LutArgs l{};
+  l.g = geom;
+  l.x = x;
+  l.y = y;
+  l.tile_info = m.mma ? tb.tiles_small : tb.tiles;
+  l.n_tiles_dev = m.mma ? tb.ntiles + 2 : tb.ntiles;
+  l.pairs = tb.pairs;
+  l.route_w = topk_weights;
+  l.N = static_cast<int>(N);
+  l.K = static_cast<int>(K);
+  l.topk = topk;
+  l.rows_out = n_pairs;
+  l.n_slabs = static_cast<int>((N + kLutRows - 1) / kLutRows);
+  set_split(&l, static_cast<int>(nb / kLutKC), 1);
+  l.flags = flags;
+  l.cluster = 0;
+  l.compact = compact;
+  l.tiles_cap = m.mma ? m.max_small : m.max_tiles;
+  l.x_rows = x_rows;
+  const long long lunits = static_cast<long long>(m.mma ? m.max_small : m.max_tiles) * l.n_slabs;
+  if (lunits >= (1LL << 31)) return STQ1_ERR_SHAPE;
+  auto launch_lut = [&](cudaStream_t st) {
+    return launch_pdl_cluster(lut_gemv_kernel<kMoeTableTokens>, dim3(static_cast<unsigned>(lunits)), kLutThreads,
+                              lut_smem_bytes(kMoeTableTokens, lut_stages(l), l.g.stage_bytes, 1), st, 1u, maps.w,
+                              maps.t, l);
+  };
+  if (!m.mma) return launch_lut(s);
   // tensor-core decode kernel: the other experts, in tiles of up to 8 pairs
   MmaArgs a{};
   a.g = geom;
@@ -802,8 +830,25 @@ int moe_compute(const MoePlan& m, const MoeTables& tb, const MoeScratch& sc, con
   a.x_rows = x_rows;
   const long long units = static_cast<long long>(m.max_tiles) * a.n_slabs;
   if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
-  return launch_pdl_cluster(mma_gemv_kernel, dim3(static_cast<unsigned>(units)), kMmaThreads,
-                            mma_smem_bytes(a.g.stage_bytes), s, 1u, maps.w, maps.t, a);
+  auto launch_mma = [&](cudaStream_t st) {
+    return launch_pdl_cluster(mma_gemv_kernel, dim3(static_cast<unsigned>(units)), kMmaThreads,
+                              mma_smem_bytes(a.g.stage_bytes), st, 1u, maps.w, maps.t, a);
+  };
+  if (m.max_small == 0) return launch_mma(s);
+  // both kernels: fork the tensor-core part onto the side stream, join after
+  SideStream* side = side_stream();
+  if (side == nullptr) {
+    rc = launch_lut(s);
+    return rc != STQ1_OK ? rc : launch_mma(s);
+  }
+  if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
+    return STQ1_ERR_CUDA;
+  rc = launch_mma(side->stream);
+  if (rc != STQ1_OK) return rc;
+  if (cudaEventRecord(side->join, side->stream) != cudaSuccess) return STQ1_ERR_CUDA;
+  rc = launch_lut(s);
+  if (rc != STQ1_OK) return rc;
+  return cudaStreamWaitEvent(s, side->join, 0) == cudaSuccess ? STQ1_OK : STQ1_ERR_CUDA;
 }
 
 }  // namespace
