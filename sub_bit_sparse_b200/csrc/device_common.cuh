@@ -186,6 +186,20 @@ __device__ __forceinline__ void st_peer_f32(uint32_t local_addr, uint32_t rank, 
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
 
+// Two fp32 additions in one instruction (the packed f32x2 add of sm_100),
+// each lane rounded to nearest as a scalar add: {a.x + b.x, a.y + b.y}.
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 template <int OFF>
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
   float v;

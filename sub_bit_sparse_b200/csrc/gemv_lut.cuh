@@ -90,9 +90,11 @@ __device__ __forceinline__ float lds_f32_addr(uint32_t addr) {
 // byte permute.
 template <int TT>
 __device__ __forceinline__ void lut_block_body(const BlockCodes& bc, uint32_t lut, float (&acc)[kLutMaxTT]) {
-  float s[TT][4];
+  // partial sums of the byte positions m = 0, 1 and m = 2, 3 of each code
+  // word, two per packed register: every update adds two lanes at once
+  float2 s[TT][2];
 #pragma unroll
-  for (int t = 0; t < TT; ++t) s[t][0] = s[t][1] = s[t][2] = s[t][3] = 0.f;
+  for (int t = 0; t < TT; ++t) s[t][0] = s[t][1] = make_float2(0.f, 0.f);
   static_for<8>([&](auto IC) {                       // qs word i: groups 8i .. 8i+7
     constexpr int i = decltype(IC)::value;
     const uint32_t Q = bc.Q[i];
@@ -100,25 +102,26 @@ __device__ __forceinline__ void lut_block_body(const BlockCodes& bc, uint32_t lu
     // table byte offsets (t << 6 | n << 2) of the 4 even / 4 odd groups
     const uint32_t ce = ((Q << 2) & 0x3C3C3C3Cu) | (((hb & 0x55u) * 0x01041040u) & 0x40404040u);
     const uint32_t co = ((Q >> 2) & 0x3C3C3C3Cu) | (((hb & 0xAAu) * 0x00820820u) & 0x40404040u);
-    static_for<4>([&](auto MC) {
-      constexpr int m = decltype(MC)::value;
-      constexpr int ge = 8 * i + 2 * m;              // even group's index in the block
-      const uint32_t ae = __byte_perm(ce, lut, 0x7650u | m);
-      const uint32_t ao = __byte_perm(co, lut, 0x7650u | m);
-      s[0][m] += lds_f32<ge * kLutGroupBytes>(ae) + lds_f32<(ge + 1) * kLutGroupBytes>(ao);
-      if constexpr (TT > 1)
-        s[1][m] += lds_f32<kLutTokenBytes + ge * kLutGroupBytes>(ae) +
-                   lds_f32<kLutTokenBytes + (ge + 1) * kLutGroupBytes>(ao);
-      if constexpr (TT > 2)
-        s[2][m] += lds_f32<2 * kLutTokenBytes + ge * kLutGroupBytes>(ae) +
-                   lds_f32<2 * kLutTokenBytes + (ge + 1) * kLutGroupBytes>(ao);
-      if constexpr (TT > 3)
-        s[3][m] += lds_f32<3 * kLutTokenBytes + ge * kLutGroupBytes>(ae) +
-                   lds_f32<3 * kLutTokenBytes + (ge + 1) * kLutGroupBytes>(ao);
+    static_for<2>([&](auto PC) {
+      constexpr int mp = decltype(PC)::value;        // byte positions 2 mp, 2 mp + 1
+      constexpr int g0 = 8 * i + 4 * mp;             // even group of position 2 mp
+      constexpr int g1 = g0 + 2;                     // even group of position 2 mp + 1
+      const uint32_t ae0 = __byte_perm(ce, lut, 0x7650u | (2 * mp));
+      const uint32_t ae1 = __byte_perm(ce, lut, 0x7650u | (2 * mp + 1));
+      const uint32_t ao0 = __byte_perm(co, lut, 0x7650u | (2 * mp));
+      const uint32_t ao1 = __byte_perm(co, lut, 0x7650u | (2 * mp + 1));
+      static_for<TT>([&](auto TC) {
+        constexpr int t = decltype(TC)::value;
+        constexpr int tb = t * kLutTokenBytes;
+        const float2 e = make_float2(lds_f32<tb + g0 * kLutGroupBytes>(ae0), lds_f32<tb + g1 * kLutGroupBytes>(ae1));
+        const float2 o = make_float2(lds_f32<tb + (g0 + 1) * kLutGroupBytes>(ao0),
+                                     lds_f32<tb + (g1 + 1) * kLutGroupBytes>(ao1));
+        s[t][mp] = fadd2(s[t][mp], fadd2(e, o));     // s_m += e_m + o_m, lane by lane
+      });
     });
   });
 #pragma unroll
-  for (int t = 0; t < TT; ++t) acc[t] = fmaf(bc.d, (s[t][0] + s[t][1]) + (s[t][2] + s[t][3]), acc[t]);
+  for (int t = 0; t < TT; ++t) acc[t] = fmaf(bc.d, (s[t][0].x + s[t][0].y) + (s[t][1].x + s[t][1].y), acc[t]);
 }
 
 // Activations of this thread's group for chunk `chunk`, TT tokens (8 bytes each).
