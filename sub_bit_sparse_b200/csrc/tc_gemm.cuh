@@ -285,6 +285,21 @@ __device__ __forceinline__ void tc_fill_tables(uint32_t* t0, uint32_t* t1) {
   }
 }
 
+// Two fp32 fused multiply-adds in one instruction (the packed f32x2 FMA of
+// sm_100), each lane rounded once as fmaf: {a.x * b.x + c.x, a.y * b.y + c.y}.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
 // Expands this thread's half of each of the block's stages into 16 TMEM
 // columns (bf16: 8 groups x 2 words of each 64-column stage; fp8: 16 groups
 // x 1 word of each 128-column stage); for each stage waits for the A stage
@@ -603,7 +618,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant
             STQ1_TMEM_LD16(tmem_lane + kTcColD + p * kTcN + kCols * chalf + 16 * c, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(d, __uint_as_float(v[i]), acc[16 * c + i]);
+            for (int i = 0; i < 16; i += 2) {         // two columns per packed fp32x2 FMA
+              const float2 r = ffma2(make_float2(d, d), make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
+                                     make_float2(acc[16 * c + i], acc[16 * c + i + 1]));
+              acc[16 * c + i] = r.x;
+              acc[16 * c + i + 1] = r.y;
+            }
           }
         }
         tc_fence_before();
