@@ -159,9 +159,9 @@ size_t stq1_gemv_workspace(int64_t N, int64_t K, int batch);
 /*
  * stq1_gemv -- y[t, j] = sum_k W^[j, k] x[t, k], fp32 accumulation.
  * The decoded weight is never materialised in memory ("Runtime" section of
- * the lemmy post: STQ1_0 CUDA kernels).  1 to 4 tokens use the lookup-table
+ * the lemmy post: STQ1_0 CUDA kernels).  1 or 2 tokens use the lookup-table
  * kernel: codes index per-group tables of the activation sums, so the weight
- * side has no multiplies (one table load per token and group).  5 to 15
+ * side has no multiplies (one table load per token and group).  3 to 15
  * tokens use the tensor-core decode kernel:
  * each group's code is expanded once in registers to bf16 +/-1 and 0 and
  * contracted against up to 8 tokens per MMA (fp32 accumulation, d applied
@@ -409,8 +409,8 @@ int stq1_gemv_noalloc(const void* W_packed, const uint16_t* x, float* y, int64_t
 
 /*
  * stq1_set_path -- process-wide choice between the matmul kernels, for testing
- * and crossover measurements: 0 = by size (default: 1 to 4 tokens use the
- * lookup-table kernel and 5 to 15 the tensor-core decode kernel; MoE calls
+ * and crossover measurements: 0 = by size (default: 1 or 2 tokens use the
+ * lookup-table kernel and 3 to 15 the tensor-core decode kernel; MoE calls
  * averaging fewer than 16 pairs per routed expert send experts with one or
  * two pairs to the lookup-table kernel and the others to the tensor-core
  * decode kernel; 16 or more tokens, and MoE calls averaging 16 or more pairs

@@ -33,9 +33,12 @@
 // 32 registers) serve 64 MMAs.  Activations for a step are staged in shared
 // memory by all threads, one step ahead, in a layout permuted so that the B
 // loads (16 bytes: two MMAs) are free of bank conflicts.  At the end the
-// four block-warps' partial sums meet in shared memory (fixed order), and
-// split-K pieces meet through the caller's workspace (the last piece to
-// finish adds them in order 0..S-1), as in the lookup-table kernel.
+// four block-warps' partial sums meet in shared memory (fixed order).  The S
+// split-K pieces of a unit normally form one thread-block cluster and push
+// their partials into the shared memory of the CTA that owns each row, one
+// cluster barrier, and the owner adds them in order 0..S-1; if the device
+// refuses the cluster, they meet through the caller's workspace (the last
+// piece to finish adds them in order), as in the lookup-table kernel.
 #pragma once
 
 #include "device_common.cuh"
@@ -53,6 +56,9 @@ constexpr int kMmaOffTable = 0;                  // 2 x 32 x 4 bytes (256-aligne
 constexpr int kMmaOffBar = 256;                  // kMmaStages mbarriers
 constexpr int kMmaOffX = 512;                    // 2 x 16 KB of staged activations
 constexpr int kMmaOffStage = kMmaOffX + 2 * kMmaXStepBytes;
+// cluster split K: S x ceil(128 / S) slots x 8 tokens of pushed partials, at
+// most (128 + S) x 32 bytes; placed after the stages
+constexpr int kMmaRedBytes = (kMmaRows + kMaxClusterRanks) * kMmaTokens * 4;
 static_assert(4 * kMmaRows * kMmaTokens * 4 <= 2 * kMmaXStepBytes, "reduction buffer must fit the x buffers");
 
 struct MmaArgs {
@@ -78,6 +84,7 @@ struct MmaArgs {
                              // (else pair id / topk).  Routing weights are always by pair id.
   int tiles_cap;             // MoE: entries the tile table holds (debug-build checks)
   int x_rows;                // rows of x (debug-build checks)
+  int cluster;               // 1: the S splits of a unit form one thread-block cluster (1, S, 1)
 };
 
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
@@ -274,6 +281,10 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
     fence_mbar_init();
   }
   __syncthreads();
+  // Cluster split K: peers write this CTA's shared memory only once it runs;
+  // announce it now and wait for every peer's announcement before the pushes.
+  const bool push = a.cluster != 0 && a.S > 1;
+  if (push) cluster_arrive_relaxed();
   auto issue = [&](int c) {
     const int st = (c - c0) % kMmaStages;
     packed_issue_chunk(a.g, &wmap, &tmap, R0, c, stage0 + st * a.g.stage_bytes, bar0 + 8u * st);
@@ -399,6 +410,10 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
       }
     }
     __syncthreads();
+    if (push) {                                    // the cluster's barriers, without pushes
+      cluster_wait();
+      cluster_sync_all();
+    }
     return;
   }
 
@@ -445,7 +460,39 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
     }
     return;
   }
-  // split K: publish the partials; the last piece of the unit adds them in order
+  if (push) {
+    // Push every (slot, token) partial into the shared memory of the CTA that
+    // owns the slot (cluster rank (slot * S) / 128, the rank equal to its
+    // split), one cluster barrier, then each owner adds its slots' S partials
+    // in order 0..S-1.
+    const uint32_t redc = stage0 + static_cast<uint32_t>(kMmaStages) * a.g.stage_bytes;
+    const int per = (kMmaRows + a.S - 1) / a.S;   // slots per owner, at most
+    cluster_wait();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int idx = threadIdx.x + 256 * k;
+      const int sl = idx >> 3, t = idx & 7;
+      const int owner = (sl * a.S) >> 7;
+      const int local = sl - (owner * kMmaRows + a.S - 1) / a.S;
+      st_peer_f32(redc + 4u * static_cast<uint32_t>((split * per + local) * kMmaTokens + t), owner, vals[k]);
+    }
+    cluster_sync_all();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int idx = threadIdx.x + 256 * k;
+      const int sl = idx >> 3, t = idx & 7;
+      if (((sl * a.S) >> 7) != split || !good[k]) continue;
+      const int local = sl - (split * kMmaRows + a.S - 1) / a.S;
+      float v = 0.f;
+      for (int sp = 0; sp < a.S; ++sp)
+        v += lds_f32_addr(redc + 4u * static_cast<uint32_t>((sp * per + local) * kMmaTokens + t));
+      if (up_flag && rows[k] >= a.N / 2) v *= a.route_w[wrows[k]];
+      a.y[static_cast<long long>(orows[k]) * a.N + rows[k]] = v;
+    }
+    return;
+  }
+  // split K through the workspace: publish the partials; the last piece of
+  // the unit adds them in order
 #pragma unroll
   for (int k = 0; k < 4; ++k)
     if (good[k]) a.partial[(static_cast<long long>(split) * a.rows_out + orows[k]) * a.N + rows[k]] = vals[k];
@@ -471,9 +518,9 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
   if (threadIdx.x == 0) a.counters[unit] = 0;
 }
 
-inline size_t mma_smem_bytes(int stage_bytes) {
-  return 256 + kMmaOffStage + static_cast<size_t>(kMmaStages) * stage_bytes;
+inline size_t mma_smem_bytes(int stage_bytes, bool cluster = false) {
+  return 256 + kMmaOffStage + static_cast<size_t>(kMmaStages) * stage_bytes + (cluster ? kMmaRedBytes : 0);
 }
-inline size_t mma_smem_bytes_max() { return mma_smem_bytes(kPackedStageMax); }
+inline size_t mma_smem_bytes_max() { return mma_smem_bytes(kPackedStageMax, true); }
 
 }  // namespace stq1

@@ -154,6 +154,7 @@ int ensure_configured() {
   cudaFuncSetAttribute(lut_gemv_kernel<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaFuncSetAttribute(lut_gemv_kernel<2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaFuncSetAttribute(lut_gemv_kernel<4>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaFuncSetAttribute(mma_gemv_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaGetLastError();
   g_configured[dev].store(true, std::memory_order_release);
   return STQ1_OK;
@@ -384,14 +385,14 @@ void plan_table(GemvPlan* p, long long N, long long K, int batch, bool one_wave)
   p->S = static_cast<int>(std::max<long long>(1, S));
 }
 
-// Tensor-core decode kernel for few tokens: 5 .. 15 tokens by default, any
+// Tensor-core decode kernel for few tokens: 3 .. 15 tokens by default, any
 // batch when forced.  Its cost per weight does not depend on the token count;
 // the table kernel's grows with it.  Measured (CUDA graphs of distinct
-// matrices): on [4096, 7168] 12.6-13.0 us at 1-8 tokens against the table
-// kernel's 5.0 / 7.2 / 10.3 / 16.5 us at 1 / 2 / 4 / 8; on [18432, 7168]
-// 26.0-26.9 us against 15.5 / 19.1 / 27.5 / 49.9 us.  Rows need an even
-// number of blocks (chunks of two).
-constexpr int kMmaMinBatch = 5;
+// matrices): on [4096, 7168] 7.7-7.8 us at 1-8 tokens against the table
+// kernel's 4.9 / 7.0 / 8.4 / 10.4 / 16.2 us at 1 / 2 / 3 / 4 / 8; on
+// [18432, 7168] 21.5-21.8 us against 14.7 / 18.4 / 21.7 / 26.8 / 48.5 us.
+// Rows need an even number of blocks (chunks of two).
+constexpr int kMmaMinBatch = 3;
 bool want_mma(long long nb, int batch) {
   if (nb % 2 != 0) return false;
   const int path = g_path;
@@ -411,11 +412,23 @@ void plan_mma(GemvPlan* p, long long N, long long K, int batch) {
   p->n_chunks = static_cast<int>(nb / 2);
   const long long steps = (p->n_chunks + 1) / 2;
   const long long units0 = static_cast<long long>(p->n_tiles) * p->n_slabs;
-  const long long target = 2LL * sm_count();
-  long long S = units0 < target ? (target + units0 - 1) / units0 : 1;
-  // split K only while the arrival counters of the units fit their region
-  if (units0 * static_cast<long long>(sizeof(int)) > static_cast<long long>(kCounterBytes)) S = 1;
-  S = std::max<long long>(1, std::min<long long>(S, steps));
+  const long long slots = 2LL * sm_count();          // two CTAs per SM
+  // The K split with the least (waves x steps per piece): a second, partial
+  // wave costs a whole piece, so for [18432, 7168] two pieces of 4 steps in
+  // one wave beat three of 3 steps in two; ties go to fewer pieces (less to
+  // reduce).  Split K only while the arrival counters of the units fit their
+  // region (the workspace fallback needs them) and a cluster holds the pieces.
+  long long S = 1;
+  if (units0 * static_cast<long long>(sizeof(int)) <= static_cast<long long>(kCounterBytes)) {
+    long long best = -1;
+    for (long long c = 1; c <= std::min<long long>(steps, kMaxClusterRanks); ++c) {
+      const long long cost = ((units0 * c + slots - 1) / slots) * ((steps + c - 1) / c);
+      if (best < 0 || cost < best) {
+        best = cost;
+        S = c;
+      }
+    }
+  }
   const long long longest = (steps + S - 1) / S;
   if (longest > 0) S = (steps + longest - 1) / longest;
   p->S = static_cast<int>(S);
@@ -537,8 +550,19 @@ int gemv_impl(const void* W_packed, const uint16_t* x, float* y, int64_t N, int6
     m.flags = 0;
     const long long units = static_cast<long long>(p.n_tiles) * p.n_slabs;
     if (units >= (1LL << 31)) return STQ1_ERR_SHAPE;
-    return launch_pdl_cluster(mma_gemv_kernel, dim3(static_cast<unsigned>(units), static_cast<unsigned>(p.S)),
-                              kMmaThreads, mma_smem_bytes(m.g.stage_bytes), s, 1u, maps.w, maps.t, m);
+    const dim3 grid(static_cast<unsigned>(units), static_cast<unsigned>(p.S));
+    // split K reduces inside a cluster of the S pieces of a unit (distributed
+    // shared memory); if the device refuses such a cluster, through the
+    // caller's workspace
+    if (p.S > 1 && p.S <= kMaxClusterRanks) {
+      m.cluster = 1;
+      if (launch_pdl_cluster(mma_gemv_kernel, grid, kMmaThreads, mma_smem_bytes(m.g.stage_bytes, true), s,
+                             static_cast<unsigned>(p.S), maps.w, maps.t, m) == STQ1_OK)
+        return STQ1_OK;
+      m.cluster = 0;
+    }
+    return launch_pdl_cluster(mma_gemv_kernel, grid, kMmaThreads, mma_smem_bytes(m.g.stage_bytes), s, 1u, maps.w,
+                              maps.t, m);
   }
   if (!p.table_path) {
     const long long warps = static_cast<long long>(batch) * N;

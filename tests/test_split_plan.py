@@ -55,11 +55,12 @@ def test_pieces_are_as_few_as_the_longest_piece_allows(table_path, n, k, b):
 
 
 # Tensor-core decode kernel: (8-token tile, 128-row slab) units, K split in
-# whole steps of four blocks (two chunks) to about two CTAs per SM.
+# whole steps of four blocks (two chunks); the split minimises waves (of two
+# CTAs per SM, 296 slots) x steps per piece, ties to fewer pieces.
 @pytest.mark.parametrize("n,k,b,want", [
-    (4096, 7168, 8, 7),     # 32 units want 10 pieces; 7 steps allow 7
-    (4096, 7168, 12, 4),    # 64 units (two token tiles) want 5 pieces of 7 steps: longest 2 -> 4 pieces
-    (18432, 7168, 8, 3),    # 144 units want 3 pieces; longest 3 steps -> 3 (3 + 2 + 2)
+    (4096, 7168, 8, 7),     # 32 units: 7 pieces of one step in one wave (cost 1)
+    (4096, 7168, 12, 4),    # 64 units: 4 pieces of 2 steps in one wave (cost 2; 7 pieces take 2 waves)
+    (18432, 7168, 8, 2),    # 144 units: 2 pieces of 4 steps in one wave (cost 4) beat 3 pieces in 2 waves (6)
     (512, 2048, 4, 2),      # 4 units, 2 steps
     (37888, 7168, 4, 1),    # 296 units: already two per SM
 ])
