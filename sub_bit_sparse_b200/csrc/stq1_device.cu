@@ -646,7 +646,14 @@ MoePlan plan_moe(int T, int topk, int E, long long K, int flags) {
   m.tiles = want_tiles(nb, n_pairs >= kTcMinPairsPerExpert * active ? kTcMinBatch : 0);
   m.mma = !m.tiles && nb % 2 == 0 && g_path != 1;
   m.tile_tokens = m.tiles ? kTcN : (m.mma ? kMmaTokens : kMoeTableTokens);
-  m.max_tiles = static_cast<int>(std::min<long long>(n_pairs, n_pairs / m.tile_tokens + active));
+  // Tiles of an expert with c pairs: ceil(c / tile_tokens) <= c / tile_tokens + 1,
+  // so at most n_pairs / tile_tokens plus the number of experts with tiles;
+  // on the tensor-core decode path only experts with more than kMoeSmallMax
+  // pairs have main tiles, at most n_pairs / (kMoeSmallMax + 1) of them.  The
+  // grid is sized by this bound (the real count is on the device), and every
+  // CTA past the real count exits at once.
+  const long long tiled = m.mma ? std::min<long long>(active, n_pairs / (kMoeSmallMax + 1)) : active;
+  m.max_tiles = static_cast<int>(std::min<long long>(n_pairs, n_pairs / m.tile_tokens + tiled));
   m.small_max = m.mma ? kMoeSmallMax : 0;
   m.max_small = m.mma ? static_cast<int>(active) : 0;
   size_t off = 0;
