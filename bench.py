@@ -674,10 +674,14 @@ def run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier):
     yd = torch.empty((STACK, 1, N_ROWS), dtype=torch.float32, device=device)
     steps = max(20, args.steps // 2)
 
+    # per-matrix views made once, as a decode loop over resident weights would
+    mats, outs = list(stack.unbind(0)), list(yd.unbind(0))
+    nxt = mats[1:] + mats[:1]
+
     def one():
         xd.copy_(xh, non_blocking=True)
-        for i in range(STACK):
-            stq1.gemv(stack[i], xd, N_ROWS, K_COLS, out=yd[i], ws=ws, prefetch=stack[(i + 1) % STACK])
+        for w, y, wn in zip(mats, outs, nxt):
+            stq1.gemv(w, xd, N_ROWS, K_COLS, out=y, ws=ws, prefetch=wn)
         yh.copy_(yd, non_blocking=True)
 
     with torch.cuda.stream(stream):

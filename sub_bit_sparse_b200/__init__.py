@@ -259,20 +259,20 @@ def gemv(w_packed, x, n: int, k: int, out=None, ws=None, prefetch=None):
     if out is None:
         out = torch.empty((b, n), dtype=torch.float32, device=x.device)
     _require(out, torch.float32, "out")
-    lib = _load()
+    lib = _lib if _lib is not None else _load()
     if ws is None:
         ws = workspace(lib.stq1_gemv_workspace(n, k, b), x.device)
+    wsp, wsn = (None, 0) if ws is None else (ws.data_ptr(), ws.numel())
     if prefetch is None:
-        rc = lib.stq1_gemv(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b,
-                           None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
-                           _stream(x))
-        _check("stq1_gemv", rc)
+        rc = lib.stq1_gemv(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b, wsp, wsn, _stream(x))
+        if rc:
+            _check("stq1_gemv", rc)
         return out
     _require(prefetch, torch.uint8, "prefetch")
-    rc = lib.stq1_gemv_prefetch(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b,
-                                None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
+    rc = lib.stq1_gemv_prefetch(w_packed.data_ptr(), x.data_ptr(), out.data_ptr(), n, k, b, wsp, wsn,
                                 prefetch.data_ptr(), prefetch.numel(), _stream(x))
-    _check("stq1_gemv_prefetch", rc)
+    if rc:
+        _check("stq1_gemv_prefetch", rc)
     return out
 
 
