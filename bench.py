@@ -108,7 +108,7 @@ class ClockSampler:
         "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80,
     }
 
-    def __init__(self, index: int, period_s: float = 0.002):
+    def __init__(self, index: int, period_s: float = 0.0005):
         self.index, self.period = index, period_s
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
