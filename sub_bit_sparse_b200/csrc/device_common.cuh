@@ -186,6 +186,19 @@ __device__ __forceinline__ void st_peer_f32(uint32_t local_addr, uint32_t rank, 
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
 
+// Asynchronous store of one fp32 into the shared memory of cluster CTA
+// `rank` (same offset as local_addr), counted as 4 bytes of completed
+// transactions on that CTA's mbarrier at local_bar's offset.  The sender does
+// not wait for it; the receiver waits on its own mbarrier.
+__device__ __forceinline__ void st_async_peer_f32(uint32_t local_addr, uint32_t local_bar, uint32_t rank, float v) {
+  uint32_t ra, rb;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(local_bar), "r"(rank));
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(ra),
+               "r"(__float_as_uint(v)), "r"(rb)
+               : "memory");
+}
+
 // Two fp32 additions in one instruction (the packed f32x2 add of sm_100),
 // each lane rounded to nearest as a scalar add: {a.x + b.x, a.y + b.y}.
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {

@@ -192,9 +192,17 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
   const uint32_t red = stage0 + ((a.cq + (a.cr > 0 ? 1 : 0)) >= 2 ? 2 : 1) * a.g.stage_bytes;
   const bool push = a.cluster && a.S > 1;
 
+  // split-K partials arrive by asynchronous stores counted on this barrier:
+  // 2 halves x S pieces x TT tokens x the rows this CTA owns, 4 bytes each
+  const uint32_t bar_red = bar0 + 16;
   if (threadIdx.x == 0) {
     mbar_init(bar0, 1);
     mbar_init(bar0 + 8, 1);
+    mbar_init(bar_red, 1);
+    if (push) {
+      const int owned = (kLutRows * (split + 1) + a.S - 1) / a.S - (kLutRows * split + a.S - 1) / a.S;
+      mbar_arrive_expect_tx(bar_red, static_cast<uint32_t>(2 * a.S * TT * owned * 4));
+    }
     fence_mbar_init();
   }
   // Peers may write this CTA's shared memory only once it runs: announce it
@@ -267,8 +275,10 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
 
   if (push) {
     // Push both halves' partials into the shared memory of the CTA that owns
-    // the row (cluster rank (row * S) / 128, the rank equal to its split),
-    // then one cluster barrier; every CTA reaches it, failed or not.
+    // the row (cluster rank (row * S) / 128, the rank equal to its split) by
+    // asynchronous stores counted on its reduction barrier; every CTA pushes,
+    // failed or not.  Each CTA then waits (bounded) on its own barrier for
+    // the partials of the rows it owns: no cluster-wide release fence.
     cluster_wait();
     const int owner = (rho * a.S) >> 7;
     // the owner's rows are ceil(128 r / S) .. ceil(128 (r + 1) / S) - 1
@@ -276,8 +286,9 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
     const int per = (kLutRows + a.S - 1) / a.S;      // rows per owner, at most
 #pragma unroll
     for (int t = 0; t < TT; ++t)
-      st_peer_f32(red + 4u * (((t * 2 * a.S) + 2 * split + half) * per + local), owner, acc[t]);
-    cluster_sync_all();
+      st_async_peer_f32(red + 4u * (((t * 2 * a.S) + 2 * split + half) * per + local), bar_red, owner, acc[t]);
+    // every thread waits, so the CTA outlives the stores still coming in
+    if (!mbar_wait_bounded(bar_red, 0)) return;
     if (half == 0 && owner == split && row_ok) {
       const bool up = (a.flags & STQ1_MOE_WEIGHT_UP) && row >= a.N / 2;
 #pragma unroll
