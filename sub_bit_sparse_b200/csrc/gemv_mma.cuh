@@ -276,14 +276,22 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(table + 128u + 4u * threadIdx.x), "r"(h[2] | (h[3] << 16))
                  : "memory");
   }
+  const bool push = a.cluster != 0 && a.S > 1;
+  // cluster split K: the pushed partials arrive by asynchronous stores counted
+  // on this barrier (S pieces x 8 tokens x the slots this CTA owns, 4 bytes each)
+  const uint32_t bar_red = bar0 + 8u * kMmaStages;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMmaStages; ++i) mbar_init(bar0 + 8u * i, 1);
+    mbar_init(bar_red, 1);
+    if (push) {
+      const int owned = (kMmaRows * (split + 1) + a.S - 1) / a.S - (kMmaRows * split + a.S - 1) / a.S;
+      mbar_arrive_expect_tx(bar_red, static_cast<uint32_t>(a.S * kMmaTokens * owned * 4));
+    }
     fence_mbar_init();
   }
   __syncthreads();
   // Cluster split K: peers write this CTA's shared memory only once it runs;
   // announce it now and wait for every peer's announcement before the pushes.
-  const bool push = a.cluster != 0 && a.S > 1;
   if (push) cluster_arrive_relaxed();
   auto issue = [&](int c) {
     const int st = (c - c0) % kMmaStages;
@@ -410,9 +418,21 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
       }
     }
     __syncthreads();
-    if (push) {                                    // the cluster's barriers, without pushes
+    if (push) {
+      // push zeros so that every owner's count completes; the error word is set
       cluster_wait();
-      cluster_sync_all();
+      const uint32_t redc = stage0 + static_cast<uint32_t>(kMmaStages) * a.g.stage_bytes;
+      const int per = (kMmaRows + a.S - 1) / a.S;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int idx = threadIdx.x + 256 * k;
+        const int sl = idx >> 3, t = idx & 7;
+        const int owner = (sl * a.S) >> 7;
+        const int local = sl - (owner * kMmaRows + a.S - 1) / a.S;
+        st_async_peer_f32(redc + 4u * static_cast<uint32_t>((split * per + local) * kMmaTokens + t), bar_red, owner,
+                          0.f);
+      }
+      mbar_wait_bounded(bar_red, 0);               // this CTA outlives the stores coming in
     }
     return;
   }
@@ -463,7 +483,8 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
   if (push) {
     // Push every (slot, token) partial into the shared memory of the CTA that
     // owns the slot (cluster rank (slot * S) / 128, the rank equal to its
-    // split), one cluster barrier, then each owner adds its slots' S partials
+    // split) by asynchronous stores counted on its reduction barrier; each
+    // CTA waits (bounded) on its own barrier, then adds its slots' S partials
     // in order 0..S-1.
     const uint32_t redc = stage0 + static_cast<uint32_t>(kMmaStages) * a.g.stage_bytes;
     const int per = (kMmaRows + a.S - 1) / a.S;   // slots per owner, at most
@@ -474,9 +495,10 @@ mma_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
       const int sl = idx >> 3, t = idx & 7;
       const int owner = (sl * a.S) >> 7;
       const int local = sl - (owner * kMmaRows + a.S - 1) / a.S;
-      st_peer_f32(redc + 4u * static_cast<uint32_t>((split * per + local) * kMmaTokens + t), owner, vals[k]);
+      st_async_peer_f32(redc + 4u * static_cast<uint32_t>((split * per + local) * kMmaTokens + t), bar_red, owner,
+                        vals[k]);
     }
-    cluster_sync_all();
+    if (!mbar_wait_bounded(bar_red, 0)) return;    // every thread: the CTA outlives the stores coming in
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int idx = threadIdx.x + 256 * k;
