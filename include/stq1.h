@@ -124,8 +124,8 @@ int stq1_quantize_ref(const float* W, const float* h, int64_t N, int64_t K, int 
  * stq1_quantize_ref for every input that function accepts (one thread per
  * 256-weight block, fp64 in the same order, no fused multiply-add).
  *   W      device, [N, K] fp32 row-major, 16-byte aligned.
- *   h      device, [K] fp32 importance (Sherry mode; NULL means h = 1;
- *          ignored in plain mode).
+ *   h      device, [K] fp32 importance, 16-byte aligned (Sherry mode;
+ *          NULL means h = 1; ignored in plain mode).
  *   out    device, N*K/256*42 bytes, 2-byte aligned (fully overwritten).
  *   rounds Sherry rounds (0..1000; the pages use 3).
  * Asynchronous on `stream`.  A NaN/Inf weight, or a negative or non-finite

@@ -16,6 +16,8 @@
 namespace stq1 {
 
 constexpr int kEncThreads = 128;                 // blocks per CTA (one thread each)
+constexpr int kEncHPitch = kBlockWeights + 4;    // floats per staged importance block (1040 B: 16 B mod 128)
+constexpr int kEncHMaxCols = 40;                 // importance rows of at most this many blocks are staged
 constexpr int kEncPitch = kBlockWeights + 1;     // floats per block staged by the STQ2 encoder (odd: conflict-free)
 
 // fp64 -> IEEE binary16 bits, round to nearest even, saturating at +/-65504:
@@ -105,9 +107,14 @@ struct WlsSums {
   }
 };
 
-// One thread encodes one block, reading it from global memory (L1/L2) once
-// per pass: no shared staging, so the number of blocks in flight per SM is set
-// by registers, which is what hides the latency of the sequential fp64 sums.
+// One thread encodes one block, reading its weights from global memory (L1/L2)
+// once per pass: no shared staging of W, so the number of blocks in flight per
+// SM is set by registers, which is what hides the latency of the sequential
+// fp64 sums.  The importances depend only on the column, so a CTA copies the
+// whole importance row (up to kEncHMaxCols blocks) into shared memory once,
+// at a pitch of 16 B mod 128 so that a quarter-warp's 16-byte loads from
+// consecutive blocks hit distinct banks; a thread's loads from its own 1 KB
+// global block would touch 32 lines per warp instruction.
 // Passes: lanes and checks; the scale of the initial lanes; then per Sherry
 // round one pass that picks every group's zero lane with that round's d and,
 // group by group in the same ascending order, adds the group's new non-zero
@@ -116,14 +123,24 @@ struct WlsSums {
 __global__ void __launch_bounds__(kEncThreads, 4)
 encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long long n_blocks, int nb, int mode,
               int rounds, uint8_t* __restrict__ out) {
+  extern __shared__ float4 hs4[];                 // staged importance row, kEncHPitch floats per block
   griddep_wait();
   griddep_launch_dependents();
+  const bool use_h = mode == STQ1_ENC_SHERRY && hcol;
+  const bool staged = use_h && nb <= kEncHMaxCols;
+  if (staged) {
+    const float4* g4 = reinterpret_cast<const float4*>(hcol);
+    for (int i = threadIdx.x; i < nb * (kBlockWeights / 4); i += kEncThreads)
+      hs4[(i / (kBlockWeights / 4)) * (kEncHPitch / 4) + i % (kBlockWeights / 4)] = __ldg(g4 + i);
+    __syncthreads();
+  }
   const long long b = static_cast<long long>(blockIdx.x) * kEncThreads + threadIdx.x;
   if (b >= n_blocks) return;
   const float4* w4 = reinterpret_cast<const float4*>(W + b * kBlockWeights);   // one group per float4
-  const float4* h4 = (mode == STQ1_ENC_SHERRY && hcol)
-                         ? reinterpret_cast<const float4*>(hcol + (b % nb) * kBlockWeights)
-                         : nullptr;
+  // generic pointer: shared (staged) or global; read with plain loads
+  const float4* h4 = !use_h ? nullptr
+                     : staged ? hs4 + (b % nb) * (kEncHPitch / 4)
+                              : reinterpret_cast<const float4*>(hcol + (b % nb) * kBlockWeights);
 
   // pass 1: zero lanes (least |w|), sign masks, amax, checks
   EncState st;
@@ -145,7 +162,7 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
         amax = fmaxf(amax, fabsf(wg[l]));
       }
       if (h4) {
-        const float4 hv = __ldg(h4 + 8 * c + i);
+        const float4 hv = h4[8 * c + i];
         const float hg[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
         for (int l = 0; l < 4; ++l) {
@@ -183,7 +200,7 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
         const float wg[4] = {v.x, v.y, v.z, v.w};
         float hg[4] = {1.f, 1.f, 1.f, 1.f};
         if (h4) {
-          const float4 hv = __ldg(h4 + 8 * c + i);
+          const float4 hv = h4[8 * c + i];
           hg[0] = hv.x; hg[1] = hv.y; hg[2] = hv.z; hg[3] = hv.w;
         }
         const int zg = static_cast<int>((z16 >> (2 * i)) & 3u);
@@ -207,7 +224,7 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
           const float wg[4] = {v.x, v.y, v.z, v.w};
           float hg[4] = {1.f, 1.f, 1.f, 1.f};
           if (h4) {
-            const float4 hv = __ldg(h4 + 8 * c + i);
+            const float4 hv = h4[8 * c + i];
             hg[0] = hv.x; hg[1] = hv.y; hg[2] = hv.z; hg[3] = hv.w;
           }
           double aw[4];
@@ -260,6 +277,10 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
   }
 }
 
-inline size_t encode_smem_bytes() { return 0; }   // blocks are read from global memory
+// Dynamic shared memory of a launch: the staged importance row, if any.
+inline size_t encode_smem_bytes(int nb, bool staged_h) {
+  return staged_h ? static_cast<size_t>(nb) * kEncHPitch * sizeof(float) : 0;
+}
+inline size_t encode_smem_bytes_max() { return static_cast<size_t>(kEncHMaxCols) * kEncHPitch * sizeof(float); }
 
 }  // namespace stq1

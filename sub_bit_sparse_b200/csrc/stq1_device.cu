@@ -139,7 +139,7 @@ int ensure_configured() {
       cudaFuncSetAttribute(tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kTcSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(encode_smem_bytes())) != cudaSuccess ||
+                           static_cast<int>(encode_smem_bytes_max())) != cudaSuccess ||
       cudaFuncSetAttribute(stq2_encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kStq2EncBlocks * kEncPitch * sizeof(float))) != cudaSuccess ||
       cudaFuncSetAttribute(hess_score_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -944,12 +944,15 @@ extern "C" int stq1_quantize(const float* W, const float* h, int64_t N, int64_t 
   if (mode == STQ1_ENC_SHERRY && (rounds < 0 || rounds > 1000)) return STQ1_ERR_ARG;
   if (N > (1LL << 40) / K) return STQ1_ERR_SHAPE;
   if (!aligned16(W) || (reinterpret_cast<uintptr_t>(out) & 1)) return STQ1_ERR_ALIGN;
+  if (mode == STQ1_ENC_SHERRY && h && !aligned16(h)) return STQ1_ERR_ALIGN;   // read as float4
   const long long n_blocks = N * (K / kBlockWeights);
   const long long grid = (n_blocks + kEncThreads - 1) / kEncThreads;
   if (grid >= (1LL << 31)) return STQ1_ERR_SHAPE;
   int rc = ensure_configured();
   if (rc != STQ1_OK) return rc;
-  return launch_pdl(encode_kernel, static_cast<unsigned>(grid), kEncThreads, encode_smem_bytes(),
+  const int nb = static_cast<int>(K / kBlockWeights);
+  const bool staged_h = mode == STQ1_ENC_SHERRY && h && nb <= kEncHMaxCols;
+  return launch_pdl(encode_kernel, static_cast<unsigned>(grid), kEncThreads, encode_smem_bytes(nb, staged_h),
                     static_cast<cudaStream_t>(stream), W, h, n_blocks, static_cast<int>(K / kBlockWeights), mode,
                     rounds, out);
 }

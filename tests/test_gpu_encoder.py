@@ -60,7 +60,9 @@ def test_encoder_matches_host_and_oracle_on_edge_blocks(rounds):
     assert np.array_equal(_gpu(w), oracle.encode_plain(w))
 
 
-@pytest.mark.parametrize("n,k", [(1, 256), (3, 512), (130, 1024), (65, 7168)])
+# 7168 and below: the importance row is staged in shared memory; 12288 (48
+# blocks per row) reads it from global memory
+@pytest.mark.parametrize("n,k", [(1, 256), (3, 512), (130, 1024), (65, 7168), (9, 10240), (7, 12288)])
 def test_encoder_small_shapes(n, k):
     w = workloads.expert_like_matrix(n, k, seeds=(n, k, n + k))
     h = workloads.calibration_importance(k, seed=n + 1)
