@@ -107,23 +107,91 @@ struct WlsSums {
   }
 };
 
-// One thread encodes one block, reading its weights from global memory (L1/L2)
-// once per pass: no shared staging of W, so the number of blocks in flight per
-// SM is set by registers, which is what hides the latency of the sequential
-// fp64 sums.  The importances depend only on the column, so a CTA copies the
-// whole importance row (up to kEncHMaxCols blocks) into shared memory once,
-// at a pitch of 16 B mod 128 so that a quarter-warp's 16-byte loads from
-// consecutive blocks hit distinct banks; a thread's loads from its own 1 KB
-// global block would touch 32 lines per warp instruction.
-// Passes: lanes and checks; the scale of the initial lanes; then per Sherry
-// round one pass that picks every group's zero lane with that round's d and,
-// group by group in the same ascending order, adds the group's new non-zero
-// lanes to the sums of the next d.  The additions happen in exactly the order
-// of a separate fit over k = 0..255, so the bytes do not change.
+// Per-warp staging of W.  A warp encodes 32 consecutive blocks, one per lane.
+// Chunk c of a block (groups 8c .. 8c+7: 128 bytes) is brought into a
+// shared slot by the whole warp with 16-byte asynchronous copies, eight lanes
+// per block, so one instruction moves four whole 128-byte lines; each lane
+// then reads its own block's slot.  Slots are 144 bytes apart (16 B mod 128),
+// so a quarter-warp's 16-byte reads from eight consecutive slots hit distinct
+// banks.  A lane reading its own 1 KB global block directly would touch 32
+// lines per warp instruction.  Each pass over a block goes through its eight
+// chunks in order and the next pass starts again at chunk 0, so the copy of
+// the next chunk is always (c + 1) mod 8.
+constexpr int kEncWarps = kEncThreads / 32;
+constexpr int kEncChunkBytes = 8 * 16;              // eight groups of one block
+constexpr int kEncWPitch = kEncChunkBytes + 16;     // bytes per block slot
+constexpr int kEncWBufBytes = 32 * kEncWPitch;      // one warp's 32 slots: 4608 B
+constexpr int kEncWBufs = 2;                        // chunks in flight per warp
+constexpr int kEncWBytes = kEncWarps * kEncWBufs * kEncWBufBytes;
+
+__device__ __forceinline__ void enc_cp_async16(uint32_t dst, const float* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ float4 enc_lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
+struct EncWPipe {
+  uint32_t buf;          // shared address of this warp's kEncWBufs buffers
+  const float* wbase;    // first weight of the warp's first block
+  int nblk;              // the warp's blocks inside the matrix (1..32)
+  int lane;
+  int q;                 // chunks consumed so far
+  int total;             // chunks this warp will consume (8 per pass)
+
+  __device__ __forceinline__ void fetch(int c, int slot) const {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int blk = 4 * j + (lane >> 3), part = lane & 7;
+      if (blk < nblk)
+        enc_cp_async16(buf + slot * kEncWBufBytes + blk * kEncWPitch + part * 16,
+                       wbase + static_cast<long long>(blk) * kBlockWeights + 32 * c + 4 * part);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  __device__ __forceinline__ void start() { q = 0; if (total > 0) fetch(0, 0); }
+  // Shared address of this lane's slot of chunk c (the q-th chunk overall).
+  // With two buffers, first queue the next chunk into the other one (read
+  // last during chunk q - 1, which every lane has released), then wait for
+  // chunk c; with one, the next chunk is queued at the release.
+  __device__ __forceinline__ uint32_t acquire(int c) {
+    if (kEncWBufs == 2 && q + 1 < total) {
+      fetch((c + 1) & 7, (q + 1) & 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncwarp();
+    return buf + (q % kEncWBufs) * kEncWBufBytes + lane * kEncWPitch;
+  }
+  __device__ __forceinline__ void release(int c) {
+    __syncwarp();
+    if (kEncWBufs == 1 && q + 1 < total) fetch((c + 1) & 7, 0);
+    ++q;
+  }
+};
+static_assert(kEncWBufs == 1 || kEncWBufs == 2, "one or two chunks in flight per warp");
+
+// One thread encodes one block.  Its weights come through the warp's staged
+// chunks, once per pass; the importances depend only on the column, so a CTA
+// copies the whole importance row (up to kEncHMaxCols blocks) into shared
+// memory once, at a pitch of 16 B mod 128 (longer rows are read from global
+// memory).  Many blocks are in flight per SM, which is what hides the latency
+// of the sequential fp64 sums.  Passes: lanes and checks; the scale of the
+// initial lanes; then per Sherry round one pass that picks every group's zero
+// lane with that round's d and, group by group in the same ascending order,
+// adds the group's new non-zero lanes to the sums of the next d.  The
+// additions happen in exactly the order of a separate fit over k = 0..255, so
+// the bytes do not change.  Every lane of a warp runs every pass (the copies
+// are shared); lanes past the matrix or with a non-finite block only skip
+// their stores.
 __global__ void __launch_bounds__(kEncThreads, 4)
 encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long long n_blocks, int nb, int mode,
               int rounds, uint8_t* __restrict__ out) {
-  extern __shared__ float4 hs4[];                 // staged importance row, kEncHPitch floats per block
+  extern __shared__ __align__(16) uint8_t enc_smem[];   // [W slots][importance row]
+  float4* hs4 = reinterpret_cast<float4*>(enc_smem + kEncWBytes);
   griddep_wait();
   griddep_launch_dependents();
   const bool use_h = mode == STQ1_ENC_SHERRY && hcol;
@@ -134,9 +202,18 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
       hs4[(i / (kBlockWeights / 4)) * (kEncHPitch / 4) + i % (kBlockWeights / 4)] = __ldg(g4 + i);
     __syncthreads();
   }
-  const long long b = static_cast<long long>(blockIdx.x) * kEncThreads + threadIdx.x;
-  if (b >= n_blocks) return;
-  const float4* w4 = reinterpret_cast<const float4*>(W + b * kBlockWeights);   // one group per float4
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long bw0 = static_cast<long long>(blockIdx.x) * kEncThreads + 32 * warp;
+  if (bw0 >= n_blocks) return;                    // whole warps only
+  const long long b = bw0 + lane;
+  const bool active = b < n_blocks;
+  EncWPipe wp;
+  wp.buf = smem_u32(enc_smem) + warp * kEncWBufs * kEncWBufBytes;
+  wp.wbase = W + bw0 * kBlockWeights;
+  wp.nblk = static_cast<int>(min(32LL, n_blocks - bw0));
+  wp.lane = lane;
+  wp.total = 8 * (mode == STQ1_ENC_PLAIN ? 1 : 2 + rounds);
+  wp.start();
   // generic pointer: shared (staged) or global; read with plain loads
   const float4* h4 = !use_h ? nullptr
                      : staged ? hs4 + (b % nb) * (kEncHPitch / 4)
@@ -148,10 +225,11 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
   float amax = 0.f;
 #pragma unroll 1
   for (int c = 0; c < 8; ++c) {
+    const uint32_t ws = wp.acquire(c);
     uint32_t z16 = 0u, n32 = 0u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float4 v = __ldg(w4 + 8 * c + i);
+      const float4 v = enc_lds_f4(ws + 16 * i);
       const float wg[4] = {v.x, v.y, v.z, v.w};
       int zl;
       uint32_t neg;
@@ -173,15 +251,16 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
       z16 |= static_cast<uint32_t>(zl) << (2 * i);
       n32 |= neg << (4 * i);
     }
+    wp.release(c);
     // fill the rotating state in chunk order: after 8 iterations chunk c sits in its place
     st.neg[0] = n32;
     st.rotate(z16);
   }
   uint16_t* o16 = reinterpret_cast<uint16_t*>(out + b * kBlockBytes);   // 2-byte aligned
-  if (!finite) {
+  const bool store = active && finite;
+  if (active && !finite) {
     flag_error(STQ1_DEV_BAD_VALUE);
     for (int i = 0; i < kBlockBytes / 2; ++i) o16[i] = 0;
-    return;
   }
   if (!hany) h4 = nullptr;                       // an all-zero importance block uses h = 1
 
@@ -193,10 +272,11 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
     WlsSums sums;
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
+      const uint32_t ws = wp.acquire(c);
       const uint32_t z16 = st.z[0] & 0xFFFFu;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float4 v = __ldg(w4 + 8 * c + i);
+        const float4 v = enc_lds_f4(ws + 16 * i);
         const float wg[4] = {v.x, v.y, v.z, v.w};
         float hg[4] = {1.f, 1.f, 1.f, 1.f};
         if (h4) {
@@ -208,6 +288,7 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
         for (int l = 0; l < 4; ++l)
           if (l != zg) sums.add(fabs(static_cast<double>(wg[l])), static_cast<double>(hg[l]));
       }
+      wp.release(c);
       st.rotate(z16);
     }
     double d = sums.scale();
@@ -217,10 +298,11 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
       WlsSums next;
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
+        const uint32_t ws = wp.acquire(c);
         uint32_t z16 = 0u;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float4 v = __ldg(w4 + 8 * c + i);
+          const float4 v = enc_lds_f4(ws + 16 * i);
           const float wg[4] = {v.x, v.y, v.z, v.w};
           float hg[4] = {1.f, 1.f, 1.f, 1.f};
           if (h4) {
@@ -245,12 +327,14 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
           for (int l = 0; l < 4; ++l)
             if (l != best_l) next.add(aw[l], static_cast<double>(hg[l]));
         }
+        wp.release(c);
         st.rotate(z16);
       }
       d = next.scale();
     }
     d_bits = enc_half_bits(d);
   }
+  if (!store) return;
   // pack: d, qs (even group in the low nibble), qh (group g at bit g & 7 of byte g >> 3);
   // chunk c gives qs bytes 4c .. 4c+3 and qh byte c (the block starts on a 2-byte boundary)
   o16[0] = d_bits;
@@ -277,10 +361,13 @@ encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long 
   }
 }
 
-// Dynamic shared memory of a launch: the staged importance row, if any.
+// Dynamic shared memory of a launch: the warps' W slots, then the staged
+// importance row, if any.
 inline size_t encode_smem_bytes(int nb, bool staged_h) {
-  return staged_h ? static_cast<size_t>(nb) * kEncHPitch * sizeof(float) : 0;
+  return kEncWBytes + (staged_h ? static_cast<size_t>(nb) * kEncHPitch * sizeof(float) : 0);
 }
-inline size_t encode_smem_bytes_max() { return static_cast<size_t>(kEncHMaxCols) * kEncHPitch * sizeof(float); }
+inline size_t encode_smem_bytes_max() {
+  return kEncWBytes + static_cast<size_t>(kEncHMaxCols) * kEncHPitch * sizeof(float);
+}
 
 }  // namespace stq1
