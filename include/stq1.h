@@ -504,7 +504,7 @@ int stq1_status(void* stream, int* device_err);
  * the stored scale is fp16 of one more fit.  All in fp64 with a fixed order,
  * so the bytes are those of the oracle's encoder.
  *   W       device, [N, K] fp32 row-major, 16-byte aligned.
- *   h       device, [K] fp32 importance per column, 4-byte aligned, or NULL
+ *   h       device, [K] fp32 importance per column, 16-byte aligned, or NULL
  *           (h = 1).  A block whose h is all zero uses h = 1.
  *   rounds  0..1000.
  *   out     device, N*K/256*66 bytes, 2-byte aligned (fully overwritten).

@@ -18,7 +18,6 @@ namespace stq1 {
 constexpr int kEncThreads = 128;                 // blocks per CTA (one thread each)
 constexpr int kEncHPitch = kBlockWeights + 4;    // floats per staged importance block (1040 B: 16 B mod 128)
 constexpr int kEncHMaxCols = 40;                 // importance rows of at most this many blocks are staged
-constexpr int kEncPitch = kBlockWeights + 1;     // floats per block staged by the STQ2 encoder (odd: conflict-free)
 
 // fp64 -> IEEE binary16 bits, round to nearest even, saturating at +/-65504:
 // 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits, subnormal quantum

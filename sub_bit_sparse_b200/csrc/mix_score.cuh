@@ -36,105 +36,142 @@ constexpr int kStq2BlockBytes = 66;
 constexpr int kStq2OffCodes = 2;
 
 // ---------------------------------------------------------------------------
-// STQ2 encoder: one thread per 256-weight block (staged in shared memory like
-// the STQ1_0 encoder).  d starts at fp16(amax) with each weight at its nearest
-// level (d m_q) / 3, m_q = 2q - 3 (ties: the lower code); then `rounds` times
-// d is refit by weighted least squares, d = 3 sum h w m / sum h m^2 (k
-// ascending), and the levels re-picked; the stored scale is fp16 of one more
-// fit.  Every real-valued step is fp64 with the round-to-nearest intrinsics,
-// so the bytes do not depend on contraction or scheduling.
+// STQ2 encoder: one thread per 256-weight block, with the STQ1_0 encoder's
+// staging (W per warp in 128-byte chunks through shared memory, the
+// importance row once per CTA).  d starts at fp16(amax) with each weight at
+// its nearest level (d m_q) / 3, m_q = 2q - 3 (ties: the lower code); then
+// `rounds` times d is refit by weighted least squares, d = 3 sum h w m /
+// sum h m^2 (k ascending), and the levels re-picked; the stored scale is fp16
+// of one more fit.  Each pass that picks the levels also adds the new levels'
+// terms to the next fit's sums, weight by weight in ascending k, which is the
+// order of a separate fit, so the bytes do not change: 2 + rounds passes over
+// W instead of 2 + 2 rounds.  Every real-valued step is fp64 with the
+// round-to-nearest intrinsics, so the bytes do not depend on contraction or
+// scheduling.
 // ---------------------------------------------------------------------------
-constexpr int kStq2EncBlocks = 64;              // blocks (threads) per CTA
-
-__device__ __forceinline__ void stq2_pick(const float* w, double d, uint32_t (&qw)[16]) {
-  double lev[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) lev[q] = __ddiv_rn(__dmul_rn(d, static_cast<double>(2 * q - 3)), 3.0);
-#pragma unroll 1
-  for (int j = 0; j < 16; ++j) {
-    uint32_t word = 0;
-#pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-      const double wk = static_cast<double>(w[16 * j + i]);
-      int best = 0;
-      double bd = fabs(__dsub_rn(wk, lev[0]));
-#pragma unroll
-      for (int q = 1; q < 4; ++q) {
-        const double dq = fabs(__dsub_rn(wk, lev[q]));
-        if (dq < bd) { bd = dq; best = q; }
-      }
-      word |= static_cast<uint32_t>(best) << (2 * i);
-    }
-    qw[j] = word;
-  }
-}
-
-__device__ __forceinline__ double stq2_wls(const float* w, const float* h, const uint32_t (&qw)[16]) {
-  double num = 0.0, den = 0.0;
-#pragma unroll 1
-  for (int j = 0; j < 16; ++j) {
-    const uint32_t word = qw[j];
-#pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-      const int k = 16 * j + i;
-      const double m = static_cast<double>(2 * static_cast<int>((word >> (2 * i)) & 3u) - 3);
-      const double hk = h ? static_cast<double>(h[k]) : 1.0;
-      num = __dadd_rn(num, __dmul_rn(__dmul_rn(hk, static_cast<double>(w[k])), m));
-      den = __dadd_rn(den, __dmul_rn(hk, __dmul_rn(m, m)));
-    }
-  }
-  return __ddiv_rn(__dmul_rn(3.0, num), den);
-}
-
-__global__ void __launch_bounds__(kStq2EncBlocks)
+__global__ void __launch_bounds__(kEncThreads, 4)
 stq2_encode_kernel(const float* __restrict__ W, const float* __restrict__ hcol, long long n_blocks, int nb,
                    int rounds, uint8_t* __restrict__ out) {
-  extern __shared__ float sw[];                   // [kStq2EncBlocks][kEncPitch]
-  const long long b0 = static_cast<long long>(blockIdx.x) * kStq2EncBlocks;
-  const int nblk = static_cast<int>(min(static_cast<long long>(kStq2EncBlocks), n_blocks - b0));
+  extern __shared__ __align__(16) uint8_t enc_smem[];   // [W slots][importance row]
+  float4* hs4 = reinterpret_cast<float4*>(enc_smem + kEncWBytes);
   griddep_wait();                                 // W may come from the previous kernel
-  const float4* src = reinterpret_cast<const float4*>(W + b0 * kBlockWeights);
-  for (int f = threadIdx.x; f < nblk * (kBlockWeights / 4); f += kStq2EncBlocks) {
-    const float4 v = __ldg(src + f);
-    float* d = sw + (f >> 6) * kEncPitch + 4 * (f & 63);
-    d[0] = v.x;
-    d[1] = v.y;
-    d[2] = v.z;
-    d[3] = v.w;
+  const bool staged = hcol && nb <= kEncHMaxCols;
+  if (staged) {
+    const float4* g4 = reinterpret_cast<const float4*>(hcol);
+    for (int i = threadIdx.x; i < nb * (kBlockWeights / 4); i += kEncThreads)
+      hs4[(i / (kBlockWeights / 4)) * (kEncHPitch / 4) + i % (kBlockWeights / 4)] = __ldg(g4 + i);
+    __syncthreads();
   }
-  __syncthreads();
-  if (threadIdx.x >= nblk) return;
-  const long long b = b0 + threadIdx.x;
-  const float* w = sw + threadIdx.x * kEncPitch;
-  const float* h = hcol ? hcol + (b % nb) * kBlockWeights : nullptr;
-  bool finite = true;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long bw0 = static_cast<long long>(blockIdx.x) * kEncThreads + 32 * warp;
+  if (bw0 >= n_blocks) return;                    // whole warps only
+  const long long b = bw0 + lane;
+  const bool active = b < n_blocks;
+  const int picks = rounds > 0 ? rounds + 1 : 1;
+  EncWPipe wp;
+  wp.buf = smem_u32(enc_smem) + warp * kEncWBufs * kEncWBufBytes;
+  wp.wbase = W + bw0 * kBlockWeights;
+  wp.nblk = static_cast<int>(min(32LL, n_blocks - bw0));
+  wp.lane = lane;
+  wp.total = 8 * (1 + picks);
+  wp.start();
+  // generic pointer: shared (staged) or global; read with plain loads
+  const float4* h4 = !hcol ? nullptr
+                     : staged ? hs4 + (b % nb) * (kEncHPitch / 4)
+                              : reinterpret_cast<const float4*>(hcol + (b % nb) * kBlockWeights);
+
+  // pass 1: amax and checks
+  bool finite = true, hany = false;
   float amax = 0.f;
-  for (int k = 0; k < kBlockWeights; ++k) {
-    finite = finite && isfinite(w[k]);
-    amax = fmaxf(amax, fabsf(w[k]));
-  }
-  if (h) {
-    bool hany = false;
-    for (int k = 0; k < kBlockWeights; ++k) {
-      const float hk = h[k];
-      finite = finite && isfinite(hk) && hk >= 0.f;
-      hany = hany || hk != 0.f;
+#pragma unroll 1
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t ws = wp.acquire(c);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 v = enc_lds_f4(ws + 16 * i);
+      const float wg[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        finite = finite && isfinite(wg[e]);
+        amax = fmaxf(amax, fabsf(wg[e]));
+      }
+      if (h4) {
+        const float4 hv = h4[8 * c + i];
+        const float hg[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          finite = finite && isfinite(hg[e]) && hg[e] >= 0.f;
+          hany = hany || hg[e] != 0.f;
+        }
+      }
     }
-    if (!hany) h = nullptr;                       // an all-zero importance block uses h = 1
+    wp.release(c);
   }
   uint16_t* o16 = reinterpret_cast<uint16_t*>(out + b * kStq2BlockBytes);   // 2-byte aligned
-  if (!finite) {
+  const bool store = active && finite;
+  if (active && !finite) {
     flag_error(STQ1_DEV_BAD_VALUE);
     for (int i = 0; i < kStq2BlockBytes / 2; ++i) o16[i] = 0;
-    return;
   }
+  if (!hany) h4 = nullptr;                        // an all-zero importance block uses h = 1
+
   uint16_t d_bits = enc_half_bits(static_cast<double>(amax));
+  double d = static_cast<double>(__half2float(__ushort_as_half(d_bits)));
+  // codes: word j = weights 16j .. 16j+15, 2 bits each; the words of the chunk
+  // in hand enter at the top and the rest move down, so after eight chunks
+  // they are back in order (no indexing with a loop variable)
   uint32_t qw[16];
-  stq2_pick(w, static_cast<double>(__half2float(__ushort_as_half(d_bits))), qw);
-  if (rounds > 0) {
-    for (int r = 0; r < rounds; ++r) stq2_pick(w, stq2_wls(w, h, qw), qw);
-    d_bits = enc_half_bits(stq2_wls(w, h, qw));
+#pragma unroll
+  for (int j = 0; j < 16; ++j) qw[j] = 0u;
+#pragma unroll 1
+  for (int p = 0; p < picks; ++p) {
+    double lev[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) lev[q] = __ddiv_rn(__dmul_rn(d, static_cast<double>(2 * q - 3)), 3.0);
+    double num = 0.0, den = 0.0;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t ws = wp.acquire(c);
+      uint32_t word[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 v = enc_lds_f4(ws + 16 * i);
+        const float wg[4] = {v.x, v.y, v.z, v.w};
+        float hg[4] = {1.f, 1.f, 1.f, 1.f};
+        if (h4) {
+          const float4 hv = h4[8 * c + i];
+          hg[0] = hv.x; hg[1] = hv.y; hg[2] = hv.z; hg[3] = hv.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int n = 4 * i + e;                 // weight of the chunk, k = 32 c + n
+          const double wk = static_cast<double>(wg[e]);
+          int best = 0;
+          double bd = fabs(__dsub_rn(wk, lev[0]));
+#pragma unroll
+          for (int q = 1; q < 4; ++q) {
+            const double dq = fabs(__dsub_rn(wk, lev[q]));
+            if (dq < bd) { bd = dq; best = q; }
+          }
+          word[n >> 4] |= static_cast<uint32_t>(best) << (2 * (n & 15));
+          if (rounds > 0) {
+            const double m = static_cast<double>(2 * best - 3);
+            const double hk = h4 ? static_cast<double>(hg[e]) : 1.0;
+            num = __dadd_rn(num, __dmul_rn(__dmul_rn(hk, wk), m));
+            den = __dadd_rn(den, __dmul_rn(hk, __dmul_rn(m, m)));
+          }
+        }
+      }
+      wp.release(c);
+#pragma unroll
+      for (int j = 0; j < 14; ++j) qw[j] = qw[j + 2];
+      qw[14] = word[0];
+      qw[15] = word[1];
+    }
+    if (rounds > 0) d = __ddiv_rn(__dmul_rn(3.0, num), den);
   }
+  if (rounds > 0) d_bits = enc_half_bits(d);
+  if (!store) return;
   o16[0] = d_bits;
 #pragma unroll
   for (int i = 0; i < 32; ++i) o16[1 + i] = static_cast<uint16_t>(qw[i >> 1] >> (16 * (i & 1)));

@@ -141,7 +141,7 @@ int ensure_configured() {
       cudaFuncSetAttribute(encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(encode_smem_bytes_max())) != cudaSuccess ||
       cudaFuncSetAttribute(stq2_encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kStq2EncBlocks * kEncPitch * sizeof(float))) != cudaSuccess ||
+                           static_cast<int>(encode_smem_bytes_max())) != cudaSuccess ||
       cudaFuncSetAttribute(hess_score_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kHsSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(hess_score_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1361,16 +1361,17 @@ extern "C" int stq1_quantize_stq2(const float* W, const float* h, int64_t N, int
   if (!W || !out) return STQ1_ERR_NULL;
   if (N <= 0 || K <= 0 || K % kBlockWeights || N > (1LL << 40) / K) return STQ1_ERR_SHAPE;
   if (rounds < 0 || rounds > 1000) return STQ1_ERR_ARG;
-  if (!aligned16(W) || (reinterpret_cast<uintptr_t>(out) & 1) || (reinterpret_cast<uintptr_t>(h) & 3))
+  if (!aligned16(W) || (reinterpret_cast<uintptr_t>(out) & 1) || (h && !aligned16(h)))   // h read as float4
     return STQ1_ERR_ALIGN;
   const long long n_blocks = N * (K / kBlockWeights);
-  const long long grid = (n_blocks + kStq2EncBlocks - 1) / kStq2EncBlocks;
+  const long long grid = (n_blocks + kEncThreads - 1) / kEncThreads;
   if (grid >= (1LL << 31)) return STQ1_ERR_SHAPE;
   int rc = ensure_configured();
   if (rc != STQ1_OK) return rc;
-  return launch_pdl(stq2_encode_kernel, static_cast<unsigned>(grid), kStq2EncBlocks,
-                    static_cast<size_t>(kStq2EncBlocks) * kEncPitch * sizeof(float), static_cast<cudaStream_t>(stream),
-                    W, h, n_blocks, static_cast<int>(K / kBlockWeights), rounds, out);
+  const int nb = static_cast<int>(K / kBlockWeights);
+  const bool staged_h = h && nb <= kEncHMaxCols;
+  return launch_pdl(stq2_encode_kernel, static_cast<unsigned>(grid), kEncThreads, encode_smem_bytes(nb, staged_h),
+                    static_cast<cudaStream_t>(stream), W, h, n_blocks, nb, rounds, out);
 }
 
 extern "C" int stq1_hessian_diag(const uint16_t* x, int64_t L, int64_t rows, int64_t K, float* h, void* stream) {

@@ -87,6 +87,7 @@ def test_host_side_argument_checks_need_no_gpu():
     assert L.stq1_quantize_stq2(1 << 20, None, 4, 256, -1, 1 << 20, None) == -8
     assert L.stq1_quantize_stq2((1 << 20) + 4, None, 4, 256, 0, 1 << 20, None) == -6
     assert L.stq1_quantize_stq2(1 << 20, (1 << 20) + 2, 4, 256, 3, 1 << 20, None) == -6
+    assert L.stq1_quantize_stq2(1 << 20, (1 << 20) + 4, 4, 256, 3, 1 << 20, None) == -6   # h read as float4
     assert L.stq1_hessian_diag(None, 1, 4, 256, 1 << 20, None) == -2
     assert L.stq1_hessian_diag(1 << 20, 0, 4, 256, 1 << 20, None) == -1
     assert L.stq1_hessian_diag(1 << 20, 1, 0, 256, 1 << 20, None) == -1

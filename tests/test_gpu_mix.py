@@ -65,7 +65,9 @@ def _stq2_edge_matrix():
 
 
 @pytest.mark.parametrize("rounds", [0, 1, 3])
-@pytest.mark.parametrize("shape", [(1, 256), (7, 1024), (129, 2048)])
+# K up to 10240: the importance row is staged in shared memory; 12288 reads
+# it from global memory; 65 x 7168 ends in a partly filled warp
+@pytest.mark.parametrize("shape", [(1, 256), (7, 1024), (129, 2048), (65, 7168), (9, 10240), (3, 12288)])
 def test_stq2_encoder_matches_oracle(shape, rounds):
     n, k = shape
     w = workloads.expert_like_matrix(n, k, seeds=(n, k, 9))
