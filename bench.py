@@ -108,10 +108,13 @@ class ClockSampler:
         "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80,
     }
 
-    def __init__(self, index: int, period_s: float = 0.0005):
+    def __init__(self, index: int, period_s: float = 0.0):
+        # period 0: sample back to back (each NVML query takes a while), so that
+        # a timed region of a few milliseconds still gets several samples
         self.index, self.period = index, period_s
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
+        self._first = threading.Event()
         self._thr = None
         try:
             import pynvml
@@ -133,12 +136,14 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
+            self._first.set()
             time.sleep(self.period)
 
     def __enter__(self):
         if self.nv is not None:
             self._thr = threading.Thread(target=self._run, daemon=True)
             self._thr.start()
+            self._first.wait(1.0)          # the sampler is running when the region starts
         return self
 
     def __exit__(self, *exc):
