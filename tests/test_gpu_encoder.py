@@ -87,6 +87,37 @@ def test_encoder_flags_non_finite_inputs():
     assert stq1.status() & stq1.DEV_BAD_VALUE
 
 
+@pytest.mark.parametrize("k", [1024, 12288])
+def test_non_finite_blocks_inside_a_warp_leave_the_others_exact(k):
+    # A warp encodes 32 consecutive blocks and shares the copies of their
+    # weights, so a lane whose block is flagged keeps running every pass; the
+    # other lanes of its warp must still write the host encoder's bytes.
+    # k = 1024 stages the importance row in shared memory, 12288 reads it from
+    # global memory.
+    n = 40 if k == 1024 else 4
+    w = workloads.expert_like_matrix(n, k, seeds=(31, 32, 33))
+    h = workloads.calibration_importance(k, seed=34)
+    nb = k // 256
+    bad = [37, 70, n * nb - 1]                          # mid-warp, mid-warp, the very last block
+    clean = w.copy()
+    for j, blk in enumerate(bad):
+        r, c = divmod(blk, nb)
+        w[r, 256 * c + 17 * j] = (np.nan, np.inf, -np.inf)[j]
+        clean[r, 256 * c:256 * (c + 1)] = 0.0
+    for mode, hh in (("plain", None), ("sherry", h)):
+        g = _gpu_raw(w, hh, mode).reshape(-1, 42)
+        assert stq1.status() & stq1.DEV_BAD_VALUE
+        ref = stq1.quantize_ref(clean, hh, mode=mode).reshape(-1, 42).copy()
+        ref[bad] = 0
+        assert np.array_equal(g, ref)
+
+
+def _gpu_raw(w, h, mode):
+    wd = torch.from_numpy(np.ascontiguousarray(w, dtype=np.float32)).cuda()
+    hd = None if h is None else torch.from_numpy(np.ascontiguousarray(h, dtype=np.float32)).cuda()
+    return stq1.quantize_gpu(wd, hd, mode=mode, rounds=3).cpu().numpy()
+
+
 def test_weighted_error_study_1200_rows():
     # Synthetic stand-in for the pages' 1,200-row study (lemmy post, "Scale and
     # zero position are fit together"; the pages report ~90% lower

@@ -96,6 +96,27 @@ def test_stq2_encoder_full_layer_sampled():
     assert np.array_equal(g[rows], oracle.encode_stq2(w[rows], h, rounds=3).reshape(64, -1))
 
 
+@pytest.mark.parametrize("k", [1024, 12288])
+def test_stq2_non_finite_blocks_inside_a_warp_leave_the_others_exact(k):
+    # lanes of a flagged block keep running the passes (the weight copies are
+    # shared by the warp); the rest of the warp must match the oracle
+    n = 40 if k == 1024 else 4
+    w = workloads.expert_like_matrix(n, k, seeds=(41, 42, 43))
+    h = workloads.calibration_importance(k, seed=44)
+    nb = k // 256
+    bad = [37, n * nb - 1]
+    clean = w.copy()
+    for j, blk in enumerate(bad):
+        r, c = divmod(blk, nb)
+        w[r, 256 * c + 5] = (np.nan, np.inf)[j]
+        clean[r, 256 * c:256 * (c + 1)] = 0.0
+    g = stq1.stq2_quantize(_dev(w), _dev(h), rounds=3).cpu().numpy().reshape(-1, 66)
+    assert stq1.status() & stq1.DEV_BAD_VALUE
+    ref = oracle.encode_stq2(clean, h, rounds=3).reshape(-1, 66).copy()
+    ref[bad] = 0
+    assert np.array_equal(g, ref)
+
+
 def test_stq2_encoder_flags_non_finite():
     w = np.zeros((2, 512), np.float32)
     w[0, 3] = np.nan
