@@ -670,8 +670,10 @@ def run_sweep(args):
 
 
 def run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier):
-    """Public API, host buffers: per step copy x in from pinned memory, run the 64
-    GEMVs, read all outputs back to pinned memory."""
+    """Host buffers: per step copy x in from pinned memory, run the 64 GEMVs, read
+    all outputs back to pinned memory.  `value` goes through the C-ABI entry point
+    (stq1_gemv_prefetch) with the pointers ready, as a C caller makes the call;
+    `python_api` is the same loop through the Python binding (`stq1.gemv`)."""
     xh = torch.empty((1, K_COLS), dtype=torch.bfloat16).pin_memory()
     xh.copy_(xs[:1].cpu())
     yh = torch.empty((STACK, 1, N_ROWS), dtype=torch.float32).pin_memory()
@@ -679,32 +681,55 @@ def run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier):
     yd = torch.empty((STACK, 1, N_ROWS), dtype=torch.float32, device=device)
     steps = max(20, args.steps // 2)
 
-    # per-matrix views made once, as a decode loop over resident weights would
+    # per-matrix views and pointers made once, as a decode loop over resident weights would
     mats, outs = list(stack.unbind(0)), list(yd.unbind(0))
     nxt = mats[1:] + mats[:1]
+    import ctypes as C
+    call = stq1.LIB.stq1_gemv_prefetch
+    vp = C.c_void_p
+    common = (vp(xd.data_ptr()),)
+    tail = (C.c_int64(N_ROWS), C.c_int64(K_COLS), C.c_int(1), vp(ws.data_ptr()), C.c_size_t(ws.numel()))
+    # argument tuples built once (ctypes objects of the declared types pass without conversion)
+    argv = [(vp(w.data_ptr()),) + common + (vp(y.data_ptr()),) + tail + (vp(wn.data_ptr()), C.c_int64(PACKED),
+                                                                           vp(stream.cuda_stream))
+            for w, y, wn in zip(mats, outs, nxt)]
 
-    def one():
+    def one_abi():
+        xd.copy_(xh, non_blocking=True)
+        for a in argv:
+            rc = call(*a)
+            if rc:
+                raise RuntimeError(f"stq1_gemv_prefetch returned {rc}")
+        yh.copy_(yd, non_blocking=True)
+
+    def one_py():
         xd.copy_(xh, non_blocking=True)
         for w, y, wn in zip(mats, outs, nxt):
             stq1.gemv(w, xd, N_ROWS, K_COLS, out=y, ws=ws, prefetch=wn)
         yh.copy_(yd, non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            one()
-    torch.cuda.synchronize()
-    barrier()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for _ in range(steps):
-            one()
-        end.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(start.elapsed_time(end), device)
-    return {"value": round(whole_job_rate(STACK * PACKED * steps, world, ms) / 1e9, 1), "unit": "GB/s",
+    def timed_loop(one):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                one()
+        torch.cuda.synchronize()
+        barrier()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(steps):
+                one()
+            end.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(start.elapsed_time(end), device)
+
+    ms = timed_loop(one_abi)
+    ms_py = timed_loop(one_py)
+    rate = lambda t: round(whole_job_rate(STACK * PACKED * steps, world, t) / 1e9, 1)
+    return {"value": rate(ms), "unit": "GB/s",
             "h2d_bytes_per_step": K_COLS * 2, "d2h_bytes_per_step": STACK * N_ROWS * 4,
-            "steps": steps, "ms_per_step": round(ms / steps, 4)}
+            "steps": steps, "ms_per_step": round(ms / steps, 4), "route": "C ABI (stq1_gemv_prefetch)",
+            "python_api": {"value": rate(ms_py), "ms_per_step": round(ms_py / steps, 4), "route": "stq1.gemv"}}
 
 
 # ---------------------------------------------------------------------------
