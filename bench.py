@@ -685,7 +685,12 @@ def run_e2e(torch, stq1, device, stream, stack, xs, ws, args, world, barrier):
     mats, outs = list(stack.unbind(0)), list(yd.unbind(0))
     nxt = mats[1:] + mats[:1]
     import ctypes as C
-    call = stq1.LIB.stq1_gemv_prefetch
+    stq1.LIB.stq1_gemv_prefetch                   # loads the library (and checks its version)
+    # the same symbol through a handle without declared argument types: the
+    # arguments below are already ctypes objects of the C types, so no per-call
+    # conversion runs
+    call = C.CDLL(stq1.LIB_PATH).stq1_gemv_prefetch
+    call.restype = C.c_int
     vp = C.c_void_p
     common = (vp(xd.data_ptr()),)
     tail = (C.c_int64(N_ROWS), C.c_int64(K_COLS), C.c_int(1), vp(ws.data_ptr()), C.c_size_t(ws.numel()))
