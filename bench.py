@@ -865,6 +865,24 @@ def profile_case(args):
         torch.cuda.synchronize()
         print("profile case done", o.cpu().numpy().tolist())
         return
+    if args.profile_case == "encode":
+        # two [4096, 7168] fp32 layers (235 MB, larger than L2) with importances;
+        # launches alternate Sherry (3 rounds) and STQ2 (3 rounds), so the first
+        # two captured launches are one of each, on a layer not read before
+        g = torch.Generator(device=device)
+        g.manual_seed(7)
+        w = torch.randn((2, N_ROWS, K_COLS), device=device, generator=g) * 0.02
+        h = torch.rand((K_COLS,), device=device, generator=g)
+        clean = torch.empty(64 << 20, dtype=torch.float32, device=device)
+        float(clean.sum())
+        del clean
+        outs = []
+        for l in range(2):
+            outs.append(stq1.quantize_gpu(w[l], h, mode="sherry", rounds=3))
+            outs.append(stq1.stq2_quantize(w[1 - l], h, rounds=3))
+        torch.cuda.synchronize()
+        print("profile case done", [int(o.view(torch.int16).sum(dtype=torch.int64)) for o in outs])
+        return
     if args.profile_case in ("moe", "prefill"):
         stream = torch.cuda.Stream(device)
         fn = run_moe if args.profile_case == "moe" else run_prefill
@@ -895,7 +913,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", default=None, choices=["gemv", "moe", "prefill", "mix"])
+    ap.add_argument("--profile-case", default=None, choices=["gemv", "moe", "prefill", "mix", "encode"])
     ap.add_argument("--sweep", action="store_true", help="crossover sweep (18432 x 7168, batch 1..1024)")
     args = ap.parse_args()
     if args.sweep:
