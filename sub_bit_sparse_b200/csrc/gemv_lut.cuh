@@ -165,7 +165,11 @@ __device__ __forceinline__ void lut_build(const uint2 (&xv)[kLutMaxTT], uint32_t
 // (expert * N + slab * 128); xr / orow = activation row pointers and output
 // rows of the tile's tokens.  Threads q and q + 128 own the same row; the
 // first decodes the chunk's first block, the second its second block.
-template <int TT>
+// DB (a one-token unit in a launch sized for two or more tokens): the unused
+// second token's table space holds a second table, so chunk c + 1's table is
+// built while slower threads still read chunk c's, and a chunk needs one
+// barrier instead of two.
+template <int TT, bool DB = false>
 __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wmap, const CUtensorMap* tmap, long long R0,
                          int slab, int split, int unit, const uint16_t* const (&xr)[kLutMaxTT],
                          const int (&orow)[kLutMaxTT], const int (&wrow)[kLutMaxTT], uint8_t* smem) {
@@ -185,7 +189,7 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t lut = (sbase + 255u) & ~255u;
-  const uint32_t bar0 = lut + TT * kLutTokenBytes;   // 2 mbarriers
+  const uint32_t bar0 = lut + (DB ? 2 : TT) * kLutTokenBytes;   // 2 mbarriers
   const uint32_t stage0 = bar0 + 128;                // 128-aligned tensor-copy destinations
   const int NS = (c1 - c0 >= 2) ? 2 : 1;
   // split-K partials pushed by the cluster, at the same offset in every CTA of it
@@ -245,33 +249,44 @@ __device__ __forceinline__ void lut_unit(const LutArgs& a, const CUtensorMap* wm
   griddep_launch_dependents();
   uint2 xv[kLutMaxTT];
   lut_load_x<TT>(xr, c0, xv);
-  const uint32_t lut_half = lut + static_cast<uint32_t>(half * kGroupsPerBlock * kLutGroupBytes);
+  const uint32_t half_off = static_cast<uint32_t>(half * kGroupsPerBlock * kLutGroupBytes);
   bool failed = false;
   for (int c = c0; c < c1; ++c) {
     const int it = c - c0;
     const int st = NS == 2 ? (it & 1) : 0;
     const uint32_t parity = static_cast<uint32_t>(NS == 2 ? (it >> 1) : it) & 1u;
-    lut_build<TT>(xv, lut);
+    // DB: chunk c's table goes to the buffer chunk c - 2 used; every thread
+    // finished reading that one before it passed chunk c - 1's barrier
+    const uint32_t lut_c = DB ? lut + static_cast<uint32_t>((it & 1) * kLutTokenBytes) : lut;
+    lut_build<TT>(xv, lut_c);
     if (c + 1 < c1) lut_load_x<TT>(xr, c + 1, xv);   // prefetch the next chunk's activations
     const bool landed = mbar_wait_bounded(bar0 + 8u * st, parity);
-    // one barrier: tables built, copies landed (agreed by every thread)
+    // one barrier: tables built, copies landed (agreed by every thread); with
+    // DB also every thread done with chunk c - 1, so its stage is free
     if (!__syncthreads_and(landed)) {
       // A copy did not complete within the bound (the error word is set).
       // Wait (bounded) for the copies already issued into the other stage, so
       // no tensor copy is still writing this CTA's shared memory when it exits.
-      if (NS == 2 && c + 1 < c1) mbar_wait_bounded(bar0 + 8u * (st ^ 1), static_cast<uint32_t>((it + 1) >> 1) & 1u);
+      // (With DB the next chunk's copy is issued only after this barrier, so
+      // the other stage has one in flight only in the first iteration.)
+      if (NS == 2 && c + 1 < c1 && (!DB || it == 0))
+        mbar_wait_bounded(bar0 + 8u * (st ^ 1), static_cast<uint32_t>((it + 1) >> 1) & 1u);
       failed = true;
       break;
     }
+    if (DB && threadIdx.x == 0 && it >= 1 && c + 1 < c1) issue(c + 1, st ^ 1);   // chunk c - 1's stage
     if (row_ok) {
       // only the extraction depends on the block's offset; one copy of the body follows
       BlockCodes b;
       load_chunk_block(stage0 + st * a.g.stage_bytes + my_slot, packed_window_offset(a.g, res, c), half, b);
-      lut_block_body<TT>(b, lut_half, acc);
+      lut_block_body<TT>(b, lut_c + half_off, acc);
     }
-    __syncthreads();
-    if (threadIdx.x == 0 && c + NS < c1) issue(c + NS, st);   // this stage is free again
+    if (!DB) {
+      __syncthreads();
+      if (threadIdx.x == 0 && c + NS < c1) issue(c + NS, st);   // this stage is free again
+    }
   }
+  if (DB) __syncthreads();                         // every lookup done: the tables are free below
 
   if (push) {
     // Push both halves' partials into the shared memory of the CTA that owns
@@ -425,7 +440,7 @@ lut_gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant_
       return;
     }
   }
-  lut_unit<1>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, wrow, smem);
+  lut_unit<1, (TTMAX >= 2)>(a, &wmap, &tmap, R0, slab, split, unit, xr, orow, wrow, smem);
 }
 
 // Dynamic shared memory: tables, barriers, stages and (cluster split K) the
