@@ -166,3 +166,21 @@ def test_table_kernel_small_batches(table_path, n, k, b):
 
 def test_table_kernel_moe(table_path):
     _moe(256, 1024, 12, 9, 4, 1, seed=9100)
+
+
+def test_table_kernel_one_token_tile_over_many_chunks(table_path):
+    # Batch 5 on the table kernel: a four-token tile and a one-token tile.
+    # With 112 slabs the split is one piece per unit, so every CTA runs all 14
+    # chunks, and the one-token unit alternates two tables (one barrier per
+    # chunk, each chunk's copy issued after the previous chunk's barrier).
+    # Rows of the first, a middle and the last slab against the oracle.
+    n, k, b = 14336, 7168, 5
+    rb = k // 256 * 42
+    packed = workloads.random_packed_blocks(n * k // 256, seed=9200)
+    x = workloads.activations_bf16(b, k, seed=9201)
+    y = stq1.gemv(_dev(packed), _bf16(x), n, k).cpu().numpy()
+    assert stq1.status() == 0
+    for r0 in (0, 7040, n - 128):
+        sub = packed[r0 * rb:(r0 + 128) * rb]
+        _assert_close(y[:, r0:r0 + 128], oracle.gemv(sub, x, 128, k), oracle.gemv_abs(sub, x, 128, k),
+                      f"rows {r0}..{r0 + 127}")
